@@ -1,0 +1,385 @@
+/*
+ * w4_oracle.c -- plain CPU oracle for group-wise INT4 weight quantization and
+ * W4A16 inference.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path (the CUDA library
+ * under int4_w4a16_b200/) includes, links or calls this file.  Only tests/,
+ * the smoke check in __graft_entry__.py and the cpu_baseline / reference arm
+ * of bench.py load it.  It shares no code, header, table or constant with the
+ * CUDA path.
+ *
+ * Every function is the plain definition of what the method computes, in the
+ * order the sources state it, with no blocking, fusion or reordering.  Loops
+ * over independent rows may run on several OpenMP threads; the arithmetic of
+ * each output element is the same sequential code whatever the thread count.
+ *
+ * Sources (cited by page title and section):
+ *   [QAT]  SGLang RL team, "INT4 QAT end-to-end" blog (re-post): fake
+ *          quantization + STE in Megatron (_FakeInt4QuantizationSTE), the
+ *          [-7, 7] simulated INT4 range, Fig. 4 "Rollout-side INT4 weight
+ *          only" (8 INT4 values packed into one INT32, 8 x 4 bits = 32 bits,
+ *          pack_int4_to_int32), moe_align_block_size, "MoE operator deep
+ *          fusion".
+ *   [TAG]  reportify.cn concept page "量化感知训练" (quantization-aware
+ *          training): para. [8][9] fake quant forward / STE backward,
+ *          [10] real quantization of the exported weights, [11] 1x32 scale
+ *          granularity, [32] two 4-bit weights per byte, [35]
+ *          moe_align_block_size.
+ *   [BAS]  "量化基础：从 FP32 到 INT4 的压缩艺术" (quantization basics):
+ *          §1.3 table (INT4 range [-8, 7], BF16 = 1+8+7 bits),
+ *          §2.2 symmetric quantization s = max|x| / q_max,
+ *               q = clamp(round(x / s), -q_max, q_max),
+ *          §2.4 error bound |x_hat - x| <= s/2,
+ *          §6.1 numpy symmetric quantizer and its printed output,
+ *          §6.2 torch.round rounds half to even.
+ *
+ * Readings where the sources are silent (each is listed in the design doc):
+ *   - groups are 32 contiguous elements along K (the reduction dim) of a
+ *     row-major [rows, K] BF16 matrix ([TAG] [11] "1x32");
+ *   - s32 = fl32(amax / 7) in IEEE fp32, then s = bf16_rne(s32) is the
+ *     stored scale, and q divides by that stored BF16 scale, so that fake
+ *     quantization and dequantized export agree bit for bit;
+ *   - q = clamp(rint_half_even(fl32(w / s)), -8, 7); with this scale the clamp
+ *     never fires, so the [-7, 7] and [-8, 7] readings coincide;
+ *   - amax == 0 or s rounding to 0 gives s = +0 and q = 0 for the group;
+ *   - Wdq = bf16_rne(q * s), +0.0 when q == 0;
+ *   - packing is low nibble first, two's complement nibbles, along K;
+ *   - moe_align: stable sort of (token, k) slots by expert, runs padded to a
+ *     multiple of the block size, sentinel T*topk, expert id -1 past the end.
+ *
+ * Inputs are assumed finite (NaN / Inf behaviour is unspecified).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------------ */
+/* BF16 <-> FP32 ([BAS] §1.3: BF16 is 1 sign, 8 exponent, 7 mantissa bits,  */
+/* i.e. the upper half of an IEEE fp32).                                     */
+/* ------------------------------------------------------------------------ */
+
+float w4o_f32_from_bf16(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* Round an fp32 to the nearest BF16, ties to even (finite inputs). */
+uint16_t w4o_bf16_from_f32(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    uint32_t upper = u >> 16;
+    uint32_t lower = u & 0xFFFFu;
+    if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u)))
+        upper += 1u;
+    return (uint16_t)upper;
+}
+
+void w4o_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+int w4o_get_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* ------------------------------------------------------------------------ */
+/* Group-32 symmetric INT4 quantization ([QAT] fake quantization / real      */
+/* quantization; [BAS] §2.2 with q_max = 7 and the INT4 clamp of §1.3).      */
+/* ------------------------------------------------------------------------ */
+
+/* One group: returns the stored BF16 scale and writes q[0..n-1]. */
+static uint16_t quantize_one_group(const uint16_t *w, int64_t n, int8_t *q)
+{
+    /* step 1: amax = max |w| over the group, on the BF16 values */
+    float amax = 0.0f;
+    for (int64_t i = 0; i < n; ++i) {
+        float a = fabsf(w4o_f32_from_bf16(w[i]));
+        if (a > amax) amax = a;
+    }
+    /* step 2: s32 = amax / 7 in IEEE fp32 */
+    volatile float seven = 7.0f;
+    float s32 = amax / seven;
+    /* step 3: the stored scale is BF16 */
+    uint16_t s_bits = w4o_bf16_from_f32(s32);
+    float s = w4o_f32_from_bf16(s_bits);
+    /* step 4: q = clamp(round_half_even(w / s), -8, 7); q = 0 when s == 0 */
+    for (int64_t i = 0; i < n; ++i) {
+        if (s == 0.0f) {
+            q[i] = 0;
+            continue;
+        }
+        float y = w4o_f32_from_bf16(w[i]) / s;      /* IEEE fp32 quotient */
+        float r = nearbyintf(y);                     /* default mode: ties to even */
+        if (r < -8.0f) r = -8.0f;
+        if (r > 7.0f) r = 7.0f;
+        q[i] = (int8_t)r;
+    }
+    return s_bits;
+}
+
+/* q[rows*K] int8 codes and S[rows*(K/group)] BF16 scales. */
+void w4o_quantize(const uint16_t *W, int64_t rows, int64_t K, int64_t group,
+                  int8_t *q, uint16_t *S)
+{
+    int64_t gpr = K / group;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t g = 0; g < gpr; ++g) {
+            int64_t base = r * K + g * group;
+            S[r * gpr + g] = quantize_one_group(W + base, group, q + base);
+        }
+}
+
+/* Dequantized value of one code: bf16_rne(q * s), +0.0 for q == 0. */
+static uint16_t dequant_one(int8_t q, uint16_t s_bits)
+{
+    float s = w4o_f32_from_bf16(s_bits);
+    float v = (float)q * s;          /* exact in fp32: <= 4 x 8 significant bits */
+    if (v == 0.0f) v = 0.0f;         /* +0.0 */
+    return w4o_bf16_from_f32(v);
+}
+
+/* Fake quantization (quantize then immediately dequantize, storage stays BF16):
+ * Wdq[rows*K]; S may be NULL. */
+void w4o_fake_quant(const uint16_t *W, int64_t rows, int64_t K, int64_t group,
+                    uint16_t *Wdq, uint16_t *S)
+{
+    int64_t gpr = K / group;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        int8_t *qg = (int8_t *)malloc((size_t)group);
+        for (int64_t g = 0; g < gpr; ++g) {
+            int64_t base = r * K + g * group;
+            uint16_t s_bits = quantize_one_group(W + base, group, qg);
+            if (S) S[r * gpr + g] = s_bits;
+            for (int64_t i = 0; i < group; ++i)
+                Wdq[base + i] = dequant_one(qg[i], s_bits);
+        }
+        free(qg);
+    }
+}
+
+/* Straight-through estimator backward: the gradient passes through the
+ * rounding unchanged ([QAT] §2.1; [TAG] [9][17]). */
+void w4o_ste_backward(const uint16_t *dWdq, int64_t n, uint16_t *dW)
+{
+    for (int64_t i = 0; i < n; ++i) dW[i] = dWdq[i];
+}
+
+/* ------------------------------------------------------------------------ */
+/* Packing ([QAT] Fig. 4: eight INT4 values in one INT32; element i of the   */
+/* eight sits at bits [4i, 4i+3] as a two's-complement nibble).              */
+/* ------------------------------------------------------------------------ */
+
+int32_t w4o_pack8(const int8_t *q8)
+{
+    uint32_t word = 0;
+    for (int i = 0; i < 8; ++i)
+        word |= ((uint32_t)q8[i] & 0xFu) << (4 * i);
+    return (int32_t)word;
+}
+
+void w4o_unpack8(int32_t word, int8_t *q8)
+{
+    uint32_t u = (uint32_t)word;
+    for (int i = 0; i < 8; ++i) {
+        int v = (int)((u >> (4 * i)) & 0xFu);
+        q8[i] = (int8_t)(v >= 8 ? v - 16 : v);
+    }
+}
+
+void w4o_pack(const int8_t *q, int64_t n, int32_t *words)
+{
+    for (int64_t j = 0; j < n / 8; ++j) words[j] = w4o_pack8(q + 8 * j);
+}
+
+void w4o_unpack(const int32_t *words, int64_t n, int8_t *q)
+{
+    for (int64_t j = 0; j < n / 8; ++j) w4o_unpack8(words[j], q + 8 * j);
+}
+
+/* Real quantization for export: codes packed along K into Wq[rows*(K/8)]
+ * plus BF16 scales S[rows*(K/group)]. */
+void w4o_quantize_pack(const uint16_t *W, int64_t rows, int64_t K, int64_t group,
+                       int32_t *Wq, uint16_t *S)
+{
+    int64_t gpr = K / group;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        int8_t *qrow = (int8_t *)malloc((size_t)K);
+        for (int64_t g = 0; g < gpr; ++g)
+            S[r * gpr + g] = quantize_one_group(W + r * K + g * group, group,
+                                                qrow + g * group);
+        w4o_pack(qrow, K, Wq + r * (K / 8));
+        free(qrow);
+    }
+}
+
+/* Inverse of the export: unpack the codes and dequantize them. */
+void w4o_dequant(const int32_t *Wq, const uint16_t *S, int64_t rows, int64_t K,
+                 int64_t group, uint16_t *Wdq)
+{
+    int64_t gpr = K / group;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        int8_t *qrow = (int8_t *)malloc((size_t)K);
+        w4o_unpack(Wq + r * (K / 8), K, qrow);
+        for (int64_t k = 0; k < K; ++k)
+            Wdq[r * K + k] = dequant_one(qrow[k], S[r * gpr + k / group]);
+        free(qrow);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Generic symmetric quantizer of [BAS] §2.2 / §6.1, in fp64, with the scale */
+/* left unrounded: s = max|x| / qmax per group, q = clip(round(x/s)).       */
+/* Used to reproduce the page's worked INT8 example.                         */
+/* ------------------------------------------------------------------------ */
+void w4o_symmetric_quantize_f64(const double *x, int64_t n, int64_t group,
+                                int qmax, int32_t *q, double *s_out)
+{
+    for (int64_t g0 = 0, gi = 0; g0 < n; g0 += group, ++gi) {
+        int64_t len = (n - g0 < group) ? n - g0 : group;
+        double amax = 0.0;
+        for (int64_t i = 0; i < len; ++i)
+            if (fabs(x[g0 + i]) > amax) amax = fabs(x[g0 + i]);
+        double s = amax / (double)qmax;
+        s_out[gi] = s;
+        for (int64_t i = 0; i < len; ++i) {
+            double r = (s == 0.0) ? 0.0 : nearbyint(x[g0 + i] / s);
+            if (r < -qmax) r = -qmax;
+            if (r > qmax) r = qmax;
+            q[g0 + i] = (int32_t)r;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* W4A16 GEMM: Y = X . dq(W)^T, FP32 accumulation in ascending k, one BF16   */
+/* rounding of the result.  R (optional) receives the fp32 sums.             */
+/* ------------------------------------------------------------------------ */
+void w4o_gemm(const uint16_t *X, const uint16_t *Wdq, int64_t M, int64_t N,
+              int64_t K, uint16_t *Y, float *R)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t m = 0; m < M; ++m) {
+            float acc = 0.0f;
+            for (int64_t k = 0; k < K; ++k) {
+                float prod = w4o_f32_from_bf16(X[m * K + k]) *
+                             w4o_f32_from_bf16(Wdq[n * K + k]);   /* exact */
+                acc = acc + prod;
+            }
+            if (R) R[m * N + n] = acc;
+            if (Y) Y[m * N + n] = w4o_bf16_from_f32(acc);
+        }
+}
+
+/* Same product, read straight from the packed export (unpack + dequant of one
+ * row of W at a time, then the plain dot products). */
+void w4o_w4a16_gemm(const uint16_t *X, const int32_t *Wq, const uint16_t *S,
+                    int64_t M, int64_t N, int64_t K, int64_t group,
+                    uint16_t *Y, float *R)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        uint16_t *wrow = (uint16_t *)malloc((size_t)K * sizeof(uint16_t));
+        w4o_dequant(Wq + n * (K / 8), S + n * (K / group), 1, K, group, wrow);
+        for (int64_t m = 0; m < M; ++m) {
+            float acc = 0.0f;
+            for (int64_t k = 0; k < K; ++k)
+                acc = acc + w4o_f32_from_bf16(X[m * K + k]) *
+                            w4o_f32_from_bf16(wrow[k]);
+            if (R) R[m * N + n] = acc;
+            if (Y) Y[m * N + n] = w4o_bf16_from_f32(acc);
+        }
+        free(wrow);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* moe_align_block_size ([QAT] "merge and align the tokens of the same       */
+/* expert"; [TAG] [35]).  Slot i = t*topk + k routes to e_i = topk_ids[i].   */
+/* Each expert's slots, in ascending slot order, form one run padded up to   */
+/* a multiple of `block`; runs follow in ascending expert id.  Padding and   */
+/* everything past the padded total hold the sentinel T*topk; expert_ids is  */
+/* the expert of each block, -1 past the end.  Slots whose expert id is out  */
+/* of [0, E) are skipped.  Returns 0, or -1 if `cap` is too small.           */
+/* ------------------------------------------------------------------------ */
+int w4o_moe_align(const int32_t *topk_ids, int64_t T, int64_t topk, int64_t E,
+                  int64_t block, int32_t *sorted_ids, int64_t cap,
+                  int32_t *expert_ids, int32_t *num_post_pad)
+{
+    int64_t slots = T * topk;
+    int64_t *cnt = (int64_t *)calloc((size_t)E, sizeof(int64_t));
+    for (int64_t i = 0; i < slots; ++i) {
+        int32_t e = topk_ids[i];
+        if (e >= 0 && e < E) cnt[e] += 1;
+    }
+    int64_t total = 0;
+    for (int64_t e = 0; e < E; ++e)
+        total += (cnt[e] + block - 1) / block * block;
+    if (total > cap) {
+        free(cnt);
+        return -1;
+    }
+    for (int64_t p = 0; p < cap; ++p) sorted_ids[p] = (int32_t)slots;
+    for (int64_t b = 0; b < cap / block; ++b) expert_ids[b] = -1;
+    int64_t off = 0;
+    for (int64_t e = 0; e < E; ++e) {
+        int64_t r = 0;
+        for (int64_t i = 0; i < slots; ++i)       /* ascending slot order */
+            if (topk_ids[i] == e) sorted_ids[off + r++] = (int32_t)i;
+        int64_t padded = (cnt[e] + block - 1) / block * block;
+        for (int64_t b = off / block; b < (off + padded) / block; ++b)
+            expert_ids[b] = (int32_t)e;
+        off += padded;
+    }
+    *num_post_pad = (int32_t)total;
+    free(cnt);
+    return 0;
+}
+
+/* Grouped W4A16 GEMM over the aligned slot list: for every block b with
+ * expert e and every real slot in it, C[slot, :] = A[slot / a_row_div, :] .
+ * dq(W_e)^T, with the same fp32 accumulation as w4o_gemm.  Wdq holds every
+ * expert's dequantized weights, [E, N, K].  Padding slots are not written. */
+void w4o_moe_gemm(const uint16_t *A, int64_t a_row_div, const uint16_t *Wdq,
+                  const int32_t *sorted_ids, const int32_t *expert_ids,
+                  int64_t num_post_pad, int64_t num_slots, int64_t block,
+                  int64_t N, int64_t K, uint16_t *C, float *R)
+{
+    #pragma omp parallel for schedule(dynamic)
+    for (int64_t p = 0; p < num_post_pad; ++p) {
+        int32_t slot = sorted_ids[p];
+        int32_t e = expert_ids[p / block];
+        if (slot < 0 || slot >= num_slots || e < 0) continue;
+        const uint16_t *a = A + (int64_t)(slot / a_row_div) * K;
+        const uint16_t *w = Wdq + (int64_t)e * N * K;
+        for (int64_t n = 0; n < N; ++n) {
+            float acc = 0.0f;
+            for (int64_t k = 0; k < K; ++k)
+                acc = acc + w4o_f32_from_bf16(a[k]) * w4o_f32_from_bf16(w[n * K + k]);
+            if (R) R[(int64_t)slot * N + n] = acc;
+            if (C) C[(int64_t)slot * N + n] = w4o_bf16_from_f32(acc);
+        }
+    }
+}
