@@ -1,0 +1,495 @@
+#!/usr/bin/env python3
+"""Benchmark of the INT4 W4A16 hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode|prefill|moe|qat]
+
+Default workload: the decode GEMV sweep -- W[12288, 4096] BF16 ~ N(0, 0.02^2)
+with 0.1 % x20 outliers, group 32, activations X[M, 4096] ~ N(0, 1) for
+M in {1, 8, 16, 32}.  One step is one pass of the whole hot path over it:
+  1. fake quantization of W (QAT forward, w4_fake_quant),
+  2. the STE backward of the gradient into a separate buffer (w4_ste_backward),
+  3. real quantization + packing of W (export, w4_quantize_pack),
+  4. the W4A16 GEMM for each M (decode, w4a16_gemm).
+The metric is the step's algorithmic HBM throughput (GB/s): the bytes each
+kernel must move at minimum, summed over the step, divided by the step time.
+Every kernel reads inputs that are not resident in L2: W and the gradients
+alternate between two copies, the decode GEMMs rotate over eight packed copies
+of the weight (each copy is about 28 MB; L2 is 126 MB).
+
+--impl reference times the CPU oracle (plain C, all host cores) on the same
+workload and metric; under torchrun only rank 0 runs it.
+
+Multi-GPU (torchrun): each rank runs an independent replica of the workload
+(weak scaling; no collective on the data path); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+# DRAM traffic per launch from ncu captures (dram__bytes_read.sum +
+# dram__bytes_write.sum), keyed by kernel; each entry records the SHA-256 of the
+# CUDA source it was measured on, so a changed kernel reports null.
+NCU_TRAFFIC = {}
+
+
+def _src_hash(fname: str) -> str:
+    with open(os.path.join(ROOT, "int4_w4a16_b200", "csrc", fname), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def _traffic(kernel: str, workload_key: str):
+    e = NCU_TRAFFIC.get((kernel, workload_key))
+    if e is None or e["src"] != _src_hash(e["file"]):
+        return None
+    return e["bytes"]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# Decode workload (default bench line)
+# ---------------------------------------------------------------------------
+
+class DecodeWorkload:
+    name = "decode"
+
+    def __init__(self, device):
+        import int4_w4a16_b200 as w4
+        self.w4 = w4
+        cfg = synth.Decode()
+        self.cfg = cfg
+        self.N, self.K, self.Ms = cfg.N, cfg.K, cfg.Ms
+        N, K = self.N, self.K
+        self.W = [cfg.weight(device), synth.normal_bf16((N, K), 0.02, cfg.seed, 1, device,
+                                                        outlier_frac=0.001)]
+        self.G = [cfg.grads(device), synth.normal_bf16((N, K), 1e-3, cfg.seed, 6, device)]
+        self.X = {M: cfg.activations(M, device) for M in self.Ms}
+        self.Wdq = torch.empty_like(self.W[0])
+        self.dW = torch.empty_like(self.W[0])
+        self.Wq = torch.empty((N, K // 8), dtype=torch.int32, device=device)
+        self.S = torch.empty((N, K // 32), dtype=torch.bfloat16, device=device)
+        # eight packed copies for the decode GEMMs (L2-cold reads)
+        self.copies = []
+        for i in range(8):
+            Wq, S = w4.quantize_pack(self.W[i % 2])
+            self.copies.append((Wq, S))
+        self.Y = {M: torch.empty((M, N), dtype=torch.bfloat16, device=device) for M in self.Ms}
+        self.step_idx = 0
+        nk = N * K
+        self.kernels = ["fake_quant", "ste_backward", "quantize_pack"] + [f"gemm_m{M}" for M in self.Ms]
+        self.bytes = {"fake_quant": 4 * nk, "ste_backward": 4 * nk,
+                      "quantize_pack": 2 * nk + nk // 2 + nk // 16}
+        self.flops = {}
+        for M in self.Ms:
+            self.bytes[f"gemm_m{M}"] = nk // 2 + nk // 16 + 2 * M * K + 2 * M * N
+            self.flops[f"gemm_m{M}"] = 2 * M * N * K
+        self.launches_per_step = 3 + len(self.Ms)
+
+    def step(self, ev=None):
+        """One pass; ev (optional) = {kernel: (start_event, end_event)} to record."""
+        w4 = self.w4
+        i = self.step_idx
+        self.step_idx += 1
+        W, G = self.W[i % 2], self.G[i % 2]
+
+        def rec(name, fn):
+            if ev is not None:
+                ev[name][0].record()
+            fn()
+            if ev is not None:
+                ev[name][1].record()
+
+        rec("fake_quant", lambda: w4.w4_fake_quant(W, self.Wdq))
+        rec("ste_backward", lambda: w4.w4_ste_backward(G, self.dW))
+        rec("quantize_pack", lambda: w4.w4_quantize_pack(W, self.Wq, self.S))
+        for j, M in enumerate(self.Ms):
+            Wq, S = self.copies[(4 * i + j) % len(self.copies)]
+            rec(f"gemm_m{M}", lambda: w4.w4a16_gemm(self.X[M], Wq, S, self.Y[M]))
+
+    def e2e_step(self, host):
+        """Same pass through the public API from pinned host buffers, with the
+        step's inputs copied in and its results copied out."""
+        w4 = self.w4
+        W = host["W"].to(self.W[0].device, non_blocking=True)
+        G = host["G"].to(self.W[0].device, non_blocking=True)
+        Xs = {M: host["X"][M].to(self.W[0].device, non_blocking=True) for M in self.Ms}
+        w4.w4_fake_quant(W, self.Wdq)
+        w4.w4_ste_backward(G, self.dW)
+        w4.w4_quantize_pack(W, self.Wq, self.S)
+        for M in self.Ms:
+            w4.w4a16_gemm(Xs[M], self.Wq, self.S, self.Y[M])
+        host["Wdq"].copy_(self.Wdq, non_blocking=True)
+        host["dW"].copy_(self.dW, non_blocking=True)
+        host["Wq"].copy_(self.Wq, non_blocking=True)
+        host["S"].copy_(self.S, non_blocking=True)
+        for M in self.Ms:
+            host["Y"][M].copy_(self.Y[M], non_blocking=True)
+
+    def host_buffers(self):
+        pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h = {"W": pin(self.W[0]), "G": pin(self.G[0]),
+             "X": {M: pin(self.X[M]) for M in self.Ms},
+             "Wdq": pin(self.Wdq), "dW": pin(self.dW), "Wq": pin(self.Wq), "S": pin(self.S),
+             "Y": {M: pin(self.Y[M]) for M in self.Ms}}
+        h["W"].copy_(self.W[0])
+        h["G"].copy_(self.G[0])
+        for M in self.Ms:
+            h["X"][M].copy_(self.X[M])
+        h2d = h["W"].nbytes + h["G"].nbytes + sum(x.nbytes for x in h["X"].values())
+        d2h = (h["Wdq"].nbytes + h["dW"].nbytes + h["Wq"].nbytes + h["S"].nbytes +
+               sum(y.nbytes for y in h["Y"].values()))
+        return h, h2d, d2h
+
+    @property
+    def step_bytes(self):
+        return sum(self.bytes.values())
+
+    @property
+    def step_flops(self):
+        return sum(self.flops.values())
+
+    def config(self):
+        return decode_config()
+
+
+def decode_config():
+    cfg = synth.Decode()
+    return {"workload": "decode GEMV sweep: W[12288,4096] BF16 N(0,0.02^2) + 0.1% x20 "
+                        "outliers, group 32, X[M,4096] N(0,1), M in {1,8,16,32}; step = "
+                        "fake_quant + STE (separate buffer) + quantize_pack of W, then "
+                        "the W4A16 GEMM for each M",
+            "N": cfg.N, "K": cfg.K, "M": list(cfg.Ms), "group": 32,
+            "l2": "inputs larger than L2: W and grads alternate over 2 copies (100 MB "
+                  "each), the GEMMs rotate over 8 packed copies (28.3 MB each)"}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle arm (cpu_baseline and --impl reference)
+# ---------------------------------------------------------------------------
+
+def oracle_decode_step(state):
+    import oracle
+    oracle.fake_quant(state["W"])
+    oracle.ste_backward(state["G"])
+    Wq, S = oracle.quantize_pack(state["W"])
+    for M, X in state["X"].items():
+        oracle.w4a16_gemm(X, Wq, S, want_r=False)
+
+
+def oracle_state(rows: int):
+    """The decode workload restricted to the first `rows` rows of W (and of the
+    gradient); the GEMMs then produce the first `rows` columns of Y."""
+    cfg = synth.Decode()
+    W = synth.bits(cfg.weight()[:rows])
+    G = synth.bits(cfg.grads()[:rows])
+    X = {M: synth.bits(cfg.activations(M)) for M in cfg.Ms}
+    K = cfg.K
+    nk = rows * K
+    b = 4 * nk + 4 * nk + (2 * nk + nk // 2 + nk // 16)
+    for M in cfg.Ms:
+        b += nk // 2 + nk // 16 + 2 * M * K + 2 * M * rows
+    return {"W": W, "G": G, "X": X}, b
+
+
+def time_oracle(target_s: float = 15.0, rows: int = 1024):
+    import oracle
+    st, nbytes = oracle_state(rows)
+    t0 = time.perf_counter()
+    oracle_decode_step(st)
+    one = time.perf_counter() - t0
+    reps = max(1, int(target_s / max(one, 1e-3)))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle_decode_step(st)
+    dt = (time.perf_counter() - t0) / reps
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": oracle.get_threads(),
+            "kind": "oracle",
+            "sample": f"decode workload restricted to W rows 0..{rows - 1} of 12288 "
+                      f"({rows / 12288:.1%} of each kernel's work), {reps} timed passes "
+                      f"after one warm pass",
+            "sec_per_pass": dt}
+
+
+# ---------------------------------------------------------------------------
+# Main
+# ---------------------------------------------------------------------------
+
+def dist_setup(n_gpus: int):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    st, nbytes = oracle_state(args.ref_rows)
+    for _ in range(args.warmup if args.warmup < 3 else 1):
+        oracle_decode_step(st)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_decode_step(st)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = nbytes / dt / 1e9
+    sample = (f"decode workload restricted to W rows 0..{args.ref_rows - 1} of 12288 per "
+              f"step ({args.ref_rows / 12288:.1%} of each kernel's work)")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": decode_config(),
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.get_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+METRIC = "W4A16 hot-path HBM throughput (decode GEMV sweep + QAT fake-quant/STE + quantize_pack), GB/s"
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode", choices=["decode"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-rows", type=int, default=512)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    args = ap.parse_args()
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        return run_reference(args, rank, 1)
+
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}))
+        return 1
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    import int4_w4a16_b200 as w4
+    w4.lib()
+    wl = DecodeWorkload(dev)
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream()
+
+    for _ in range(max(3, args.warmup)):
+        wl.step()
+    w4.w4_device_status()
+
+    sampler = ClockSampler(local) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    # pre-roll so that the clock sampler sees the GPU under this load
+    t_end = time.perf_counter() + 0.6
+    while time.perf_counter() < t_end:
+        wl.step()
+    torch.cuda.synchronize()
+
+    evs = [{k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for k in wl.kernels} for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s in range(args.steps):
+        wl.step(evs[s])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    elapsed_ms = t0.elapsed_time(t1)
+    # post-roll for the sampler
+    t_end = time.perf_counter() + 0.4
+    while time.perf_counter() < t_end:
+        wl.step()
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    w4.w4_device_status()
+
+    elapsed_ms = max_over_ranks(elapsed_ms, world)
+    ms_per_step = elapsed_ms / args.steps
+    value = world * wl.step_bytes * args.steps / (elapsed_ms * 1e-3) / 1e9
+
+    # per-kernel averages over the timed region
+    per = {}
+    for k in wl.kernels:
+        ts = [e[k][0].elapsed_time(e[k][1]) for e in evs]
+        per[k] = sum(ts) / len(ts)
+    rooflines = {}
+    for k in wl.kernels:
+        us = per[k] * 1e3
+        gbs = wl.bytes[k] / (per[k] * 1e-3) / 1e9
+        r = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+             "frac": gbs / peaks["hbm_gbs"], "us": us, "algorithmic_bytes": wl.bytes[k],
+             "traffic": _traffic(k, "decode")}
+        if k in wl.flops:
+            r["tflops"] = wl.flops[k] / (per[k] * 1e-3) / 1e12
+        rooflines[k] = r
+    dominant = max(wl.kernels, key=lambda k: per[k])
+    gemm_us = sum(per[k] for k in wl.kernels if k.startswith("gemm")) * 1e3
+    gemm_bytes = sum(wl.bytes[k] for k in wl.kernels if k.startswith("gemm"))
+
+    # end to end through the public API, from pinned host memory
+    host, h2d, d2h = wl.host_buffers()
+    for _ in range(2):
+        wl.e2e_step(host)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        wl.e2e_step(host)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.e2e_steps
+    e2e_value = world * wl.step_bytes / (e2e_ms * 1e-3) / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = time_oracle()
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic", "config": wl.config(),
+            "roofline": {"kernel": dominant, **{k: v for k, v in rooflines[dominant].items()
+                                                  if k in ("bound", "achieved", "peak", "unit",
+                                                           "frac", "traffic")},
+                         "peak_source": peaks["source"]},
+            "rooflines": rooflines,
+            "decode_gemm": {"GB/s": gemm_bytes / (gemm_us * 1e-6) / 1e9,
+                            "frac": gemm_bytes / (gemm_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+                            "us_sum_4M": gemm_us},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": wl.launches_per_step * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

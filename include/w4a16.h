@@ -1,0 +1,178 @@
+/*
+ * w4a16.h -- C ABI of the B200 (sm_100a) library for group-wise INT4 weight
+ * quantization and W4A16 inference (libw4a16.so).
+ *
+ * Sources, by page title and section:
+ *   [QAT] SGLang RL team, "INT4 QAT end-to-end" blog (re-post): fake
+ *         quantization with a straight-through estimator in Megatron
+ *         (_FakeInt4QuantizationSTE), Fig. 4 "Rollout-side INT4 weight only"
+ *         (eight INT4 values packed into one INT32: 8 x 4 bits = 32 bits,
+ *         pack_int4_to_int32), "minimal packing and zero-overhead unpacking",
+ *         moe_align_block_size, "MoE operator deep fusion".
+ *   [TAG] reportify.cn concept page "量化感知训练": [8][9][16][17] fake
+ *         quantization forward / STE backward, [10] real quantization of the
+ *         exported weights, [11] 1x32 scale granularity, [32] W4A16 with two
+ *         4-bit weights per byte, [35] moe_align_block_size.
+ *   [BAS] "量化基础：从 FP32 到 INT4 的压缩艺术": §1.3 (INT4 range [-8, 7],
+ *         BF16 1+8+7 bits), §2.2 (s = max|x| / q_max, q = clamp(round(x/s))),
+ *         §2.4 (|x_hat - x| <= s/2), §6.2 (round half to even).
+ *
+ * Data formats (all row-major, all buffers owned by the caller):
+ *   W    [rows, K]        BF16 weights (w4_bf16 = raw BF16 bits), K contiguous.
+ *   S    [rows, K/32]     BF16 scales, one per group of 32 consecutive elements
+ *                         along K: S = bf16_rne(fl32(amax / 7)).
+ *   Wq   [rows, K/8]      int32 words; word j of a row holds codes
+ *                         q[8j .. 8j+7], code i of the eight in bits
+ *                         [4i, 4i+3] as a two's-complement nibble (low nibble
+ *                         first).  q = clamp(rint_half_even(w / S), -8, 7).
+ *   Wdq  [rows, K]        BF16 dequantized weights bf16_rne(q * S) (+0.0 for
+ *                         q == 0).
+ *   X    [M, K], Y [M, N] BF16 activations and outputs; Y = X . Wdq^T with
+ *                         FP32 accumulation and one BF16 rounding.
+ *
+ * Conventions for every call:
+ *   - Pointers are device pointers (cudaMalloc / PyTorch CUDA tensors) unless
+ *     stated otherwise; they must be non-null and 16-byte aligned, or the call
+ *     returns W4_ERR_INVALID_ARG without launching anything.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call validates its arguments on the host, then only
+ *     enqueues kernels on `stream` and returns; it never synchronizes, never
+ *     allocates device memory and keeps no pointer after it returns.
+ *   - group must be 32 (else W4_ERR_UNSUPPORTED); K must be a positive
+ *     multiple of 32.
+ *   - A kernel launch failure returns W4_ERR_CUDA (w4_last_cuda_error() gives
+ *     the cudaError_t).  Device-side waits are bounded: a kernel whose wait
+ *     runs out sets a device status flag and exits cleanly; w4_device_status()
+ *     reports it as W4_ERR_TIMEOUT.
+ *   - Inputs are assumed finite; NaN / Inf inputs give unspecified codes.
+ *   - Results are deterministic: run-to-run identical bits.
+ */
+#ifndef W4A16_H
+#define W4A16_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum w4_status {
+    W4_OK = 0,
+    W4_ERR_INVALID_ARG = 1, /* null / misaligned pointer, bad size or shape   */
+    W4_ERR_UNSUPPORTED = 2, /* well-formed request outside what is built      */
+    W4_ERR_CUDA = 3,        /* a CUDA runtime / driver call failed            */
+    W4_ERR_TIMEOUT = 4      /* a device-side bounded wait gave up             */
+} w4_status;
+
+typedef uint16_t w4_bf16; /* raw BF16 bits */
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int w4_version(void);
+
+/* Human-readable name of a status code (static string). */
+const char *w4_status_string(w4_status s);
+
+/* The cudaError_t of the last W4_ERR_CUDA returned on this host thread. */
+int w4_last_cuda_error(void);
+
+/* Synchronizes `stream`, then reports and clears the device status flag:
+ * W4_ERR_TIMEOUT if any kernel of this library gave up a bounded wait since
+ * the last call, W4_ERR_CUDA if the synchronization itself failed, else W4_OK. */
+w4_status w4_device_status(void *stream);
+
+/*
+ * Fake quantization (QDQ) forward -- [QAT] fake quantization ("mapped to INT4
+ * and immediately restored"), [TAG] [8][16], [BAS] §2.2.
+ *   W    in   [rows, K] BF16
+ *   Wdq  out  [rows, K] BF16, bf16_rne(q * S); may not alias W
+ *   S    out  [rows, K/32] BF16 scales, or NULL to skip writing them
+ * Memory-bound: reads 2 bytes and writes 2 (+1/16) bytes per element.
+ */
+w4_status w4_fake_quant(const w4_bf16 *W, w4_bf16 *Wdq, w4_bf16 *S,
+                        int64_t rows, int64_t K, int group, void *stream);
+
+/*
+ * Straight-through-estimator backward -- [QAT] §2.1 (gradients skip the
+ * rounding layer), [TAG] [9][17]: dW = dWdq bit for bit.  When dW == dWdq the
+ * call is a no-op (zero-copy); otherwise it copies n BF16 values.
+ */
+w4_status w4_ste_backward(const w4_bf16 *dWdq, w4_bf16 *dW, int64_t n, void *stream);
+
+/*
+ * Real quantization + packing for export -- [TAG] [10][32], [QAT] Fig. 4.
+ *   W    in   [rows, K] BF16
+ *   Wq   out  [rows, K/8] int32, low-nibble-first two's-complement codes
+ *   S    out  [rows, K/32] BF16 scales
+ * The codes and scales are the same as w4_fake_quant's, so
+ * w4_dequant(w4_quantize_pack(W)) == w4_fake_quant(W) bit for bit.
+ */
+w4_status w4_quantize_pack(const w4_bf16 *W, int32_t *Wq, w4_bf16 *S,
+                           int64_t rows, int64_t K, int group, void *stream);
+
+/*
+ * Unpack + dequantize ([QAT] "zero-overhead unpacking"): Wdq = bf16_rne(q * S),
+ * with the same register-level unpack the GEMMs use.  Mainly a test helper.
+ */
+w4_status w4_dequant(const int32_t *Wq, const w4_bf16 *S, w4_bf16 *Wdq,
+                     int64_t rows, int64_t K, int group, void *stream);
+
+/*
+ * W4A16 GEMM -- [TAG] [32] (W4A16 inference), [QAT] Fig. 4 and "zero-overhead
+ * unpacking"; the product runs on BF16 tensor cores with FP32 accumulation.
+ *   X   in   [M, K] BF16        Wq  in  [N, K/8] int32   S  in  [N, K/32] BF16
+ *   Y   out  [M, N] BF16, Y = X . dq(Wq, S)^T
+ * Any M >= 1, N >= 1.  Y may not alias an input.
+ */
+w4_status w4a16_gemm(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S,
+                     w4_bf16 *Y, int64_t M, int64_t N, int64_t K, int group,
+                     void *stream);
+
+/* Padded capacity the caller must provide for w4_moe_align's sorted_ids:
+ * T*topk + E*(block-1), rounded up to a multiple of block.  Host-only. */
+int64_t w4_moe_capacity(int64_t T, int topk, int E, int block);
+
+/*
+ * moe_align_block_size -- [QAT] "merge and align the tokens routed to the same
+ * expert", [TAG] [35].  Slot i = t*topk + k is routed to expert
+ * topk_ids[t*topk + k].  Each expert's slots, in ascending slot order, form
+ * one run padded up to a multiple of `block`; runs follow in ascending expert
+ * id.
+ *   topk_ids      in   [T, topk] int32 expert ids (ids outside [0, E) are skipped)
+ *   sorted_ids    out  [cap] int32 slot ids; padding and the tail hold T*topk
+ *   expert_ids    out  [cap/block] int32 expert of each block, -1 past the end
+ *   num_post_pad  out  [1] int32 padded total (a multiple of block)
+ * block must be a power of two in [1, 256]; cap >= w4_moe_capacity(...) and a
+ * multiple of block; E in [1, 1024]; topk in [1, 64].  Single-block kernel
+ * with no scratch memory.
+ */
+w4_status w4_moe_align(const int32_t *topk_ids, int64_t T, int topk, int E, int block,
+                       int32_t *sorted_ids, int64_t cap, int32_t *expert_ids,
+                       int32_t *num_post_pad, void *stream);
+
+/*
+ * Grouped W4A16 GEMM over the aligned slot list -- [QAT] "MoE operator deep
+ * fusion", [TAG] [35].  For every block b < num_post_pad/block with expert
+ * e = expert_ids[b], and every real slot = sorted_ids[b*block + j]
+ * (slot < num_slots):
+ *     C[slot, :] = A[slot / a_row_div, :] . dq(Wq[e], S[e])^T
+ *   A             in   [ceil(num_slots / a_row_div), K] BF16 (tokens for the
+ *                      gate_up projection with a_row_div = topk; per-slot
+ *                      rows for the down projection with a_row_div = 1)
+ *   Wq, S         in   [E, N, K/8] int32, [E, N, K/32] BF16
+ *   sorted_ids, expert_ids, num_post_pad   in (device), as written by w4_moe_align
+ *   C             out  [num_slots, N] BF16; rows of padding slots are never written
+ * block must be one of 16, 32, 64; cap is the length of sorted_ids.  The
+ * number of blocks is read on the device, so the call needs no host sync.
+ */
+w4_status w4_moe_w4a16_gemm(const w4_bf16 *A, int a_row_div, const int32_t *Wq,
+                            const w4_bf16 *S, const int32_t *sorted_ids,
+                            const int32_t *expert_ids, const int32_t *num_post_pad,
+                            int64_t cap, int block, int64_t num_slots, w4_bf16 *C,
+                            int64_t N, int64_t K, int E, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A16_H */

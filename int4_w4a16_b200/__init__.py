@@ -1,0 +1,260 @@
+"""int4_w4a16_b200 -- group-wise INT4 weight quantization and W4A16 inference on
+B200 (sm_100a).
+
+This module is the thin Python binding of ``libw4a16.so`` (C ABI declared in
+``include/w4a16.h``).  Each ``w4_*`` function has the name of the C entry point
+it calls and only marshals arguments: tensor data pointers, sizes and the
+current CUDA stream.  Every step of the computation runs in the library's CUDA
+kernels; there is no CPU or PyTorch fallback -- if the library or a CUDA device
+is missing, calls raise.
+
+PyTorch is used for device memory and streams only.  BF16 tensors are passed as
+``torch.bfloat16``; packed weights as ``torch.int32``.
+
+Sources (page titles): SGLang RL team "INT4 QAT end-to-end" blog (fake
+quantization + STE, Fig. 4 packing, moe_align_block_size, MoE operator
+fusion); reportify.cn "量化感知训练" [8]-[11], [32], [35]; "量化基础：从 FP32
+到 INT4 的压缩艺术" §2.2, §2.4.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "W4Error", "lib", "w4_version", "w4_device_status", "w4_fake_quant", "w4_ste_backward",
+    "w4_quantize_pack", "w4_dequant", "w4a16_gemm", "w4_moe_capacity", "w4_moe_align",
+    "w4_moe_w4a16_gemm", "fake_quant", "quantize_pack", "dequant", "gemm", "moe_align",
+    "moe_gemm", "FakeInt4STE", "GROUP",
+]
+
+GROUP = 32
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libw4a16.so")
+
+_STATUS = {0: "W4_OK", 1: "W4_ERR_INVALID_ARG", 2: "W4_ERR_UNSUPPORTED", 3: "W4_ERR_CUDA",
+           4: "W4_ERR_TIMEOUT"}
+
+
+class W4Error(RuntimeError):
+    def __init__(self, fn: str, code: int, cuda_err: int = 0):
+        msg = f"{fn} returned {_STATUS.get(code, code)}"
+        if code == 3:
+            msg += f" (cudaError {cuda_err})"
+        super().__init__(msg)
+        self.code = code
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_INT = ctypes.c_int
+
+
+def lib() -> ctypes.CDLL:
+    """Load libw4a16.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m int4_w4a16_b200.build` "
+                "(there is no fallback path)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, args in {
+            "w4_fake_quant": [_P, _P, _P, _I64, _I64, _INT, _P],
+            "w4_ste_backward": [_P, _P, _I64, _P],
+            "w4_quantize_pack": [_P, _P, _P, _I64, _I64, _INT, _P],
+            "w4_dequant": [_P, _P, _P, _I64, _I64, _INT, _P],
+            "w4a16_gemm": [_P, _P, _P, _P, _I64, _I64, _I64, _INT, _P],
+            "w4_moe_align": [_P, _I64, _INT, _INT, _INT, _P, _I64, _P, _P, _P],
+            "w4_moe_w4a16_gemm": [_P, _INT, _P, _P, _P, _P, _P, _I64, _INT, _I64, _P, _I64,
+                                  _I64, _INT, _P],
+            "w4_device_status": [_P],
+        }.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = ctypes.c_int
+        L.w4_moe_capacity.argtypes = [_I64, _INT, _INT, _INT]
+        L.w4_moe_capacity.restype = ctypes.c_int64
+        L.w4_version.restype = ctypes.c_int
+        L.w4_last_cuda_error.restype = ctypes.c_int
+        L.w4_status_string.argtypes = [_INT]
+        L.w4_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != 0:
+        raise W4Error(fn, rc, lib().w4_last_cuda_error() if rc == 3 else 0)
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libw4a16 takes CUDA tensors (device memory)")
+    if not t.is_contiguous():
+        raise ValueError("libw4a16 takes contiguous tensors")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+
+
+def _dtype(t: torch.Tensor, dt: torch.dtype, what: str) -> None:
+    if t.dtype != dt:
+        raise TypeError(f"{what} must be {dt}, got {t.dtype}")
+
+
+# ---------------------------------------------------------------------------
+# C-ABI calls (same names as include/w4a16.h)
+# ---------------------------------------------------------------------------
+
+def w4_version() -> int:
+    return int(lib().w4_version())
+
+
+def w4_device_status(stream=None) -> None:
+    """Synchronize the stream and raise if a kernel gave up a bounded wait."""
+    _check("w4_device_status", lib().w4_device_status(_stream(stream)))
+
+
+def w4_fake_quant(W, Wdq, S=None, group: int = GROUP, stream=None) -> None:
+    _dtype(W, torch.bfloat16, "W")
+    _dtype(Wdq, torch.bfloat16, "Wdq")
+    rows, K = W.shape
+    _check("w4_fake_quant", lib().w4_fake_quant(_ptr(W), _ptr(Wdq), _ptr(S), rows, K, group,
+                                                _stream(stream)))
+
+
+def w4_ste_backward(dWdq, dW, stream=None) -> None:
+    _dtype(dWdq, torch.bfloat16, "dWdq")
+    _dtype(dW, torch.bfloat16, "dW")
+    _check("w4_ste_backward", lib().w4_ste_backward(_ptr(dWdq), _ptr(dW), dWdq.numel(),
+                                                    _stream(stream)))
+
+
+def w4_quantize_pack(W, Wq, S, group: int = GROUP, stream=None) -> None:
+    _dtype(W, torch.bfloat16, "W")
+    _dtype(Wq, torch.int32, "Wq")
+    _dtype(S, torch.bfloat16, "S")
+    rows, K = W.shape
+    _check("w4_quantize_pack", lib().w4_quantize_pack(_ptr(W), _ptr(Wq), _ptr(S), rows, K,
+                                                      group, _stream(stream)))
+
+
+def w4_dequant(Wq, S, Wdq, group: int = GROUP, stream=None) -> None:
+    _dtype(Wq, torch.int32, "Wq")
+    rows, K = Wdq.shape
+    _check("w4_dequant", lib().w4_dequant(_ptr(Wq), _ptr(S), _ptr(Wdq), rows, K, group,
+                                          _stream(stream)))
+
+
+def w4a16_gemm(X, Wq, S, Y, group: int = GROUP, stream=None) -> None:
+    _dtype(X, torch.bfloat16, "X")
+    _dtype(Wq, torch.int32, "Wq")
+    M, K = X.shape
+    N = Wq.shape[0]
+    if Wq.shape[1] * 8 != K or tuple(Y.shape) != (M, N):
+        raise ValueError("shape mismatch")
+    _check("w4a16_gemm", lib().w4a16_gemm(_ptr(X), _ptr(Wq), _ptr(S), _ptr(Y), M, N, K, group,
+                                          _stream(stream)))
+
+
+def w4_moe_capacity(T: int, topk: int, E: int, block: int) -> int:
+    return int(lib().w4_moe_capacity(T, topk, E, block))
+
+
+def w4_moe_align(topk_ids, E: int, block: int, sorted_ids, expert_ids, num_post_pad,
+                 stream=None) -> None:
+    _dtype(topk_ids, torch.int32, "topk_ids")
+    T, topk = topk_ids.shape
+    _check("w4_moe_align", lib().w4_moe_align(_ptr(topk_ids), T, topk, E, block,
+                                              _ptr(sorted_ids), sorted_ids.numel(),
+                                              _ptr(expert_ids), _ptr(num_post_pad),
+                                              _stream(stream)))
+
+
+def w4_moe_w4a16_gemm(A, a_row_div: int, Wq, S, sorted_ids, expert_ids, num_post_pad,
+                      block: int, num_slots: int, C, stream=None) -> None:
+    E, N, K8 = Wq.shape
+    _check("w4_moe_w4a16_gemm", lib().w4_moe_w4a16_gemm(
+        _ptr(A), a_row_div, _ptr(Wq), _ptr(S), _ptr(sorted_ids), _ptr(expert_ids),
+        _ptr(num_post_pad), sorted_ids.numel(), block, num_slots, _ptr(C), N, K8 * 8, E,
+        _stream(stream)))
+
+
+# ---------------------------------------------------------------------------
+# Allocating conveniences (outputs from torch.empty on the input's device)
+# ---------------------------------------------------------------------------
+
+def fake_quant(W: torch.Tensor, want_scales: bool = False):
+    rows, K = W.shape
+    Wdq = torch.empty_like(W)
+    S = torch.empty((rows, K // GROUP), dtype=torch.bfloat16, device=W.device) if want_scales else None
+    w4_fake_quant(W, Wdq, S)
+    return (Wdq, S) if want_scales else Wdq
+
+
+def quantize_pack(W: torch.Tensor):
+    rows, K = W.shape
+    Wq = torch.empty((rows, K // 8), dtype=torch.int32, device=W.device)
+    S = torch.empty((rows, K // GROUP), dtype=torch.bfloat16, device=W.device)
+    w4_quantize_pack(W, Wq, S)
+    return Wq, S
+
+
+def dequant(Wq: torch.Tensor, S: torch.Tensor) -> torch.Tensor:
+    rows, K8 = Wq.shape
+    Wdq = torch.empty((rows, K8 * 8), dtype=torch.bfloat16, device=Wq.device)
+    w4_dequant(Wq, S, Wdq)
+    return Wdq
+
+
+def gemm(X: torch.Tensor, Wq: torch.Tensor, S: torch.Tensor) -> torch.Tensor:
+    Y = torch.empty((X.shape[0], Wq.shape[0]), dtype=torch.bfloat16, device=X.device)
+    w4a16_gemm(X, Wq, S, Y)
+    return Y
+
+
+def moe_align(topk_ids: torch.Tensor, E: int, block: int):
+    T, topk = topk_ids.shape
+    cap = w4_moe_capacity(T, topk, E, block)
+    dev = topk_ids.device
+    sorted_ids = torch.empty(cap, dtype=torch.int32, device=dev)
+    expert_ids = torch.empty(cap // block, dtype=torch.int32, device=dev)
+    npp = torch.empty(4, dtype=torch.int32, device=dev)[:1]
+    w4_moe_align(topk_ids, E, block, sorted_ids, expert_ids, npp)
+    return sorted_ids, expert_ids, npp
+
+
+def moe_gemm(A, a_row_div, Wq, S, sorted_ids, expert_ids, num_post_pad, block, num_slots,
+             C=None):
+    if C is None:
+        C = torch.empty((num_slots, Wq.shape[1]), dtype=torch.bfloat16, device=A.device)
+    w4_moe_w4a16_gemm(A, a_row_div, Wq, S, sorted_ids, expert_ids, num_post_pad, block,
+                      num_slots, C)
+    return C
+
+
+class FakeInt4STE(torch.autograd.Function):
+    """Fake INT4 quantization with a straight-through estimator.
+
+    Forward: Wdq = w4_fake_quant(W) (group-32 QDQ, BF16 in and out).
+    Backward: the gradient passes through the rounding unchanged (identity,
+    zero-copy), as in the INT4 QAT blog's _FakeInt4QuantizationSTE.
+    """
+
+    @staticmethod
+    def forward(ctx, W):
+        return fake_quant(W.contiguous())
+
+    @staticmethod
+    def backward(ctx, grad_out):
+        return grad_out

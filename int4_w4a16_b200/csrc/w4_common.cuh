@@ -1,0 +1,334 @@
+// w4_common.cuh -- shared device helpers of libw4a16 (sm_100a only).
+//
+// Thin inline-PTX wrappers for mbarriers, TMA tensor loads, cp.async and the
+// 5th-generation tensor-core instructions (tcgen05.*), plus the bounded-wait
+// and device-status machinery.  Every spin on an mbarrier is bounded by a
+// global-timer deadline; on expiry the kernel records W4_ERR_TIMEOUT in the
+// device status word and the calling role stops waiting.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/w4a16.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "libw4a16 is built for sm_100a only"
+#endif
+
+namespace w4 {
+
+// ---------------------------------------------------------------------------
+// Device status word: set (never cleared) by kernels, read/cleared by the host
+// through w4_device_status().
+// ---------------------------------------------------------------------------
+extern __device__ unsigned int g_device_status;
+
+constexpr unsigned int kStatusTimeout = 1u;
+// A bounded wait gives up after this many nanoseconds of %globaltimer.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void record_timeout() {
+    atomicOr(&g_device_status, kStatusTimeout);
+}
+
+// ---------------------------------------------------------------------------
+// Shared-memory addresses and mbarriers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .b64 st;\n\t"
+        "mbarrier.arrive.release.cta.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile(
+        "{\n\t.reg .b64 st;\n\t"
+        "mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(bar),
+        "r"(bytes)
+        : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity.  Returns false (after
+// recording the timeout and raising *abort_flag) if the deadline passes or if
+// another thread of the CTA already raised *abort_flag.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          volatile int *abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 255u) == 0u) {
+            if (*abort_flag) return false;
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                record_timeout();
+                *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Proxy fences
+// ---------------------------------------------------------------------------
+// Generic-proxy shared-memory writes -> later async-proxy (TMA / tensor core) reads.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
+// TMA (cp.async.bulk.tensor), no multicast
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *m) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *m, uint32_t bar,
+                                            int32_t x, int32_t y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cta.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *m, uint32_t bar,
+                                            int32_t x, int32_t y, int32_t z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cta.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// cp.async (16-byte global -> shared copies) with mbarrier completion
+// ---------------------------------------------------------------------------
+// Copies src_bytes (0 or 16) bytes and zero-fills the rest of the 16.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+
+// The barrier receives one arrival once all prior cp.async of this thread land.
+__device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Tensor memory (tcgen05) -- cta_group::1 only
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     dst_smem),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before_sync() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after_sync() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]; kind::f16 (BF16 inputs, FP32 accumulator).
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(
+            d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u),
+        "r"(0u)
+        : "memory");
+}
+
+// The barrier receives one arrival when all previously issued tcgen05.mma of
+// this thread have completed.
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+        : "memory");
+}
+
+// Store 8 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st_x8(uint32_t taddr, const uint32_t (&v)[8]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
+            taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Load 16 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+          "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
+// UMMA descriptors
+// ---------------------------------------------------------------------------
+// Shared-memory matrix descriptor for a K-major operand stored in the 128-byte
+// swizzled canonical layout: rows of 128 bytes (64 BF16 along K), 8-row atoms
+// of 1024 bytes stacked at a 1024-byte stride.
+__device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);          // start address
+    d |= (uint64_t)1u << 16;                           // leading byte offset (unused)
+    d |= (uint64_t)(1024u >> 4) << 32;                 // stride byte offset: 8-row atom
+    d |= (uint64_t)1u << 46;                           // descriptor version (sm_100)
+    d |= (uint64_t)2u << 61;                           // layout: 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor: kind::f16, A = B = BF16, D = FP32, both K-major,
+// M = 128, N = n.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t m, uint32_t n) {
+    return (1u << 4)            // D format: F32
+           | (1u << 7)          // A format: BF16
+           | (1u << 10)         // B format: BF16
+           | ((n >> 3) << 17)   // N / 8
+           | ((m >> 4) << 24);  // M / 16
+}
+
+// ---------------------------------------------------------------------------
+// INT4 -> BF16 unpack + dequant of one packed word (register level).
+//
+// Input: w = eight two's-complement codes q_0..q_7 (q_i in bits [4i, 4i+3]);
+// s2 = the group's BF16 scale in both halves.  Output: four BF16x2 words,
+// out[j] = (q_{2j} * s, q_{2j+1} * s), low half = even element.
+//
+// Step 1 (one LOP3 per pair): (w >> 4i) & 0x000F000F selects codes i and i+4;
+// XOR with 0x43084308 flips the code's sign bit (two's complement -> offset
+// binary, n ^ 8 = q + 8) and sets the BF16 exponent of 128, whose ulp is 1, so
+// each half reads 136 + q exactly.  Step 2: byte permutes pair codes (2j,
+// 2j+1).  Step 3: subtract 136 (exact), multiply by the scale (one rounding
+// to nearest even: the product of a 4-bit and an 8-bit significand is exact
+// before rounding), i.e. bf16_rne(q * s); q == 0 gives +0.0.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t lop3_and_xor(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    // (a & b) ^ c  -> truth table 0x6A
+    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+__device__ __forceinline__ void dequant_word(uint32_t w, uint32_t s2, uint32_t (&out)[4]) {
+    const uint32_t m = 0x000F000Fu, x = 0x43084308u;
+    uint32_t t0 = lop3_and_xor(w, m, x);          // codes 0, 4
+    uint32_t t1 = lop3_and_xor(w >> 4, m, x);     // codes 1, 5
+    uint32_t t2 = lop3_and_xor(w >> 8, m, x);     // codes 2, 6
+    uint32_t t3 = lop3_and_xor(w >> 12, m, x);    // codes 3, 7
+    uint32_t p01 = __byte_perm(t0, t1, 0x5410);
+    uint32_t p23 = __byte_perm(t2, t3, 0x5410);
+    uint32_t p45 = __byte_perm(t0, t1, 0x7632);
+    uint32_t p67 = __byte_perm(t2, t3, 0x7632);
+    const __nv_bfloat162 bias = __floats2bfloat162_rn(136.0f, 136.0f);
+    const __nv_bfloat162 sc = *reinterpret_cast<const __nv_bfloat162 *>(&s2);
+    uint32_t in[4] = {p01, p23, p45, p67};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162 *>(&in[j]);
+        v = __hsub2(v, bias);
+        v = __hmul2(v, sc);
+        out[j] = *reinterpret_cast<uint32_t *>(&v);
+    }
+}
+
+__device__ __forceinline__ uint32_t bf16x2_splat(uint16_t s) {
+    return (uint32_t)s | ((uint32_t)s << 16);
+}
+
+}  // namespace w4
+
+// ---------------------------------------------------------------------------
+// Host-side helpers shared by the ABI entry points
+// ---------------------------------------------------------------------------
+namespace w4host {
+
+void set_cuda_error(cudaError_t e);
+
+inline bool aligned16(const void *p) {
+    return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+inline w4_status launch_status() {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        set_cuda_error(e);
+        return W4_ERR_CUDA;
+    }
+    return W4_OK;
+}
+
+int num_sms();
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+CUresult encode_tiled(CUtensorMap *map, CUtensorMapDataType dtype, cuuint32_t rank,
+                      void *gaddr, const cuuint64_t *dims, const cuuint64_t *strides_bytes,
+                      const cuuint32_t *box, CUtensorMapSwizzle swizzle);
+
+}  // namespace w4host

@@ -1,0 +1,587 @@
+// w4_gemm.cu -- W4A16 GEMM (dense) and grouped MoE W4A16 GEMM on 5th-generation
+// tensor cores (tcgen05, sm_100a).
+//
+// What it computes (INT4 QAT blog, Fig. 4 and "zero-overhead unpacking";
+// reportify.cn "量化感知训练" [32][35]):  Y[m, n] = sum_k X[m, k] * dq(W)[n, k],
+// dq(W)[n, k] = bf16_rne(q[n, k] * S[n, k/32]), FP32 accumulation, one BF16
+// rounding of the result.  The MoE variant runs the same product per aligned
+// block of slots with the block's expert weights and gathered activation rows.
+//
+// Design (B200-first; the pages' Marlin kernel targets H-series mma.sync and
+// is prior art only):
+//  * swap-AB: the MMA's A operand (M = 128 rows) is the dequantized weight
+//    tile, the B operand (N = MT columns) is the activation tile, so decode
+//    shapes with 1..64 tokens still use a full-height MMA;
+//  * the weights never exist as BF16 in memory or shared memory: packed words
+//    arrive by TMA (128-byte swizzle, bank-conflict-free row reads), four
+//    dequant warps unpack them in registers (LOP3 + PRMT + 2 packed BF16 ops
+//    per pair) and store the BF16 A tile straight into tensor memory with
+//    tcgen05.st; tcgen05.mma then reads A from TMEM and B from shared memory,
+//    which keeps the shared-memory traffic of a decode step at the packed
+//    bytes plus the activations;
+//  * activations arrive by TMA in the canonical K-major 128-byte-swizzled
+//    layout (dense), or by cp.async row gathers into the same layout (MoE);
+//  * warp specialization: warp 0 = loads, warp 1 = TMEM allocation + MMA
+//    issue (one thread), warps 2-5 = dequant, warps 6-9 = epilogue
+//    (tcgen05.ld -> BF16 -> global), with mbarrier rings between them and
+//    double-buffered accumulators where TMEM allows;
+//  * persistent CTAs (one per SM) walk a static list of work items; for decode
+//    the N rows are split evenly over the SMs (rows per tile = ceil(N / SMs))
+//    so every SM streams the same number of weight bytes and no split-K
+//    reduction (and no scratch memory) is needed.
+// Every mbarrier wait is bounded (w4_common.cuh); a timed-out CTA records the
+// device status, drains its own in-flight copies and MMAs, frees its TMEM and
+// exits.
+#include <algorithm>
+
+#include "w4_common.cuh"
+
+namespace w4 {
+namespace {
+
+constexpr int kWarps = 10;
+constexpr int kThreadsGemm = kWarps * 32;
+constexpr int kTmemCols = 512;
+
+struct GemmParams {
+    const uint16_t *S;           // scales (direct loads when KB < 256)
+    uint16_t *Y;                 // dense: Y [M, N]; MoE: C [num_slots, N]
+    const uint16_t *A;           // MoE: activation rows [a_rows, K]
+    const int32_t *sorted_ids;   // MoE
+    const int32_t *expert_ids;   // MoE
+    const int32_t *num_post_pad; // MoE
+    int64_t M, N, K;
+    int64_t num_slots;           // MoE
+    int64_t a_rows;              // MoE
+    int a_row_div;               // MoE
+    int cap_blocks;              // MoE: length of expert_ids (bounds num_post_pad / MT)
+    int rows_per_tile;           // R <= 128
+    int n_row_tiles;
+    int n_tok_tiles;             // dense
+    int num_kb;
+};
+
+// Shared-memory layout, all offsets from a 1024-aligned base.
+template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE>
+struct Layout {
+    static constexpr int kWBytes = 128 * KB / 2;            // packed tile, up to 128 rows
+    static constexpr int kSBytes = (KB == 256) ? 128 * 16 : 0;
+    static constexpr int kXSub = MT * 128;                  // one 64-wide K slice
+    static constexpr int kXBytes = (KB / 64) * kXSub;
+    static constexpr int kStage = kWBytes + kSBytes + kXBytes;
+    static constexpr int kBarOff = NSTAGE * kStage;
+    static constexpr int kNumBars = 2 * NSTAGE + 2 * NASTAGE + 2 * NACC + 1;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+    static constexpr int kBytes = kMiscOff + 16;
+    static constexpr int kAlloc = kBytes + 1024;            // slack for 1024-alignment
+    static_assert(kWBytes % 1024 == 0 && kXSub % 1024 == 0, "1024-byte aligned tiles");
+    static_assert(kStage % 1024 == 0, "stage size");
+    static_assert(NACC * MT + NASTAGE * (KB / 2) <= kTmemCols, "TMEM budget");
+};
+
+__device__ __forceinline__ uint32_t swz(uint32_t off, uint32_t sw_bytes) {
+    // TMA / UMMA swizzle: 16-byte chunk index XOR address bits [7, ...).
+    return off ^ (((off >> 7) & (sw_bytes / 16 - 1)) << 4);
+}
+
+// Bounded wait executed by every lane of a warp; the verdict is warp-uniform.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
+    bool ok = mbar_wait(bar, parity, abort_flag);
+    return __all_sync(0xFFFFFFFFu, ok);
+}
+
+// Drain wait used on the way out of an aborted CTA (does not look at the abort flag).
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+    const unsigned long long t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs / 4) {
+            record_timeout();
+            return;
+        }
+    }
+}
+
+template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, bool MOE>
+__global__ void __launch_bounds__(kThreadsGemm, 1)
+    w4a16_tc_kernel(const __grid_constant__ CUtensorMap tm_w,
+                    const __grid_constant__ CUtensorMap tm_s,
+                    const __grid_constant__ CUtensorMap tm_x, const GemmParams p) {
+    using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE>;
+    constexpr int kWords = KB / 8;             // packed words per row per k-block
+    constexpr int kAStageCols = KB / 2;        // TMEM columns per A stage
+    constexpr int kABase = NACC * MT;          // first A column
+    constexpr uint32_t kIdesc = idesc_bf16_f32(128, MT);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar0 = sbase + L::kBarOff;
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (NSTAGE + s); };
+    auto afull_bar = [&](int a) { return bar0 + 8u * (2 * NSTAGE + a); };
+    auto aempty_bar = [&](int a) { return bar0 + 8u * (2 * NSTAGE + NASTAGE + a); };
+    auto accfull_bar = [&](int d) { return bar0 + 8u * (2 * NSTAGE + 2 * NASTAGE + d); };
+    auto accempty_bar = [&](int d) {
+        return bar0 + 8u * (2 * NSTAGE + 2 * NASTAGE + NACC + d);
+    };
+    const uint32_t mmadone_bar = bar0 + 8u * (2 * NSTAGE + 2 * NASTAGE + 2 * NACC);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
+
+    auto w_stage = [&](int s) { return sbase + (uint32_t)(s * L::kStage); };
+    auto s_stage = [&](int s) { return sbase + (uint32_t)(s * L::kStage + L::kWBytes); };
+    auto x_stage = [&](int s) {
+        return sbase + (uint32_t)(s * L::kStage + L::kWBytes + L::kSBytes);
+    };
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NSTAGE; ++s) {
+            mbar_init(full_bar(s), MOE ? 33u : 1u);
+            mbar_init(empty_bar(s), 1u);
+        }
+        for (int a = 0; a < NASTAGE; ++a) {
+            mbar_init(afull_bar(a), 128u);
+            mbar_init(aempty_bar(a), 1u);
+        }
+        for (int d = 0; d < NACC; ++d) {
+            mbar_init(accfull_bar(d), 1u);
+            mbar_init(accempty_bar(d), 128u);
+        }
+        mbar_init(mmadone_bar, 1u);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_w);
+        if (KB == 256) tma_prefetch_desc(&tm_s);
+        if (!MOE) tma_prefetch_desc(&tm_x);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int R = p.rows_per_tile;
+    const int num_kb = p.num_kb;
+    int num_items;
+    if (MOE) {
+        const int npp = *p.num_post_pad;
+        const int nblocks = min(max(npp, 0) / MT, p.cap_blocks);
+        num_items = nblocks * p.n_row_tiles;
+    } else {
+        num_items = p.n_row_tiles * p.n_tok_tiles;
+    }
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ loads
+        uint32_t it = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < num_items && ok; item += gridDim.x) {
+            const int rt = item % p.n_row_tiles;
+            const int tt = item / p.n_row_tiles;
+            const int row0 = rt * R;
+            int expert = 0;
+            if (MOE) expert = __ldg(p.expert_ids + tt);
+            for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                const int s = it % NSTAGE;
+                if (!warp_wait(empty_bar(s), ((it / NSTAGE) & 1u) ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    const uint32_t wbytes = (uint32_t)R * (KB / 2);
+                    const uint32_t sbytes = (KB == 256) ? (uint32_t)R * 16u : 0u;
+                    const uint32_t xbytes = MOE ? 0u : (uint32_t)L::kXBytes;
+                    mbar_arrive_expect_tx(full_bar(s), wbytes + sbytes + xbytes);
+                    if (MOE) {
+                        tma_load_3d(w_stage(s), &tm_w, full_bar(s), kb * kWords, row0, expert);
+                        if (KB == 256)
+                            tma_load_3d(s_stage(s), &tm_s, full_bar(s), kb * 8, row0, expert);
+                    } else {
+                        tma_load_2d(w_stage(s), &tm_w, full_bar(s), kb * kWords, row0);
+                        if (KB == 256) tma_load_2d(s_stage(s), &tm_s, full_bar(s), kb * 8, row0);
+#pragma unroll
+                        for (int u = 0; u < KB / 64; ++u)
+                            tma_load_2d(x_stage(s) + u * L::kXSub, &tm_x, full_bar(s),
+                                        kb * KB + u * 64, tt * MT);
+                    }
+                }
+                if (MOE) {
+                    // Gather the block's activation rows: lane = 16-byte chunk along K.
+                    const int c = lane;                   // KB == 256: 32 chunks per row
+                    const int64_t k = (int64_t)kb * KB + c * 8;
+                    for (int t = 0; t < MT; ++t) {
+                        const int slot = __ldg(p.sorted_ids + (int64_t)tt * MT + t);
+                        const int64_t row =
+                            (slot >= 0 && slot < p.num_slots) ? slot / p.a_row_div : -1;
+                        const bool in = row >= 0 && row < p.a_rows && k < p.K;
+                        const uint16_t *src = in ? p.A + row * p.K + k : p.A;
+                        const uint32_t dst = x_stage(s) + (c >> 3) * L::kXSub + t * 128 +
+                                             ((((uint32_t)c & 7u) ^ ((uint32_t)t & 7u)) << 4);
+                        cp_async_16(dst, src, in ? 16u : 0u);
+                    }
+                    cp_async_mbar_arrive(full_bar(s));
+                }
+            }
+        }
+        // Drain: wait (bounded) until the loads this warp issued have landed.
+        if (lane == 0) {
+            const uint32_t first = it > (uint32_t)NSTAGE ? it - NSTAGE : 0u;
+            for (uint32_t j = first; j < it; ++j) drain_wait(full_bar(j % NSTAGE), (j / NSTAGE) & 1u);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------- MMA
+        if (lane == 0) {
+            uint32_t it = 0, acc_it = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < num_items && ok; item += gridDim.x, ++acc_it) {
+                const int d = acc_it % NACC;
+                if (!mbar_wait(accempty_bar(d), ((acc_it / NACC) & 1u) ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(d * MT);
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    const int s = it % NSTAGE;
+                    const int a = it % NASTAGE;
+                    if (!mbar_wait(full_bar(s), (it / NSTAGE) & 1u, abort_flag) ||
+                        !mbar_wait(afull_bar(a), (it / NASTAGE) & 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    if (MOE) fence_proxy_async_smem();   // cp.async (generic proxy) -> MMA
+                    const uint32_t a_tmem = tmem_base + (uint32_t)(kABase + a * kAStageCols);
+#pragma unroll
+                    for (int u = 0; u < KB / 16; ++u) {
+                        const uint32_t baddr = x_stage(s) + (u >> 2) * L::kXSub + (u & 3) * 32;
+                        tc_mma_ts(d_tmem, a_tmem + u * 8, smem_desc_k_sw128(baddr), kIdesc,
+                                  (kb > 0 || u > 0) ? 1u : 0u);
+                    }
+                    tc_commit(empty_bar(s));
+                    tc_commit(aempty_bar(a));
+                }
+                if (!ok) break;
+                tc_commit(accfull_bar(d));
+            }
+            // All MMAs issued by this thread complete before TMEM is released.
+            tc_commit(mmadone_bar);
+            drain_wait(mmadone_bar, 0u);
+        }
+    } else if (warp < 6) {
+        // --------------------------------------------------------- dequant
+        const int q4 = warp & 3;                    // TMEM lane quarter of this warp
+        const int lrow = q4 * 32 + lane;            // A row of this thread
+        const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
+        const int64_t gpr = p.K / 32;               // groups per row
+        uint32_t it = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < num_items && ok; item += gridDim.x) {
+            const int rt = item % p.n_row_tiles;
+            const int tt = item / p.n_row_tiles;
+            const int64_t row = (int64_t)rt * R + lrow;
+            const bool valid = lrow < R && row < p.N;
+            const uint16_t *srow = nullptr;
+            if (KB != 256 && valid) {
+                int64_t base = row * gpr;
+                if (MOE) base += (int64_t)__ldg(p.expert_ids + tt) * p.N * gpr;
+                srow = p.S + base;
+            }
+            for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                const int s = it % NSTAGE;
+                const int a = it % NASTAGE;
+                // scales of this k-block (direct loads when the tile has no TMA scales)
+                uint32_t sc[KB / 32];
+                if (KB != 256) {
+#pragma unroll
+                    for (int g = 0; g < KB / 32; ++g) {
+                        const int64_t gi = (int64_t)kb * (KB / 32) + g;
+                        const uint16_t v = (srow != nullptr && gi < gpr) ? __ldg(srow + gi) : 0;
+                        sc[g] = bf16x2_splat(v);
+                    }
+                }
+                if (!warp_wait(full_bar(s), (it / NSTAGE) & 1u, abort_flag) ||
+                    !warp_wait(aempty_bar(a), ((it / NASTAGE) & 1u) ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                if (KB == 256) {
+                    const uint4 sv = *reinterpret_cast<const uint4 *>(smem + (s_stage(s) - sbase) +
+                                                                     lrow * 16);
+                    const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+                    for (int g = 0; g < 8; ++g)
+                        sc[g % (KB / 32)] = bf16x2_splat((uint16_t)(sw[g >> 1] >> (16 * (g & 1))));
+                    // (the loop above fills all eight entries when KB == 256)
+                }
+                const uint8_t *wrow = smem + (w_stage(s) - sbase);
+                const uint32_t a_col = tmem_base + lane_addr + (uint32_t)(kABase + a * kAStageCols);
+#pragma unroll
+                for (int g = 0; g < KB / 32; ++g) {
+                    // 16-byte chunk g of this row = 4 words = one group of 32 codes
+                    const uint32_t off = swz((uint32_t)(lrow * (KB / 2) + g * 16), KB / 2);
+                    const uint4 wv = *reinterpret_cast<const uint4 *>(wrow + off);
+                    const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
+                    uint32_t o[16];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        uint32_t t4[4];
+                        dequant_word(ws[j], sc[g], t4);
+                        o[4 * j + 0] = t4[0];
+                        o[4 * j + 1] = t4[1];
+                        o[4 * j + 2] = t4[2];
+                        o[4 * j + 3] = t4[3];
+                    }
+                    // columns: 2 BF16 per 32-bit column, ascending k
+                    uint32_t lo[8], hi[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        lo[j] = o[j];
+                        hi[j] = o[8 + j];
+                    }
+                    tmem_st_x8(a_col + g * 16, lo);
+                    tmem_st_x8(a_col + g * 16 + 8, hi);
+                }
+                tmem_wait_st();
+                tc_fence_before_sync();
+                mbar_arrive(afull_bar(a));
+            }
+        }
+    } else {
+        // -------------------------------------------------------- epilogue
+        const int q4 = warp & 3;
+        const int lrow = q4 * 32 + lane;
+        const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
+        uint32_t acc_it = 0;
+        for (int item = blockIdx.x; item < num_items; item += gridDim.x, ++acc_it) {
+            const int rt = item % p.n_row_tiles;
+            const int tt = item / p.n_row_tiles;
+            const int d = acc_it % NACC;
+            if (!warp_wait(accfull_bar(d), (acc_it / NACC) & 1u, abort_flag)) break;
+            tc_fence_after_sync();
+            const int64_t row = (int64_t)rt * R + lrow;
+            const bool valid = lrow < R && row < p.N;
+#pragma unroll 1
+            for (int c0 = 0; c0 < MT; c0 += 16) {
+                uint32_t v[16];
+                tmem_ld_x16(tmem_base + lane_addr + (uint32_t)(d * MT + c0), v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int tok = c0 + j;
+                    int64_t out_row;
+                    if (MOE) {
+                        const int slot = __ldg(p.sorted_ids + (int64_t)tt * MT + tok);
+                        out_row = (slot >= 0 && slot < p.num_slots) ? slot : -1;
+                    } else {
+                        const int64_t m = (int64_t)tt * MT + tok;
+                        out_row = (m < p.M) ? m : -1;
+                    }
+                    if (valid && out_row >= 0) {
+                        const __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(v[j]));
+                        p.Y[out_row * p.N + row] = *reinterpret_cast<const uint16_t *>(&h);
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            mbar_arrive(accempty_bar(d));
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+
+template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, bool MOE>
+w4_status launch_cfg(const CUtensorMap &tw, const CUtensorMap &ts, const CUtensorMap &tx,
+                     const GemmParams &p, int num_items_max, cudaStream_t stream) {
+    using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE>;
+    auto kern = w4a16_tc_kernel<KB, MT, NSTAGE, NACC, NASTAGE, MOE>;
+    // At least half of the SM's shared memory, so one CTA (and one TMEM
+    // allocation of 512 columns) per SM.
+    const int smem = std::max(L::kAlloc, 120 * 1024);
+    static bool configured = false;
+    if (!configured) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess)
+            return w4host::launch_status();
+        configured = true;
+    }
+    const int grid = std::max(1, std::min(num_items_max, w4host::num_sms()));
+    kern<<<grid, kThreadsGemm, smem, stream>>>(tw, ts, tx, p);
+    return w4host::launch_status();
+}
+
+bool make_map(CUtensorMap *m, CUtensorMapDataType dt, int rank, const void *ptr,
+              const cuuint64_t *dims, const cuuint64_t *strides, const cuuint32_t *box,
+              CUtensorMapSwizzle sw) {
+    return w4host::encode_tiled(m, dt, (cuuint32_t)rank, const_cast<void *>(ptr), dims, strides,
+                                box, sw) == CUDA_SUCCESS;
+}
+
+int ceil_div_i(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
+
+}  // namespace
+}  // namespace w4
+
+using namespace w4;
+
+extern "C" w4_status w4a16_gemm(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S,
+                                w4_bf16 *Y, int64_t M, int64_t N, int64_t K, int group,
+                                void *stream) {
+    if (group != 32) return W4_ERR_UNSUPPORTED;
+    if (M < 0 || N < 0 || K <= 0 || (K % 32) != 0) return W4_ERR_INVALID_ARG;
+    if (!w4host::aligned16(X) || !w4host::aligned16(Wq) || !w4host::aligned16(S) ||
+        !w4host::aligned16(Y))
+        return W4_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return W4_OK;
+    if (N > (1 << 30) || M > (1 << 30) || K > (1 << 24)) return W4_ERR_UNSUPPORTED;
+    cudaStream_t st = (cudaStream_t)stream;
+
+    GemmParams p = {};
+    p.S = reinterpret_cast<const uint16_t *>(S);
+    p.Y = reinterpret_cast<uint16_t *>(Y);
+    p.M = M;
+    p.N = N;
+    p.K = K;
+
+    const int sms = w4host::num_sms();
+    const bool wide_k = (K % 256) == 0;
+    CUtensorMap tw, ts, tx;
+    memset(&ts, 0, sizeof ts);
+
+    // X: [M, K] BF16, 64-wide K boxes of MT rows, 128-byte swizzle.
+    auto map_x = [&](int mt) {
+        cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+        cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+        cuuint32_t box[2] = {64u, (cuuint32_t)mt};
+        return make_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, dims, strides, box,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
+    };
+    auto map_w = [&](int kb, int R) {
+        cuuint64_t dims[2] = {(cuuint64_t)(K / 8), (cuuint64_t)N};
+        cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+        cuuint32_t box[2] = {(cuuint32_t)(kb / 8), (cuuint32_t)R};
+        return make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_INT32, 2, Wq, dims, strides, box,
+                        kb == 256 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B);
+    };
+    auto map_s = [&](int R) {
+        cuuint64_t dims[2] = {(cuuint64_t)(K / 32), (cuuint64_t)N};
+        cuuint64_t strides[1] = {(cuuint64_t)(K / 16)};
+        cuuint32_t box[2] = {8u, (cuuint32_t)R};
+        return make_map(&ts, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, S, dims, strides, box,
+                        CU_TENSOR_MAP_SWIZZLE_NONE);
+    };
+
+    if (M <= 64 && wide_k) {
+        // Decode: one token tile, N split evenly over the SMs.
+        const int mt = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+        int R = ceil_div_i(N, sms);
+        R = std::min(128, std::max(16, (R + 7) / 8 * 8));
+        p.rows_per_tile = R;
+        p.n_row_tiles = ceil_div_i(N, R);
+        p.n_tok_tiles = 1;
+        p.num_kb = ceil_div_i(K, 256);
+        if (!map_x(mt) || !map_w(256, R) || !map_s(R)) return W4_ERR_CUDA;
+        const int items = p.n_row_tiles;
+        if (mt == 16) return launch_cfg<256, 16, 6, 2, 3, false>(tw, ts, tx, p, items, st);
+        if (mt == 32) return launch_cfg<256, 32, 6, 2, 3, false>(tw, ts, tx, p, items, st);
+        return launch_cfg<256, 64, 4, 2, 3, false>(tw, ts, tx, p, items, st);
+    }
+    // Prefill (and any K that is not a multiple of 256): 128-row tiles,
+    // 64-wide K blocks, scales read directly.
+    const int mt = M <= 64 ? 64 : 256;
+    p.rows_per_tile = 128;
+    p.n_row_tiles = ceil_div_i(N, 128);
+    p.n_tok_tiles = ceil_div_i(M, mt);
+    p.num_kb = ceil_div_i(K, 64);
+    if (!map_x(mt) || !map_w(64, 128)) return W4_ERR_CUDA;
+    const int64_t items = (int64_t)p.n_row_tiles * p.n_tok_tiles;
+    if (items > (1 << 30)) return W4_ERR_UNSUPPORTED;
+    if (mt == 64) return launch_cfg<64, 64, 8, 2, 8, false>(tw, ts, tx, p, (int)items, st);
+    return launch_cfg<64, 256, 6, 1, 8, false>(tw, ts, tx, p, (int)items, st);
+}
+
+extern "C" int64_t w4_moe_capacity(int64_t T, int topk, int E, int block) {
+    if (T < 0 || topk <= 0 || E <= 0 || block <= 0) return 0;
+    const int64_t cap = T * topk + (int64_t)E * (block - 1);
+    return (cap + block - 1) / block * block;
+}
+
+extern "C" w4_status w4_moe_w4a16_gemm(const w4_bf16 *A, int a_row_div, const int32_t *Wq,
+                                       const w4_bf16 *S, const int32_t *sorted_ids,
+                                       const int32_t *expert_ids, const int32_t *num_post_pad,
+                                       int64_t cap, int block, int64_t num_slots, w4_bf16 *C,
+                                       int64_t N, int64_t K, int E, void *stream) {
+    if (!w4host::aligned16(A) || !w4host::aligned16(Wq) || !w4host::aligned16(S) ||
+        !w4host::aligned16(sorted_ids) || !w4host::aligned16(expert_ids) ||
+        !w4host::aligned16(num_post_pad) || !w4host::aligned16(C))
+        return W4_ERR_INVALID_ARG;
+    if (a_row_div <= 0 || N <= 0 || K <= 0 || (K % 32) != 0 || E <= 0 || num_slots < 0 ||
+        cap < 0 || block <= 0 || (cap % block) != 0)
+        return W4_ERR_INVALID_ARG;
+    if (block != 16 && block != 32 && block != 64) return W4_ERR_UNSUPPORTED;
+    if ((K % 256) != 0) return W4_ERR_UNSUPPORTED;
+    if (num_slots == 0 || cap == 0) return W4_OK;
+    cudaStream_t st = (cudaStream_t)stream;
+
+    GemmParams p = {};
+    p.S = reinterpret_cast<const uint16_t *>(S);
+    p.Y = reinterpret_cast<uint16_t *>(C);
+    p.A = reinterpret_cast<const uint16_t *>(A);
+    p.sorted_ids = sorted_ids;
+    p.expert_ids = expert_ids;
+    p.num_post_pad = num_post_pad;
+    p.M = num_slots;
+    p.N = N;
+    p.K = K;
+    p.num_slots = num_slots;
+    p.a_row_div = a_row_div;
+    p.a_rows = (num_slots + a_row_div - 1) / a_row_div;
+    if (cap / block > (1 << 30)) return W4_ERR_UNSUPPORTED;
+    p.cap_blocks = (int)(cap / block);
+    p.rows_per_tile = 128;
+    p.n_row_tiles = ceil_div_i(N, 128);
+    p.n_tok_tiles = 0;
+    p.num_kb = ceil_div_i(K, 256);
+
+    CUtensorMap tw, ts, tx;
+    memset(&tx, 0, sizeof tx);
+    {
+        cuuint64_t dims[3] = {(cuuint64_t)(K / 8), (cuuint64_t)N, (cuuint64_t)E};
+        cuuint64_t strides[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N * (K / 2)};
+        cuuint32_t box[3] = {32u, 128u, 1u};
+        if (!make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_INT32, 3, Wq, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+            return W4_ERR_CUDA;
+    }
+    {
+        cuuint64_t dims[3] = {(cuuint64_t)(K / 32), (cuuint64_t)N, (cuuint64_t)E};
+        cuuint64_t strides[2] = {(cuuint64_t)(K / 16), (cuuint64_t)N * (K / 16)};
+        cuuint32_t box[3] = {8u, 128u, 1u};
+        if (!make_map(&ts, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, S, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+            return W4_ERR_CUDA;
+    }
+    const int64_t items_max = (cap / block) * p.n_row_tiles;
+    const int items = (int)std::min<int64_t>(items_max, 1 << 30);
+    if (block == 16) return launch_cfg<256, 16, 6, 2, 3, true>(tw, ts, tx, p, items, st);
+    if (block == 32) return launch_cfg<256, 32, 6, 2, 3, true>(tw, ts, tx, p, items, st);
+    return launch_cfg<256, 64, 4, 2, 3, true>(tw, ts, tx, p, items, st);
+}

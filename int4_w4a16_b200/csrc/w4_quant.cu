@@ -1,0 +1,272 @@
+// w4_quant.cu -- group-32 INT4 quantizers: fake quantization (QDQ), real
+// quantization + packing, the STE backward copy and the unpack/dequant helper.
+//
+// Method (INT4 QAT blog, fake quantization and Fig. 4; reportify.cn
+// "量化感知训练" [10][11][32]; "量化基础" §2.2): per group of 32 consecutive
+// BF16 weights along K, s = bf16_rne(fl32(amax / 7)),
+// q = clamp(rint_half_even(w / s), -8, 7), Wdq = bf16_rne(q * s), codes packed
+// low nibble first, eight per int32.
+//
+// Layout of the work: one thread owns 8 consecutive elements (one 16-byte
+// load, one packed word); 4 lanes own a group and reduce its amax with two
+// xor-shuffles.  Grid-stride loop, four 16-byte loads in flight per thread,
+// streaming (evict-first) loads and stores: the kernels are HBM-bound.
+//
+// Division-free exact rounding.  The codes must equal rint_half_even of the
+// IEEE fp32 quotient fl32(w / s).  With w and s both BF16 (8-bit significands)
+// the exact quotient y = w / s is either exactly a half-integer or at least
+// 1/510 away from every half-integer (write both as integer * 2^e; the
+// numerator of y - (j + 1/2) is a nonzero integer multiple of a power of two
+// that the denominator bounds), and fl32 never moves y across or onto a
+// half-integer.  The kernel forms t = w * r with r = rcp_rn(s) (relative error
+// < 2^-23, so |t - y| < 1e-6 for |y| <= 7.03), snaps t to the 2^-10 grid with
+// one fused multiply-add against 1.5 * 2^13, and then rounds the snapped
+// value to an integer, ties to even, by adding the constant that brings it to
+// 1.5 * 2^23.  Snapping maps exact ties onto the half-integer and keeps every
+// other quotient strictly on its own side, so the result equals
+// rint_half_even(y).  The code is then the low byte of the float's bits
+// (bits = 0x4B400000 + q).  Scales below 2^-126 (subnormal) take the plain
+// IEEE-division path.
+#include <algorithm>
+
+#include "w4_common.cuh"
+
+namespace w4 {
+
+__device__ unsigned int g_device_status = 0;
+
+namespace {
+
+constexpr float kSnap = 12288.0f;         // 1.5 * 2^13: ulp 2^-10 around it
+constexpr float kToInt = 12570624.0f;     // 1.5 * 2^23 - 1.5 * 2^13 (exact in fp32)
+constexpr float kMagic = 12582912.0f;     // 1.5 * 2^23: ulp 1 around it
+
+__device__ __forceinline__ float lo_f(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float hi_f(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Group amax over the 4 lanes that share a group; returns the BF16 bits of amax.
+__device__ __forceinline__ uint32_t group_amax_bits(const uint4 &v) {
+    // |w| as BF16 (sign bit cleared); max of BF16 magnitudes is exact.
+    const uint32_t m = 0x7FFF7FFFu;
+    const uint32_t u[4] = {v.x & m, v.y & m, v.z & m, v.w & m};
+    const __nv_bfloat162 *a = reinterpret_cast<const __nv_bfloat162 *>(u);
+    __nv_bfloat162 mx = __hmax2(__hmax2(a[0], a[1]), __hmax2(a[2], a[3]));
+    const uint32_t mb = *reinterpret_cast<uint32_t *>(&mx);
+    // non-negative BF16 values order like their bit patterns
+    uint32_t am = max(mb & 0xFFFFu, mb >> 16);
+    am = max(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
+    am = max(am, __shfl_xor_sync(0xFFFFFFFFu, am, 2));
+    return am;
+}
+
+struct GroupScale {
+    float s;        // the stored BF16 scale, widened
+    float r;        // rcp_rn(s) on the fast path
+    uint16_t bits;  // BF16 bits of s
+    int mode;       // 0: s == 0, 1: normal s (fast path), 2: subnormal s
+};
+
+__device__ __forceinline__ GroupScale make_scale(uint32_t amax_bits) {
+    GroupScale g;
+    const float a = __uint_as_float(amax_bits << 16);
+    const float s32 = __fdiv_rn(a, 7.0f);
+    const __nv_bfloat16 sb = __float2bfloat16_rn(s32);
+    g.bits = *reinterpret_cast<const uint16_t *>(&sb);
+    g.s = __bfloat162float(sb);
+    g.mode = (g.s == 0.0f) ? 0 : (g.s < 1.17549435e-38f ? 2 : 1);
+    g.r = (g.mode == 1) ? __frcp_rn(g.s) : 0.0f;
+    return g;
+}
+
+// c = 1.5 * 2^23 + q as an fp32 (so bits(c) = 0x4B400000 + q).
+__device__ __forceinline__ float code_float(float x, const GroupScale &g) {
+    if (g.mode == 1) return __fadd_rn(__fmaf_rn(x, g.r, kSnap), kToInt);
+    if (g.mode == 0) return kMagic;
+    const float q = (float)__float2int_rn(__fdiv_rn(x, g.s));  // IEEE path, tiny scales
+    return __fadd_rn(q, kMagic);
+}
+
+__device__ __forceinline__ void codes8(const uint4 &v, const GroupScale &g, float (&c)[8]) {
+    c[0] = code_float(lo_f(v.x), g);
+    c[1] = code_float(hi_f(v.x), g);
+    c[2] = code_float(lo_f(v.y), g);
+    c[3] = code_float(hi_f(v.y), g);
+    c[4] = code_float(lo_f(v.z), g);
+    c[5] = code_float(hi_f(v.z), g);
+    c[6] = code_float(lo_f(v.w), g);
+    c[7] = code_float(hi_f(v.w), g);
+}
+
+// Eight codes (low bytes of the floats' bits) -> one low-nibble-first word.
+__device__ __forceinline__ uint32_t pack8(const float (&c)[8]) {
+    const uint32_t b0 = __float_as_uint(c[0]), b1 = __float_as_uint(c[1]);
+    const uint32_t b2 = __float_as_uint(c[2]), b3 = __float_as_uint(c[3]);
+    const uint32_t b4 = __float_as_uint(c[4]), b5 = __float_as_uint(c[5]);
+    const uint32_t b6 = __float_as_uint(c[6]), b7 = __float_as_uint(c[7]);
+    // even = bytes [q0, q2, q4, q6], odd = [q1, q3, q5, q7]
+    const uint32_t even = __byte_perm(__byte_perm(b0, b2, 0x0040), __byte_perm(b4, b6, 0x0040),
+                                      0x5410);
+    const uint32_t odd = __byte_perm(__byte_perm(b1, b3, 0x0040), __byte_perm(b5, b7, 0x0040),
+                                     0x5410);
+    return (even & 0x0F0F0F0Fu) | ((odd << 4) & 0xF0F0F0F0u);
+}
+
+// Eight codes -> four BF16x2 words of bf16_rne(q * s).
+__device__ __forceinline__ uint4 dequant8(const float (&c)[8], float s) {
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float v0 = __fmul_rn(__fsub_rn(c[2 * j], kMagic), s);       // exact
+        const float v1 = __fmul_rn(__fsub_rn(c[2 * j + 1], kMagic), s);
+        __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
+        o[j] = *reinterpret_cast<uint32_t *>(&h);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+constexpr int kUnroll = 4;
+constexpr int kThreads = 256;
+
+// MODE 0: quantize + pack (Wq, S).  MODE 1: fake quant (Wdq, optional S).
+template <int MODE>
+__global__ void __launch_bounds__(kThreads) quant_kernel(const uint4 *__restrict__ W,
+                                                         uint4 *__restrict__ Wdq,
+                                                         uint32_t *__restrict__ Wq,
+                                                         uint16_t *__restrict__ S, int64_t n8) {
+    const int lane = threadIdx.x & 31;
+    const int64_t T = (int64_t)gridDim.x * blockDim.x;
+    const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    // The loop bound is tested on the warp's first item, so all 32 lanes run
+    // every iteration together (the shuffles need the full warp); n8 is a
+    // multiple of 4, so the 4 lanes of a group are valid or invalid together.
+    for (int64_t base = gt - lane; base < n8; base += kUnroll * T) {
+        uint4 v[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t i = base + lane + u * T;
+            v[u] = (i < n8) ? __ldcs(W + i) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t i = base + lane + u * T;
+            const GroupScale g = make_scale(group_amax_bits(v[u]));
+            if (i < n8) {
+                float c[8];
+                codes8(v[u], g, c);
+                if (MODE == 0) {
+                    __stcs(reinterpret_cast<unsigned int *>(Wq + i), pack8(c));
+                } else {
+                    __stcs(Wdq + i, dequant8(c, g.s));
+                }
+                if (S != nullptr && (lane & 3) == 0) S[i >> 2] = g.bits;
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kThreads) copy16_kernel(const uint4 *__restrict__ src,
+                                                          uint4 *__restrict__ dst, int64_t n16) {
+    const int64_t T = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += T)
+        __stcs(dst + i, __ldcs(src + i));
+}
+
+__global__ void copy2_tail_kernel(const uint16_t *__restrict__ src, uint16_t *__restrict__ dst,
+                                  int64_t begin, int64_t n) {
+    const int64_t i = begin + (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) dst[i] = src[i];
+}
+
+// One thread = 4 words = one group of 32 codes sharing one scale.
+__global__ void __launch_bounds__(kThreads) dequant_kernel(const uint4 *__restrict__ Wq,
+                                                           const uint16_t *__restrict__ S,
+                                                           uint4 *__restrict__ Wdq,
+                                                           int64_t ngroups) {
+    const int64_t T = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < ngroups; g += T) {
+        const uint4 w = __ldcs(Wq + g);
+        const uint32_t s2 = bf16x2_splat(S[g]);
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint32_t o[4];
+            dequant_word(ws[j], s2, o);
+            __stcs(Wdq + 4 * g + j, make_uint4(o[0], o[1], o[2], o[3]));
+        }
+    }
+}
+
+int grid_for(int64_t work_items, int per_thread) {
+    const int64_t need = (work_items + (int64_t)kThreads * per_thread - 1) /
+                         ((int64_t)kThreads * per_thread);
+    const int64_t cap = (int64_t)w4host::num_sms() * 4;
+    return (int)std::max<int64_t>(1, std::min<int64_t>(need, cap));
+}
+
+w4_status check_quant_args(const void *in, const void *out, int64_t rows, int64_t K, int group) {
+    if (group != 32) return W4_ERR_UNSUPPORTED;
+    if (rows < 0 || K <= 0 || (K % 32) != 0) return W4_ERR_INVALID_ARG;
+    if (rows > 0 && K > ((int64_t)1 << 60) / rows) return W4_ERR_INVALID_ARG;
+    if (!w4host::aligned16(in) || !w4host::aligned16(out)) return W4_ERR_INVALID_ARG;
+    return W4_OK;
+}
+
+}  // namespace
+}  // namespace w4
+
+using namespace w4;
+
+extern "C" w4_status w4_fake_quant(const w4_bf16 *W, w4_bf16 *Wdq, w4_bf16 *S, int64_t rows,
+                                   int64_t K, int group, void *stream) {
+    w4_status st = check_quant_args(W, Wdq, rows, K, group);
+    if (st != W4_OK) return st;
+    if (S != nullptr && !w4host::aligned16(S)) return W4_ERR_INVALID_ARG;
+    if ((const void *)W == (const void *)Wdq) return W4_ERR_INVALID_ARG;
+    const int64_t n8 = rows * K / 8;
+    if (n8 == 0) return W4_OK;
+    quant_kernel<1><<<grid_for(n8, kUnroll), kThreads, 0, (cudaStream_t)stream>>>(
+        reinterpret_cast<const uint4 *>(W), reinterpret_cast<uint4 *>(Wdq), nullptr,
+        reinterpret_cast<uint16_t *>(S), n8);
+    return w4host::launch_status();
+}
+
+extern "C" w4_status w4_quantize_pack(const w4_bf16 *W, int32_t *Wq, w4_bf16 *S, int64_t rows,
+                                      int64_t K, int group, void *stream) {
+    w4_status st = check_quant_args(W, Wq, rows, K, group);
+    if (st != W4_OK) return st;
+    if (!w4host::aligned16(S)) return W4_ERR_INVALID_ARG;
+    const int64_t n8 = rows * K / 8;
+    if (n8 == 0) return W4_OK;
+    quant_kernel<0><<<grid_for(n8, kUnroll), kThreads, 0, (cudaStream_t)stream>>>(
+        reinterpret_cast<const uint4 *>(W), nullptr, reinterpret_cast<uint32_t *>(Wq),
+        reinterpret_cast<uint16_t *>(S), n8);
+    return w4host::launch_status();
+}
+
+extern "C" w4_status w4_ste_backward(const w4_bf16 *dWdq, w4_bf16 *dW, int64_t n, void *stream) {
+    if (n < 0 || !w4host::aligned16(dWdq) || !w4host::aligned16(dW)) return W4_ERR_INVALID_ARG;
+    if ((const void *)dWdq == (const void *)dW || n == 0) return W4_OK;  // zero-copy identity
+    const uint16_t *a = reinterpret_cast<const uint16_t *>(dWdq);
+    uint16_t *b = reinterpret_cast<uint16_t *>(dW);
+    if (a < b + n && b < a + n) return W4_ERR_INVALID_ARG;  // partial overlap
+    const int64_t n16 = n / 8;
+    if (n16 > 0)
+        copy16_kernel<<<grid_for(n16, 1), kThreads, 0, (cudaStream_t)stream>>>(
+            reinterpret_cast<const uint4 *>(a), reinterpret_cast<uint4 *>(b), n16);
+    if (n16 * 8 < n)
+        copy2_tail_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(a, b, n16 * 8, n);
+    return w4host::launch_status();
+}
+
+extern "C" w4_status w4_dequant(const int32_t *Wq, const w4_bf16 *S, w4_bf16 *Wdq, int64_t rows,
+                                int64_t K, int group, void *stream) {
+    w4_status st = check_quant_args(Wq, Wdq, rows, K, group);
+    if (st != W4_OK) return st;
+    if (!w4host::aligned16(S)) return W4_ERR_INVALID_ARG;
+    const int64_t ngroups = rows * K / 32;
+    if (ngroups == 0) return W4_OK;
+    dequant_kernel<<<grid_for(ngroups, 1), kThreads, 0, (cudaStream_t)stream>>>(
+        reinterpret_cast<const uint4 *>(Wq), reinterpret_cast<const uint16_t *>(S),
+        reinterpret_cast<uint4 *>(Wdq), ngroups);
+    return w4host::launch_status();
+}

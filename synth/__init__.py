@@ -53,8 +53,10 @@ def normal_bf16(shape, std: float, seed: int, index: int = 0, device="cpu",
 def laplace_bf16(shape, b: float, seed: int, index: int = 0, device="cpu") -> torch.Tensor:
     """Laplace(0, b) BF16 tensor (location 0, scale b), by inverse CDF."""
     g = _gen(seed, index, device)
-    u = torch.rand(shape, generator=g, device=device, dtype=torch.float32) - 0.5
-    # u in [-0.5, 0.5); 1 - 2|u| in (0, 1]
+    # u in [-0.5 + 2^-25, 0.5): strictly inside (-1/2, 1/2), so 1 - 2|u| > 0 and
+    # every draw is finite (a draw of exactly -1/2 would map to infinity).
+    u = (torch.rand(shape, generator=g, device=device, dtype=torch.float32) - 0.5) \
+        * (1.0 - 2.0 ** -24)
     x = -b * torch.sign(u) * torch.log1p(-2.0 * u.abs())
     return x.to(torch.bfloat16)
 

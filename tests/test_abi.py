@@ -1,0 +1,100 @@
+"""The C-ABI library loads, exports every entry point include/w4a16.h declares,
+and rejects malformed calls on the host before launching anything (no GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import int4_w4a16_b200 as w4
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "w4a16.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(w4\w*)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ["w4_fake_quant", "w4_ste_backward", "w4_quantize_pack", "w4_dequant",
+                     "w4a16_gemm", "w4_moe_align", "w4_moe_w4a16_gemm", "w4_moe_capacity",
+                     "w4_device_status", "w4_status_string", "w4_version",
+                     "w4_last_cuda_error"]:
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = ctypes.CDLL(w4.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(L, name), f"{name} declared in w4a16.h but not exported"
+
+
+def test_status_strings_and_version():
+    L = w4.lib()
+    assert [L.w4_status_string(i) for i in range(5)] == [
+        b"W4_OK", b"W4_ERR_INVALID_ARG", b"W4_ERR_UNSUPPORTED", b"W4_ERR_CUDA",
+        b"W4_ERR_TIMEOUT"]
+    assert w4.w4_version() >= 100
+
+
+def test_moe_capacity_host_only():
+    L = w4.lib()
+    assert L.w4_moe_capacity(16, 8, 128, 16) == 16 * 8 + 128 * 15
+    assert L.w4_moe_capacity(3, 2, 4, 4) == 20          # 6 + 12 = 18 -> 20
+    assert L.w4_moe_capacity(-1, 8, 128, 16) == 0
+
+
+A16 = 0x10000          # a 16-byte-aligned fake address: never dereferenced, the
+MIS = 0x10002          # calls below all fail validation before any CUDA call
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((A16, A16, None, 4, 64, 16, None), 2),      # group != 32 -> unsupported
+    ((A16, A16, None, 4, 48, 32, None), 1),      # K not a multiple of 32
+    ((None, A16, None, 4, 64, 32, None), 1),     # null input
+    ((MIS, A16, None, 4, 64, 32, None), 1),      # misaligned input
+    ((A16, A16, None, 4, 64, 32, None), 1),      # output aliases input
+    ((A16, A16 + 0x1000, MIS, 4, 64, 32, None), 1),  # misaligned scales
+    ((A16, A16 + 0x1000, None, -1, 64, 32, None), 1),  # negative rows
+])
+def test_fake_quant_validation(args, expect):
+    assert w4.lib().w4_fake_quant(*args) == expect
+
+
+def test_other_validation():
+    L = w4.lib()
+    assert L.w4_quantize_pack(A16, A16 + 0x100, None, 4, 64, 32, None) == 1
+    assert L.w4_quantize_pack(A16, A16 + 0x100, A16 + 0x200, 4, 64, 8, None) == 2
+    assert L.w4_dequant(A16, MIS, A16 + 0x100, 4, 64, 32, None) == 1
+    assert L.w4_ste_backward(A16, MIS, 8, None) == 1
+    assert L.w4_ste_backward(A16, A16, 8, None) == 0           # aliased: zero-copy no-op
+    assert L.w4_ste_backward(A16, A16 + 2 * 8, 64, None) == 1  # partial overlap
+    assert L.w4a16_gemm(A16, A16, A16, None, 1, 8, 64, 32, None) == 1
+    assert L.w4a16_gemm(A16, A16, A16, A16, 1, 8, 40, 32, None) == 1
+    assert L.w4a16_gemm(A16, A16, A16, A16, 1, 8, 64, 64, None) == 2
+    assert L.w4a16_gemm(A16, A16, A16, A16, 0, 8, 64, 32, None) == 0   # empty: no launch
+    # moe_align: block not a power of two, E too large, capacity too small
+    assert L.w4_moe_align(A16, 4, 2, 8, 24, A16, 1024, A16, A16, None) == 1
+    assert L.w4_moe_align(A16, 4, 2, 2048, 16, A16, 1 << 20, A16, A16, None) == 1
+    assert L.w4_moe_align(A16, 4, 2, 8, 16, A16, 16, A16, A16, None) == 1
+    # grouped GEMM: unsupported block size / K, misaligned pointers
+    args = [A16, 8, A16, A16, A16, A16, A16, 1024, 16, 128, A16, 3072, 4096, 128, None]
+    a = list(args); a[8] = 8
+    assert L.w4_moe_w4a16_gemm(*a) == 2
+    a = list(args); a[12] = 4096 + 32
+    assert L.w4_moe_w4a16_gemm(*a) == 2
+    a = list(args); a[10] = MIS
+    assert L.w4_moe_w4a16_gemm(*a) == 1
+    a = list(args); a[1] = 0
+    assert L.w4_moe_w4a16_gemm(*a) == 1
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    W = torch.zeros(4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        w4.w4_fake_quant(W, torch.empty_like(W))
