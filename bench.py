@@ -314,12 +314,21 @@ def dist_setup(n_gpus: int):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Max of a scalar over the ranks (the only collective: timing plumbing)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def shard(n_items: int, rank: int, world: int) -> range:
+    """Contiguous, balanced share of n independent items for this rank."""
+    lo = n_items * rank // world
+    hi = n_items * (rank + 1) // world
+    return range(lo, hi)
 
 
 def barrier(world: int):
@@ -356,6 +365,141 @@ def run_reference(args, rank, world):
     return 0
 
 
+# ---------------------------------------------------------------------------
+# Extra workloads (their own lines; not the default bench line)
+# ---------------------------------------------------------------------------
+
+def _flush_l2(buf):
+    buf.zero_()
+
+
+def _time_kernel(fn, reps, flush):
+    """Median CUDA-event time (ms) of fn over reps, L2 flushed before each."""
+    ts = []
+    for _ in range(reps):
+        flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    ts.sort()
+    return ts[len(ts) // 2], ts[len(ts) // 10], ts[(9 * len(ts)) // 10]
+
+
+def run_extra(args):
+    import int4_w4a16_b200 as w4
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w4.lib()
+    peaks = load_peaks()
+    l2 = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    flush = lambda: _flush_l2(l2)
+    reps = max(5, args.steps)
+    out = {"workload": args.workload, "peaks": peaks, "l2": "256 MB buffer written before "
+           "every timed launch", "reps": reps, "results": []}
+    if args.workload == "prefill":
+        cfg = synth.Prefill()
+        W = cfg.weight(dev)
+        Wq, S = w4.quantize_pack(W)
+        del W
+        for M in cfg.Ms:
+            X = cfg.activations(M, dev)
+            Y = torch.empty((M, cfg.N), dtype=torch.bfloat16, device=dev)
+            fn = lambda: w4.w4a16_gemm(X, Wq, S, Y)
+            for _ in range(3):
+                fn()
+            med, p10, p90 = _time_kernel(fn, reps, flush)
+            fl = 2.0 * M * cfg.N * cfg.K
+            tf = fl / (med * 1e-3) / 1e12
+            out["results"].append({"M": M, "N": cfg.N, "K": cfg.K, "ms": med, "p10": p10,
+                                   "p90": p90, "TFLOP/s": tf,
+                                   "frac_bf16_burst": tf / peaks["bf16_tflops"],
+                                   "frac_bf16_sustained": tf / peaks["bf16_tflops_sustained"]})
+    elif args.workload == "moe":
+        cfg = synth.MoEDecode()
+        Wg = cfg.gate_up_weight(dev)
+        Wd = cfg.down_weight(dev)
+        E = cfg.E
+        Wq_g = torch.empty((E, 2 * cfg.inter, cfg.hidden // 8), dtype=torch.int32, device=dev)
+        S_g = torch.empty((E, 2 * cfg.inter, cfg.hidden // 32), dtype=torch.bfloat16, device=dev)
+        Wq_d = torch.empty((E, cfg.hidden, cfg.inter // 8), dtype=torch.int32, device=dev)
+        S_d = torch.empty((E, cfg.hidden, cfg.inter // 32), dtype=torch.bfloat16, device=dev)
+        for e in range(E):
+            w4.w4_quantize_pack(Wg[e], Wq_g[e], S_g[e])
+            w4.w4_quantize_pack(Wd[e], Wq_d[e], S_d[e])
+        del Wg, Wd
+        per_gu = 2 * cfg.inter * cfg.hidden * 9 // 16
+        per_dn = cfg.hidden * cfg.inter * 9 // 16
+        for T in cfg.Ts:
+            ids, _ = cfg.routing(T)
+            ids_d = ids.to(dev)
+            active = len(set(ids.view(-1).tolist()))
+            X = cfg.tokens(T, dev)
+            H = synth.normal_bf16((T * cfg.topk, cfg.inter), 1.0, 0, 300 + T, dev)
+            for block in cfg.blocks:
+                s_ids, e_ids, npp = w4.moe_align(ids_d, E, block)
+                C1 = torch.empty((T * cfg.topk, 2 * cfg.inter), dtype=torch.bfloat16, device=dev)
+                C2 = torch.empty((T * cfg.topk, cfg.hidden), dtype=torch.bfloat16, device=dev)
+                f_align = lambda: w4.w4_moe_align(ids_d, E, block, s_ids, e_ids, npp)
+                f_gu = lambda: w4.w4_moe_w4a16_gemm(X, cfg.topk, Wq_g, S_g, s_ids, e_ids, npp,
+                                                    block, T * cfg.topk, C1)
+                f_dn = lambda: w4.w4_moe_w4a16_gemm(H, 1, Wq_d, S_d, s_ids, e_ids, npp, block,
+                                                    T * cfg.topk, C2)
+                for f in (f_align, f_gu, f_dn):
+                    f()
+                t_al = _time_kernel(f_align, reps, flush)[0]
+                t_gu = _time_kernel(f_gu, reps, flush)[0]
+                t_dn = _time_kernel(f_dn, reps, flush)[0]
+                npad = int(npp.item())
+                b_gu = active * per_gu + X.nbytes + C1.nbytes
+                b_dn = active * per_dn + H.nbytes + C2.nbytes
+                out["results"].append({
+                    "T": T, "block": block, "active_experts": active, "padded_slots": npad,
+                    "moe_align_us": t_al * 1e3,
+                    "gate_up_us": t_gu * 1e3, "gate_up_GB/s": b_gu / (t_gu * 1e-3) / 1e9,
+                    "gate_up_frac": b_gu / (t_gu * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                    "down_us": t_dn * 1e3, "down_GB/s": b_dn / (t_dn * 1e-3) / 1e9,
+                    "down_frac": b_dn / (t_dn * 1e-3) / 1e9 / peaks["hbm_gbs"]})
+    elif args.workload == "qat":
+        cfg = synth.QATStack()
+        mats = []
+        for layer in range(cfg.layers):
+            for which in range(2):
+                W = cfg.weight(layer, which, dev)
+                G = cfg.grad(layer, which, dev)
+                rows, K = W.shape
+                mats.append((W, G, torch.empty_like(W), torch.empty_like(W),
+                             torch.empty((rows, K // 8), dtype=torch.int32, device=dev),
+                             torch.empty((rows, K // 32), dtype=torch.bfloat16, device=dev)))
+        n = cfg.elements
+
+        def fq():
+            for (W, G, Wdq, dW, Wq, S) in mats:
+                w4.w4_fake_quant(W, Wdq)
+
+        def ste():
+            for (W, G, Wdq, dW, Wq, S) in mats:
+                w4.w4_ste_backward(G, dW)
+
+        def qp():
+            for (W, G, Wdq, dW, Wq, S) in mats:
+                w4.w4_quantize_pack(W, Wq, S)
+
+        for name, f, bpe in (("fake_quant", fq, 4.0), ("ste_backward", ste, 4.0),
+                             ("quantize_pack", qp, 2.5625)):
+            f()
+            med, p10, p90 = _time_kernel(f, max(3, reps // 10), flush)
+            gbs = n * bpe / (med * 1e-3) / 1e9
+            out["results"].append({"kernel": name, "elements": n, "ms": med, "GB/s": gbs,
+                                   "frac": gbs / peaks["hbm_gbs"]})
+    w4.w4_device_status()
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 METRIC = "W4A16 hot-path HBM throughput (decode GEMV sweep + QAT fake-quant/STE + quantize_pack), GB/s"
 
 
@@ -365,7 +509,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decode", choices=["decode"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "moe", "qat"],
+                    help="decode is the bench line; the others print their own lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--e2e-steps", type=int, default=5)
@@ -378,6 +523,8 @@ def main():
     if not torch.cuda.is_available():
         print(json.dumps({"error": "no CUDA device"}))
         return 1
+    if args.workload != "decode":
+        return run_extra(args)
     rank, world, local = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)

@@ -39,8 +39,9 @@
 namespace w4 {
 namespace {
 
-constexpr int kWarps = 10;
-constexpr int kThreadsGemm = kWarps * 32;
+// Warp roles: 0 = loads, 1 = TMEM allocation + MMA issue, then 4 * NDQ
+// dequant warps (NDQ per TMEM lane quarter), then 4 epilogue warps.
+__host__ __device__ constexpr int gemm_threads(int ndq) { return 32 * (2 + 4 * ndq + 4); }
 constexpr int kTmemCols = 512;
 
 struct GemmParams {
@@ -62,7 +63,7 @@ struct GemmParams {
 };
 
 // Shared-memory layout, all offsets from a 1024-aligned base.
-template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE>
+template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT>
 struct Layout {
     static constexpr int kWBytes = 128 * KB / 2;            // packed tile, up to 128 rows
     static constexpr int kSBytes = (KB == 256) ? 128 * 16 : 0;
@@ -76,8 +77,29 @@ struct Layout {
     static constexpr int kAlloc = kBytes + 1024;            // slack for 1024-alignment
     static_assert(kWBytes % 1024 == 0 && kXSub % 1024 == 0, "1024-byte aligned tiles");
     static_assert(kStage % 1024 == 0, "stage size");
-    static_assert(NACC * MT + NASTAGE * (KB / 2) <= kTmemCols, "TMEM budget");
+    static_assert(NACC * NSPLIT * MT + NASTAGE * (KB / 2) <= kTmemCols, "TMEM budget");
 };
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
+    return v;
+}
 
 __device__ __forceinline__ uint32_t swz(uint32_t off, uint32_t sw_bytes) {
     // TMA / UMMA swizzle: 16-byte chunk index XOR address bits [7, ...).
@@ -101,15 +123,22 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
     }
 }
 
-template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, bool MOE>
-__global__ void __launch_bounds__(kThreadsGemm, 1)
+// NSPLIT: independent accumulators per work item; consecutive 16-wide K steps
+// of the MMA go round-robin to them, so small-N MMAs do not wait on each
+// other, and the epilogue adds them in a fixed order.
+template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT, int NDQ, bool MOE>
+__global__ void __launch_bounds__(gemm_threads(NDQ), 1)
     w4a16_tc_kernel(const __grid_constant__ CUtensorMap tm_w,
                     const __grid_constant__ CUtensorMap tm_s,
                     const __grid_constant__ CUtensorMap tm_x, const GemmParams p) {
-    using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE>;
+    using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE, NSPLIT>;
     constexpr int kWords = KB / 8;             // packed words per row per k-block
     constexpr int kAStageCols = KB / 2;        // TMEM columns per A stage
-    constexpr int kABase = NACC * MT;          // first A column
+    constexpr int kAccCols = NSPLIT * MT;      // TMEM columns per work item accumulator
+    constexpr int kABase = NACC * kAccCols;    // first A column
+    constexpr int kDqWarps = 4 * NDQ;
+    constexpr int kEpiWarp0 = 2 + kDqWarps;
+    static_assert((KB / 32) % NDQ == 0, "k-block chunks split evenly over the dequant warps");
     constexpr uint32_t kIdesc = idesc_bf16_f32(128, MT);
 
     extern __shared__ uint8_t smem_raw[];
@@ -144,7 +173,7 @@ __global__ void __launch_bounds__(kThreadsGemm, 1)
             mbar_init(empty_bar(s), 1u);
         }
         for (int a = 0; a < NASTAGE; ++a) {
-            mbar_init(afull_bar(a), 128u);
+            mbar_init(afull_bar(a), 32u * kDqWarps);
             mbar_init(aempty_bar(a), 1u);
         }
         for (int d = 0; d < NACC; ++d) {
@@ -247,7 +276,7 @@ __global__ void __launch_bounds__(kThreadsGemm, 1)
                     break;
                 }
                 tc_fence_after_sync();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(d * MT);
+                const uint32_t d_tmem = tmem_base + (uint32_t)(d * kAccCols);
                 for (int kb = 0; kb < num_kb; ++kb, ++it) {
                     const int s = it % NSTAGE;
                     const int a = it % NASTAGE;
@@ -262,8 +291,9 @@ __global__ void __launch_bounds__(kThreadsGemm, 1)
 #pragma unroll
                     for (int u = 0; u < KB / 16; ++u) {
                         const uint32_t baddr = x_stage(s) + (u >> 2) * L::kXSub + (u & 3) * 32;
-                        tc_mma_ts(d_tmem, a_tmem + u * 8, smem_desc_k_sw128(baddr), kIdesc,
-                                  (kb > 0 || u > 0) ? 1u : 0u);
+                        tc_mma_ts(d_tmem + (uint32_t)((u % NSPLIT) * MT), a_tmem + u * 8,
+                                  smem_desc_k_sw128(baddr), kIdesc,
+                                  (kb > 0 || u >= NSPLIT) ? 1u : 0u);
                     }
                     tc_commit(empty_bar(s));
                     tc_commit(aempty_bar(a));
@@ -275,9 +305,15 @@ __global__ void __launch_bounds__(kThreadsGemm, 1)
             tc_commit(mmadone_bar);
             drain_wait(mmadone_bar, 0u);
         }
-    } else if (warp < 6) {
+    } else if (warp < kEpiWarp0) {
         // --------------------------------------------------------- dequant
+        // NDQ warps per TMEM lane quarter; warp part h takes chunks
+        // [h*GH, (h+1)*GH) of every k-block (a chunk = 16 bytes of a row =
+        // 4 packed words = one group of 32 codes).
+        constexpr int G = KB / 32;
+        constexpr int GH = G / NDQ;
         const int q4 = warp & 3;                    // TMEM lane quarter of this warp
+        const int half = (warp - 2) >> 2;           // part index in [0, NDQ)
         const int lrow = q4 * 32 + lane;            // A row of this thread
         const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
         const int64_t gpr = p.K / 32;               // groups per row
@@ -297,14 +333,14 @@ __global__ void __launch_bounds__(kThreadsGemm, 1)
             for (int kb = 0; kb < num_kb; ++kb, ++it) {
                 const int s = it % NSTAGE;
                 const int a = it % NASTAGE;
-                // scales of this k-block (direct loads when the tile has no TMA scales)
-                uint32_t sc[KB / 32];
+                uint32_t sc[GH];
                 if (KB != 256) {
+                    // scales of this k-block (direct loads when the tile has no TMA scales)
 #pragma unroll
-                    for (int g = 0; g < KB / 32; ++g) {
-                        const int64_t gi = (int64_t)kb * (KB / 32) + g;
+                    for (int j = 0; j < GH; ++j) {
+                        const int64_t gi = (int64_t)kb * G + half * GH + j;
                         const uint16_t v = (srow != nullptr && gi < gpr) ? __ldg(srow + gi) : 0;
-                        sc[g] = bf16x2_splat(v);
+                        sc[j] = bf16x2_splat(v);
                     }
                 }
                 if (!warp_wait(full_bar(s), (it / NSTAGE) & 1u, abort_flag) ||
@@ -313,42 +349,44 @@ __global__ void __launch_bounds__(kThreadsGemm, 1)
                     break;
                 }
                 tc_fence_after_sync();
-                if (KB == 256) {
-                    const uint4 sv = *reinterpret_cast<const uint4 *>(smem + (s_stage(s) - sbase) +
-                                                                     lrow * 16);
-                    const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+                // all shared-memory reads of this k-block first
+                uint4 wv[GH];
 #pragma unroll
-                    for (int g = 0; g < 8; ++g)
-                        sc[g % (KB / 32)] = bf16x2_splat((uint16_t)(sw[g >> 1] >> (16 * (g & 1))));
-                    // (the loop above fills all eight entries when KB == 256)
+                for (int j = 0; j < GH; ++j) {
+                    const uint32_t off =
+                        swz((uint32_t)(lrow * (KB / 2) + (half * GH + j) * 16), KB / 2);
+                    wv[j] = lds128(w_stage(s) + off);
                 }
-                const uint8_t *wrow = smem + (w_stage(s) - sbase);
+                if (KB == 256) {
+                    // this part's GH scales of the row (2 * GH bytes, naturally aligned)
+                    const uint32_t saddr = s_stage(s) + lrow * 16 + half * GH * 2;
+                    uint32_t sw[4];
+                    if (GH == 8) {
+                        const uint4 v4 = lds128(saddr);
+                        sw[0] = v4.x; sw[1] = v4.y; sw[2] = v4.z; sw[3] = v4.w;
+                    } else if (GH == 4) {
+                        const uint2 v2 = lds64(saddr);
+                        sw[0] = v2.x; sw[1] = v2.y; sw[2] = 0; sw[3] = 0;
+                    } else {
+                        sw[0] = lds32(saddr); sw[1] = 0; sw[2] = 0; sw[3] = 0;
+                    }
+#pragma unroll
+                    for (int j = 0; j < GH; ++j)
+                        sc[j] = bf16x2_splat((uint16_t)(sw[j >> 1] >> (16 * (j & 1))));
+                }
                 const uint32_t a_col = tmem_base + lane_addr + (uint32_t)(kABase + a * kAStageCols);
 #pragma unroll
-                for (int g = 0; g < KB / 32; ++g) {
-                    // 16-byte chunk g of this row = 4 words = one group of 32 codes
-                    const uint32_t off = swz((uint32_t)(lrow * (KB / 2) + g * 16), KB / 2);
-                    const uint4 wv = *reinterpret_cast<const uint4 *>(wrow + off);
-                    const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
-                    uint32_t o[16];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        uint32_t t4[4];
-                        dequant_word(ws[j], sc[g], t4);
-                        o[4 * j + 0] = t4[0];
-                        o[4 * j + 1] = t4[1];
-                        o[4 * j + 2] = t4[2];
-                        o[4 * j + 3] = t4[3];
-                    }
-                    // columns: 2 BF16 per 32-bit column, ascending k
+                for (int j = 0; j < GH; ++j) {
+                    const uint32_t ws[4] = {wv[j].x, wv[j].y, wv[j].z, wv[j].w};
                     uint32_t lo[8], hi[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        lo[j] = o[j];
-                        hi[j] = o[8 + j];
-                    }
-                    tmem_st_x8(a_col + g * 16, lo);
-                    tmem_st_x8(a_col + g * 16 + 8, hi);
+                    dequant_word(ws[0], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&lo[0]));
+                    dequant_word(ws[1], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&lo[4]));
+                    dequant_word(ws[2], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&hi[0]));
+                    dequant_word(ws[3], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&hi[4]));
+                    // columns: 2 BF16 per 32-bit column, ascending k
+                    const uint32_t col = a_col + (uint32_t)((half * GH + j) * 16);
+                    tmem_st_x8(col, lo);
+                    tmem_st_x8(col + 8, hi);
                 }
                 tmem_wait_st();
                 tc_fence_before_sync();
@@ -372,8 +410,17 @@ __global__ void __launch_bounds__(kThreadsGemm, 1)
 #pragma unroll 1
             for (int c0 = 0; c0 < MT; c0 += 16) {
                 uint32_t v[16];
-                tmem_ld_x16(tmem_base + lane_addr + (uint32_t)(d * MT + c0), v);
+                tmem_ld_x16(tmem_base + lane_addr + (uint32_t)(d * kAccCols + c0), v);
                 tmem_wait_ld();
+#pragma unroll
+                for (int sp = 1; sp < NSPLIT; ++sp) {
+                    uint32_t w2[16];
+                    tmem_ld_x16(tmem_base + lane_addr + (uint32_t)(d * kAccCols + sp * MT + c0), w2);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(w2[j]));
+                }
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
                     const int tok = c0 + j;
@@ -408,11 +455,11 @@ __global__ void __launch_bounds__(kThreadsGemm, 1)
 // Host side
 // ---------------------------------------------------------------------------
 
-template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, bool MOE>
+template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT, int NDQ, bool MOE>
 w4_status launch_cfg(const CUtensorMap &tw, const CUtensorMap &ts, const CUtensorMap &tx,
                      const GemmParams &p, int num_items_max, cudaStream_t stream) {
-    using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE>;
-    auto kern = w4a16_tc_kernel<KB, MT, NSTAGE, NACC, NASTAGE, MOE>;
+    using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE, NSPLIT>;
+    auto kern = w4a16_tc_kernel<KB, MT, NSTAGE, NACC, NASTAGE, NSPLIT, NDQ, MOE>;
     // At least half of the SM's shared memory, so one CTA (and one TMEM
     // allocation of 512 columns) per SM.
     const int smem = std::max(L::kAlloc, 120 * 1024);
@@ -424,7 +471,7 @@ w4_status launch_cfg(const CUtensorMap &tw, const CUtensorMap &ts, const CUtenso
         configured = true;
     }
     const int grid = std::max(1, std::min(num_items_max, w4host::num_sms()));
-    kern<<<grid, kThreadsGemm, smem, stream>>>(tw, ts, tx, p);
+    kern<<<grid, gemm_threads(NDQ), smem, stream>>>(tw, ts, tx, p);
     return w4host::launch_status();
 }
 
@@ -492,17 +539,18 @@ extern "C" w4_status w4a16_gemm(const w4_bf16 *X, const int32_t *Wq, const w4_bf
     if (M <= 64 && wide_k) {
         // Decode: one token tile, N split evenly over the SMs.
         const int mt = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
-        int R = ceil_div_i(N, sms);
-        R = std::min(128, std::max(16, (R + 7) / 8 * 8));
+        // rows per tile: every SM streams the same number of weight rows
+        int R = std::min<int64_t>(128, std::max<int64_t>(1, ceil_div_i(N, sms)));
+        while (R < 128 && ceil_div_i(N, R) > sms) ++R;
         p.rows_per_tile = R;
         p.n_row_tiles = ceil_div_i(N, R);
         p.n_tok_tiles = 1;
         p.num_kb = ceil_div_i(K, 256);
         if (!map_x(mt) || !map_w(256, R) || !map_s(R)) return W4_ERR_CUDA;
         const int items = p.n_row_tiles;
-        if (mt == 16) return launch_cfg<256, 16, 6, 2, 3, false>(tw, ts, tx, p, items, st);
-        if (mt == 32) return launch_cfg<256, 32, 6, 2, 3, false>(tw, ts, tx, p, items, st);
-        return launch_cfg<256, 64, 4, 2, 3, false>(tw, ts, tx, p, items, st);
+        if (mt == 16) return launch_cfg<256, 16, 6, 1, 3, 4, 4, false>(tw, ts, tx, p, items, st);
+        if (mt == 32) return launch_cfg<256, 32, 6, 1, 3, 4, 4, false>(tw, ts, tx, p, items, st);
+        return launch_cfg<256, 64, 4, 1, 2, 4, 4, false>(tw, ts, tx, p, items, st);
     }
     // Prefill (and any K that is not a multiple of 256): 128-row tiles,
     // 64-wide K blocks, scales read directly.
@@ -514,8 +562,8 @@ extern "C" w4_status w4a16_gemm(const w4_bf16 *X, const int32_t *Wq, const w4_bf
     if (!map_x(mt) || !map_w(64, 128)) return W4_ERR_CUDA;
     const int64_t items = (int64_t)p.n_row_tiles * p.n_tok_tiles;
     if (items > (1 << 30)) return W4_ERR_UNSUPPORTED;
-    if (mt == 64) return launch_cfg<64, 64, 8, 2, 8, false>(tw, ts, tx, p, (int)items, st);
-    return launch_cfg<64, 256, 6, 1, 8, false>(tw, ts, tx, p, (int)items, st);
+    if (mt == 64) return launch_cfg<64, 64, 8, 1, 8, 4, 2, false>(tw, ts, tx, p, (int)items, st);
+    return launch_cfg<64, 256, 6, 1, 8, 1, 2, false>(tw, ts, tx, p, (int)items, st);
 }
 
 extern "C" int64_t w4_moe_capacity(int64_t T, int topk, int E, int block) {
@@ -581,7 +629,7 @@ extern "C" w4_status w4_moe_w4a16_gemm(const w4_bf16 *A, int a_row_div, const in
     }
     const int64_t items_max = (cap / block) * p.n_row_tiles;
     const int items = (int)std::min<int64_t>(items_max, 1 << 30);
-    if (block == 16) return launch_cfg<256, 16, 6, 2, 3, true>(tw, ts, tx, p, items, st);
-    if (block == 32) return launch_cfg<256, 32, 6, 2, 3, true>(tw, ts, tx, p, items, st);
-    return launch_cfg<256, 64, 4, 2, 3, true>(tw, ts, tx, p, items, st);
+    if (block == 16) return launch_cfg<256, 16, 6, 2, 3, 4, 4, true>(tw, ts, tx, p, items, st);
+    if (block == 32) return launch_cfg<256, 32, 6, 2, 2, 4, 4, true>(tw, ts, tx, p, items, st);
+    return launch_cfg<256, 64, 4, 1, 2, 4, 4, true>(tw, ts, tx, p, items, st);
 }

@@ -12,21 +12,27 @@
 // xor-shuffles.  Grid-stride loop, four 16-byte loads in flight per thread,
 // streaming (evict-first) loads and stores: the kernels are HBM-bound.
 //
-// Division-free exact rounding.  The codes must equal rint_half_even of the
-// IEEE fp32 quotient fl32(w / s).  With w and s both BF16 (8-bit significands)
-// the exact quotient y = w / s is either exactly a half-integer or at least
-// 1/510 away from every half-integer (write both as integer * 2^e; the
-// numerator of y - (j + 1/2) is a nonzero integer multiple of a power of two
-// that the denominator bounds), and fl32 never moves y across or onto a
-// half-integer.  The kernel forms t = w * r with r = rcp_rn(s) (relative error
-// < 2^-23, so |t - y| < 1e-6 for |y| <= 7.03), snaps t to the 2^-10 grid with
-// one fused multiply-add against 1.5 * 2^13, and then rounds the snapped
-// value to an integer, ties to even, by adding the constant that brings it to
-// 1.5 * 2^23.  Snapping maps exact ties onto the half-integer and keeps every
-// other quotient strictly on its own side, so the result equals
-// rint_half_even(y).  The code is then the low byte of the float's bits
-// (bits = 0x4B400000 + q).  Scales below 2^-126 (subnormal) take the plain
-// IEEE-division path.
+// Division-free exact arithmetic.
+//  * Scale: s32 = fl32(amax / 7) is formed by quotient refinement with one FMA
+//    residual step (Markstein): q0 = fl(a * c), r = fma(-q0, 7, a),
+//    s32 = fma(r, c, q0), c = fl32(1/7).  This equals the IEEE quotient for
+//    every finite BF16 amax (checked exhaustively on the host by
+//    tests/test_kernel_arith.py).
+//  * Codes: they must equal rint_half_even of the IEEE fp32 quotient
+//    fl32(w / s).  With w and s both BF16 (8-bit significands) the exact
+//    quotient y = w / s is either exactly a half-integer or at least 1/510 away
+//    from every half-integer (write both as integer * 2^e; the numerator of
+//    y - (j + 1/2) is a nonzero integer multiple of a power of two that the
+//    denominator bounds), and fl32 never moves y across or onto a
+//    half-integer.  The kernel forms t = w * r with r = rcp.approx(s) (relative
+//    error <= 2^-23, so |t - y| < 1e-6 for |y| <= 7.03), snaps t to the 2^-10
+//    grid with one fused multiply-add against 1.5 * 2^13, then rounds the
+//    snapped value to an integer, ties to even, by adding the constant that
+//    brings it to 1.5 * 2^23.  Snapping maps exact ties onto the half-integer
+//    and keeps every other quotient strictly on its own side, so the result
+//    equals rint_half_even(y).  The code is then the low byte of the float's
+//    bits (bits = 0x4B400000 + q).  Scales below 2^-126 (subnormal) take the
+//    plain IEEE-division path.
 #include <algorithm>
 
 #include "w4_common.cuh"
@@ -66,35 +72,43 @@ struct GroupScale {
     int mode;       // 0: s == 0, 1: normal s (fast path), 2: subnormal s
 };
 
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ GroupScale make_scale(uint32_t amax_bits) {
     GroupScale g;
     const float a = __uint_as_float(amax_bits << 16);
-    const float s32 = __fdiv_rn(a, 7.0f);
+    // fl32(a / 7) by one refinement step (exact for every BF16 a)
+    const float c = __uint_as_float(0x3E124925u);     // fl32(1/7)
+    const float q0 = __fmul_rn(a, c);
+    const float rr = __fmaf_rn(-q0, 7.0f, a);
+    const float s32 = __fmaf_rn(rr, c, q0);
     const __nv_bfloat16 sb = __float2bfloat16_rn(s32);
     g.bits = *reinterpret_cast<const uint16_t *>(&sb);
     g.s = __bfloat162float(sb);
     g.mode = (g.s == 0.0f) ? 0 : (g.s < 1.17549435e-38f ? 2 : 1);
-    g.r = (g.mode == 1) ? __frcp_rn(g.s) : 0.0f;
+    g.r = (g.mode == 1) ? rcp_approx(g.s) : 0.0f;
     return g;
 }
 
+// --- fast path: normal scale, straight-line, no per-element branches -------
 // c = 1.5 * 2^23 + q as an fp32 (so bits(c) = 0x4B400000 + q).
-__device__ __forceinline__ float code_float(float x, const GroupScale &g) {
-    if (g.mode == 1) return __fadd_rn(__fmaf_rn(x, g.r, kSnap), kToInt);
-    if (g.mode == 0) return kMagic;
-    const float q = (float)__float2int_rn(__fdiv_rn(x, g.s));  // IEEE path, tiny scales
-    return __fadd_rn(q, kMagic);
+__device__ __forceinline__ float code_fast(float x, float r) {
+    return __fadd_rn(__fmaf_rn(x, r, kSnap), kToInt);
 }
 
-__device__ __forceinline__ void codes8(const uint4 &v, const GroupScale &g, float (&c)[8]) {
-    c[0] = code_float(lo_f(v.x), g);
-    c[1] = code_float(hi_f(v.x), g);
-    c[2] = code_float(lo_f(v.y), g);
-    c[3] = code_float(hi_f(v.y), g);
-    c[4] = code_float(lo_f(v.z), g);
-    c[5] = code_float(hi_f(v.z), g);
-    c[6] = code_float(lo_f(v.w), g);
-    c[7] = code_float(hi_f(v.w), g);
+__device__ __forceinline__ void codes8_fast(const uint4 &v, float r, float (&c)[8]) {
+    c[0] = code_fast(lo_f(v.x), r);
+    c[1] = code_fast(hi_f(v.x), r);
+    c[2] = code_fast(lo_f(v.y), r);
+    c[3] = code_fast(hi_f(v.y), r);
+    c[4] = code_fast(lo_f(v.z), r);
+    c[5] = code_fast(hi_f(v.z), r);
+    c[6] = code_fast(lo_f(v.w), r);
+    c[7] = code_fast(hi_f(v.w), r);
 }
 
 // Eight codes (low bytes of the floats' bits) -> one low-nibble-first word.
@@ -111,17 +125,51 @@ __device__ __forceinline__ uint32_t pack8(const float (&c)[8]) {
     return (even & 0x0F0F0F0Fu) | ((odd << 4) & 0xF0F0F0F0u);
 }
 
-// Eight codes -> four BF16x2 words of bf16_rne(q * s).
-__device__ __forceinline__ uint4 dequant8(const float (&c)[8], float s) {
+// Eight codes -> four BF16x2 words of bf16_rne(q * s).  With
+// neg_cs = -(1.5 * 2^23) * s (exact: s has 8 significant bits and 3 * s has
+// at most 10, as long as s <= 2^100), fma(c, s, neg_cs) = (c - 1.5 * 2^23) * s
+// = q * s exactly, rounded once to BF16 by the conversion; q == 0 gives +0.
+__device__ __forceinline__ uint4 dequant8_fast(const float (&c)[8], float s, float neg_cs) {
     uint32_t o[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        const float v0 = __fmul_rn(__fsub_rn(c[2 * j], kMagic), s);       // exact
-        const float v1 = __fmul_rn(__fsub_rn(c[2 * j + 1], kMagic), s);
+        const float v0 = __fmaf_rn(c[2 * j], s, neg_cs);
+        const float v1 = __fmaf_rn(c[2 * j + 1], s, neg_cs);
         __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
         o[j] = *reinterpret_cast<uint32_t *>(&h);
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// --- slow path: zero, subnormal or huge scale; codes by IEEE division -------
+// Handles one whole 8-element item and writes its outputs (kept out of line so
+// that the fast path's registers are unaffected).
+template <int MODE>
+__device__ __forceinline__ void item_slow(uint4 v, float s, uint32_t *Wq, uint4 *Wdq, int64_t i) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float c[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float xs[2] = {lo_f(w[j]), hi_f(w[j])};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const float q = (s == 0.0f) ? 0.0f : (float)__float2int_rn(__fdiv_rn(xs[h], s));
+            c[2 * j + h] = __fadd_rn(q, kMagic);
+        }
+    }
+    if (MODE == 0) {
+        Wq[i] = pack8(c);
+    } else {
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float v0 = __fmul_rn(__fsub_rn(c[2 * j], kMagic), s);       // exact
+            const float v1 = __fmul_rn(__fsub_rn(c[2 * j + 1], kMagic), s);
+            __nv_bfloat162 hh = __floats2bfloat162_rn(v0, v1);
+            o[j] = *reinterpret_cast<uint32_t *>(&hh);
+        }
+        Wdq[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
 }
 
 constexpr int kUnroll = 4;
@@ -129,7 +177,7 @@ constexpr int kThreads = 256;
 
 // MODE 0: quantize + pack (Wq, S).  MODE 1: fake quant (Wdq, optional S).
 template <int MODE>
-__global__ void __launch_bounds__(kThreads) quant_kernel(const uint4 *__restrict__ W,
+__global__ void __launch_bounds__(kThreads, 4) quant_kernel(const uint4 *__restrict__ W,
                                                          uint4 *__restrict__ Wdq,
                                                          uint32_t *__restrict__ Wq,
                                                          uint16_t *__restrict__ S, int64_t n8) {
@@ -150,25 +198,45 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const uint4 *__restrict
         for (int u = 0; u < kUnroll; ++u) {
             const int64_t i = base + lane + u * T;
             const GroupScale g = make_scale(group_amax_bits(v[u]));
+            // the fast path needs a normal scale (and, for the BF16 output, no
+            // overflow of 1.5 * 2^23 * s); all lanes take the same branch
+            const bool fast = g.mode == 1 && (MODE == 0 || g.s <= 1.2676506e30f);
             if (i < n8) {
-                float c[8];
-                codes8(v[u], g, c);
-                if (MODE == 0) {
-                    __stcs(reinterpret_cast<unsigned int *>(Wq + i), pack8(c));
+                if (fast) {
+                    float c[8];
+                    codes8_fast(v[u], g.r, c);
+                    if (MODE == 0) {
+                        __stcs(reinterpret_cast<unsigned int *>(Wq + i), pack8(c));
+                    } else {
+                        __stcs(Wdq + i, dequant8_fast(c, g.s, -kMagic * g.s));
+                    }
                 } else {
-                    __stcs(Wdq + i, dequant8(c, g.s));
+                    item_slow<MODE>(v[u], g.s, Wq, Wdq, i);
                 }
-                if (S != nullptr && (lane & 3) == 0) S[i >> 2] = g.bits;
             }
+            if (i < n8 && S != nullptr && (lane & 3) == 0) S[i >> 2] = g.bits;
         }
     }
 }
 
-__global__ void __launch_bounds__(kThreads) copy16_kernel(const uint4 *__restrict__ src,
-                                                          uint4 *__restrict__ dst, int64_t n16) {
+__global__ void __launch_bounds__(kThreads, 4) copy16_kernel(const uint4 *__restrict__ src,
+                                                             uint4 *__restrict__ dst,
+                                                             int64_t n16) {
     const int64_t T = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += T)
-        __stcs(dst + i, __ldcs(src + i));
+    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < n16;
+         base += kUnroll * T) {
+        uint4 v[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t i = base + u * T;
+            if (i < n16) v[u] = __ldcs(src + i);
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t i = base + u * T;
+            if (i < n16) __stcs(dst + i, v[u]);
+        }
+    }
 }
 
 __global__ void copy2_tail_kernel(const uint16_t *__restrict__ src, uint16_t *__restrict__ dst,
@@ -251,7 +319,7 @@ extern "C" w4_status w4_ste_backward(const w4_bf16 *dWdq, w4_bf16 *dW, int64_t n
     if (a < b + n && b < a + n) return W4_ERR_INVALID_ARG;  // partial overlap
     const int64_t n16 = n / 8;
     if (n16 > 0)
-        copy16_kernel<<<grid_for(n16, 1), kThreads, 0, (cudaStream_t)stream>>>(
+        copy16_kernel<<<grid_for(n16, kUnroll), kThreads, 0, (cudaStream_t)stream>>>(
             reinterpret_cast<const uint4 *>(a), reinterpret_cast<uint4 *>(b), n16);
     if (n16 * 8 < n)
         copy2_tail_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(a, b, n16 * 8, n);

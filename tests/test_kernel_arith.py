@@ -1,0 +1,61 @@
+"""Host-side checks of the arithmetic the quantizer kernels use in place of
+divisions (no GPU).  The fp32 fused operations are emulated exactly: every
+product and sum below is exact in float64 for these operand sizes, and one
+cast to float32 is the single rounding of the fused operation.
+
+1. s32 = fl32(amax / 7) is formed as q0 = fl(a * c), r = fma(-q0, 7, a),
+   q = fma(r, c, q0) with c = fl32(1/7) (quotient refinement with one FMA
+   residual step, Markstein's method).  Checked for every finite BF16 amax.
+2. The code rint_half_even(fl32(w / s)) is formed as
+   fl(fl(fma(w, r, 1.5*2^13)) + (1.5*2^23 - 1.5*2^13)) with r an approximate
+   reciprocal of s (relative error up to 2^-21 allowed): the FMA snaps w*r to
+   the 2^-10 grid, which lands exact ties on the half-integer and leaves every
+   other BF16/BF16 quotient (at least 1/510 from any half-integer) on its side;
+   the add then rounds to an integer, ties to even.  Checked on every BF16
+   magnitude below 128 group maxima, with the reciprocal perturbed both ways.
+"""
+import numpy as np
+import pytest
+
+import oracle
+
+F32 = np.float32
+SNAP = 12288.0                 # 1.5 * 2^13
+TOINT = 12582912.0 - 12288.0   # 1.5 * 2^23 - 1.5 * 2^13
+MAGIC = 12582912.0             # 1.5 * 2^23
+
+
+def _f32(x):
+    return np.asarray(x, dtype=np.float64).astype(np.float32)
+
+
+def test_div7_refinement_exact_for_all_bf16():
+    b = np.arange(0, 0x7F80, dtype=np.uint32)
+    a = (b << 16).view(np.float32)
+    ref = a / F32(7.0)
+    c = float(F32(1.0) / F32(7.0))
+    q0 = _f32(a.astype(np.float64) * c)
+    r = _f32(a.astype(np.float64) - q0.astype(np.float64) * 7.0)
+    q = _f32(r.astype(np.float64) * c + q0.astype(np.float64))
+    assert np.array_equal(q.view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("rel", [0.0, 2.0 ** -21, -(2.0 ** -21)])
+def test_snap_rounding_matches_ieee_quotient(rel):
+    all_bits = np.arange(0, 0x7F80, dtype=np.uint32)
+    mags = (all_bits << 16).view(np.float32)
+    for mant in range(0, 128, 3):
+        amax = float(((np.uint32(0x4080 + mant)) << 16).view(np.float32))   # [4, 8)
+        s_bits = oracle.bf16_from_f32_scalar(float(F32(amax) / F32(7.0)))
+        s = float((np.uint32(s_bits) << 16).view(np.float32))
+        w = mags[(mags <= amax)].astype(np.float64)
+        w = np.concatenate([w, -w])
+        ref = np.clip(np.rint((w.astype(np.float32) / F32(s)).astype(np.float64)), -8, 7)
+        r = float(F32(1.0 / s)) * (1.0 + rel)
+        a = _f32(w * r + SNAP)                       # fma(w, r, SNAP)
+        c = _f32(a.astype(np.float64) + TOINT)       # fadd
+        q = c.astype(np.float64) - MAGIC
+        assert np.array_equal(q, ref), mant
+        # the code is the low byte of the float's bits
+        low = (c.view(np.uint32) & 0xFF).astype(np.uint8).view(np.int8)
+        assert np.array_equal(low.astype(np.float64), ref)
