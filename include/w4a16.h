@@ -37,7 +37,8 @@
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Every call validates its arguments on the host, then only
  *     enqueues kernels on `stream` and returns; it never synchronizes, never
- *     allocates device memory and keeps no pointer after it returns.
+ *     allocates device memory and keeps no pointer after it returns.  Scratch
+ *     memory, where a schedule uses some, is passed in by the caller.
  *   - group must be 32 (else W4_ERR_UNSUPPORTED); K must be a positive
  *     multiple of 32.
  *   - A kernel launch failure returns W4_ERR_CUDA (w4_last_cuda_error() gives
@@ -122,11 +123,22 @@ w4_status w4_dequant(const int32_t *Wq, const w4_bf16 *S, w4_bf16 *Wdq,
  * unpacking"; the product runs on BF16 tensor cores with FP32 accumulation.
  *   X   in   [M, K] BF16        Wq  in  [N, K/8] int32   S  in  [N, K/32] BF16
  *   Y   out  [M, N] BF16, Y = X . dq(Wq, S)^T
+ *   workspace, workspace_bytes: optional device scratch (256-byte aligned) for
+ *        the decode-shaped split (M <= 64, K % 256 == 0, few 128-row tiles
+ *        per SM).  NULL, or fewer bytes than w4a16_gemm_workspace_bytes(M, N, K)
+ *        reports, selects the unsplit schedule instead (same results).  The
+ *        workspace must be all zero before its first use; every call leaves
+ *        its counters at zero again.  Calls that may overlap on the GPU must
+ *        not share a workspace.  After W4_ERR_TIMEOUT, zero it again.
  * Any M >= 1, N >= 1.  Y may not alias an input.
  */
 w4_status w4a16_gemm(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S,
                      w4_bf16 *Y, int64_t M, int64_t N, int64_t K, int group,
-                     void *stream);
+                     void *workspace, size_t workspace_bytes, void *stream);
+
+/* Bytes of workspace the split schedule of w4a16_gemm uses for this shape on
+ * the current device (0 when that schedule does not apply).  Host-only. */
+size_t w4a16_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* Padded capacity the caller must provide for w4_moe_align's sorted_ids:
  * T*topk + E*(block-1), rounded up to a multiple of block.  Host-only. */

@@ -24,7 +24,8 @@ import os
 import torch
 
 __all__ = [
-    "W4Error", "lib", "w4_version", "w4_device_status", "w4_fake_quant", "w4_ste_backward",
+    "W4Error", "lib", "workspace", "w4a16_gemm_workspace_bytes", "w4_version",
+    "w4_device_status", "w4_fake_quant", "w4_ste_backward",
     "w4_quantize_pack", "w4_dequant", "w4a16_gemm", "w4_moe_capacity", "w4_moe_align",
     "w4_moe_w4a16_gemm", "fake_quant", "quantize_pack", "dequant", "gemm", "moe_align",
     "moe_gemm", "FakeInt4STE", "GROUP",
@@ -67,7 +68,7 @@ def lib() -> ctypes.CDLL:
             "w4_ste_backward": [_P, _P, _I64, _P],
             "w4_quantize_pack": [_P, _P, _P, _I64, _I64, _INT, _P],
             "w4_dequant": [_P, _P, _P, _I64, _I64, _INT, _P],
-            "w4a16_gemm": [_P, _P, _P, _P, _I64, _I64, _I64, _INT, _P],
+            "w4a16_gemm": [_P, _P, _P, _P, _I64, _I64, _I64, _INT, _P, ctypes.c_size_t, _P],
             "w4_moe_align": [_P, _I64, _INT, _INT, _INT, _P, _I64, _P, _P, _P],
             "w4_moe_w4a16_gemm": [_P, _INT, _P, _P, _P, _P, _P, _I64, _INT, _I64, _P, _I64,
                                   _I64, _INT, _P],
@@ -76,6 +77,8 @@ def lib() -> ctypes.CDLL:
             f = getattr(L, name)
             f.argtypes = args
             f.restype = ctypes.c_int
+        L.w4a16_gemm_workspace_bytes.argtypes = [_I64, _I64, _I64]
+        L.w4a16_gemm_workspace_bytes.restype = ctypes.c_size_t
         L.w4_moe_capacity.argtypes = [_I64, _INT, _INT, _INT]
         L.w4_moe_capacity.restype = ctypes.c_int64
         L.w4_version.restype = ctypes.c_int
@@ -156,15 +159,39 @@ def w4_dequant(Wq, S, Wdq, group: int = GROUP, stream=None) -> None:
                                           _stream(stream)))
 
 
-def w4a16_gemm(X, Wq, S, Y, group: int = GROUP, stream=None) -> None:
+_WORKSPACE = {}
+
+
+def workspace(device, nbytes: int) -> torch.Tensor:
+    """A zeroed per-device scratch buffer of at least nbytes for the split GEMM
+    schedule (the kernels leave it zeroed after every call)."""
+    idx = torch.device(device).index
+    t = _WORKSPACE.get(idx)
+    if t is None or t.numel() < nbytes:
+        t = torch.zeros(max(int(nbytes), 1 << 20), dtype=torch.uint8, device=device)
+        _WORKSPACE[idx] = t
+    return t
+
+
+def w4a16_gemm_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().w4a16_gemm_workspace_bytes(M, N, K))
+
+
+def w4a16_gemm(X, Wq, S, Y, group: int = GROUP, ws="auto", stream=None) -> None:
+    """ws: "auto" (the module's zeroed per-device buffer), None (unsplit
+    schedule), or a zeroed uint8 CUDA tensor."""
     _dtype(X, torch.bfloat16, "X")
     _dtype(Wq, torch.int32, "Wq")
     M, K = X.shape
     N = Wq.shape[0]
     if Wq.shape[1] * 8 != K or tuple(Y.shape) != (M, N):
         raise ValueError("shape mismatch")
+    if isinstance(ws, str):
+        need = w4a16_gemm_workspace_bytes(M, N, K)
+        ws = workspace(X.device, need) if need > 0 else None
+    wptr, wbytes = (_ptr(ws), ws.numel() * ws.element_size()) if ws is not None else (None, 0)
     _check("w4a16_gemm", lib().w4a16_gemm(_ptr(X), _ptr(Wq), _ptr(S), _ptr(Y), M, N, K, group,
-                                          _stream(stream)))
+                                          wptr, wbytes, _stream(stream)))
 
 
 def w4_moe_capacity(T: int, topk: int, E: int, block: int) -> int:
@@ -217,9 +244,9 @@ def dequant(Wq: torch.Tensor, S: torch.Tensor) -> torch.Tensor:
     return Wdq
 
 
-def gemm(X: torch.Tensor, Wq: torch.Tensor, S: torch.Tensor) -> torch.Tensor:
+def gemm(X: torch.Tensor, Wq: torch.Tensor, S: torch.Tensor, ws="auto") -> torch.Tensor:
     Y = torch.empty((X.shape[0], Wq.shape[0]), dtype=torch.bfloat16, device=X.device)
-    w4a16_gemm(X, Wq, S, Y)
+    w4a16_gemm(X, Wq, S, Y, ws=ws)
     return Y
 
 

@@ -70,14 +70,19 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
         : "memory");
 }
 
+// try_wait with a suspend-time hint: a thread whose phase has not completed
+// is suspended (it stops competing for issue slots) until the phase completes
+// or the hint elapses, whichever comes first.
+constexpr uint32_t kSuspendHintNs = 1000000u;   // 1 ms
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     return ok != 0;
 }
@@ -89,15 +94,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile int *abort_flag) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
+    for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 0u) {
-            if (*abort_flag) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                record_timeout();
-                *abort_flag = 1;
-                return false;
-            }
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            record_timeout();
+            *abort_flag = 1;
+            return false;
         }
     }
 }
@@ -296,6 +299,38 @@ __device__ __forceinline__ void dequant_word(uint32_t w, uint32_t s2, uint32_t (
         v = __hmul2(v, sc);
         out[j] = *reinterpret_cast<uint32_t *>(&v);
     }
+}
+
+// Same unpack without the pairing permutes: out[j] = (q_j * s, q_{j+4} * s).
+// Used with activations whose 8-element chunks are stored in the matching order
+// [x0, x4, x1, x5, x2, x6, x3, x7] (see permute_chunk8), which leaves the
+// product unchanged because the K sum does not depend on the order of its terms.
+__device__ __forceinline__ void dequant_word_k8perm(uint32_t w, uint32_t s2, uint32_t (&out)[4]) {
+    const uint32_t m = 0x000F000Fu, x = 0x43084308u;
+    uint32_t in[4];
+    in[0] = lop3_and_xor(w, m, x);          // codes 0, 4
+    in[1] = lop3_and_xor(w >> 4, m, x);     // codes 1, 5
+    in[2] = lop3_and_xor(w >> 8, m, x);     // codes 2, 6
+    in[3] = lop3_and_xor(w >> 12, m, x);    // codes 3, 7
+    const __nv_bfloat162 bias = __floats2bfloat162_rn(136.0f, 136.0f);
+    const __nv_bfloat162 sc = *reinterpret_cast<const __nv_bfloat162 *>(&s2);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162 *>(&in[j]);
+        v = __hsub2(v, bias);
+        v = __hmul2(v, sc);
+        out[j] = *reinterpret_cast<uint32_t *>(&v);
+    }
+}
+
+// 8 BF16 values [x0..x7] (16 bytes) -> [x0, x4, x1, x5, x2, x6, x3, x7].
+__device__ __forceinline__ uint4 permute_chunk8(uint4 v) {
+    uint4 o;
+    o.x = __byte_perm(v.x, v.z, 0x5410);
+    o.y = __byte_perm(v.x, v.z, 0x7632);
+    o.z = __byte_perm(v.y, v.w, 0x5410);
+    o.w = __byte_perm(v.y, v.w, 0x7632);
+    return o;
 }
 
 __device__ __forceinline__ uint32_t bf16x2_splat(uint16_t s) {

@@ -39,9 +39,13 @@
 namespace w4 {
 namespace {
 
-// Warp roles: 0 = loads, 1 = TMEM allocation + MMA issue, then 4 * NDQ
-// dequant warps (NDQ per TMEM lane quarter), then 4 epilogue warps.
-__host__ __device__ constexpr int gemm_threads(int ndq) { return 32 * (2 + 4 * ndq + 4); }
+// Warp roles: warp 0 = loads (and TMEM allocation), then 4 * NDQ dequant warps
+// (NDQ per TMEM lane quarter), then 4 MMA + epilogue warps: lane 0 of the
+// first NMMA of them issues MMAs (each into its own accumulator, every NMMA-th
+// 16-wide K step), and all four drain the accumulators of their lane quarter.
+// A single thread issues at most about one small tcgen05.mma per ~120 cycles,
+// so small-N tiles need several issuers to keep up with HBM.
+__host__ __device__ constexpr int gemm_threads(int ndq) { return 32 * (1 + 4 * ndq + 4); }
 constexpr int kTmemCols = 512;
 
 struct GemmParams {
@@ -60,7 +64,61 @@ struct GemmParams {
     int n_row_tiles;
     int n_tok_tiles;             // dense
     int num_kb;
+    // stream-K split of the (row tile, k-block) units of a one-token-tile GEMM
+    int split;                   // 0: whole-K work items; 1: split units
+    int64_t units;               // n_row_tiles * num_kb
+    int ctas;                    // grid size the split was planned for
+    int max_contrib;             // most CTAs sharing one row tile
+    float *ws_part;              // [n_row_tiles][max_contrib][128][MT] partial sums
+    unsigned int *ws_cnt;        // [n_row_tiles][4] arrival counters (zero between calls)
 };
+
+// Work items: (row tile rt, token tile tt, k-blocks [kb0, kb1)).  Dense and MoE
+// kernels walk whole-K items blockIdx.x, blockIdx.x + gridDim.x, ...; a split
+// kernel walks the CTA's contiguous range of (row tile, k-block) units, cut at
+// row-tile boundaries.
+struct ItemIter {
+    int64_t cur, end;
+    int step;
+};
+
+__device__ __forceinline__ ItemIter make_iter(const GemmParams &p, int num_items) {
+    ItemIter I;
+    if (p.split) {
+        I.cur = (int64_t)blockIdx.x * p.units / p.ctas;
+        I.end = ((int64_t)blockIdx.x + 1) * p.units / p.ctas;
+        I.step = 0;
+    } else {
+        I.cur = blockIdx.x;
+        I.end = num_items;
+        I.step = gridDim.x;
+    }
+    return I;
+}
+
+__device__ __forceinline__ bool next_item(ItemIter &I, const GemmParams &p, int &rt, int &tt,
+                                          int &kb0, int &kb1) {
+    if (I.cur >= I.end) return false;
+    if (p.split) {
+        rt = (int)(I.cur / p.num_kb);
+        kb0 = (int)(I.cur % p.num_kb);
+        kb1 = (int)((I.end - I.cur) < (int64_t)(p.num_kb - kb0) ? kb0 + (I.end - I.cur) : p.num_kb);
+        tt = 0;
+        I.cur += kb1 - kb0;
+    } else {
+        rt = (int)(I.cur % p.n_row_tiles);
+        tt = (int)(I.cur / p.n_row_tiles);
+        kb0 = 0;
+        kb1 = p.num_kb;
+        I.cur += I.step;
+    }
+    return true;
+}
+
+// CTA that owns split unit x (CTA c owns [c*U/P, (c+1)*U/P)).
+__device__ __forceinline__ int unit_owner(int64_t x, const GemmParams &p) {
+    return (int)(((x + 1) * p.ctas - 1) / p.units);
+}
 
 // Shared-memory layout, all offsets from a 1024-aligned base.
 template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT>
@@ -101,6 +159,12 @@ __device__ __forceinline__ uint2 lds64(uint32_t addr) {
     return v;
 }
 
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
 __device__ __forceinline__ uint32_t swz(uint32_t off, uint32_t sw_bytes) {
     // TMA / UMMA swizzle: 16-byte chunk index XOR address bits [7, ...).
     return off ^ (((off >> 7) & (sw_bytes / 16 - 1)) << 4);
@@ -123,9 +187,9 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
     }
 }
 
-// NSPLIT: independent accumulators per work item; consecutive 16-wide K steps
-// of the MMA go round-robin to them, so small-N MMAs do not wait on each
-// other, and the epilogue adds them in a fixed order.
+// NSPLIT: MMA issuers = accumulators per work item; 16-wide K step u goes to
+// issuer / accumulator u % NSPLIT, and the epilogue adds the accumulators in
+// a fixed order.
 template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT, int NDQ, bool MOE>
 __global__ void __launch_bounds__(gemm_threads(NDQ), 1)
     w4a16_tc_kernel(const __grid_constant__ CUtensorMap tm_w,
@@ -137,7 +201,11 @@ __global__ void __launch_bounds__(gemm_threads(NDQ), 1)
     constexpr int kAccCols = NSPLIT * MT;      // TMEM columns per work item accumulator
     constexpr int kABase = NACC * kAccCols;    // first A column
     constexpr int kDqWarps = 4 * NDQ;
-    constexpr int kEpiWarp0 = 2 + kDqWarps;
+    constexpr int kEpiWarp0 = 1 + kDqWarps;
+    static_assert(NSPLIT >= 1 && NSPLIT <= 4, "one to four MMA issuers");
+    // 256-wide k-blocks (decode / MoE, few activation rows per tile): reorder the
+    // activation chunks in shared memory instead of pairing the unpacked codes.
+    constexpr bool kXPerm = (KB == 256);
     static_assert((KB / 32) % NDQ == 0, "k-block chunks split evenly over the dequant warps");
     constexpr uint32_t kIdesc = idesc_bf16_f32(128, MT);
 
@@ -170,24 +238,24 @@ __global__ void __launch_bounds__(gemm_threads(NDQ), 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < NSTAGE; ++s) {
             mbar_init(full_bar(s), MOE ? 33u : 1u);
-            mbar_init(empty_bar(s), 1u);
+            mbar_init(empty_bar(s), (uint32_t)NSPLIT);
         }
         for (int a = 0; a < NASTAGE; ++a) {
             mbar_init(afull_bar(a), 32u * kDqWarps);
-            mbar_init(aempty_bar(a), 1u);
+            mbar_init(aempty_bar(a), (uint32_t)NSPLIT);
         }
         for (int d = 0; d < NACC; ++d) {
-            mbar_init(accfull_bar(d), 1u);
+            mbar_init(accfull_bar(d), (uint32_t)NSPLIT);
             mbar_init(accempty_bar(d), 128u);
         }
-        mbar_init(mmadone_bar, 1u);
+        mbar_init(mmadone_bar, (uint32_t)NSPLIT);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tm_w);
         if (KB == 256) tma_prefetch_desc(&tm_s);
         if (!MOE) tma_prefetch_desc(&tm_x);
     }
-    if (warp == 1) {
+    if (warp == 0) {
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
         tmem_relinquish();
     }
@@ -211,13 +279,31 @@ __global__ void __launch_bounds__(gemm_threads(NDQ), 1)
         // ------------------------------------------------------------ loads
         uint32_t it = 0;
         bool ok = true;
-        for (int item = blockIdx.x; item < num_items && ok; item += gridDim.x) {
-            const int rt = item % p.n_row_tiles;
-            const int tt = item / p.n_row_tiles;
+        ItemIter I = make_iter(p, num_items);
+        int rt, tt, kb0, kb1;
+        while (ok && next_item(I, p, rt, tt, kb0, kb1)) {
             const int row0 = rt * R;
             int expert = 0;
-            if (MOE) expert = __ldg(p.expert_ids + tt);
-            for (int kb = 0; kb < num_kb; ++kb, ++it) {
+            // MoE: activation row of each of the block's MT slots (-1 for padding),
+            // lane t % 32 of register t / 32, loaded once per work item
+            int gather_row[(MT + 31) / 32];
+            if (MOE) {
+                expert = __ldg(p.expert_ids + tt);
+#pragma unroll
+                for (int r = 0; r < (MT + 31) / 32; ++r) {
+                    const int t = r * 32 + lane;
+                    int row = -1;
+                    if (t < MT) {
+                        const int slot = __ldg(p.sorted_ids + (int64_t)tt * MT + t);
+                        if (slot >= 0 && slot < p.num_slots) {
+                            row = slot / p.a_row_div;
+                            if (row >= p.a_rows) row = -1;
+                        }
+                    }
+                    gather_row[r] = row;
+                }
+            }
+            for (int kb = kb0; kb < kb1; ++kb, ++it) {
                 const int s = it % NSTAGE;
                 if (!warp_wait(empty_bar(s), ((it / NSTAGE) & 1u) ^ 1u, abort_flag)) {
                     ok = false;
@@ -242,15 +328,15 @@ __global__ void __launch_bounds__(gemm_threads(NDQ), 1)
                     }
                 }
                 if (MOE) {
-                    // Gather the block's activation rows: lane = 16-byte chunk along K.
+                    // Gather the block's activation rows: lane = 16-byte chunk along K;
+                    // the rows come from the per-item table in registers.
                     const int c = lane;                   // KB == 256: 32 chunks per row
                     const int64_t k = (int64_t)kb * KB + c * 8;
+#pragma unroll
                     for (int t = 0; t < MT; ++t) {
-                        const int slot = __ldg(p.sorted_ids + (int64_t)tt * MT + t);
-                        const int64_t row =
-                            (slot >= 0 && slot < p.num_slots) ? slot / p.a_row_div : -1;
-                        const bool in = row >= 0 && row < p.a_rows && k < p.K;
-                        const uint16_t *src = in ? p.A + row * p.K + k : p.A;
+                        const int row = __shfl_sync(0xFFFFFFFFu, gather_row[t >> 5], t & 31);
+                        const bool in = row >= 0 && k < p.K;
+                        const uint16_t *src = in ? p.A + (int64_t)row * p.K + k : p.A;
                         const uint32_t dst = x_stage(s) + (c >> 3) * L::kXSub + t * 128 +
                                              ((((uint32_t)c & 7u) ^ ((uint32_t)t & 7u)) << 4);
                         cp_async_16(dst, src, in ? 16u : 0u);
@@ -264,47 +350,6 @@ __global__ void __launch_bounds__(gemm_threads(NDQ), 1)
             const uint32_t first = it > (uint32_t)NSTAGE ? it - NSTAGE : 0u;
             for (uint32_t j = first; j < it; ++j) drain_wait(full_bar(j % NSTAGE), (j / NSTAGE) & 1u);
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------- MMA
-        if (lane == 0) {
-            uint32_t it = 0, acc_it = 0;
-            bool ok = true;
-            for (int item = blockIdx.x; item < num_items && ok; item += gridDim.x, ++acc_it) {
-                const int d = acc_it % NACC;
-                if (!mbar_wait(accempty_bar(d), ((acc_it / NACC) & 1u) ^ 1u, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after_sync();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(d * kAccCols);
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
-                    const int s = it % NSTAGE;
-                    const int a = it % NASTAGE;
-                    if (!mbar_wait(full_bar(s), (it / NSTAGE) & 1u, abort_flag) ||
-                        !mbar_wait(afull_bar(a), (it / NASTAGE) & 1u, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after_sync();
-                    if (MOE) fence_proxy_async_smem();   // cp.async (generic proxy) -> MMA
-                    const uint32_t a_tmem = tmem_base + (uint32_t)(kABase + a * kAStageCols);
-#pragma unroll
-                    for (int u = 0; u < KB / 16; ++u) {
-                        const uint32_t baddr = x_stage(s) + (u >> 2) * L::kXSub + (u & 3) * 32;
-                        tc_mma_ts(d_tmem + (uint32_t)((u % NSPLIT) * MT), a_tmem + u * 8,
-                                  smem_desc_k_sw128(baddr), kIdesc,
-                                  (kb > 0 || u >= NSPLIT) ? 1u : 0u);
-                    }
-                    tc_commit(empty_bar(s));
-                    tc_commit(aempty_bar(a));
-                }
-                if (!ok) break;
-                tc_commit(accfull_bar(d));
-            }
-            // All MMAs issued by this thread complete before TMEM is released.
-            tc_commit(mmadone_bar);
-            drain_wait(mmadone_bar, 0u);
-        }
     } else if (warp < kEpiWarp0) {
         // --------------------------------------------------------- dequant
         // NDQ warps per TMEM lane quarter; warp part h takes chunks
@@ -313,15 +358,15 @@ __global__ void __launch_bounds__(gemm_threads(NDQ), 1)
         constexpr int G = KB / 32;
         constexpr int GH = G / NDQ;
         const int q4 = warp & 3;                    // TMEM lane quarter of this warp
-        const int half = (warp - 2) >> 2;           // part index in [0, NDQ)
+        const int half = (warp - 1) >> 2;           // part index in [0, NDQ)
         const int lrow = q4 * 32 + lane;            // A row of this thread
         const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
         const int64_t gpr = p.K / 32;               // groups per row
         uint32_t it = 0;
         bool ok = true;
-        for (int item = blockIdx.x; item < num_items && ok; item += gridDim.x) {
-            const int rt = item % p.n_row_tiles;
-            const int tt = item / p.n_row_tiles;
+        ItemIter I = make_iter(p, num_items);
+        int rt, tt, kb0, kb1;
+        while (ok && next_item(I, p, rt, tt, kb0, kb1)) {
             const int64_t row = (int64_t)rt * R + lrow;
             const bool valid = lrow < R && row < p.N;
             const uint16_t *srow = nullptr;
@@ -330,7 +375,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ), 1)
                 if (MOE) base += (int64_t)__ldg(p.expert_ids + tt) * p.N * gpr;
                 srow = p.S + base;
             }
-            for (int kb = 0; kb < num_kb; ++kb, ++it) {
+            for (int kb = kb0; kb < kb1; ++kb, ++it) {
                 const int s = it % NSTAGE;
                 const int a = it % NASTAGE;
                 uint32_t sc[GH];
@@ -349,6 +394,19 @@ __global__ void __launch_bounds__(gemm_threads(NDQ), 1)
                     break;
                 }
                 tc_fence_after_sync();
+                if (kXPerm) {
+                    // reorder this thread's share of the stage's activation chunks
+                    // to match the A columns of dequant_word_k8perm
+                    const int dq_tid = (warp - 1) * 32 + lane;
+#pragma unroll 1
+                    for (int ci = dq_tid; ci < MT * 32; ci += 32 * kDqWarps) {
+                        const int t = ci >> 5, c = ci & 31;
+                        const uint32_t addr = x_stage(s) + (c >> 3) * L::kXSub + t * 128 +
+                                              ((((uint32_t)c & 7u) ^ ((uint32_t)t & 7u)) << 4);
+                        sts128(addr, permute_chunk8(lds128(addr)));
+                    }
+                    fence_proxy_async_smem();   // generic writes -> tensor-core reads
+                }
                 // all shared-memory reads of this k-block first
                 uint4 wv[GH];
 #pragma unroll
@@ -379,10 +437,17 @@ __global__ void __launch_bounds__(gemm_threads(NDQ), 1)
                 for (int j = 0; j < GH; ++j) {
                     const uint32_t ws[4] = {wv[j].x, wv[j].y, wv[j].z, wv[j].w};
                     uint32_t lo[8], hi[8];
-                    dequant_word(ws[0], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&lo[0]));
-                    dequant_word(ws[1], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&lo[4]));
-                    dequant_word(ws[2], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&hi[0]));
-                    dequant_word(ws[3], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&hi[4]));
+                    if (kXPerm) {
+                        dequant_word_k8perm(ws[0], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&lo[0]));
+                        dequant_word_k8perm(ws[1], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&lo[4]));
+                        dequant_word_k8perm(ws[2], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&hi[0]));
+                        dequant_word_k8perm(ws[3], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&hi[4]));
+                    } else {
+                        dequant_word(ws[0], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&lo[0]));
+                        dequant_word(ws[1], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&lo[4]));
+                        dequant_word(ws[2], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&hi[0]));
+                        dequant_word(ws[3], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&hi[4]));
+                    }
                     // columns: 2 BF16 per 32-bit column, ascending k
                     const uint32_t col = a_col + (uint32_t)((half * GH + j) * 16);
                     tmem_st_x8(col, lo);
@@ -394,19 +459,70 @@ __global__ void __launch_bounds__(gemm_threads(NDQ), 1)
             }
         }
     } else {
-        // -------------------------------------------------------- epilogue
+        // ------------------------------------------------- MMA + epilogue
+        const int j = warp - kEpiWarp0;             // 0..3
+        const bool issuer = j < NSPLIT;             // warp-uniform
         const int q4 = warp & 3;
         const int lrow = q4 * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
-        uint32_t acc_it = 0;
-        for (int item = blockIdx.x; item < num_items; item += gridDim.x, ++acc_it) {
-            const int rt = item % p.n_row_tiles;
-            const int tt = item / p.n_row_tiles;
+        uint32_t it = 0, acc_it = 0;
+        bool ok = true;
+        ItemIter I = make_iter(p, num_items);
+        int rt, tt, kb0, kb1;
+        for (; ok && next_item(I, p, rt, tt, kb0, kb1); ++acc_it) {
             const int d = acc_it % NACC;
+            if (issuer) {
+                if (!warp_wait(accempty_bar(d), ((acc_it / NACC) & 1u) ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(d * kAccCols + j * MT);
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                    const int s = it % NSTAGE;
+                    const int a = it % NASTAGE;
+                    if (!warp_wait(full_bar(s), (it / NSTAGE) & 1u, abort_flag) ||
+                        !warp_wait(afull_bar(a), (it / NASTAGE) & 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    if (lane == 0) {
+                        if (MOE) fence_proxy_async_smem();   // cp.async (generic proxy) -> MMA
+                        const uint32_t a_tmem =
+                            tmem_base + (uint32_t)(kABase + a * kAStageCols);
+#pragma unroll
+                        for (int u = j; u < KB / 16; u += NSPLIT) {
+                            const uint32_t baddr =
+                                x_stage(s) + (u >> 2) * L::kXSub + (u & 3) * 32;
+                            tc_mma_ts(d_tmem, a_tmem + u * 8, smem_desc_k_sw128(baddr), kIdesc,
+                                      (kb > kb0 || u >= NSPLIT) ? 1u : 0u);
+                        }
+                        tc_commit(empty_bar(s));
+                        tc_commit(aempty_bar(a));
+                    }
+                    __syncwarp();
+                }
+                if (!ok) break;
+                if (lane == 0) tc_commit(accfull_bar(d));
+                __syncwarp();
+            }
+            // epilogue of this lane quarter: sum the NSPLIT accumulators in order
             if (!warp_wait(accfull_bar(d), (acc_it / NACC) & 1u, abort_flag)) break;
             tc_fence_after_sync();
             const int64_t row = (int64_t)rt * R + lrow;
             const bool valid = lrow < R && row < p.N;
+            // split item: this CTA holds only part of the row tile's K range
+            const bool partial = p.split && !(kb0 == 0 && kb1 == p.num_kb);
+            int contrib = 1, my_idx = 0;
+            float *my_part = nullptr;
+            if (partial) {
+                const int c_first = unit_owner((int64_t)rt * p.num_kb, p);
+                const int c_last = unit_owner((int64_t)rt * p.num_kb + p.num_kb - 1, p);
+                contrib = c_last - c_first + 1;
+                my_idx = blockIdx.x - c_first;
+                my_part = p.ws_part + (((int64_t)rt * p.max_contrib + my_idx) * 128 + lrow) * MT;
+            }
 #pragma unroll 1
             for (int c0 = 0; c0 < MT; c0 += 16) {
                 uint32_t v[16];
@@ -418,12 +534,22 @@ __global__ void __launch_bounds__(gemm_threads(NDQ), 1)
                     tmem_ld_x16(tmem_base + lane_addr + (uint32_t)(d * kAccCols + sp * MT + c0), w2);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(w2[j]));
+                    for (int jj = 0; jj < 16; ++jj)
+                        v[jj] = __float_as_uint(__uint_as_float(v[jj]) + __uint_as_float(w2[jj]));
+                }
+                if (partial) {
+                    // park this CTA's partial sums (fp32) for the row tile's last arriver
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        __stcg(reinterpret_cast<float4 *>(my_part + c0) + q,
+                               make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                           __uint_as_float(v[4 * q + 2]),
+                                           __uint_as_float(v[4 * q + 3])));
+                    continue;
                 }
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int tok = c0 + j;
+                for (int jj = 0; jj < 16; ++jj) {
+                    const int tok = c0 + jj;
                     int64_t out_row;
                     if (MOE) {
                         const int slot = __ldg(p.sorted_ids + (int64_t)tt * MT + tok);
@@ -433,19 +559,64 @@ __global__ void __launch_bounds__(gemm_threads(NDQ), 1)
                         out_row = (m < p.M) ? m : -1;
                     }
                     if (valid && out_row >= 0) {
-                        const __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(v[j]));
+                        const __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(v[jj]));
                         p.Y[out_row * p.N + row] = *reinterpret_cast<const uint16_t *>(&h);
                     }
                 }
             }
             tc_fence_before_sync();
             mbar_arrive(accempty_bar(d));
+            if (partial) {
+                // The last of the row tile's contributing warps (per lane quarter)
+                // adds all partials in ascending K order and writes Y.
+                __threadfence();
+                __syncwarp();
+                unsigned int *cnt = p.ws_cnt + (int64_t)rt * 4 + q4;
+                unsigned int old = 0;
+                if (lane == 0) old = atomicAdd(cnt, 1u);
+                old = __shfl_sync(0xFFFFFFFFu, old, 0);
+                if (old == (unsigned int)(contrib - 1)) {
+                    __threadfence();
+                    const float *base =
+                        p.ws_part + ((int64_t)rt * p.max_contrib * 128 + lrow) * MT;
+#pragma unroll 1
+                    for (int c0 = 0; c0 < MT; c0 += 4) {
+                        float4 acc = __ldcg(reinterpret_cast<const float4 *>(base + c0));
+                        for (int ci = 1; ci < contrib; ++ci) {
+                            const float4 t = __ldcg(
+                                reinterpret_cast<const float4 *>(base + (int64_t)ci * 128 * MT + c0));
+                            acc.x += t.x;
+                            acc.y += t.y;
+                            acc.z += t.z;
+                            acc.w += t.w;
+                        }
+                        const float av[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const int64_t m = c0 + q;
+                            if (valid && m < p.M) {
+                                const __nv_bfloat16 h = __float2bfloat16_rn(av[q]);
+                                p.Y[m * p.N + row] = *reinterpret_cast<const uint16_t *>(&h);
+                            }
+                        }
+                    }
+                    if (lane == 0) *cnt = 0u;       // ready for the next call
+                }
+            }
+        }
+        // all MMAs issued by this warp complete before TMEM is released
+        if (issuer) {
+            if (lane == 0) {
+                tc_commit(mmadone_bar);
+                drain_wait(mmadone_bar, 0u);
+            }
+            __syncwarp();
         }
     }
 
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == 0) {
         tc_fence_after_sync();
         tmem_dealloc(tmem_base, kTmemCols);
     }
@@ -466,7 +637,9 @@ w4_status launch_cfg(const CUtensorMap &tw, const CUtensorMap &ts, const CUtenso
     static bool configured = false;
     if (!configured) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-            cudaSuccess)
+                cudaSuccess ||
+            cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared) != cudaSuccess)
             return w4host::launch_status();
         configured = true;
     }
@@ -489,13 +662,55 @@ int ceil_div_i(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
 
 using namespace w4;
 
+namespace w4 {
+namespace {
+
+// Plan of the stream-K split for a decode-shaped GEMM (M <= 64, K % 256 == 0)
+// on `sms` CTAs; returns false when the split does not apply.
+struct SplitPlan {
+    int n_rt, nkb, ctas, max_contrib, mt;
+    size_t cnt_bytes, part_bytes;
+};
+
+bool plan_split(int64_t M, int64_t N, int64_t K, int sms, SplitPlan *sp) {
+    if (M > 64 || (K % 256) != 0) return false;
+    const int64_t n_rt = (N + 127) / 128, nkb = K / 256;
+    if (n_rt >= sms || nkb < 2 || n_rt > (1 << 20)) return false;
+    const int64_t units = n_rt * nkb;
+    const int ctas = (int)std::min<int64_t>(sms, units);
+    auto owner = [&](int64_t x) { return (int)(((x + 1) * ctas - 1) / units); };
+    int mc = 1;
+    for (int64_t rt = 0; rt < n_rt; ++rt)
+        mc = std::max(mc, owner(rt * nkb + nkb - 1) - owner(rt * nkb) + 1);
+    sp->n_rt = (int)n_rt;
+    sp->nkb = (int)nkb;
+    sp->ctas = ctas;
+    sp->max_contrib = mc;
+    sp->mt = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+    sp->cnt_bytes = ((size_t)n_rt * 4 * sizeof(unsigned int) + 255) / 256 * 256;
+    sp->part_bytes = (size_t)n_rt * mc * 128 * sp->mt * sizeof(float);
+    return true;
+}
+
+}  // namespace
+}  // namespace w4
+
+extern "C" size_t w4a16_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    SplitPlan sp;
+    if (M <= 0 || N <= 0 || K <= 0) return 0;
+    if (!plan_split(M, N, K, w4host::num_sms(), &sp)) return 0;
+    return sp.cnt_bytes + sp.part_bytes;
+}
+
 extern "C" w4_status w4a16_gemm(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S,
                                 w4_bf16 *Y, int64_t M, int64_t N, int64_t K, int group,
-                                void *stream) {
+                                void *workspace, size_t workspace_bytes, void *stream) {
     if (group != 32) return W4_ERR_UNSUPPORTED;
     if (M < 0 || N < 0 || K <= 0 || (K % 32) != 0) return W4_ERR_INVALID_ARG;
     if (!w4host::aligned16(X) || !w4host::aligned16(Wq) || !w4host::aligned16(S) ||
         !w4host::aligned16(Y))
+        return W4_ERR_INVALID_ARG;
+    if (workspace != nullptr && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return W4_ERR_INVALID_ARG;
     if (M == 0 || N == 0) return W4_OK;
     if (N > (1 << 30) || M > (1 << 30) || K > (1 << 24)) return W4_ERR_UNSUPPORTED;
@@ -537,20 +752,40 @@ extern "C" w4_status w4a16_gemm(const w4_bf16 *X, const int32_t *Wq, const w4_bf
     };
 
     if (M <= 64 && wide_k) {
-        // Decode: one token tile, N split evenly over the SMs.
         const int mt = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
-        // rows per tile: every SM streams the same number of weight rows
-        int R = std::min<int64_t>(128, std::max<int64_t>(1, ceil_div_i(N, sms)));
-        while (R < 128 && ceil_div_i(N, R) > sms) ++R;
-        p.rows_per_tile = R;
-        p.n_row_tiles = ceil_div_i(N, R);
         p.n_tok_tiles = 1;
         p.num_kb = ceil_div_i(K, 256);
-        if (!map_x(mt) || !map_w(256, R) || !map_s(R)) return W4_ERR_CUDA;
-        const int items = p.n_row_tiles;
-        if (mt == 16) return launch_cfg<256, 16, 6, 1, 3, 4, 4, false>(tw, ts, tx, p, items, st);
-        if (mt == 32) return launch_cfg<256, 32, 6, 1, 3, 4, 4, false>(tw, ts, tx, p, items, st);
-        return launch_cfg<256, 64, 4, 1, 2, 4, 4, false>(tw, ts, tx, p, items, st);
+        SplitPlan sp;
+        int items;
+        if (workspace != nullptr && plan_split(M, N, K, sms, &sp) &&
+            workspace_bytes >= sp.cnt_bytes + sp.part_bytes) {
+            // Decode, stream-K: full 128-row tiles, the (row tile, k-block)
+            // units cut evenly over the SMs, partial tiles reduced in a fixed
+            // order by the last arriving CTA.
+            p.rows_per_tile = 128;
+            p.n_row_tiles = sp.n_rt;
+            p.split = 1;
+            p.units = (int64_t)sp.n_rt * sp.nkb;
+            p.ctas = sp.ctas;
+            p.max_contrib = sp.max_contrib;
+            p.ws_cnt = reinterpret_cast<unsigned int *>(workspace);
+            p.ws_part = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) +
+                                                  sp.cnt_bytes);
+            items = sp.ctas;
+            if (!map_x(mt) || !map_w(256, 128) || !map_s(128)) return W4_ERR_CUDA;
+        } else {
+            // Decode without a workspace: one token tile, N split evenly over
+            // the SMs (rows per tile = ceil(N / SMs)).
+            int R = std::min<int64_t>(128, std::max<int64_t>(1, ceil_div_i(N, sms)));
+            while (R < 128 && ceil_div_i(N, R) > sms) ++R;
+            p.rows_per_tile = R;
+            p.n_row_tiles = ceil_div_i(N, R);
+            items = p.n_row_tiles;
+            if (!map_x(mt) || !map_w(256, R) || !map_s(R)) return W4_ERR_CUDA;
+        }
+        if (mt == 16) return launch_cfg<256, 16, 6, 1, 3, 4, 2, false>(tw, ts, tx, p, items, st);
+        if (mt == 32) return launch_cfg<256, 32, 6, 1, 3, 4, 2, false>(tw, ts, tx, p, items, st);
+        return launch_cfg<256, 64, 4, 1, 2, 4, 2, false>(tw, ts, tx, p, items, st);
     }
     // Prefill (and any K that is not a multiple of 256): 128-row tiles,
     // 64-wide K blocks, scales read directly.
@@ -629,7 +864,7 @@ extern "C" w4_status w4_moe_w4a16_gemm(const w4_bf16 *A, int a_row_div, const in
     }
     const int64_t items_max = (cap / block) * p.n_row_tiles;
     const int items = (int)std::min<int64_t>(items_max, 1 << 30);
-    if (block == 16) return launch_cfg<256, 16, 6, 2, 3, 4, 4, true>(tw, ts, tx, p, items, st);
-    if (block == 32) return launch_cfg<256, 32, 6, 2, 2, 4, 4, true>(tw, ts, tx, p, items, st);
-    return launch_cfg<256, 64, 4, 1, 2, 4, 4, true>(tw, ts, tx, p, items, st);
+    if (block == 16) return launch_cfg<256, 16, 6, 2, 3, 4, 2, true>(tw, ts, tx, p, items, st);
+    if (block == 32) return launch_cfg<256, 32, 6, 2, 2, 4, 2, true>(tw, ts, tx, p, items, st);
+    return launch_cfg<256, 64, 4, 1, 2, 4, 2, true>(tw, ts, tx, p, items, st);
 }

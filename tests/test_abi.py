@@ -21,7 +21,8 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for required in ["w4_fake_quant", "w4_ste_backward", "w4_quantize_pack", "w4_dequant",
-                     "w4a16_gemm", "w4_moe_align", "w4_moe_w4a16_gemm", "w4_moe_capacity",
+                     "w4a16_gemm", "w4a16_gemm_workspace_bytes", "w4_moe_align",
+                     "w4_moe_w4a16_gemm", "w4_moe_capacity",
                      "w4_device_status", "w4_status_string", "w4_version",
                      "w4_last_cuda_error"]:
         assert required in names
@@ -73,10 +74,11 @@ def test_other_validation():
     assert L.w4_ste_backward(A16, MIS, 8, None) == 1
     assert L.w4_ste_backward(A16, A16, 8, None) == 0           # aliased: zero-copy no-op
     assert L.w4_ste_backward(A16, A16 + 2 * 8, 64, None) == 1  # partial overlap
-    assert L.w4a16_gemm(A16, A16, A16, None, 1, 8, 64, 32, None) == 1
-    assert L.w4a16_gemm(A16, A16, A16, A16, 1, 8, 40, 32, None) == 1
-    assert L.w4a16_gemm(A16, A16, A16, A16, 1, 8, 64, 64, None) == 2
-    assert L.w4a16_gemm(A16, A16, A16, A16, 0, 8, 64, 32, None) == 0   # empty: no launch
+    assert L.w4a16_gemm(A16, A16, A16, None, 1, 8, 64, 32, None, 0, None) == 1
+    assert L.w4a16_gemm(A16, A16, A16, A16, 1, 8, 40, 32, None, 0, None) == 1
+    assert L.w4a16_gemm(A16, A16, A16, A16, 1, 8, 64, 64, None, 0, None) == 2
+    assert L.w4a16_gemm(A16, A16, A16, A16, 1, 8, 64, 32, A16 + 16, 4096, None) == 1  # ws not 256-aligned
+    assert L.w4a16_gemm(A16, A16, A16, A16, 0, 8, 64, 32, None, 0, None) == 0   # empty: no launch
     # moe_align: block not a power of two, E too large, capacity too small
     assert L.w4_moe_align(A16, 4, 2, 8, 24, A16, 1024, A16, A16, None) == 1
     assert L.w4_moe_align(A16, 4, 2, 2048, 16, A16, 1 << 20, A16, A16, None) == 1

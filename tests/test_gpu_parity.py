@@ -208,15 +208,48 @@ def test_gemm_tiny_layer_config():
     assert_gemm_close(Y, R, "tiny layer")
 
 
-@pytest.mark.parametrize("M", [1, 8, 16, 32])
-def test_gemm_decode_config(M):
+_DECODE = {}
+
+
+def _decode_weight():
+    if "w" not in _DECODE:
+        cfg = synth.Decode()
+        _DECODE["w"] = oracle.quantize_pack(bits(cfg.weight()))
+    return _DECODE["w"]
+
+
+@pytest.mark.parametrize("split", [True, False])
+@pytest.mark.parametrize("M", [1, 8, 16, 32, 64])
+def test_gemm_decode_config(M, split):
+    """Decode GEMV sweep, with the stream-K split (workspace) and without."""
     cfg = synth.Decode()
-    W = cfg.weight()
-    Wq, S = oracle.quantize_pack(bits(W))
+    Wq, S = _decode_weight()
     X = cfg.activations(M)
-    Y = bits(w4.gemm(X.to(DEV), torch.from_numpy(Wq).to(DEV), _np_bf16(S).to(DEV)))
+    ws = "auto" if split else None
+    if split:
+        assert w4.w4a16_gemm_workspace_bytes(M, cfg.N, cfg.K) > 0
+    Y = bits(w4.gemm(X.to(DEV), torch.from_numpy(Wq).to(DEV), _np_bf16(S).to(DEV), ws=ws))
     _, R = oracle.w4a16_gemm(bits(X), Wq, S)
-    assert_gemm_close(Y, R, f"decode M={M}")
+    assert_gemm_close(Y, R, f"decode M={M} split={split}")
+
+
+def test_gemm_split_workspace_left_zero_and_deterministic():
+    M, N, K = 16, 4096 + 200, 2048          # ragged last row tile, 8 k-blocks
+    X, Wq, S, Y1 = _gemm_case(M, N, K, seed=5)
+    need = w4.w4a16_gemm_workspace_bytes(M, N, K)
+    assert need > 0
+    ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
+    Xd, Wqd, Sd = _np_bf16(X).to(DEV), torch.from_numpy(Wq).to(DEV), _np_bf16(S).to(DEV)
+    outs = [bits(w4.gemm(Xd, Wqd, Sd, ws=ws)) for _ in range(3)]
+    w4.w4_device_status()
+    n_rt = (N + 127) // 128
+    assert int(ws[: n_rt * 16].count_nonzero()) == 0, "split counters not reset"
+    assert all(np.array_equal(o, outs[0]) for o in outs)
+    _, R = oracle.w4a16_gemm(X, Wq, S)
+    assert_gemm_close(outs[0], R, "split ragged")
+    # the unsplit schedule gives the same product within tolerance
+    Y0 = bits(w4.gemm(Xd, Wqd, Sd, ws=None))
+    assert_gemm_close(Y0, R, "unsplit ragged")
 
 
 @pytest.mark.parametrize("M", [512, 2048, 8192])
