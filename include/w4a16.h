@@ -140,6 +140,34 @@ w4_status w4a16_gemm(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S,
  * the current device (0 when that schedule does not apply).  Host-only. */
 size_t w4a16_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
+/*
+ * W4A16 GEMM for callers that cannot allocate device memory.  (The pages have
+ * no counterpart: this is a deployment variant of w4a16_gemm.)
+ *
+ * Some callers cannot hand the library a workspace: an inference engine that
+ * budgets all device memory at start-up and forbids later allocations, a
+ * plug-in whose host framework owns the allocator, or code that must not call
+ * cudaMalloc because it can synchronize the device.  This entry point computes
+ * exactly what w4a16_gemm computes, using as its scratch a fixed 8 MiB array
+ * inside the library's device image, which every GPU that loads the library
+ * holds until the process exits.  It allocates nothing and calls no
+ * allocating routine.
+ *   - Shapes whose split schedule would need more than 8 MiB of scratch
+ *     (e.g. M = 64 with K = 4096, N = 12288) return W4_ERR_UNSUPPORTED;
+ *     w4a16_gemm with a caller-provided workspace handles them.
+ *   - The first call on a device looks up the array's device address (a
+ *     one-time set-up per device); make that first call before any stream
+ *     capture.
+ *   - Every call shares the one array per device: the call zeroes the part that
+ *     must start at zero (asynchronously, on `stream`), and calls that may
+ *     overlap on the GPU (different streams) race on it and must be serialized
+ *     by the caller.
+ * Arguments as in w4a16_gemm.
+ */
+w4_status w4a16_gemm_noalloc(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S,
+                             w4_bf16 *Y, int64_t M, int64_t N, int64_t K, int group,
+                             void *stream);
+
 /* Padded capacity the caller must provide for w4_moe_align's sorted_ids:
  * T*topk + E*(block-1), rounded up to a multiple of block.  Host-only. */
 int64_t w4_moe_capacity(int64_t T, int topk, int E, int block);

@@ -69,6 +69,7 @@ def lib() -> ctypes.CDLL:
             "w4_quantize_pack": [_P, _P, _P, _I64, _I64, _INT, _P],
             "w4_dequant": [_P, _P, _P, _I64, _I64, _INT, _P],
             "w4a16_gemm": [_P, _P, _P, _P, _I64, _I64, _I64, _INT, _P, ctypes.c_size_t, _P],
+            "w4a16_gemm_noalloc": [_P, _P, _P, _P, _I64, _I64, _I64, _INT, _P],
             "w4_moe_align": [_P, _I64, _INT, _INT, _INT, _P, _I64, _P, _P, _P],
             "w4_moe_w4a16_gemm": [_P, _INT, _P, _P, _P, _P, _P, _I64, _INT, _I64, _P, _I64,
                                   _I64, _INT, _P],
@@ -192,6 +193,20 @@ def w4a16_gemm(X, Wq, S, Y, group: int = GROUP, ws="auto", stream=None) -> None:
     wptr, wbytes = (_ptr(ws), ws.numel() * ws.element_size()) if ws is not None else (None, 0)
     _check("w4a16_gemm", lib().w4a16_gemm(_ptr(X), _ptr(Wq), _ptr(S), _ptr(Y), M, N, K, group,
                                           wptr, wbytes, _stream(stream)))
+
+
+def w4a16_gemm_noalloc(X, Wq, S, Y, group: int = GROUP, stream=None) -> None:
+    """w4a16_gemm without any workspace argument or allocation: the library uses
+    a fixed 8 MiB scratch array of its own per device (see include/w4a16.h for
+    who needs this and its limits)."""
+    _dtype(X, torch.bfloat16, "X")
+    _dtype(Wq, torch.int32, "Wq")
+    M, K = X.shape
+    N = Wq.shape[0]
+    if Wq.shape[1] * 8 != K or tuple(Y.shape) != (M, N):
+        raise ValueError("shape mismatch")
+    _check("w4a16_gemm_noalloc", lib().w4a16_gemm_noalloc(_ptr(X), _ptr(Wq), _ptr(S), _ptr(Y),
+                                                          M, N, K, group, _stream(stream)))
 
 
 def w4_moe_capacity(T: int, topk: int, E: int, block: int) -> int:

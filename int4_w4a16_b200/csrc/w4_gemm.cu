@@ -33,6 +33,7 @@
 // device status, drains its own in-flight copies and MMAs, frees its TMEM and
 // exits.
 #include <algorithm>
+#include <mutex>
 
 #include "w4_common.cuh"
 
@@ -867,4 +868,81 @@ extern "C" w4_status w4_moe_w4a16_gemm(const w4_bf16 *A, int a_row_div, const in
     if (block == 16) return launch_cfg<256, 16, 6, 2, 3, 4, 2, true>(tw, ts, tx, p, items, st);
     if (block == 32) return launch_cfg<256, 32, 6, 2, 2, 4, 2, true>(tw, ts, tx, p, items, st);
     return launch_cfg<256, 64, 4, 1, 2, 4, 2, true>(tw, ts, tx, p, items, st);
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of the decode GEMM.
+//
+// Some callers cannot give this library device memory for scratch: an
+// inference engine that budgets every byte of device memory at start-up and
+// forbids allocations afterwards, a plug-in whose host framework owns the
+// allocator, or a caller that must not call cudaMalloc because it can
+// synchronize the device.  w4a16_gemm_noalloc serves them with a fixed scratch
+// array that lives in this library's device image: every GPU that loads the
+// library holds these bytes until the process exits, and no call allocates.
+// ---------------------------------------------------------------------------
+namespace w4 {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 8u << 20;   // 8 MiB per device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch, looked up once per device with that
+// device current (in host code the symbol is only a host-side stand-in).
+std::mutex g_noalloc_mutex;
+void *g_noalloc_ptr[64] = {nullptr};
+
+w4_status noalloc_scratch(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        w4host::set_cuda_error(e);
+        return W4_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= 64) return W4_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess || ptr == nullptr) {
+            w4host::set_cuda_error(e);
+            return W4_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = ptr;
+    }
+    *out = g_noalloc_ptr[dev];
+    return W4_OK;
+}
+
+}  // namespace
+}  // namespace w4
+
+extern "C" w4_status w4a16_gemm_noalloc(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S,
+                                        w4_bf16 *Y, int64_t M, int64_t N, int64_t K, int group,
+                                        void *stream) {
+    if (group != 32) return W4_ERR_UNSUPPORTED;
+    if (M < 0 || N < 0 || K <= 0 || (K % 32) != 0) return W4_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return W4_OK;
+    // The scratch this shape's schedule needs must fit the fixed array.
+    SplitPlan sp;
+    size_t need = 0, zero_bytes = 0;
+    if (plan_split(M, N, K, w4host::num_sms(), &sp)) {
+        need = sp.cnt_bytes + sp.part_bytes;
+        zero_bytes = sp.cnt_bytes;
+    }
+    if (need > kNoAllocScratchBytes) return W4_ERR_UNSUPPORTED;
+    void *scratch = nullptr;
+    const w4_status st = noalloc_scratch(&scratch);
+    if (st != W4_OK) return st;
+    // The split's arrival counters must start at zero; the array keeps whatever
+    // the previous call (or an aborted one) left there.
+    if (zero_bytes > 0) {
+        const cudaError_t e = cudaMemsetAsync(scratch, 0, zero_bytes, (cudaStream_t)stream);
+        if (e != cudaSuccess) {
+            w4host::set_cuda_error(e);
+            return W4_ERR_CUDA;
+        }
+    }
+    return w4a16_gemm(X, Wq, S, Y, M, N, K, group, need > 0 ? scratch : nullptr,
+                      need > 0 ? kNoAllocScratchBytes : 0, stream);
 }

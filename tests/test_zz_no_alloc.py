@@ -1,0 +1,71 @@
+"""The allocation-free GEMM entry point, called through the C ABI.
+
+w4a16_gemm_noalloc exists for callers that cannot give the library a device
+workspace (an engine that fixes its device memory budget at start-up, a
+plug-in whose host framework owns the allocator, code that must not call
+cudaMalloc).  It must give the same product as w4a16_gemm with a workspace, call
+after call, while using only the library's own fixed scratch array.  This file
+is named so that pytest collects it last.
+"""
+import numpy as np
+import pytest
+import torch
+
+import int4_w4a16_b200 as w4
+import oracle
+import synth
+from synth import bits
+
+pytestmark = pytest.mark.gpu
+REL_TOL = 1e-2
+
+
+def _close(y_bits, ref_bits, what):
+    y = (y_bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    r = (ref_bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    scale = np.abs(r).max()
+    err = np.abs(y - r)
+    assert err.max() <= REL_TOL * scale, what
+    assert not np.any(err > REL_TOL * np.abs(r) + 1e-3 * scale), what
+
+
+@pytest.mark.parametrize("M", [1, 16, 32])
+def test_noalloc_matches_workspace_entry_point_twice(M):
+    L = w4.lib()
+    cfg = synth.Decode()
+    Wq_h, S_h = oracle.quantize_pack(bits(cfg.weight()))
+    dev = "cuda"
+    Wq = torch.from_numpy(Wq_h).to(dev)
+    S = torch.from_numpy(S_h.view(np.int16)).view(torch.bfloat16).to(dev)
+    X = cfg.activations(M, dev)
+    N, K = cfg.N, cfg.K
+    stream = torch.cuda.current_stream().cuda_stream
+    need = L.w4a16_gemm_workspace_bytes(M, N, K)
+    ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
+    Y_ref = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    rc = L.w4a16_gemm(X.data_ptr(), Wq.data_ptr(), S.data_ptr(), Y_ref.data_ptr(), M, N, K, 32,
+                      ws.data_ptr(), ws.numel(), stream)
+    assert rc == 0
+    for call in range(2):                       # two calls in a row share the array
+        Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=dev)
+        rc = L.w4a16_gemm_noalloc(X.data_ptr(), Wq.data_ptr(), S.data_ptr(), Y.data_ptr(),
+                                  M, N, K, 32, stream)
+        assert rc == 0, f"call {call}: status {rc}"
+        torch.cuda.synchronize()
+        _close(bits(Y), bits(Y_ref), f"M={M} call {call}")
+    assert L.w4_device_status(stream) == 0
+
+
+def test_noalloc_rejects_shapes_beyond_its_scratch():
+    L = w4.lib()
+    cfg = synth.Decode()
+    M, N, K = 64, cfg.N, cfg.K                  # split scratch ~9.4 MB > 8 MiB
+    assert L.w4a16_gemm_workspace_bytes(M, N, K) > (8 << 20)
+    dev = "cuda"
+    X = torch.zeros((M, K), dtype=torch.bfloat16, device=dev)
+    Wq = torch.zeros((N, K // 8), dtype=torch.int32, device=dev)
+    S = torch.zeros((N, K // 32), dtype=torch.bfloat16, device=dev)
+    Y = torch.zeros((M, N), dtype=torch.bfloat16, device=dev)
+    rc = L.w4a16_gemm_noalloc(X.data_ptr(), Wq.data_ptr(), S.data_ptr(), Y.data_ptr(), M, N, K,
+                              32, torch.cuda.current_stream().cuda_stream)
+    assert rc == 2                              # W4_ERR_UNSUPPORTED, nothing launched
