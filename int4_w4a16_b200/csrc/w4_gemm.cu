@@ -13,22 +13,29 @@
 //    tile, the B operand (N = MT columns) is the activation tile, so decode
 //    shapes with 1..64 tokens still use a full-height MMA;
 //  * the weights never exist as BF16 in memory or shared memory: packed words
-//    arrive by TMA (128-byte swizzle, bank-conflict-free row reads), four
-//    dequant warps unpack them in registers (LOP3 + PRMT + 2 packed BF16 ops
-//    per pair) and store the BF16 A tile straight into tensor memory with
+//    arrive by TMA (128-byte swizzle, bank-conflict-free row reads), dequant
+//    warps unpack them in registers (LOP3 + 2 packed BF16 ops per pair of
+//    codes) and store the BF16 A tile straight into tensor memory with
 //    tcgen05.st; tcgen05.mma then reads A from TMEM and B from shared memory,
 //    which keeps the shared-memory traffic of a decode step at the packed
 //    bytes plus the activations;
+//  * with 256-wide k-blocks a register pair holds codes (j, j + 4) of a packed
+//    word, which saves the PRMT that natural order needs; the MMA issuers
+//    reorder their activation chunks in shared memory to match, overlapped
+//    with the unpacking of the same stage;
 //  * activations arrive by TMA in the canonical K-major 128-byte-swizzled
 //    layout (dense), or by cp.async row gathers into the same layout (MoE);
-//  * warp specialization: warp 0 = loads, warp 1 = TMEM allocation + MMA
-//    issue (one thread), warps 2-5 = dequant, warps 6-9 = epilogue
-//    (tcgen05.ld -> BF16 -> global), with mbarrier rings between them and
-//    double-buffered accumulators where TMEM allows;
-//  * persistent CTAs (one per SM) walk a static list of work items; for decode
-//    the N rows are split evenly over the SMs (rows per tile = ceil(N / SMs))
-//    so every SM streams the same number of weight bytes and no split-K
-//    reduction (and no scratch memory) is needed.
+//  * warp specialization: warp 0 = loads + TMEM allocation, then groups of
+//    four dequant warps that take turns over the k-blocks, then four MMA +
+//    epilogue warps (several MMA issuers, each into its own accumulator,
+//    because one thread issues a small tcgen05.mma only every ~100 cycles),
+//    with mbarrier rings between the roles;
+//  * persistent CTAs (one per SM) walk a static list of work items.  A decode
+//    GEMM given a workspace splits the (row tile, k-block) units evenly over
+//    the SMs (stream-K); the last CTA to finish a row tile adds the parked
+//    FP32 partial sums in ascending K order, so the result is deterministic.
+//    Without a workspace the N rows are split evenly (rows per tile =
+//    ceil(N / SMs)) and no reduction is needed.
 // Every mbarrier wait is bounded (w4_common.cuh); a timed-out CTA records the
 // device status, drains its own in-flight copies and MMAs, frees its TMEM and
 // exits.
@@ -41,12 +48,17 @@ namespace w4 {
 namespace {
 
 // Warp roles: warp 0 = loads (and TMEM allocation), then 4 * NDQ dequant warps
-// (NDQ per TMEM lane quarter), then 4 MMA + epilogue warps: lane 0 of the
+// (NDQ groups of four that take turns over the k-blocks), then (256-wide
+// k-blocks only) kPermWarps warps that reorder the activation chunks, then
+// 4 MMA + epilogue warps: lane 0 of the
 // first NMMA of them issues MMAs (each into its own accumulator, every NMMA-th
 // 16-wide K step), and all four drain the accumulators of their lane quarter.
 // A single thread issues at most about one small tcgen05.mma per ~120 cycles,
 // so small-N tiles need several issuers to keep up with HBM.
-__host__ __device__ constexpr int gemm_threads(int ndq) { return 32 * (1 + 4 * ndq + 4); }
+__host__ __device__ constexpr int perm_warps(int kb) { return kb == 256 ? 2 : 0; }
+__host__ __device__ constexpr int gemm_threads(int ndq, int kb) {
+    return 32 * (1 + 4 * ndq + perm_warps(kb) + 4);
+}
 constexpr int kTmemCols = 512;
 
 struct GemmParams {
@@ -78,20 +90,22 @@ struct GemmParams {
 // kernels walk whole-K items blockIdx.x, blockIdx.x + gridDim.x, ...; a split
 // kernel walks the CTA's contiguous range of (row tile, k-block) units, cut at
 // row-tile boundaries.
+// 32-bit unsigned arithmetic throughout: the host enables the split only when
+// units * (ctas + 1) < 2^32, and the item count of the other modes is an int.
 struct ItemIter {
-    int64_t cur, end;
-    int step;
+    uint32_t cur, end, step;
 };
 
 __device__ __forceinline__ ItemIter make_iter(const GemmParams &p, int num_items) {
     ItemIter I;
     if (p.split) {
-        I.cur = (int64_t)blockIdx.x * p.units / p.ctas;
-        I.end = ((int64_t)blockIdx.x + 1) * p.units / p.ctas;
+        const uint32_t units = (uint32_t)p.units, ctas = (uint32_t)p.ctas;
+        I.cur = blockIdx.x * units / ctas;
+        I.end = (blockIdx.x + 1) * units / ctas;
         I.step = 0;
     } else {
         I.cur = blockIdx.x;
-        I.end = num_items;
+        I.end = (uint32_t)num_items;
         I.step = gridDim.x;
     }
     return I;
@@ -101,14 +115,20 @@ __device__ __forceinline__ bool next_item(ItemIter &I, const GemmParams &p, int 
                                           int &kb0, int &kb1) {
     if (I.cur >= I.end) return false;
     if (p.split) {
-        rt = (int)(I.cur / p.num_kb);
-        kb0 = (int)(I.cur % p.num_kb);
-        kb1 = (int)((I.end - I.cur) < (int64_t)(p.num_kb - kb0) ? kb0 + (I.end - I.cur) : p.num_kb);
+        const uint32_t nkb = (uint32_t)p.num_kb;
+        const uint32_t r = I.cur / nkb;
+        const uint32_t k0 = I.cur - r * nkb;
+        const uint32_t k1 = min(nkb, k0 + (I.end - I.cur));
+        rt = (int)r;
+        kb0 = (int)k0;
+        kb1 = (int)k1;
         tt = 0;
-        I.cur += kb1 - kb0;
+        I.cur += k1 - k0;
     } else {
-        rt = (int)(I.cur % p.n_row_tiles);
-        tt = (int)(I.cur / p.n_row_tiles);
+        const uint32_t nrt = (uint32_t)p.n_row_tiles;
+        const uint32_t q = I.cur / nrt;
+        rt = (int)(I.cur - q * nrt);
+        tt = (int)q;
         kb0 = 0;
         kb1 = p.num_kb;
         I.cur += I.step;
@@ -117,8 +137,8 @@ __device__ __forceinline__ bool next_item(ItemIter &I, const GemmParams &p, int 
 }
 
 // CTA that owns split unit x (CTA c owns [c*U/P, (c+1)*U/P)).
-__device__ __forceinline__ int unit_owner(int64_t x, const GemmParams &p) {
-    return (int)(((x + 1) * p.ctas - 1) / p.units);
+__device__ __forceinline__ int unit_owner(uint32_t x, const GemmParams &p) {
+    return (int)(((x + 1) * (uint32_t)p.ctas - 1) / (uint32_t)p.units);
 }
 
 // Shared-memory layout, all offsets from a 1024-aligned base.
@@ -130,7 +150,7 @@ struct Layout {
     static constexpr int kXBytes = (KB / 64) * kXSub;
     static constexpr int kStage = kWBytes + kSBytes + kXBytes;
     static constexpr int kBarOff = NSTAGE * kStage;
-    static constexpr int kNumBars = 2 * NSTAGE + 2 * NASTAGE + 2 * NACC + 1;
+    static constexpr int kNumBars = 3 * NSTAGE + 2 * NASTAGE + 2 * NACC + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kBytes = kMiscOff + 16;
     static constexpr int kAlloc = kBytes + 1024;            // slack for 1024-alignment
@@ -180,8 +200,8 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 // Drain wait used on the way out of an aborted CTA (does not look at the abort flag).
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
     const unsigned long long t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs / 4) {
+    for (uint32_t n = 1; !mbar_try_wait(bar, parity); ++n) {
+        if (n % kPollsPerCheck == 0 && globaltimer_ns() - t0 > kWaitLimitNs / 4) {
             record_timeout();
             return;
         }
@@ -192,7 +212,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 // issuer / accumulator u % NSPLIT, and the epilogue adds the accumulators in
 // a fixed order.
 template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT, int NDQ, bool MOE>
-__global__ void __launch_bounds__(gemm_threads(NDQ), 1)
+__global__ void __launch_bounds__(gemm_threads(NDQ, KB), 1)
     w4a16_tc_kernel(const __grid_constant__ CUtensorMap tm_w,
                     const __grid_constant__ CUtensorMap tm_s,
                     const __grid_constant__ CUtensorMap tm_x, const GemmParams p) {
@@ -202,12 +222,12 @@ __global__ void __launch_bounds__(gemm_threads(NDQ), 1)
     constexpr int kAccCols = NSPLIT * MT;      // TMEM columns per work item accumulator
     constexpr int kABase = NACC * kAccCols;    // first A column
     constexpr int kDqWarps = 4 * NDQ;
-    constexpr int kEpiWarp0 = 1 + kDqWarps;
+    constexpr int kPermWarps = perm_warps(KB);
+    constexpr int kEpiWarp0 = 1 + kDqWarps + kPermWarps;
     static_assert(NSPLIT >= 1 && NSPLIT <= 4, "one to four MMA issuers");
     // 256-wide k-blocks (decode / MoE, few activation rows per tile): reorder the
     // activation chunks in shared memory instead of pairing the unpacked codes.
     constexpr bool kXPerm = (KB == 256);
-    static_assert((KB / 32) % NDQ == 0, "k-block chunks split evenly over the dequant warps");
     constexpr uint32_t kIdesc = idesc_bf16_f32(128, MT);
 
     extern __shared__ uint8_t smem_raw[];
@@ -224,6 +244,10 @@ __global__ void __launch_bounds__(gemm_threads(NDQ), 1)
         return bar0 + 8u * (2 * NSTAGE + 2 * NASTAGE + NACC + d);
     };
     const uint32_t mmadone_bar = bar0 + 8u * (2 * NSTAGE + 2 * NASTAGE + 2 * NACC);
+    // stage s's activation chunks reordered (256-wide k-blocks)
+    auto xfull_bar = [&](int s) {
+        return bar0 + 8u * (2 * NSTAGE + 2 * NASTAGE + 2 * NACC + 1 + s);
+    };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
 
@@ -242,7 +266,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ), 1)
             mbar_init(empty_bar(s), (uint32_t)NSPLIT);
         }
         for (int a = 0; a < NASTAGE; ++a) {
-            mbar_init(afull_bar(a), 32u * kDqWarps);
+            mbar_init(afull_bar(a), 128u);   // one dequant group
             mbar_init(aempty_bar(a), (uint32_t)NSPLIT);
         }
         for (int d = 0; d < NACC; ++d) {
@@ -250,6 +274,8 @@ __global__ void __launch_bounds__(gemm_threads(NDQ), 1)
             mbar_init(accempty_bar(d), 128u);
         }
         mbar_init(mmadone_bar, (uint32_t)NSPLIT);
+        if (kXPerm)
+            for (int s = 0; s < NSTAGE; ++s) mbar_init(xfull_bar(s), 32u * kPermWarps);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tm_w);
@@ -351,15 +377,17 @@ __global__ void __launch_bounds__(gemm_threads(NDQ), 1)
             const uint32_t first = it > (uint32_t)NSTAGE ? it - NSTAGE : 0u;
             for (uint32_t j = first; j < it; ++j) drain_wait(full_bar(j % NSTAGE), (j / NSTAGE) & 1u);
         }
-    } else if (warp < kEpiWarp0) {
+    } else if (warp < 1 + kDqWarps) {
         // --------------------------------------------------------- dequant
-        // NDQ warps per TMEM lane quarter; warp part h takes chunks
-        // [h*GH, (h+1)*GH) of every k-block (a chunk = 16 bytes of a row =
-        // 4 packed words = one group of 32 codes).
+        // NDQ groups of 4 warps, one warp per TMEM lane quarter.  Group g takes
+        // every NDQ-th k-block of the CTA's work in full, so one group's barrier
+        // waits and shared-memory latency overlap another group's arithmetic.
+        // A thread owns one A row (TMEM lane) and unpacks its G chunks (a chunk =
+        // 16 bytes of the row = 4 packed words = one group of 32 codes).
         constexpr int G = KB / 32;
-        constexpr int GH = G / NDQ;
+        static_assert(G % 2 == 0, "chunks are stored in pairs (32 TMEM columns)");
         const int q4 = warp & 3;                    // TMEM lane quarter of this warp
-        const int half = (warp - 1) >> 2;           // part index in [0, NDQ)
+        const uint32_t grp = (uint32_t)(warp - 1) >> 2;   // group index in [0, NDQ)
         const int lrow = q4 * 32 + lane;            // A row of this thread
         const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
         const int64_t gpr = p.K / 32;               // groups per row
@@ -377,86 +405,117 @@ __global__ void __launch_bounds__(gemm_threads(NDQ), 1)
                 srow = p.S + base;
             }
             for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                if (it % NDQ != grp) continue;
                 const int s = it % NSTAGE;
                 const int a = it % NASTAGE;
-                uint32_t sc[GH];
+                uint32_t sc[G];
                 if (KB != 256) {
                     // scales of this k-block (direct loads when the tile has no TMA scales)
 #pragma unroll
-                    for (int j = 0; j < GH; ++j) {
-                        const int64_t gi = (int64_t)kb * G + half * GH + j;
+                    for (int j = 0; j < G; ++j) {
+                        const int64_t gi = (int64_t)kb * G + j;
                         const uint16_t v = (srow != nullptr && gi < gpr) ? __ldg(srow + gi) : 0;
                         sc[j] = bf16x2_splat(v);
                     }
                 }
-                if (!warp_wait(full_bar(s), (it / NSTAGE) & 1u, abort_flag) ||
-                    !warp_wait(aempty_bar(a), ((it / NASTAGE) & 1u) ^ 1u, abort_flag)) {
+                if (!warp_wait(full_bar(s), (it / NSTAGE) & 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                // The row's 16-byte chunks are read one pair ahead of their use, which
+                // keeps the register footprint at two pairs plus the 32 outputs.
+                auto load_pair = [&](int j, uint4 (&w)[2]) {
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj)
+                        w[jj] = lds128(w_stage(s) +
+                                       swz((uint32_t)(lrow * (KB / 2) + (j + jj) * 16), KB / 2));
+                };
+                uint4 cur[2], nxt[2];
+                load_pair(0, cur);
+                if (KB == 256) {
+                    // the row's 8 scales (16 bytes)
+                    const uint4 v4 = lds128(s_stage(s) + lrow * 16);
+                    const uint32_t sw[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+                    for (int j = 0; j < G; ++j)
+                        sc[j] = bf16x2_splat((uint16_t)(sw[j >> 1] >> (16 * (j & 1))));
+                }
+                if (!warp_wait(aempty_bar(a), ((it / NASTAGE) & 1u) ^ 1u, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after_sync();
-                if (kXPerm) {
-                    // reorder this thread's share of the stage's activation chunks
-                    // to match the A columns of dequant_word_k8perm
-                    const int dq_tid = (warp - 1) * 32 + lane;
-#pragma unroll 1
-                    for (int ci = dq_tid; ci < MT * 32; ci += 32 * kDqWarps) {
-                        const int t = ci >> 5, c = ci & 31;
-                        const uint32_t addr = x_stage(s) + (c >> 3) * L::kXSub + t * 128 +
-                                              ((((uint32_t)c & 7u) ^ ((uint32_t)t & 7u)) << 4);
-                        sts128(addr, permute_chunk8(lds128(addr)));
-                    }
-                    fence_proxy_async_smem();   // generic writes -> tensor-core reads
-                }
-                // all shared-memory reads of this k-block first
-                uint4 wv[GH];
-#pragma unroll
-                for (int j = 0; j < GH; ++j) {
-                    const uint32_t off =
-                        swz((uint32_t)(lrow * (KB / 2) + (half * GH + j) * 16), KB / 2);
-                    wv[j] = lds128(w_stage(s) + off);
-                }
-                if (KB == 256) {
-                    // this part's GH scales of the row (2 * GH bytes, naturally aligned)
-                    const uint32_t saddr = s_stage(s) + lrow * 16 + half * GH * 2;
-                    uint32_t sw[4];
-                    if (GH == 8) {
-                        const uint4 v4 = lds128(saddr);
-                        sw[0] = v4.x; sw[1] = v4.y; sw[2] = v4.z; sw[3] = v4.w;
-                    } else if (GH == 4) {
-                        const uint2 v2 = lds64(saddr);
-                        sw[0] = v2.x; sw[1] = v2.y; sw[2] = 0; sw[3] = 0;
-                    } else {
-                        sw[0] = lds32(saddr); sw[1] = 0; sw[2] = 0; sw[3] = 0;
-                    }
-#pragma unroll
-                    for (int j = 0; j < GH; ++j)
-                        sc[j] = bf16x2_splat((uint16_t)(sw[j >> 1] >> (16 * (j & 1))));
-                }
                 const uint32_t a_col = tmem_base + lane_addr + (uint32_t)(kABase + a * kAStageCols);
+                // Two chunks (8 packed words) become 32 TMEM columns, 2 BF16 per column.
 #pragma unroll
-                for (int j = 0; j < GH; ++j) {
-                    const uint32_t ws[4] = {wv[j].x, wv[j].y, wv[j].z, wv[j].w};
-                    uint32_t lo[8], hi[8];
-                    if (kXPerm) {
-                        dequant_word_k8perm(ws[0], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&lo[0]));
-                        dequant_word_k8perm(ws[1], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&lo[4]));
-                        dequant_word_k8perm(ws[2], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&hi[0]));
-                        dequant_word_k8perm(ws[3], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&hi[4]));
-                    } else {
-                        dequant_word(ws[0], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&lo[0]));
-                        dequant_word(ws[1], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&lo[4]));
-                        dequant_word(ws[2], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&hi[0]));
-                        dequant_word(ws[3], sc[j], *reinterpret_cast<uint32_t(*)[4]>(&hi[4]));
+                for (int j = 0; j < G; j += 2) {
+                    if (j + 2 < G) load_pair(j + 2, nxt);
+                    uint32_t o[32];
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const uint32_t ws[4] = {cur[jj].x, cur[jj].y, cur[jj].z, cur[jj].w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint32_t t4[4];
+                            if (kXPerm) dequant_word_k8perm(ws[q], sc[j + jj], t4);
+                            else dequant_word(ws[q], sc[j + jj], t4);
+#pragma unroll
+                            for (int z = 0; z < 4; ++z) o[jj * 16 + q * 4 + z] = t4[z];
+                        }
                     }
-                    // columns: 2 BF16 per 32-bit column, ascending k
-                    const uint32_t col = a_col + (uint32_t)((half * GH + j) * 16);
-                    tmem_st_x8(col, lo);
-                    tmem_st_x8(col + 8, hi);
+                    tmem_st_x32(a_col + (uint32_t)(j * 16), o);
+                    if (j + 2 < G) {
+                        cur[0] = nxt[0];
+                        cur[1] = nxt[1];
+                    }
                 }
                 tmem_wait_st();
                 tc_fence_before_sync();
                 mbar_arrive(afull_bar(a));
+            }
+        }
+    } else if (warp < kEpiWarp0) {
+        // ------------------------------------------------ activation reorder
+        // 256-wide k-blocks: the dequant warps leave codes (j, j + 4) of a packed
+        // word in one register pair (dequant_word_k8perm), so every 16-byte
+        // activation chunk [x0..x7] of the stage is rewritten in place as
+        // [x0, x4, x1, x5, x2, x6, x3, x7].  These warps issue no asynchronous
+        // copies or MMAs, so their proxy fence waits only for their own stores.
+        const int pw = warp - 1 - kDqWarps;
+        uint32_t it = 0;
+        bool ok = true;
+        ItemIter I = make_iter(p, num_items);
+        int rt, tt, kb0, kb1;
+        while (ok && next_item(I, p, rt, tt, kb0, kb1)) {
+            for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                const int s = it % NSTAGE;
+                if (!warp_wait(full_bar(s), (it / NSTAGE) & 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                constexpr int kChunks = MT * (KB / 8);
+                // batches of 8 chunks per thread: all loads first, so their
+                // latencies overlap
+                constexpr int kBatch = 8;
+                constexpr int kStride = 32 * (kPermWarps > 0 ? kPermWarps : 1);
+                static_assert(kChunks % (kStride * kBatch) == 0, "whole batches");
+#pragma unroll 1
+                for (int c0 = pw * 32 + lane; c0 < kChunks; c0 += kStride * kBatch) {
+                    uint32_t addr[kBatch];
+                    uint4 v[kBatch];
+#pragma unroll
+                    for (int b = 0; b < kBatch; ++b) {
+                        const int ci = c0 + b * kStride;
+                        const int t = ci / (KB / 8), c = ci % (KB / 8);
+                        addr[b] = x_stage(s) + (c >> 3) * L::kXSub + t * 128 +
+                                  ((((uint32_t)c & 7u) ^ ((uint32_t)t & 7u)) << 4);
+                        v[b] = lds128(addr[b]);
+                    }
+#pragma unroll
+                    for (int b = 0; b < kBatch; ++b) sts128(addr[b], permute_chunk8(v[b]));
+                }
+                fence_proxy_async_smem();   // generic writes -> tensor-core reads
+                mbar_arrive(xfull_bar(s));
             }
         }
     } else {
@@ -482,8 +541,14 @@ __global__ void __launch_bounds__(gemm_threads(NDQ), 1)
                 for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % NSTAGE;
                     const int a = it % NASTAGE;
-                    if (!warp_wait(full_bar(s), (it / NSTAGE) & 1u, abort_flag) ||
-                        !warp_wait(afull_bar(a), (it / NASTAGE) & 1u, abort_flag)) {
+                    // the stage's loads landed (and, for 256-wide k-blocks, its
+                    // activation chunks are reordered)
+                    if (!warp_wait(kXPerm ? xfull_bar(s) : full_bar(s), (it / NSTAGE) & 1u,
+                                   abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (!warp_wait(afull_bar(a), (it / NASTAGE) & 1u, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -518,8 +583,8 @@ __global__ void __launch_bounds__(gemm_threads(NDQ), 1)
             int contrib = 1, my_idx = 0;
             float *my_part = nullptr;
             if (partial) {
-                const int c_first = unit_owner((int64_t)rt * p.num_kb, p);
-                const int c_last = unit_owner((int64_t)rt * p.num_kb + p.num_kb - 1, p);
+                const int c_first = unit_owner((uint32_t)rt * (uint32_t)p.num_kb, p);
+                const int c_last = unit_owner((uint32_t)rt * (uint32_t)p.num_kb + (uint32_t)p.num_kb - 1u, p);
                 contrib = c_last - c_first + 1;
                 my_idx = blockIdx.x - c_first;
                 my_part = p.ws_part + (((int64_t)rt * p.max_contrib + my_idx) * 128 + lrow) * MT;
@@ -645,7 +710,7 @@ w4_status launch_cfg(const CUtensorMap &tw, const CUtensorMap &ts, const CUtenso
         configured = true;
     }
     const int grid = std::max(1, std::min(num_items_max, w4host::num_sms()));
-    kern<<<grid, gemm_threads(NDQ), smem, stream>>>(tw, ts, tx, p);
+    kern<<<grid, gemm_threads(NDQ, KB), smem, stream>>>(tw, ts, tx, p);
     return w4host::launch_status();
 }
 
@@ -679,6 +744,7 @@ bool plan_split(int64_t M, int64_t N, int64_t K, int sms, SplitPlan *sp) {
     if (n_rt >= sms || nkb < 2 || n_rt > (1 << 20)) return false;
     const int64_t units = n_rt * nkb;
     const int ctas = (int)std::min<int64_t>(sms, units);
+    if (units * (ctas + 1) >= ((int64_t)1 << 32)) return false;   // device math is 32-bit
     auto owner = [&](int64_t x) { return (int)(((x + 1) * ctas - 1) / units); };
     int mc = 1;
     for (int64_t rt = 0; rt < n_rt; ++rt)

@@ -7,10 +7,13 @@
 // q = clamp(rint_half_even(w / s), -8, 7), Wdq = bf16_rne(q * s), codes packed
 // low nibble first, eight per int32.
 //
-// Layout of the work: one thread owns 8 consecutive elements (one 16-byte
-// load, one packed word); 4 lanes own a group and reduce its amax with two
-// xor-shuffles.  Grid-stride loop, four 16-byte loads in flight per thread,
-// streaming (evict-first) loads and stores: the kernels are HBM-bound.
+// Layout of the work: one thread owns one group (32 consecutive elements,
+// 64 bytes read as two 32-byte loads when W is 32-byte aligned), so the amax
+// needs no shuffles and the scale is formed once per group; the packed output
+// is one 16-byte store per thread (consecutive across the warp).  Grid-stride
+// loop with two groups (128 bytes) in flight per thread and streaming loads
+// and stores: the kernels are HBM-bound, and per-element integer work is what
+// limits them short of that, so it is kept to the minimum.
 //
 // Division-free exact arithmetic.
 //  * Scale: s32 = fl32(amax / 7) is formed by quotient refinement with one FMA
@@ -50,19 +53,25 @@ constexpr float kMagic = 12582912.0f;     // 1.5 * 2^23: ulp 1 around it
 __device__ __forceinline__ float lo_f(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float hi_f(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Group amax over the 4 lanes that share a group; returns the BF16 bits of amax.
-__device__ __forceinline__ uint32_t group_amax_bits(const uint4 &v) {
-    // |w| as BF16 (sign bit cleared); max of BF16 magnitudes is exact.
-    const uint32_t m = 0x7FFF7FFFu;
-    const uint32_t u[4] = {v.x & m, v.y & m, v.z & m, v.w & m};
-    const __nv_bfloat162 *a = reinterpret_cast<const __nv_bfloat162 *>(u);
-    __nv_bfloat162 mx = __hmax2(__hmax2(a[0], a[1]), __hmax2(a[2], a[3]));
-    const uint32_t mb = *reinterpret_cast<uint32_t *>(&mx);
-    // non-negative BF16 values order like their bit patterns
-    uint32_t am = max(mb & 0xFFFFu, mb >> 16);
-    am = max(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
-    am = max(am, __shfl_xor_sync(0xFFFFFFFFu, am, 2));
-    return am;
+// max(|a|, |b|) per BF16 half (the sign bit of each half is the XOR of the
+// inputs' signs and is masked off by the caller).
+__device__ __forceinline__ uint32_t absmax2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// amax of a group of 32 BF16 values (16 words); returns the BF16 bits of amax.
+// The max of BF16 magnitudes is exact, and non-negative BF16 values order like
+// their bit patterns.
+__device__ __forceinline__ uint32_t group_amax_bits(const uint32_t (&v)[16]) {
+    uint32_t m[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m[j] = absmax2(v[2 * j], v[2 * j + 1]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) m[j] = absmax2(m[2 * j], m[2 * j + 1]);
+    m[0] = absmax2(absmax2(m[0], m[1]), absmax2(m[2], m[3])) & 0x7FFF7FFFu;
+    return max(m[0] & 0xFFFFu, m[0] >> 16);
 }
 
 struct GroupScale {
@@ -172,49 +181,140 @@ __device__ __forceinline__ void item_slow(uint4 v, float s, uint32_t *Wq, uint4 
     }
 }
 
+// A whole group on the slow path, out of line so that the fast path keeps its
+// registers.
+template <int MODE>
+__device__ __noinline__ void group_slow(uint4 c0, uint4 c1, uint4 c2, uint4 c3, float s,
+                                        uint32_t *Wq, uint4 *Wdq, int64_t i0) {
+    item_slow<MODE>(c0, s, Wq, Wdq, i0);
+    item_slow<MODE>(c1, s, Wq, Wdq, i0 + 1);
+    item_slow<MODE>(c2, s, Wq, Wdq, i0 + 2);
+    item_slow<MODE>(c3, s, Wq, Wdq, i0 + 3);
+}
+
 constexpr int kUnroll = 4;
 constexpr int kThreads = 256;
+constexpr int kGroupsInFlight = 2;
+constexpr int kQuantBlocksPerSm = 3;
+
+// 32-byte streaming (evict-first) global load / store; 32-byte aligned address.
+struct u32x8 {
+    uint32_t v[8];
+};
+
+__device__ __forceinline__ u32x8 ld256_cs(const void *p) {
+    u32x8 r;
+    asm volatile("ld.global.cs.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r.v[0]), "=r"(r.v[1]), "=r"(r.v[2]), "=r"(r.v[3]), "=r"(r.v[4]),
+                   "=r"(r.v[5]), "=r"(r.v[6]), "=r"(r.v[7])
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ void st256_cs(void *p, const u32x8 &r) {
+    asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p),
+                 "r"(r.v[0]), "r"(r.v[1]), "r"(r.v[2]), "r"(r.v[3]), "r"(r.v[4]), "r"(r.v[5]),
+                 "r"(r.v[6]), "r"(r.v[7])
+                 : "memory");
+}
+
+// 64 bytes (one group) from global memory: two 32-byte loads (V8, 32-byte
+// aligned source) or four 16-byte loads; streaming (evict-first).
+template <bool V8>
+__device__ __forceinline__ void load_group(const uint32_t *p, uint32_t (&v)[16]) {
+    if (V8) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const u32x8 r = ld256_cs(p + 8 * h);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[8 * h + j] = r.v[j];
+        }
+    } else {
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const uint4 t = __ldcs(reinterpret_cast<const uint4 *>(p) + h);
+            v[4 * h] = t.x; v[4 * h + 1] = t.y; v[4 * h + 2] = t.z; v[4 * h + 3] = t.w;
+        }
+    }
+}
+
+template <bool V8>
+__device__ __forceinline__ void store_group(uint32_t *p, const uint32_t (&v)[16]) {
+    if (V8) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            u32x8 r;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) r.v[j] = v[8 * h + j];
+            st256_cs(p + 8 * h, r);
+        }
+    } else {
+#pragma unroll
+        for (int h = 0; h < 4; ++h)
+            __stcs(reinterpret_cast<uint4 *>(p) + h,
+                   make_uint4(v[4 * h], v[4 * h + 1], v[4 * h + 2], v[4 * h + 3]));
+    }
+}
 
 // MODE 0: quantize + pack (Wq, S).  MODE 1: fake quant (Wdq, optional S).
-template <int MODE>
-__global__ void __launch_bounds__(kThreads, 4) quant_kernel(const uint4 *__restrict__ W,
-                                                         uint4 *__restrict__ Wdq,
+// One thread per group of 32 weights; V8: W (and Wdq) 32-byte aligned.
+template <int MODE, bool V8>
+__global__ void __launch_bounds__(kThreads, kQuantBlocksPerSm) quant_kernel(const uint32_t *__restrict__ W,
+                                                         uint32_t *__restrict__ Wdq,
                                                          uint32_t *__restrict__ Wq,
-                                                         uint16_t *__restrict__ S, int64_t n8) {
-    const int lane = threadIdx.x & 31;
+                                                         uint16_t *__restrict__ S,
+                                                         int64_t ngroups) {
     const int64_t T = (int64_t)gridDim.x * blockDim.x;
-    const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    // The loop bound is tested on the warp's first item, so all 32 lanes run
-    // every iteration together (the shuffles need the full warp); n8 is a
-    // multiple of 4, so the 4 lanes of a group are valid or invalid together.
-    for (int64_t base = gt - lane; base < n8; base += kUnroll * T) {
-        uint4 v[kUnroll];
+    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < ngroups;
+         base += kGroupsInFlight * T) {
+        uint32_t v[kGroupsInFlight][16];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int64_t i = base + lane + u * T;
-            v[u] = (i < n8) ? __ldcs(W + i) : make_uint4(0, 0, 0, 0);
+        for (int u = 0; u < kGroupsInFlight; ++u) {
+            const int64_t g = base + u * T;
+            if (g < ngroups) load_group<V8>(W + 16 * g, v[u]);
         }
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int64_t i = base + lane + u * T;
-            const GroupScale g = make_scale(group_amax_bits(v[u]));
+        for (int u = 0; u < kGroupsInFlight; ++u) {
+            const int64_t g = base + u * T;
+            if (g >= ngroups) break;
+            const GroupScale gs = make_scale(group_amax_bits(v[u]));
             // the fast path needs a normal scale (and, for the BF16 output, no
-            // overflow of 1.5 * 2^23 * s); all lanes take the same branch
-            const bool fast = g.mode == 1 && (MODE == 0 || g.s <= 1.2676506e30f);
-            if (i < n8) {
-                if (fast) {
-                    float c[8];
-                    codes8_fast(v[u], g.r, c);
-                    if (MODE == 0) {
-                        __stcs(reinterpret_cast<unsigned int *>(Wq + i), pack8(c));
-                    } else {
-                        __stcs(Wdq + i, dequant8_fast(c, g.s, -kMagic * g.s));
+            // overflow of 1.5 * 2^23 * s)
+            const bool fast = gs.mode == 1 && (MODE == 0 || gs.s <= 1.2676506e30f);
+            if (fast) {
+                if (MODE == 0) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        float cd[8];
+                        codes8_fast(make_uint4(v[u][4 * c], v[u][4 * c + 1], v[u][4 * c + 2],
+                                               v[u][4 * c + 3]),
+                                    gs.r, cd);
+                        w[c] = pack8(cd);
                     }
+                    __stcs(reinterpret_cast<uint4 *>(Wq) + g, make_uint4(w[0], w[1], w[2], w[3]));
                 } else {
-                    item_slow<MODE>(v[u], g.s, Wq, Wdq, i);
+                    uint32_t o[16];
+                    const float neg_cs = -kMagic * gs.s;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        float cd[8];
+                        codes8_fast(make_uint4(v[u][4 * c], v[u][4 * c + 1], v[u][4 * c + 2],
+                                               v[u][4 * c + 3]),
+                                    gs.r, cd);
+                        const uint4 d = dequant8_fast(cd, gs.s, neg_cs);
+                        o[4 * c] = d.x; o[4 * c + 1] = d.y; o[4 * c + 2] = d.z; o[4 * c + 3] = d.w;
+                    }
+                    store_group<V8>(Wdq + 16 * g, o);
                 }
+            } else {
+                group_slow<MODE>(make_uint4(v[u][0], v[u][1], v[u][2], v[u][3]),
+                                 make_uint4(v[u][4], v[u][5], v[u][6], v[u][7]),
+                                 make_uint4(v[u][8], v[u][9], v[u][10], v[u][11]),
+                                 make_uint4(v[u][12], v[u][13], v[u][14], v[u][15]), gs.s, Wq,
+                                 reinterpret_cast<uint4 *>(Wdq), 4 * g);
             }
-            if (i < n8 && S != nullptr && (lane & 3) == 0) S[i >> 2] = g.bits;
+            if (S != nullptr) S[g] = gs.bits;
         }
     }
 }
@@ -235,6 +335,28 @@ __global__ void __launch_bounds__(kThreads, 4) copy16_kernel(const uint4 *__rest
         for (int u = 0; u < kUnroll; ++u) {
             const int64_t i = base + u * T;
             if (i < n16) __stcs(dst + i, v[u]);
+        }
+    }
+}
+
+// The same copy in 32-byte units (both pointers 32-byte aligned): twice the
+// bytes in flight per thread.
+__global__ void __launch_bounds__(kThreads, 4) copy32_kernel(const u32x8 *__restrict__ src,
+                                                             u32x8 *__restrict__ dst,
+                                                             int64_t n32) {
+    const int64_t T = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < n32;
+         base += kUnroll * T) {
+        u32x8 v[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t i = base + u * T;
+            if (i < n32) v[u] = ld256_cs(src + i);
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t i = base + u * T;
+            if (i < n32) st256_cs(dst + i, v[u]);
         }
     }
 }
@@ -264,10 +386,13 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint4 *__restri
     }
 }
 
-int grid_for(int64_t work_items, int per_thread) {
+bool aligned32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
+
+// At most one wave of resident CTAs (blocks_per_sm per SM), grid-stride beyond.
+int grid_for(int64_t work_items, int per_thread, int blocks_per_sm = 4) {
     const int64_t need = (work_items + (int64_t)kThreads * per_thread - 1) /
                          ((int64_t)kThreads * per_thread);
-    const int64_t cap = (int64_t)w4host::num_sms() * 4;
+    const int64_t cap = (int64_t)w4host::num_sms() * blocks_per_sm;
     return (int)std::max<int64_t>(1, std::min<int64_t>(need, cap));
 }
 
@@ -290,11 +415,16 @@ extern "C" w4_status w4_fake_quant(const w4_bf16 *W, w4_bf16 *Wdq, w4_bf16 *S, i
     if (st != W4_OK) return st;
     if (S != nullptr && !w4host::aligned16(S)) return W4_ERR_INVALID_ARG;
     if ((const void *)W == (const void *)Wdq) return W4_ERR_INVALID_ARG;
-    const int64_t n8 = rows * K / 8;
-    if (n8 == 0) return W4_OK;
-    quant_kernel<1><<<grid_for(n8, kUnroll), kThreads, 0, (cudaStream_t)stream>>>(
-        reinterpret_cast<const uint4 *>(W), reinterpret_cast<uint4 *>(Wdq), nullptr,
-        reinterpret_cast<uint16_t *>(S), n8);
+    const int64_t ngroups = rows * K / 32;
+    if (ngroups == 0) return W4_OK;
+    const int grid = grid_for(ngroups, kGroupsInFlight, kQuantBlocksPerSm);
+    const uint32_t *w = reinterpret_cast<const uint32_t *>(W);
+    uint32_t *o = reinterpret_cast<uint32_t *>(Wdq);
+    uint16_t *s = reinterpret_cast<uint16_t *>(S);
+    if (aligned32(W) && aligned32(Wdq))
+        quant_kernel<1, true><<<grid, kThreads, 0, (cudaStream_t)stream>>>(w, o, nullptr, s, ngroups);
+    else
+        quant_kernel<1, false><<<grid, kThreads, 0, (cudaStream_t)stream>>>(w, o, nullptr, s, ngroups);
     return w4host::launch_status();
 }
 
@@ -303,11 +433,16 @@ extern "C" w4_status w4_quantize_pack(const w4_bf16 *W, int32_t *Wq, w4_bf16 *S,
     w4_status st = check_quant_args(W, Wq, rows, K, group);
     if (st != W4_OK) return st;
     if (!w4host::aligned16(S)) return W4_ERR_INVALID_ARG;
-    const int64_t n8 = rows * K / 8;
-    if (n8 == 0) return W4_OK;
-    quant_kernel<0><<<grid_for(n8, kUnroll), kThreads, 0, (cudaStream_t)stream>>>(
-        reinterpret_cast<const uint4 *>(W), nullptr, reinterpret_cast<uint32_t *>(Wq),
-        reinterpret_cast<uint16_t *>(S), n8);
+    const int64_t ngroups = rows * K / 32;
+    if (ngroups == 0) return W4_OK;
+    const int grid = grid_for(ngroups, kGroupsInFlight, kQuantBlocksPerSm);
+    const uint32_t *w = reinterpret_cast<const uint32_t *>(W);
+    uint32_t *q = reinterpret_cast<uint32_t *>(Wq);
+    uint16_t *s = reinterpret_cast<uint16_t *>(S);
+    if (aligned32(W))
+        quant_kernel<0, true><<<grid, kThreads, 0, (cudaStream_t)stream>>>(w, nullptr, q, s, ngroups);
+    else
+        quant_kernel<0, false><<<grid, kThreads, 0, (cudaStream_t)stream>>>(w, nullptr, q, s, ngroups);
     return w4host::launch_status();
 }
 
@@ -317,12 +452,22 @@ extern "C" w4_status w4_ste_backward(const w4_bf16 *dWdq, w4_bf16 *dW, int64_t n
     const uint16_t *a = reinterpret_cast<const uint16_t *>(dWdq);
     uint16_t *b = reinterpret_cast<uint16_t *>(dW);
     if (a < b + n && b < a + n) return W4_ERR_INVALID_ARG;  // partial overlap
-    const int64_t n16 = n / 8;
-    if (n16 > 0)
-        copy16_kernel<<<grid_for(n16, kUnroll), kThreads, 0, (cudaStream_t)stream>>>(
-            reinterpret_cast<const uint4 *>(a), reinterpret_cast<uint4 *>(b), n16);
-    if (n16 * 8 < n)
-        copy2_tail_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(a, b, n16 * 8, n);
+    int64_t done = 0;
+    if (aligned32(a) && aligned32(b)) {
+        const int64_t n32 = n / 16;
+        if (n32 > 0)
+            copy32_kernel<<<grid_for(n32, kUnroll), kThreads, 0, (cudaStream_t)stream>>>(
+                reinterpret_cast<const u32x8 *>(a), reinterpret_cast<u32x8 *>(b), n32);
+        done = n32 * 16;
+    } else {
+        const int64_t n16 = n / 8;
+        if (n16 > 0)
+            copy16_kernel<<<grid_for(n16, kUnroll), kThreads, 0, (cudaStream_t)stream>>>(
+                reinterpret_cast<const uint4 *>(a), reinterpret_cast<uint4 *>(b), n16);
+        done = n16 * 8;
+    }
+    if (done < n)
+        copy2_tail_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(a, b, done, n);
     return w4host::launch_status();
 }
 

@@ -145,6 +145,36 @@ def test_ste_backward():
     assert torch.equal(W.grad.view(torch.int16), grad.view(torch.int16))
 
 
+def test_16_byte_aligned_buffers():
+    """Buffers aligned to 16 but not 32 bytes take the 16-byte load/store kernels;
+    results are identical to the oracle either way."""
+    n = 4099 * 9                                   # not a multiple of 16: tail copy
+    src = synth.normal_bf16((n + 16,), 1e-3, seed=21).to(DEV)
+    dst = torch.zeros(n + 16, dtype=torch.bfloat16, device=DEV)
+    for so in (0, 8):
+        for do in (0, 8):
+            dst.zero_()
+            w4.w4_ste_backward(src[so:so + n], dst[do:do + n])
+            assert torch.equal(src[so:so + n].view(torch.int16), dst[do:do + n].view(torch.int16))
+            assert not dst[:do].view(torch.int16).any() and not dst[do + n:].view(torch.int16).any()
+    rows, K = 96, 512
+    W_cpu = synth.laplace_bf16((rows, K), 0.02, seed=22)
+    Wq_o, S_o = oracle.quantize_pack(bits(W_cpu))
+    Wdq_o, _ = oracle.fake_quant(bits(W_cpu))
+    buf = torch.zeros(rows * K + 8, dtype=torch.bfloat16, device=DEV)
+    buf[8:] = W_cpu.reshape(-1).to(DEV)
+    W = buf[8:].view(rows, K)                      # 16-byte but not 32-byte aligned
+    assert W.data_ptr() % 32 == 16
+    Wq, S = w4.quantize_pack(W)
+    out = torch.zeros(rows * K + 8, dtype=torch.bfloat16, device=DEV)
+    Wdq = out[8:].view(rows, K)
+    w4.w4_fake_quant(W, Wdq)
+    w4.w4_device_status()
+    assert np.array_equal(Wq.cpu().numpy(), Wq_o)
+    assert np.array_equal(bits(S), S_o)
+    assert np.array_equal(bits(Wdq), Wdq_o)
+
+
 def test_dequant_exhaustive_words():
     """Every code value at every nibble position, times a spread of scales."""
     rng = np.random.default_rng(1)
