@@ -97,16 +97,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 constexpr uint32_t kPollsPerCheck = 64;
 // Back-off between polls: a waiting warp then takes no issue slots and no
 // shared-memory bandwidth from the warps doing the work, at the price of up to
-// about this much extra latency when the phase completes.
+// about this much extra latency when the phase completes.  Waiters off the
+// critical path pass a longer back-off.
 constexpr uint32_t kPollSleepNs = 32;
 
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
-                                          volatile int *abort_flag) {
+                                          volatile int *abort_flag,
+                                          uint32_t sleep_ns = kPollSleepNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     for (uint32_t n = 1;; ++n) {
         if (mbar_try_wait(bar, parity)) return true;
-        __nanosleep(kPollSleepNs);
+        __nanosleep(sleep_ns);
         if (n % kPollsPerCheck == 0) {
             if (*abort_flag) return false;
             if (globaltimer_ns() - t0 > kWaitLimitNs) {
@@ -200,10 +202,8 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(
-            d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u),
-        "r"(0u)
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 

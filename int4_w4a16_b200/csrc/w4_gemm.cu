@@ -50,14 +50,14 @@ namespace {
 // Warp roles: warp 0 = loads (and TMEM allocation), then 4 * NDQ dequant warps
 // (NDQ groups of four that take turns over the k-blocks), then (256-wide
 // k-blocks only) kPermWarps warps that reorder the activation chunks, then
-// 4 MMA + epilogue warps: lane 0 of the
-// first NMMA of them issues MMAs (each into its own accumulator, every NMMA-th
-// 16-wide K step), and all four drain the accumulators of their lane quarter.
-// A single thread issues at most about one small tcgen05.mma per ~120 cycles,
-// so small-N tiles need several issuers to keep up with HBM.
+// 4 epilogue warps (each drains the accumulators of its TMEM lane quarter),
+// then NSPLIT MMA issuer warps: lane 0 of issuer i issues every NSPLIT-th
+// 16-wide K step into accumulator i.  A thread issues a small tcgen05.mma only
+// about every 110 cycles (issue latency, not the tensor core), so small-N
+// tiles need several issuers to keep up with HBM.
 __host__ __device__ constexpr int perm_warps(int kb) { return kb == 256 ? 2 : 0; }
-__host__ __device__ constexpr int gemm_threads(int ndq, int kb) {
-    return 32 * (1 + 4 * ndq + perm_warps(kb) + 4);
+__host__ __device__ constexpr int gemm_threads(int ndq, int kb, int nsplit) {
+    return 32 * (1 + 4 * ndq + perm_warps(kb) + 4 + nsplit);
 }
 constexpr int kTmemCols = 512;
 
@@ -150,7 +150,7 @@ struct Layout {
     static constexpr int kXBytes = (KB / 64) * kXSub;
     static constexpr int kStage = kWBytes + kSBytes + kXBytes;
     static constexpr int kBarOff = NSTAGE * kStage;
-    static constexpr int kNumBars = 3 * NSTAGE + 2 * NASTAGE + 2 * NACC + 1;
+    static constexpr int kNumBars = 2 * NSTAGE + 2 * NASTAGE + 2 * NACC + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kBytes = kMiscOff + 16;
     static constexpr int kAlloc = kBytes + 1024;            // slack for 1024-alignment
@@ -192,10 +192,17 @@ __device__ __forceinline__ uint32_t swz(uint32_t off, uint32_t sw_bytes) {
 }
 
 // Bounded wait executed by every lane of a warp; the verdict is warp-uniform.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
-    bool ok = mbar_wait(bar, parity, abort_flag);
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                          uint32_t sleep_ns = kPollSleepNs) {
+    bool ok = mbar_wait(bar, parity, abort_flag, sleep_ns);
     return __all_sync(0xFFFFFFFFu, ok);
 }
+
+// Back-off per kind of waiter: the dequant warps and the MMA issuers are on the
+// critical path (default back-off); the loads, the activation reorder and the
+// accumulator hand-over run ahead of it; the epilogue waits a whole work item.
+constexpr uint32_t kSleepAhead = 128;
+constexpr uint32_t kSleepLong = 256;
 
 // Drain wait used on the way out of an aborted CTA (does not look at the abort flag).
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
@@ -212,7 +219,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 // issuer / accumulator u % NSPLIT, and the epilogue adds the accumulators in
 // a fixed order.
 template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT, int NDQ, bool MOE>
-__global__ void __launch_bounds__(gemm_threads(NDQ, KB), 1)
+__global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT), 1)
     w4a16_tc_kernel(const __grid_constant__ CUtensorMap tm_w,
                     const __grid_constant__ CUtensorMap tm_s,
                     const __grid_constant__ CUtensorMap tm_x, const GemmParams p) {
@@ -224,7 +231,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB), 1)
     constexpr int kDqWarps = 4 * NDQ;
     constexpr int kPermWarps = perm_warps(KB);
     constexpr int kEpiWarp0 = 1 + kDqWarps + kPermWarps;
-    static_assert(NSPLIT >= 1 && NSPLIT <= 4, "one to four MMA issuers");
+    static_assert(NSPLIT >= 1 && NSPLIT <= 8, "one to eight MMA issuers");
     // 256-wide k-blocks (decode / MoE, few activation rows per tile): reorder the
     // activation chunks in shared memory instead of pairing the unpacked codes.
     constexpr bool kXPerm = (KB == 256);
@@ -244,10 +251,6 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB), 1)
         return bar0 + 8u * (2 * NSTAGE + 2 * NASTAGE + NACC + d);
     };
     const uint32_t mmadone_bar = bar0 + 8u * (2 * NSTAGE + 2 * NASTAGE + 2 * NACC);
-    // stage s's activation chunks reordered (256-wide k-blocks)
-    auto xfull_bar = [&](int s) {
-        return bar0 + 8u * (2 * NSTAGE + 2 * NASTAGE + 2 * NACC + 1 + s);
-    };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
 
@@ -266,7 +269,8 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB), 1)
             mbar_init(empty_bar(s), (uint32_t)NSPLIT);
         }
         for (int a = 0; a < NASTAGE; ++a) {
-            mbar_init(afull_bar(a), 128u);   // one dequant group
+            // one dequant group, plus the activation-reorder warps
+            mbar_init(afull_bar(a), 128u + (kXPerm ? 32u * kPermWarps : 0u));
             mbar_init(aempty_bar(a), (uint32_t)NSPLIT);
         }
         for (int d = 0; d < NACC; ++d) {
@@ -274,8 +278,6 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB), 1)
             mbar_init(accempty_bar(d), 128u);
         }
         mbar_init(mmadone_bar, (uint32_t)NSPLIT);
-        if (kXPerm)
-            for (int s = 0; s < NSTAGE; ++s) mbar_init(xfull_bar(s), 32u * kPermWarps);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tm_w);
@@ -332,7 +334,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB), 1)
             }
             for (int kb = kb0; kb < kb1; ++kb, ++it) {
                 const int s = it % NSTAGE;
-                if (!warp_wait(empty_bar(s), ((it / NSTAGE) & 1u) ^ 1u, abort_flag)) {
+                if (!warp_wait(empty_bar(s), ((it / NSTAGE) & 1u) ^ 1u, abort_flag, kSleepAhead)) {
                     ok = false;
                     break;
                 }
@@ -408,6 +410,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB), 1)
                 if (it % NDQ != grp) continue;
                 const int s = it % NSTAGE;
                 const int a = it % NASTAGE;
+                static_assert(KB == 256 || G == 2, "direct-load scales: one chunk pair per k-block");
                 uint32_t sc[G];
                 if (KB != 256) {
                     // scales of this k-block (direct loads when the tile has no TMA scales)
@@ -422,24 +425,22 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB), 1)
                     ok = false;
                     break;
                 }
-                // The row's 16-byte chunks are read one pair ahead of their use, which
-                // keeps the register footprint at two pairs plus the 32 outputs.
+                // The row's 16-byte chunks (and, with TMA-loaded scales, their two
+                // scales) are read one pair ahead of their use.  The pair loop stays
+                // rolled: one compact body run G / 2 times stays in the instruction
+                // cache, where the unrolled k-block would be refetched every time.
                 auto load_pair = [&](int j, uint4 (&w)[2]) {
 #pragma unroll
                     for (int jj = 0; jj < 2; ++jj)
                         w[jj] = lds128(w_stage(s) +
                                        swz((uint32_t)(lrow * (KB / 2) + (j + jj) * 16), KB / 2));
                 };
+                auto load_scales = [&](int j) -> uint32_t {
+                    return KB == 256 ? lds32(s_stage(s) + lrow * 16 + j * 2) : 0u;
+                };
                 uint4 cur[2], nxt[2];
                 load_pair(0, cur);
-                if (KB == 256) {
-                    // the row's 8 scales (16 bytes)
-                    const uint4 v4 = lds128(s_stage(s) + lrow * 16);
-                    const uint32_t sw[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-                    for (int j = 0; j < G; ++j)
-                        sc[j] = bf16x2_splat((uint16_t)(sw[j >> 1] >> (16 * (j & 1))));
-                }
+                uint32_t s_cur = load_scales(0);
                 if (!warp_wait(aempty_bar(a), ((it / NASTAGE) & 1u) ^ 1u, abort_flag)) {
                     ok = false;
                     break;
@@ -447,9 +448,23 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB), 1)
                 tc_fence_after_sync();
                 const uint32_t a_col = tmem_base + lane_addr + (uint32_t)(kABase + a * kAStageCols);
                 // Two chunks (8 packed words) become 32 TMEM columns, 2 BF16 per column.
-#pragma unroll
-                for (int j = 0; j < G; j += 2) {
-                    if (j + 2 < G) load_pair(j + 2, nxt);
+                constexpr int kPairs = G / 2;
+#pragma unroll 1
+                for (int jp = 0; jp < kPairs; ++jp) {
+                    const int j = 2 * jp;
+                    uint32_t s_nxt = 0;
+                    if (jp + 1 < kPairs) {
+                        load_pair(j + 2, nxt);
+                        s_nxt = load_scales(j + 2);
+                    }
+                    uint32_t scp[2];
+                    if (KB == 256) {
+                        scp[0] = bf16x2_splat((uint16_t)(s_cur & 0xFFFFu));
+                        scp[1] = bf16x2_splat((uint16_t)(s_cur >> 16));
+                    } else {
+                        scp[0] = sc[0];     // G == 2: a single pair
+                        scp[1] = sc[1];
+                    }
                     uint32_t o[32];
 #pragma unroll
                     for (int jj = 0; jj < 2; ++jj) {
@@ -457,16 +472,17 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB), 1)
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             uint32_t t4[4];
-                            if (kXPerm) dequant_word_k8perm(ws[q], sc[j + jj], t4);
-                            else dequant_word(ws[q], sc[j + jj], t4);
+                            if (kXPerm) dequant_word_k8perm(ws[q], scp[jj], t4);
+                            else dequant_word(ws[q], scp[jj], t4);
 #pragma unroll
                             for (int z = 0; z < 4; ++z) o[jj * 16 + q * 4 + z] = t4[z];
                         }
                     }
                     tmem_st_x32(a_col + (uint32_t)(j * 16), o);
-                    if (j + 2 < G) {
+                    if (jp + 1 < kPairs) {
                         cur[0] = nxt[0];
                         cur[1] = nxt[1];
+                        s_cur = s_nxt;
                     }
                 }
                 tmem_wait_st();
@@ -489,7 +505,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB), 1)
         while (ok && next_item(I, p, rt, tt, kb0, kb1)) {
             for (int kb = kb0; kb < kb1; ++kb, ++it) {
                 const int s = it % NSTAGE;
-                if (!warp_wait(full_bar(s), (it / NSTAGE) & 1u, abort_flag)) {
+                if (!warp_wait(full_bar(s), (it / NSTAGE) & 1u, abort_flag, kSleepAhead)) {
                     ok = false;
                     break;
                 }
@@ -515,13 +531,23 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB), 1)
                     for (int b = 0; b < kBatch; ++b) sts128(addr[b], permute_chunk8(v[b]));
                 }
                 fence_proxy_async_smem();   // generic writes -> tensor-core reads
-                mbar_arrive(xfull_bar(s));
+                // Join the dequant group's arrival on the A slot's "full" barrier.
+                // Waiting for the slot to be free first keeps this arrival in the
+                // slot's current phase (these warps may run ahead of the dequant).
+                const int a = it % NASTAGE;
+                if (!warp_wait(aempty_bar(a), ((it / NASTAGE) & 1u) ^ 1u, abort_flag, kSleepAhead)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive(afull_bar(a));
             }
         }
     } else {
         // ------------------------------------------------- MMA + epilogue
-        const int j = warp - kEpiWarp0;             // 0..3
-        const bool issuer = j < NSPLIT;             // warp-uniform
+        // four epilogue warps (one per TMEM lane quarter), then NSPLIT MMA issuers:
+        // the epilogue of one work item overlaps the MMAs of the next
+        const int ji = warp - kEpiWarp0 - 4;        // issuer index, < 0 for the epilogue
+        const bool issuer = ji >= 0;                // warp-uniform
         const int q4 = warp & 3;
         const int lrow = q4 * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
@@ -532,19 +558,19 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB), 1)
         for (; ok && next_item(I, p, rt, tt, kb0, kb1); ++acc_it) {
             const int d = acc_it % NACC;
             if (issuer) {
-                if (!warp_wait(accempty_bar(d), ((acc_it / NACC) & 1u) ^ 1u, abort_flag)) {
+                if (!warp_wait(accempty_bar(d), ((acc_it / NACC) & 1u) ^ 1u, abort_flag, kSleepAhead)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after_sync();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(d * kAccCols + j * MT);
+                const uint32_t d_tmem = tmem_base + (uint32_t)(d * kAccCols + ji * MT);
                 for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % NSTAGE;
                     const int a = it % NASTAGE;
-                    // the stage's loads landed (and, for 256-wide k-blocks, its
-                    // activation chunks are reordered)
-                    if (!warp_wait(kXPerm ? xfull_bar(s) : full_bar(s), (it / NSTAGE) & 1u,
-                                   abort_flag)) {
+                    // the stage's loads landed (with 256-wide k-blocks the A slot's
+                    // barrier also covers the activation reorder, which itself
+                    // waited for the loads)
+                    if (!kXPerm && !warp_wait(full_bar(s), (it / NSTAGE) & 1u, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -558,7 +584,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB), 1)
                         const uint32_t a_tmem =
                             tmem_base + (uint32_t)(kABase + a * kAStageCols);
 #pragma unroll
-                        for (int u = j; u < KB / 16; u += NSPLIT) {
+                        for (int u = ji; u < KB / 16; u += NSPLIT) {
                             const uint32_t baddr =
                                 x_stage(s) + (u >> 2) * L::kXSub + (u & 3) * 32;
                             tc_mma_ts(d_tmem, a_tmem + u * 8, smem_desc_k_sw128(baddr), kIdesc,
@@ -572,9 +598,10 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB), 1)
                 if (!ok) break;
                 if (lane == 0) tc_commit(accfull_bar(d));
                 __syncwarp();
+                continue;                           // issuers do no epilogue
             }
             // epilogue of this lane quarter: sum the NSPLIT accumulators in order
-            if (!warp_wait(accfull_bar(d), (acc_it / NACC) & 1u, abort_flag)) break;
+            if (!warp_wait(accfull_bar(d), (acc_it / NACC) & 1u, abort_flag, kSleepLong)) break;
             tc_fence_after_sync();
             const int64_t row = (int64_t)rt * R + lrow;
             const bool valid = lrow < R && row < p.N;
@@ -591,17 +618,27 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB), 1)
             }
 #pragma unroll 1
             for (int c0 = 0; c0 < MT; c0 += 16) {
+                // all NSPLIT accumulator loads in flight, one wait, then the sum in
+                // accumulator order (two at a time, to bound the registers)
                 uint32_t v[16];
-                tmem_ld_x16(tmem_base + lane_addr + (uint32_t)(d * kAccCols + c0), v);
-                tmem_wait_ld();
+                constexpr int kLd = NSPLIT < 2 ? NSPLIT : 2;
 #pragma unroll
-                for (int sp = 1; sp < NSPLIT; ++sp) {
-                    uint32_t w2[16];
-                    tmem_ld_x16(tmem_base + lane_addr + (uint32_t)(d * kAccCols + sp * MT + c0), w2);
+                for (int sp0 = 0; sp0 < NSPLIT; sp0 += kLd) {
+                    uint32_t w2[kLd][16];
+#pragma unroll
+                    for (int sp = 0; sp < kLd; ++sp)
+                        tmem_ld_x16(tmem_base + lane_addr +
+                                        (uint32_t)(d * kAccCols + (sp0 + sp) * MT + c0),
+                                    w2[sp]);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int jj = 0; jj < 16; ++jj)
-                        v[jj] = __float_as_uint(__uint_as_float(v[jj]) + __uint_as_float(w2[jj]));
+                    for (int sp = 0; sp < kLd; ++sp)
+#pragma unroll
+                        for (int jj = 0; jj < 16; ++jj)
+                            v[jj] = (sp0 + sp == 0)
+                                        ? w2[0][jj]
+                                        : __float_as_uint(__uint_as_float(v[jj]) +
+                                                          __uint_as_float(w2[sp][jj]));
                 }
                 if (partial) {
                     // park this CTA's partial sums (fp32) for the row tile's last arriver
@@ -645,24 +682,39 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB), 1)
                     __threadfence();
                     const float *base =
                         p.ws_part + ((int64_t)rt * p.max_contrib * 128 + lrow) * MT;
+                    // 16 columns at a time: the four loads of one contribution are in
+                    // flight together, so the sum costs one memory round trip per
+                    // contribution rather than one per 4 columns
 #pragma unroll 1
-                    for (int c0 = 0; c0 < MT; c0 += 4) {
-                        float4 acc = __ldcg(reinterpret_cast<const float4 *>(base + c0));
+                    for (int c0 = 0; c0 < MT; c0 += 16) {
+                        float4 acc[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            acc[q] = __ldcg(reinterpret_cast<const float4 *>(base + c0) + q);
                         for (int ci = 1; ci < contrib; ++ci) {
-                            const float4 t = __ldcg(
-                                reinterpret_cast<const float4 *>(base + (int64_t)ci * 128 * MT + c0));
-                            acc.x += t.x;
-                            acc.y += t.y;
-                            acc.z += t.z;
-                            acc.w += t.w;
+                            float4 t[4];
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                t[q] = __ldcg(reinterpret_cast<const float4 *>(
+                                                  base + (int64_t)ci * 128 * MT + c0) + q);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                acc[q].x += t[q].x;
+                                acc[q].y += t[q].y;
+                                acc[q].z += t[q].z;
+                                acc[q].w += t[q].w;
+                            }
                         }
-                        const float av[4] = {acc.x, acc.y, acc.z, acc.w};
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
-                            const int64_t m = c0 + q;
-                            if (valid && m < p.M) {
-                                const __nv_bfloat16 h = __float2bfloat16_rn(av[q]);
-                                p.Y[m * p.N + row] = *reinterpret_cast<const uint16_t *>(&h);
+                            const float av[4] = {acc[q].x, acc[q].y, acc[q].z, acc[q].w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int64_t m = c0 + 4 * q + e;
+                                if (valid && m < p.M) {
+                                    const __nv_bfloat16 h = __float2bfloat16_rn(av[e]);
+                                    p.Y[m * p.N + row] = *reinterpret_cast<const uint16_t *>(&h);
+                                }
                             }
                         }
                     }
@@ -710,7 +762,7 @@ w4_status launch_cfg(const CUtensorMap &tw, const CUtensorMap &ts, const CUtenso
         configured = true;
     }
     const int grid = std::max(1, std::min(num_items_max, w4host::num_sms()));
-    kern<<<grid, gemm_threads(NDQ, KB), smem, stream>>>(tw, ts, tx, p);
+    kern<<<grid, gemm_threads(NDQ, KB, NSPLIT), smem, stream>>>(tw, ts, tx, p);
     return w4host::launch_status();
 }
 
@@ -850,8 +902,8 @@ extern "C" w4_status w4a16_gemm(const w4_bf16 *X, const int32_t *Wq, const w4_bf
             items = p.n_row_tiles;
             if (!map_x(mt) || !map_w(256, R) || !map_s(R)) return W4_ERR_CUDA;
         }
-        if (mt == 16) return launch_cfg<256, 16, 6, 1, 3, 4, 2, false>(tw, ts, tx, p, items, st);
-        if (mt == 32) return launch_cfg<256, 32, 6, 1, 3, 4, 2, false>(tw, ts, tx, p, items, st);
+        if (mt == 16) return launch_cfg<256, 16, 6, 2, 3, 4, 2, false>(tw, ts, tx, p, items, st);
+        if (mt == 32) return launch_cfg<256, 32, 6, 2, 2, 4, 2, false>(tw, ts, tx, p, items, st);
         return launch_cfg<256, 64, 4, 1, 2, 4, 2, false>(tw, ts, tx, p, items, st);
     }
     // Prefill (and any K that is not a multiple of 256): 128-row tiles,
