@@ -115,15 +115,31 @@ __device__ __forceinline__ bool next_item(ItemIter &I, const GemmParams &p, int 
                                           int &kb0, int &kb1) {
     if (I.cur >= I.end) return false;
     if (p.split) {
+        // The CTA's units [a, b) touch at most two row tiles (fewer units than
+        // k-blocks per tile).  The piece in the later tile (its first k-blocks)
+        // goes first: its partial sums are parked early, while the CTA works on
+        // the piece in the earlier tile (that tile's last k-blocks), which the
+        // previous CTA started first, so this CTA usually arrives last there and
+        // does the tile's fixup at its end with the other partials already
+        // parked.  I.step: 0 = later piece next, 1 = earlier piece next.
         const uint32_t nkb = (uint32_t)p.num_kb;
-        const uint32_t r = I.cur / nkb;
-        const uint32_t k0 = I.cur - r * nkb;
-        const uint32_t k1 = min(nkb, k0 + (I.end - I.cur));
-        rt = (int)r;
-        kb0 = (int)k0;
-        kb1 = (int)k1;
+        const uint32_t a = I.cur, b = I.end;
+        const uint32_t t1 = (b - 1) / nkb;
+        const uint32_t split_at = max(a, t1 * nkb);
+        if (I.step == 0) {
+            rt = (int)t1;
+            kb0 = (int)(split_at - t1 * nkb);
+            kb1 = (int)(b - t1 * nkb);
+            I.step = 1;
+            if (split_at == a) I.cur = I.end;       // a single piece
+        } else {
+            const uint32_t t0 = a / nkb;
+            rt = (int)t0;
+            kb0 = (int)(a - t0 * nkb);
+            kb1 = (int)(split_at - t0 * nkb);
+            I.cur = I.end;
+        }
         tt = 0;
-        I.cur += k1 - k0;
     } else {
         const uint32_t nrt = (uint32_t)p.n_row_tiles;
         const uint32_t q = I.cur / nrt;
@@ -134,6 +150,12 @@ __device__ __forceinline__ bool next_item(ItemIter &I, const GemmParams &p, int 
         I.cur += I.step;
     }
     return true;
+}
+
+__device__ __forceinline__ unsigned int atom_add_acq_rel_gpu(unsigned int *p, unsigned int v) {
+    unsigned int old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
 }
 
 // CTA that owns split unit x (CTA c owns [c*U/P, (c+1)*U/P)).
@@ -438,37 +460,19 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT), 1)
                 auto load_scales = [&](int j) -> uint32_t {
                     return KB == 256 ? lds32(s_stage(s) + lrow * 16 + j * 2) : 0u;
                 };
-                uint4 cur[2], nxt[2];
-                load_pair(0, cur);
-                uint32_t s_cur = load_scales(0);
-                if (!warp_wait(aempty_bar(a), ((it / NASTAGE) & 1u) ^ 1u, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after_sync();
-                const uint32_t a_col = tmem_base + lane_addr + (uint32_t)(kABase + a * kAStageCols);
                 // Two chunks (8 packed words) become 32 TMEM columns, 2 BF16 per column.
-                constexpr int kPairs = G / 2;
-#pragma unroll 1
-                for (int jp = 0; jp < kPairs; ++jp) {
-                    const int j = 2 * jp;
-                    uint32_t s_nxt = 0;
-                    if (jp + 1 < kPairs) {
-                        load_pair(j + 2, nxt);
-                        s_nxt = load_scales(j + 2);
-                    }
+                auto unpack_pair = [&](const uint4 (&w)[2], uint32_t s_pair, uint32_t (&o)[32]) {
                     uint32_t scp[2];
                     if (KB == 256) {
-                        scp[0] = bf16x2_splat((uint16_t)(s_cur & 0xFFFFu));
-                        scp[1] = bf16x2_splat((uint16_t)(s_cur >> 16));
+                        scp[0] = bf16x2_splat((uint16_t)(s_pair & 0xFFFFu));
+                        scp[1] = bf16x2_splat((uint16_t)(s_pair >> 16));
                     } else {
                         scp[0] = sc[0];     // G == 2: a single pair
                         scp[1] = sc[1];
                     }
-                    uint32_t o[32];
 #pragma unroll
                     for (int jj = 0; jj < 2; ++jj) {
-                        const uint32_t ws[4] = {cur[jj].x, cur[jj].y, cur[jj].z, cur[jj].w};
+                        const uint32_t ws[4] = {w[jj].x, w[jj].y, w[jj].z, w[jj].w};
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             uint32_t t4[4];
@@ -478,12 +482,31 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT), 1)
                             for (int z = 0; z < 4; ++z) o[jj * 16 + q * 4 + z] = t4[z];
                         }
                     }
-                    tmem_st_x32(a_col + (uint32_t)(j * 16), o);
+                };
+                // The first pair is unpacked before the A slot is known to be free,
+                // so the wait for the slot overlaps that arithmetic; each later
+                // pair is loaded and unpacked while the previous one is stored.
+                uint4 cur[2];
+                load_pair(0, cur);
+                uint32_t o[32];
+                unpack_pair(cur, load_scales(0), o);
+                if (!warp_wait(aempty_bar(a), ((it / NASTAGE) & 1u) ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t a_col = tmem_base + lane_addr + (uint32_t)(kABase + a * kAStageCols);
+                constexpr int kPairs = G / 2;
+#pragma unroll 1
+                for (int jp = 0; jp < kPairs; ++jp) {
+                    const int j = 2 * jp;
+                    uint32_t s_nxt = 0;
                     if (jp + 1 < kPairs) {
-                        cur[0] = nxt[0];
-                        cur[1] = nxt[1];
-                        s_cur = s_nxt;
+                        load_pair(j + 2, cur);
+                        s_nxt = load_scales(j + 2);
                     }
+                    tmem_st_x32(a_col + (uint32_t)(j * 16), o);
+                    if (jp + 1 < kPairs) unpack_pair(cur, s_nxt, o);
                 }
                 tmem_wait_st();
                 tc_fence_before_sync();
@@ -672,19 +695,21 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT), 1)
             if (partial) {
                 // The last of the row tile's contributing warps (per lane quarter)
                 // adds all partials in ascending K order and writes Y.
-                __threadfence();
+                // __syncwarp orders the lanes' partial stores before lane 0's
+                // count update, whose release makes them visible GPU-wide; the
+                // acquire side of the same update, then __syncwarp, orders the
+                // last arriver's reads of the other partials after it.
                 __syncwarp();
                 unsigned int *cnt = p.ws_cnt + (int64_t)rt * 4 + q4;
                 unsigned int old = 0;
-                if (lane == 0) old = atomicAdd(cnt, 1u);
+                if (lane == 0) old = atom_add_acq_rel_gpu(cnt, 1u);
                 old = __shfl_sync(0xFFFFFFFFu, old, 0);
                 if (old == (unsigned int)(contrib - 1)) {
-                    __threadfence();
+                    __syncwarp();
                     const float *base =
                         p.ws_part + ((int64_t)rt * p.max_contrib * 128 + lrow) * MT;
-                    // 16 columns at a time: the four loads of one contribution are in
-                    // flight together, so the sum costs one memory round trip per
-                    // contribution rather than one per 4 columns
+                    // 16 columns at a time, contributions in ascending K order: the
+                    // four loads of one contribution are in flight together
 #pragma unroll 1
                     for (int c0 = 0; c0 < MT; c0 += 16) {
                         float4 acc[4];
