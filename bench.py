@@ -49,7 +49,15 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # DRAM traffic per launch from ncu captures (dram__bytes_read.sum +
 # dram__bytes_write.sum), keyed by kernel; each entry records the SHA-256 of the
 # CUDA source it was measured on, so a changed kernel reports null.
-NCU_TRAFFIC = {}
+# DRAM bytes (read + write) per launch from one ncu capture of the kernel
+# (profiles/ holds the summaries and commands); an entry is used only while the
+# kernel's source file is unchanged since the capture.
+NCU_TRAFFIC = {
+    ("gemm_m16", "decode"): {"bytes": 28496896 + 0, "file": "w4_gemm.cu", "src": "3a1a84011c400dbf"},
+    ("fake_quant", "decode"): {"bytes": 100675072 + 51477248, "file": "w4_quant.cu", "src": "71486a6e4f64248c"},
+    ("ste_backward", "decode"): {"bytes": 100671232 + 50535936, "file": "w4_quant.cu", "src": "71486a6e4f64248c"},
+    ("quantize_pack", "decode"): {"bytes": 100687104 + 9147392, "file": "w4_quant.cu", "src": "71486a6e4f64248c"},
+}
 
 
 def _src_hash(fname: str) -> str:
@@ -470,6 +478,43 @@ def run_extra(args):
                     "gate_up_frac": b_gu / (t_gu * 1e-3) / 1e9 / peaks["hbm_gbs"],
                     "down_us": t_dn * 1e3, "down_GB/s": b_dn / (t_dn * 1e-3) / 1e9,
                     "down_frac": b_dn / (t_dn * 1e-3) / 1e9 / peaks["hbm_gbs"]})
+    elif args.workload == "gemv":
+        # the decode GEMM alone, one activation height at a time (--m picks one)
+        cfg = synth.Decode()
+        W = cfg.weight(dev)
+        Wq, S = w4.quantize_pack(W)
+        del W
+        for M in ([args.m] if args.m else cfg.Ms):
+            X = cfg.activations(M, dev)
+            Y = torch.empty((M, cfg.N), dtype=torch.bfloat16, device=dev)
+            fn = lambda: w4.w4a16_gemm(X, Wq, S, Y)
+            for _ in range(3):
+                fn()
+            med, p10, p90 = _time_kernel(fn, reps, flush)
+            nb = Wq.nbytes + S.nbytes + X.nbytes + Y.nbytes
+            gbs = nb / (med * 1e-3) / 1e9
+            out["results"].append({"M": M, "N": cfg.N, "K": cfg.K, "us": med * 1e3,
+                                   "p10_us": p10 * 1e3, "p90_us": p90 * 1e3,
+                                   "algorithmic_bytes": nb, "GB/s": gbs,
+                                   "frac": gbs / peaks["hbm_gbs"]})
+    elif args.workload == "quant":
+        # the decode-weight quantizers one at a time
+        cfg = synth.Decode()
+        W = cfg.weight(dev)
+        G = synth.normal_bf16(W.shape, 1e-3, 0, 1, dev)
+        Wdq, dW = torch.empty_like(W), torch.empty_like(W)
+        Wq = torch.empty((cfg.N, cfg.K // 8), dtype=torch.int32, device=dev)
+        S = torch.empty((cfg.N, cfg.K // 32), dtype=torch.bfloat16, device=dev)
+        n = W.numel()
+        for name, f, bpe in (("fake_quant", lambda: w4.w4_fake_quant(W, Wdq), 4.0),
+                             ("ste_backward", lambda: w4.w4_ste_backward(G, dW), 4.0),
+                             ("quantize_pack", lambda: w4.w4_quantize_pack(W, Wq, S), 2.5625)):
+            for _ in range(3):
+                f()
+            med, p10, p90 = _time_kernel(f, reps, flush)
+            gbs = n * bpe / (med * 1e-3) / 1e9
+            out["results"].append({"kernel": name, "elements": n, "us": med * 1e3,
+                                   "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"]})
     elif args.workload == "qat":
         cfg = synth.QATStack()
         mats = []
@@ -516,7 +561,9 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "moe", "qat"],
+    ap.add_argument("--m", type=int, default=0, help="--workload gemv: one activation height")
+    ap.add_argument("--workload", default="decode",
+                    choices=["decode", "prefill", "moe", "qat", "gemv", "quant"],
                     help="decode is the bench line; the others print their own lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=512)
