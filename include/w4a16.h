@@ -82,6 +82,16 @@ int w4_last_cuda_error(void);
  * the last call, W4_ERR_CUDA if the synchronization itself failed, else W4_OK. */
 w4_status w4_device_status(void *stream);
 
+/* Self-test of the bounded device waits (an operational check of this
+ * library; the pages have no counterpart).  Launches one warp on `stream`
+ * that waits on a shared-memory mbarrier phase nothing completes, with the
+ * same polling code as the GEMM's waits but a limit of `limit_us`
+ * microseconds (1 .. 1e6).  The wait gives up, records the timeout and the
+ * kernel exits, so the next w4_device_status() returns W4_ERR_TIMEOUT and the
+ * CUDA context stays usable.  No memory is touched outside the kernel's own
+ * shared memory.  Returns W4_ERR_INVALID_ARG for a limit out of range. */
+w4_status w4_wait_selftest(uint32_t limit_us, void *stream);
+
 /*
  * Fake quantization (QDQ) forward -- [QAT] fake quantization ("mapped to INT4
  * and immediately restored"), [TAG] [8][16], [BAS] §2.2.

@@ -25,7 +25,7 @@ import torch
 
 __all__ = [
     "W4Error", "lib", "workspace", "w4a16_gemm_workspace_bytes", "w4_version",
-    "w4_device_status", "w4_fake_quant", "w4_ste_backward",
+    "w4_device_status", "w4_wait_selftest", "w4_fake_quant", "w4_ste_backward",
     "w4_quantize_pack", "w4_dequant", "w4a16_gemm", "w4_moe_capacity", "w4_moe_align",
     "w4_moe_w4a16_gemm", "fake_quant", "quantize_pack", "dequant", "gemm", "moe_align",
     "moe_gemm", "FakeInt4STE", "GROUP",
@@ -74,6 +74,7 @@ def lib() -> ctypes.CDLL:
             "w4_moe_w4a16_gemm": [_P, _INT, _P, _P, _P, _P, _P, _I64, _INT, _I64, _P, _I64,
                                   _I64, _INT, _P],
             "w4_device_status": [_P],
+            "w4_wait_selftest": [ctypes.c_uint32, _P],
         }.items():
             f = getattr(L, name)
             f.argtypes = args
@@ -127,6 +128,12 @@ def w4_version() -> int:
 def w4_device_status(stream=None) -> None:
     """Synchronize the stream and raise if a kernel gave up a bounded wait."""
     _check("w4_device_status", lib().w4_device_status(_stream(stream)))
+
+
+def w4_wait_selftest(limit_us: int, stream=None) -> None:
+    """Launch the bounded-wait self-test (see include/w4a16.h); the next
+    w4_device_status() raises W4Error with status W4_ERR_TIMEOUT."""
+    _check("w4_wait_selftest", lib().w4_wait_selftest(int(limit_us), _stream(stream)))
 
 
 def w4_fake_quant(W, Wdq, S=None, group: int = GROUP, stream=None) -> None:

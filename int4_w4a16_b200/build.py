@@ -2,8 +2,9 @@
 
     python -m int4_w4a16_b200.build [--force]
 
-Every .cu under csrc/ is compiled with relocatable device code and linked by
-nvcc into ``int4_w4a16_b200/libw4a16.so``.  No fast-math: the quantizers rely
+Every .cu under csrc/ is compiled to a complete device image (no relocatable
+device code, so the compiler sees each kernel whole) and linked by nvcc into
+``int4_w4a16_b200/libw4a16.so``.  No fast-math: the quantizers rely
 on IEEE division / reciprocal and round-to-nearest-even conversions.
 """
 from __future__ import annotations
@@ -23,7 +24,7 @@ OBJ_DIR = os.path.join(HERE, "_build")
 HEADERS = [os.path.join(ROOT, "include", "w4a16.h")] + glob.glob(os.path.join(CSRC, "*.cuh"))
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-NVCC_FLAGS = ARCH + ["-O3", "-std=c++17", "-lineinfo", "-rdc=true", "-Xcompiler", "-fPIC",
+NVCC_FLAGS = ARCH + ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC",
                      "-Xcompiler", "-Wall", "--expt-relaxed-constexpr",
                      "-I" + os.path.join(ROOT, "include")]
 
@@ -69,7 +70,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
                     print(log)
     if force or jobs or not os.path.exists(OUT) or os.path.getmtime(OUT) < _newest(objs):
         tmp = OUT + ".tmp"
-        cmd = [nvcc(), *ARCH, "-shared", "-rdc=true", *objs, "-o", tmp]
+        cmd = [nvcc(), *ARCH, "-shared", *objs, "-o", tmp]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"nvcc link failed:\n{r.stderr}")

@@ -76,10 +76,8 @@ extern "C" w4_status w4_device_status(void *stream) {
         w4host::set_cuda_error(e);
         return W4_ERR_CUDA;
     }
-    unsigned int flag = 0, zero = 0;
-    e = cudaMemcpyFromSymbol(&flag, w4::g_device_status, sizeof flag);
-    if (e == cudaSuccess && flag != 0)
-        e = cudaMemcpyToSymbol(w4::g_device_status, &zero, sizeof zero);
+    unsigned int flag = 0;
+    e = w4host::gemm_device_status(&flag);
     if (e != cudaSuccess) {
         w4host::set_cuda_error(e);
         return W4_ERR_CUDA;

@@ -22,9 +22,11 @@ namespace w4 {
 
 // ---------------------------------------------------------------------------
 // Device status word: set (never cleared) by kernels, read/cleared by the host
-// through w4_device_status().
+// through w4_device_status().  Each translation unit has its own copy (the
+// library is built without relocatable device code); the one that kernels
+// set is the GEMM's, read through w4host::gemm_device_status.
 // ---------------------------------------------------------------------------
-extern __device__ unsigned int g_device_status;
+static __device__ unsigned int g_device_status = 0;
 
 constexpr unsigned int kStatusTimeout = 1u;
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
@@ -103,7 +105,8 @@ constexpr uint32_t kPollSleepNs = 32;
 
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile int *abort_flag,
-                                          uint32_t sleep_ns = kPollSleepNs) {
+                                          uint32_t sleep_ns = kPollSleepNs,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     for (uint32_t n = 1;; ++n) {
@@ -111,7 +114,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
         __nanosleep(sleep_ns);
         if (n % kPollsPerCheck == 0) {
             if (*abort_flag) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 record_timeout();
                 *abort_flag = 1;
                 return false;
@@ -383,6 +386,8 @@ __device__ __forceinline__ uint32_t bf16x2_splat(uint16_t s) {
 namespace w4host {
 
 void set_cuda_error(cudaError_t e);
+// Reads the GEMM translation unit's device status word into *flag and clears it.
+cudaError_t gemm_device_status(unsigned int *flag);
 
 inline bool aligned16(const void *p) {
     return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0;

@@ -839,6 +839,42 @@ bool plan_split(int64_t M, int64_t N, int64_t K, int sms, SplitPlan *sp) {
 }  // namespace
 }  // namespace w4
 
+namespace w4 {
+namespace {
+
+// One warp waits, with the GEMM's bounded wait, for a phase of an mbarrier
+// that nothing completes: the wait gives up after limit_ns, records the
+// timeout in the device status word and the kernel returns.
+__global__ void wait_selftest_kernel(unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1u);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncwarp();
+    mbar_wait(smem_u32(&bar), 0u, &abort_flag, kPollSleepNs, limit_ns);
+}
+
+}  // namespace
+}  // namespace w4
+
+extern "C" w4_status w4_wait_selftest(uint32_t limit_us, void *stream) {
+    if (limit_us == 0 || limit_us > 1000000u) return W4_ERR_INVALID_ARG;
+    w4::wait_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(1000ull * limit_us);
+    return w4host::launch_status();
+}
+
+cudaError_t w4host::gemm_device_status(unsigned int *flag) {
+    cudaError_t e = cudaMemcpyFromSymbol(flag, w4::g_device_status, sizeof *flag);
+    if (e == cudaSuccess && *flag != 0) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(w4::g_device_status, &zero, sizeof zero);
+    }
+    return e;
+}
+
 extern "C" size_t w4a16_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
     SplitPlan sp;
     if (M <= 0 || N <= 0 || K <= 0) return 0;

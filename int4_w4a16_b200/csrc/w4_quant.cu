@@ -42,8 +42,6 @@
 
 namespace w4 {
 
-__device__ unsigned int g_device_status = 0;
-
 namespace {
 
 constexpr float kSnap = 12288.0f;         // 1.5 * 2^13: ulp 2^-10 around it

@@ -72,6 +72,8 @@ def test_other_validation():
     assert L.w4_quantize_pack(A16, A16 + 0x100, A16 + 0x200, 4, 64, 8, None) == 2
     assert L.w4_dequant(A16, MIS, A16 + 0x100, 4, 64, 32, None) == 1
     assert L.w4_ste_backward(A16, MIS, 8, None) == 1
+    assert L.w4_wait_selftest(0, None) == 1                    # limit out of range
+    assert L.w4_wait_selftest(2000000, None) == 1
     assert L.w4_ste_backward(A16, A16, 8, None) == 0           # aliased: zero-copy no-op
     assert L.w4_ste_backward(A16, A16 + 2 * 8, 64, None) == 1  # partial overlap
     assert L.w4a16_gemm(A16, A16, A16, None, 1, 8, 64, 32, None, 0, None) == 1
