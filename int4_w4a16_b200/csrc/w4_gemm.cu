@@ -158,6 +158,12 @@ __device__ __forceinline__ unsigned int atom_add_acq_rel_gpu(unsigned int *p, un
     return old;
 }
 
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int *p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 // CTA that owns split unit x (CTA c owns [c*U/P, (c+1)*U/P)).
 __device__ __forceinline__ int unit_owner(uint32_t x, const GemmParams &p) {
     return (int)(((x + 1) * (uint32_t)p.ctas - 1) / (uint32_t)p.units);
@@ -486,10 +492,12 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT), 1)
                 // The first pair is unpacked before the A slot is known to be free,
                 // so the wait for the slot overlaps that arithmetic; each later
                 // pair is loaded and unpacked while the previous one is stored.
+                // Two output buffers alternate, so unpacking a pair never has to
+                // wait for the store of the previous pair to read its registers.
                 uint4 cur[2];
                 load_pair(0, cur);
-                uint32_t o[32];
-                unpack_pair(cur, load_scales(0), o);
+                uint32_t o[2][32];
+                unpack_pair(cur, load_scales(0), o[0]);
                 if (!warp_wait(aempty_bar(a), ((it / NASTAGE) & 1u) ^ 1u, abort_flag)) {
                     ok = false;
                     break;
@@ -497,7 +505,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT), 1)
                 tc_fence_after_sync();
                 const uint32_t a_col = tmem_base + lane_addr + (uint32_t)(kABase + a * kAStageCols);
                 constexpr int kPairs = G / 2;
-#pragma unroll 1
+#pragma unroll
                 for (int jp = 0; jp < kPairs; ++jp) {
                     const int j = 2 * jp;
                     uint32_t s_nxt = 0;
@@ -505,8 +513,8 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT), 1)
                         load_pair(j + 2, cur);
                         s_nxt = load_scales(j + 2);
                     }
-                    tmem_st_x32(a_col + (uint32_t)(j * 16), o);
-                    if (jp + 1 < kPairs) unpack_pair(cur, s_nxt, o);
+                    tmem_st_x32(a_col + (uint32_t)(j * 16), o[jp & 1]);
+                    if (jp + 1 < kPairs) unpack_pair(cur, s_nxt, o[(jp + 1) & 1]);
                 }
                 tmem_wait_st();
                 tc_fence_before_sync();
@@ -639,6 +647,20 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT), 1)
                 my_idx = blockIdx.x - c_first;
                 my_part = p.ws_part + (((int64_t)rt * p.max_contrib + my_idx) * 128 + lrow) * MT;
             }
+            unsigned int *cnt = partial ? p.ws_cnt + (int64_t)rt * 4 + q4 : nullptr;
+            // 16-column tiles: when every other contributor has already parked its
+            // partial (the usual case for the CTA's last item), this warp sums
+            // them with its own, still in registers, without parking or counting.
+            constexpr bool kDirect = MT == 16 && !MOE;
+            bool last_now = false;
+            uint32_t own[16];
+            if (kDirect && partial) {
+                unsigned int seen = 0;
+                if (lane == 0) seen = ld_acquire_gpu(cnt);
+                seen = __shfl_sync(0xFFFFFFFFu, seen, 0);
+                __syncwarp();
+                last_now = seen == (unsigned int)(contrib - 1);
+            }
 #pragma unroll 1
             for (int c0 = 0; c0 < MT; c0 += 16) {
                 // all NSPLIT accumulator loads in flight, one wait, then the sum in
@@ -664,6 +686,11 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT), 1)
                                                           __uint_as_float(w2[sp][jj]));
                 }
                 if (partial) {
+                    if (kDirect && last_now) {
+#pragma unroll
+                        for (int jj = 0; jj < 16; ++jj) own[jj] = v[jj];
+                        continue;
+                    }
                     // park this CTA's partial sums (fp32) for the row tile's last arriver
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
@@ -692,7 +719,38 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT), 1)
             }
             tc_fence_before_sync();
             mbar_arrive(accempty_bar(d));
-            if (partial) {
+            if (kDirect && partial && last_now) {
+                // Sum in ascending K order: the parked partials, with this CTA's own
+                // values in its place, then write Y and reset the counter.
+                const float *base = p.ws_part + ((int64_t)rt * p.max_contrib * 128 + lrow) * MT;
+                float acc[16];
+                for (int ci = 0; ci < contrib; ++ci) {
+                    if (ci == my_idx) {
+#pragma unroll
+                        for (int jj = 0; jj < 16; ++jj)
+                            acc[jj] = ci == 0 ? __uint_as_float(own[jj])
+                                              : acc[jj] + __uint_as_float(own[jj]);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float4 f = __ldcg(
+                                reinterpret_cast<const float4 *>(base + (int64_t)ci * 128 * MT) + q);
+                            const float fv[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                acc[4 * q + e] = ci == 0 ? fv[e] : acc[4 * q + e] + fv[e];
+                        }
+                    }
+                }
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                    if (valid && jj < p.M) {
+                        const __nv_bfloat16 h = __float2bfloat16_rn(acc[jj]);
+                        p.Y[(int64_t)jj * p.N + row] = *reinterpret_cast<const uint16_t *>(&h);
+                    }
+                }
+                if (lane == 0) *cnt = 0u;           // ready for the next call
+            } else if (partial) {
                 // The last of the row tile's contributing warps (per lane quarter)
                 // adds all partials in ascending K order and writes Y.
                 // __syncwarp orders the lanes' partial stores before lane 0's
@@ -700,7 +758,6 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT), 1)
                 // acquire side of the same update, then __syncwarp, orders the
                 // last arriver's reads of the other partials after it.
                 __syncwarp();
-                unsigned int *cnt = p.ws_cnt + (int64_t)rt * 4 + q4;
                 unsigned int old = 0;
                 if (lane == 0) old = atom_add_acq_rel_gpu(cnt, 1u);
                 old = __shfl_sync(0xFFFFFFFFu, old, 0);
