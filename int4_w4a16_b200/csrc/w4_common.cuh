@@ -199,6 +199,26 @@ __device__ __forceinline__ void tc_fence_after_sync() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+// Warpgroup register resizing; all four warps of a warpgroup execute it.
+// .inc waits until registers released by .dec elsewhere in the CTA cover it,
+// so a split must fit in what the CTA was launched with.
+template <int N>
+__device__ __forceinline__ void reg_alloc() {
+    static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg range");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void reg_dealloc() {
+    static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg range");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+// From the launch count LAUNCH to N: .inc above it, .dec below it.
+template <int N, int LAUNCH>
+__device__ __forceinline__ void reg_set() {
+    if constexpr (N > LAUNCH) reg_alloc<N>();
+    else if constexpr (N < LAUNCH) reg_dealloc<N>();
+}
+
 // D[tmem] (+)= A[tmem] * B[smem desc]; kind::f16 (BF16 inputs, FP32 accumulator).
 __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                           uint32_t idesc, uint32_t accumulate) {

@@ -41,6 +41,7 @@
 // exits.
 #include <algorithm>
 #include <mutex>
+#include <type_traits>
 
 #include "w4_common.cuh"
 
@@ -56,8 +57,29 @@ namespace {
 // about every 110 cycles (issue latency, not the tensor core), so small-N
 // tiles need several issuers to keep up with HBM.
 __host__ __device__ constexpr int perm_warps(int kb) { return kb == 256 ? 2 : 0; }
-__host__ __device__ constexpr int gemm_threads(int ndq, int kb, int nsplit) {
-    return 32 * (1 + 4 * ndq + perm_warps(kb) + 4 + nsplit);
+__host__ __device__ constexpr int gemm_threads(int ndq, int kb, int nsplit, bool wgl) {
+    return wgl ? 128 * (ndq + 4) : 32 * (1 + 4 * ndq + perm_warps(kb) + 4 + nsplit);
+}
+// Warpgroup layout (WGL, for the decode tiles that need eight issuers): aligned
+// warpgroups of four warps, each resizing its register file with setmaxnreg:
+//   WG 0 .. NDQ-1: dequant groups;  WG NDQ: epilogue;  WG NDQ+1, NDQ+2: up to
+//   eight MMA issuers;  WG NDQ+3: loads (warp 0, also the TMEM allocation) and
+//   the activation reorder (the next kPermWarps warps).
+// Each SM sub-partition holds one warp of every warpgroup, so its register
+// file is shared by ndq + 4 warps at launch; the dequant warpgroups take what
+// the others give back.
+__host__ __device__ constexpr int launch_regs_wgl(int ndq) {
+    return 16384 / (32 * (ndq + 4)) / 8 * 8;
+}
+constexpr int kRegsEpi = 88, kRegsIssue = 40, kRegsLoad = 64;
+__host__ __device__ constexpr int dequant_regs_wgl(int ndq) {
+    return (launch_regs_wgl(ndq) * (ndq + 4) - kRegsEpi - 2 * kRegsIssue - kRegsLoad) / ndq / 8 *
+           8;
+}
+// registers the split takes per sub-partition lane slot (checked on the host
+// against what the launch allocates: setmaxnreg.inc would wait forever otherwise)
+__host__ __device__ constexpr int split_regs_wgl(int ndq) {
+    return ndq * dequant_regs_wgl(ndq) + kRegsEpi + 2 * kRegsIssue + kRegsLoad;
 }
 constexpr int kTmemCols = 512;
 
@@ -246,8 +268,9 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 // NSPLIT: MMA issuers = accumulators per work item; 16-wide K step u goes to
 // issuer / accumulator u % NSPLIT, and the epilogue adds the accumulators in
 // a fixed order.
-template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT, int NDQ, bool MOE>
-__global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT), 1)
+template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT, int NDQ, bool MOE,
+          bool WGL>
+__global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
     w4a16_tc_kernel(const __grid_constant__ CUtensorMap tm_w,
                     const __grid_constant__ CUtensorMap tm_s,
                     const __grid_constant__ CUtensorMap tm_x, const GemmParams p) {
@@ -259,7 +282,12 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT), 1)
     constexpr int kDqWarps = 4 * NDQ;
     constexpr int kPermWarps = perm_warps(KB);
     constexpr int kEpiWarp0 = 1 + kDqWarps + kPermWarps;
-    static_assert(NSPLIT >= 1 && NSPLIT <= 8, "one to eight MMA issuers");
+    constexpr int kWgLoad = NDQ + 3;                        // (warpgroup layout)
+    constexpr int kAllocWarp = WGL ? 4 * kWgLoad : 0;      // loads + TMEM allocation
+    static_assert(NSPLIT >= 1 && NSPLIT <= (WGL ? 8 : 4), "MMA issuers");
+    static_assert(!WGL || (kPermWarps <= 3 && dequant_regs_wgl(NDQ) >= 96 &&
+                           split_regs_wgl(NDQ) <= launch_regs_wgl(NDQ) * (NDQ + 4)),
+                  "warpgroup register split");
     // 256-wide k-blocks (decode / MoE, few activation rows per tile): reorder the
     // activation chunks in shared memory instead of pairing the unpacked codes.
     constexpr bool kXPerm = (KB == 256);
@@ -312,7 +340,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT), 1)
         if (KB == 256) tma_prefetch_desc(&tm_s);
         if (!MOE) tma_prefetch_desc(&tm_x);
     }
-    if (warp == 0) {
+    if (warp == kAllocWarp) {
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
         tmem_relinquish();
     }
@@ -332,7 +360,8 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT), 1)
         num_items = p.n_row_tiles * p.n_tok_tiles;
     }
 
-    if (warp == 0) {
+    // ---- role bodies (inlined at each call site below)
+    auto role_loads = [&]() {
         // ------------------------------------------------------------ loads
         uint32_t it = 0;
         bool ok = true;
@@ -407,7 +436,9 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT), 1)
             const uint32_t first = it > (uint32_t)NSTAGE ? it - NSTAGE : 0u;
             for (uint32_t j = first; j < it; ++j) drain_wait(full_bar(j % NSTAGE), (j / NSTAGE) & 1u);
         }
-    } else if (warp < 1 + kDqWarps) {
+    };
+    // grp: dequant group in [0, NDQ)
+    auto role_dequant = [&](const uint32_t grp) {
         // --------------------------------------------------------- dequant
         // NDQ groups of 4 warps, one warp per TMEM lane quarter.  Group g takes
         // every NDQ-th k-block of the CTA's work in full, so one group's barrier
@@ -417,7 +448,6 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT), 1)
         constexpr int G = KB / 32;
         static_assert(G % 2 == 0, "chunks are stored in pairs (32 TMEM columns)");
         const int q4 = warp & 3;                    // TMEM lane quarter of this warp
-        const uint32_t grp = (uint32_t)(warp - 1) >> 2;   // group index in [0, NDQ)
         const int lrow = q4 * 32 + lane;            // A row of this thread
         const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
         const int64_t gpr = p.K / 32;               // groups per row
@@ -521,14 +551,15 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT), 1)
                 mbar_arrive(afull_bar(a));
             }
         }
-    } else if (warp < kEpiWarp0) {
+    };
+    // pw: index of the activation-reorder warp
+    auto role_perm = [&](const int pw) {
         // ------------------------------------------------ activation reorder
         // 256-wide k-blocks: the dequant warps leave codes (j, j + 4) of a packed
         // word in one register pair (dequant_word_k8perm), so every 16-byte
         // activation chunk [x0..x7] of the stage is rewritten in place as
         // [x0, x4, x1, x5, x2, x6, x3, x7].  These warps issue no asynchronous
         // copies or MMAs, so their proxy fence waits only for their own stores.
-        const int pw = warp - 1 - kDqWarps;
         uint32_t it = 0;
         bool ok = true;
         ItemIter I = make_iter(p, num_items);
@@ -573,12 +604,14 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT), 1)
                 mbar_arrive(afull_bar(a));
             }
         }
-    } else {
+    };
+    // kIss: std::true_type for an MMA issuer (index ji), std::false_type for an
+    // epilogue warp; each instantiation keeps only its own role's code
+    auto role_mma = [&](auto kIss, const int ji) {
         // ------------------------------------------------- MMA + epilogue
         // four epilogue warps (one per TMEM lane quarter), then NSPLIT MMA issuers:
         // the epilogue of one work item overlaps the MMAs of the next
-        const int ji = warp - kEpiWarp0 - 4;        // issuer index, < 0 for the epilogue
-        const bool issuer = ji >= 0;                // warp-uniform
+        constexpr bool issuer = decltype(kIss)::value;
         const int q4 = warp & 3;
         const int lrow = q4 * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
@@ -588,7 +621,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT), 1)
         int rt, tt, kb0, kb1;
         for (; ok && next_item(I, p, rt, tt, kb0, kb1); ++acc_it) {
             const int d = acc_it % NACC;
-            if (issuer) {
+            if constexpr (issuer) {
                 if (!warp_wait(accempty_bar(d), ((acc_it / NACC) & 1u) ^ 1u, abort_flag, kSleepAhead)) {
                     ok = false;
                     break;
@@ -805,18 +838,47 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT), 1)
             }
         }
         // all MMAs issued by this warp complete before TMEM is released
-        if (issuer) {
+        if constexpr (issuer) {
             if (lane == 0) {
                 tc_commit(mmadone_bar);
                 drain_wait(mmadone_bar, 0u);
             }
             __syncwarp();
         }
+    };
+
+    if constexpr (WGL) {
+        // Each warpgroup first resizes its register file (every warp of the
+        // warpgroup executes its setmaxnreg), so the compiler fits each role
+        // into that count.
+        const int wg = warp >> 2;
+        constexpr int kLaunch = launch_regs_wgl(NDQ);
+        if (wg == kWgLoad) {
+            reg_set<kRegsLoad, kLaunch>();
+            if (warp == kAllocWarp) role_loads();
+            else if (warp - kAllocWarp <= kPermWarps) role_perm(warp - kAllocWarp - 1);
+        } else if (wg < NDQ) {
+            reg_set<dequant_regs_wgl(NDQ), kLaunch>();
+            role_dequant((uint32_t)wg);
+        } else if (wg == NDQ) {
+            reg_set<kRegsEpi, kLaunch>();
+            role_mma(std::false_type{}, -1);
+        } else {
+            reg_set<kRegsIssue, kLaunch>();
+            const int ji = warp - 4 * (NDQ + 1);
+            if (ji < NSPLIT) role_mma(std::true_type{}, ji);
+        }
+    } else {
+        if (warp == 0) role_loads();
+        else if (warp < 1 + kDqWarps) role_dequant((uint32_t)(warp - 1) >> 2);
+        else if (warp < kEpiWarp0) role_perm(warp - 1 - kDqWarps);
+        else if (warp < kEpiWarp0 + 4) role_mma(std::false_type{}, -1);
+        else role_mma(std::true_type{}, warp - kEpiWarp0 - 4);
     }
 
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == kAllocWarp) {
         tc_fence_after_sync();
         tmem_dealloc(tmem_base, kTmemCols);
     }
@@ -826,11 +888,12 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT), 1)
 // Host side
 // ---------------------------------------------------------------------------
 
-template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT, int NDQ, bool MOE>
+template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT, int NDQ, bool MOE,
+          bool WGL = false>
 w4_status launch_cfg(const CUtensorMap &tw, const CUtensorMap &ts, const CUtensorMap &tx,
                      const GemmParams &p, int num_items_max, cudaStream_t stream) {
     using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE, NSPLIT>;
-    auto kern = w4a16_tc_kernel<KB, MT, NSTAGE, NACC, NASTAGE, NSPLIT, NDQ, MOE>;
+    auto kern = w4a16_tc_kernel<KB, MT, NSTAGE, NACC, NASTAGE, NSPLIT, NDQ, MOE, WGL>;
     // At least half of the SM's shared memory, so one CTA (and one TMEM
     // allocation of 512 columns) per SM.
     const int smem = std::max(L::kAlloc, 120 * 1024);
@@ -843,8 +906,21 @@ w4_status launch_cfg(const CUtensorMap &tw, const CUtensorMap &ts, const CUtenso
             return w4host::launch_status();
         configured = true;
     }
+    if (WGL) {
+        // setmaxnreg draws on the registers the CTA was launched with: refuse to
+        // launch (rather than wait forever) if the build gave fewer than the
+        // split needs.
+        static int regs_built = -1;
+        if (regs_built < 0) {
+            cudaFuncAttributes fa;
+            if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return w4host::launch_status();
+            regs_built = fa.numRegs;
+        }
+        if (regs_built * gemm_threads(NDQ, KB, NSPLIT, WGL) < 128 * split_regs_wgl(NDQ))
+            return W4_ERR_UNSUPPORTED;
+    }
     const int grid = std::max(1, std::min(num_items_max, w4host::num_sms()));
-    kern<<<grid, gemm_threads(NDQ, KB, NSPLIT), smem, stream>>>(tw, ts, tx, p);
+    kern<<<grid, gemm_threads(NDQ, KB, NSPLIT, WGL), smem, stream>>>(tw, ts, tx, p);
     return w4host::launch_status();
 }
 
@@ -1020,8 +1096,8 @@ extern "C" w4_status w4a16_gemm(const w4_bf16 *X, const int32_t *Wq, const w4_bf
             items = p.n_row_tiles;
             if (!map_x(mt) || !map_w(256, R) || !map_s(R)) return W4_ERR_CUDA;
         }
-        if (mt == 16) return launch_cfg<256, 16, 6, 2, 3, 4, 2, false>(tw, ts, tx, p, items, st);
-        if (mt == 32) return launch_cfg<256, 32, 6, 2, 2, 4, 2, false>(tw, ts, tx, p, items, st);
+        if (mt == 16) return launch_cfg<256, 16, 6, 1, 3, 8, 2, false, true>(tw, ts, tx, p, items, st);
+        if (mt == 32) return launch_cfg<256, 32, 6, 1, 2, 8, 2, false, true>(tw, ts, tx, p, items, st);
         return launch_cfg<256, 64, 4, 1, 2, 4, 2, false>(tw, ts, tx, p, items, st);
     }
     // Prefill (and any K that is not a multiple of 256): 128-row tiles,
