@@ -46,14 +46,12 @@ import synth  # noqa: E402
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
-# DRAM traffic per launch from ncu captures (dram__bytes_read.sum +
-# dram__bytes_write.sum), keyed by kernel; each entry records the SHA-256 of the
-# CUDA source it was measured on, so a changed kernel reports null.
 # DRAM bytes (read + write) per launch from one ncu capture of the kernel
 # (profiles/ holds the summaries and commands); an entry is used only while the
 # kernel's source file is unchanged since the capture.
 NCU_TRAFFIC = {
-    ("gemm_m16", "decode"): {"bytes": 28496896 + 0, "file": "w4_gemm.cu", "src": "3a1a84011c400dbf"},
+    ("gemm_m16", "decode"): {"bytes": 28509696 + 0, "file": "w4_gemm.cu", "src": "54b19eef2ee33544"},
+    ("gemm_m1", "decode"): {"bytes": 28345088 + 0, "file": "w4_gemv.cu", "src": "d7c1dfe0481fe22a"},
     ("fake_quant", "decode"): {"bytes": 100675072 + 51477248, "file": "w4_quant.cu", "src": "71486a6e4f64248c"},
     ("ste_backward", "decode"): {"bytes": 100671232 + 50535936, "file": "w4_quant.cu", "src": "71486a6e4f64248c"},
     ("quantize_pack", "decode"): {"bytes": 100687104 + 9147392, "file": "w4_quant.cu", "src": "71486a6e4f64248c"},

@@ -76,8 +76,10 @@ extern "C" w4_status w4_device_status(void *stream) {
         w4host::set_cuda_error(e);
         return W4_ERR_CUDA;
     }
-    unsigned int flag = 0;
+    unsigned int flag = 0, flag_gemv = 0;
     e = w4host::gemm_device_status(&flag);
+    if (e == cudaSuccess) e = w4host::gemv_device_status(&flag_gemv);
+    flag |= flag_gemv;
     if (e != cudaSuccess) {
         w4host::set_cuda_error(e);
         return W4_ERR_CUDA;

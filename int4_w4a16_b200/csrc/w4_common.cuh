@@ -408,6 +408,14 @@ namespace w4host {
 void set_cuda_error(cudaError_t e);
 // Reads the GEMM translation unit's device status word into *flag and clears it.
 cudaError_t gemm_device_status(unsigned int *flag);
+// Same for the warp-level MMA (decode) translation unit.
+cudaError_t gemv_device_status(unsigned int *flag);
+
+// Decode-shaped W4A16 GEMM on the warp-level MMA path (w4_gemv.cu): whether it
+// takes the shape, and the launch (arguments already validated by the caller).
+bool gemv_supported(int64_t M, int64_t N, int64_t K);
+w4_status gemv_launch(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S, w4_bf16 *Y,
+                      int64_t M, int64_t N, int64_t K, void *stream);
 
 inline bool aligned16(const void *p) {
     return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0;

@@ -1011,6 +1011,7 @@ cudaError_t w4host::gemm_device_status(unsigned int *flag) {
 extern "C" size_t w4a16_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
     SplitPlan sp;
     if (M <= 0 || N <= 0 || K <= 0) return 0;
+    if (w4host::gemv_supported(M, N, K)) return 0;
     if (!plan_split(M, N, K, w4host::num_sms(), &sp)) return 0;
     return sp.cnt_bytes + sp.part_bytes;
 }
@@ -1028,6 +1029,12 @@ extern "C" w4_status w4a16_gemm(const w4_bf16 *X, const int32_t *Wq, const w4_bf
     if (M == 0 || N == 0) return W4_OK;
     if (N > (1 << 30) || M > (1 << 30) || K > (1 << 24)) return W4_ERR_UNSUPPORTED;
     cudaStream_t st = (cudaStream_t)stream;
+    // 1..8 activation rows: the warp-level MMA kernel unpacks straight into
+    // MMA fragments (w4_gemv.cu), no tensor memory.
+    if (w4host::gemv_supported(M, N, K)) {
+        const w4_status gs = w4host::gemv_launch(X, Wq, S, Y, M, N, K, stream);
+        if (gs != W4_ERR_UNSUPPORTED) return gs;     // else: too many rows per SM, below
+    }
 
     GemmParams p = {};
     p.S = reinterpret_cast<const uint16_t *>(S);

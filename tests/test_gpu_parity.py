@@ -248,16 +248,17 @@ def _decode_weight():
     return _DECODE["w"]
 
 
-@pytest.mark.parametrize("split", [True, False])
-@pytest.mark.parametrize("M", [1, 8, 16, 32, 64])
+@pytest.mark.parametrize("M,split", [(1, False), (8, False), (16, True), (16, False),
+                                     (32, True), (32, False), (64, True), (64, False)])
 def test_gemm_decode_config(M, split):
-    """Decode GEMV sweep, with the stream-K split (workspace) and without."""
+    """Decode GEMV sweep: 1..8 rows take the warp-level MMA kernel (no
+    workspace); 16..64 rows the tensor-memory kernel, with the stream-K split
+    (workspace) and without."""
     cfg = synth.Decode()
     Wq, S = _decode_weight()
     X = cfg.activations(M)
     ws = "auto" if split else None
-    if split:
-        assert w4.w4a16_gemm_workspace_bytes(M, cfg.N, cfg.K) > 0
+    assert (w4.w4a16_gemm_workspace_bytes(M, cfg.N, cfg.K) > 0) == (M > 8)
     Y = bits(w4.gemm(X.to(DEV), torch.from_numpy(Wq).to(DEV), _np_bf16(S).to(DEV), ws=ws))
     _, R = oracle.w4a16_gemm(bits(X), Wq, S)
     assert_gemm_close(Y, R, f"decode M={M} split={split}")
