@@ -177,8 +177,10 @@ class DecodeWorkload:
             self.flops[f"gemm_m{M}"] = 2 * M * N * K
         self.launches_per_step = 3 + len(self.Ms)
 
-    def step(self, ev=None):
-        """One pass; ev (optional) = {kernel: (start_event, end_event)} to record."""
+    def step(self, ev=None, gemm_ev=None):
+        """One pass; ev (optional) = {kernel: (start_event, end_event)} to record
+        around each launch; gemm_ev (optional) = (start, end) recorded once
+        around the decode GEMM launches together."""
         w4 = self.w4
         i = self.step_idx
         self.step_idx += 1
@@ -194,9 +196,13 @@ class DecodeWorkload:
         rec("fake_quant", lambda: w4.w4_fake_quant(W, self.Wdq))
         rec("ste_backward", lambda: w4.w4_ste_backward(G, self.dW))
         rec("quantize_pack", lambda: w4.w4_quantize_pack(W, self.Wq, self.S))
+        if gemm_ev is not None:
+            gemm_ev[0].record()
         for j, M in enumerate(self.Ms):
             Wq, S = self.copies[(4 * i + j) % len(self.copies)]
             rec(f"gemm_m{M}", lambda: w4.w4a16_gemm(self.X[M], Wq, S, self.Y[M]))
+        if gemm_ev is not None:
+            gemm_ev[1].record()
 
     def e2e_step(self, host):
         """Same pass through the public API from pinned host buffers, with the
@@ -511,6 +517,10 @@ def run_extra(args):
         W = cfg.weight(dev)
         Wq, S = w4.quantize_pack(W)
         del W
+        # 16 copies of the packed weight (453 MB, several times the L2) for the
+        # rotation measurement below
+        n_rot = 16
+        rot = [(Wq.clone(), S.clone()) for _ in range(n_rot)]
         for M in ([args.m] if args.m else cfg.Ms):
             X = cfg.activations(M, dev)
             Y = torch.empty((M, cfg.N), dtype=torch.bfloat16, device=dev)
@@ -520,10 +530,19 @@ def run_extra(args):
             med, p10, p90 = _time_kernel(fn, reps, flush)
             nb = Wq.nbytes + S.nbytes + X.nbytes + Y.nbytes
             gbs = nb / (med * 1e-3) / 1e9
+            # the same GEMM over the 16 copies in turn, one CUDA graph between one
+            # event pair: every launch reads weights that are not in L2, and no
+            # flush kernel or event sits between launches
+            rot_fn = lambda: [w4.w4a16_gemm(X, q, s_, Y) for q, s_ in rot]
+            rot_fn()
+            rmed, _, _ = _time_kernel(rot_fn, max(5, reps // 4), lambda: None)
+            rus = rmed * 1e3 / n_rot
             out["results"].append({"M": M, "N": cfg.N, "K": cfg.K, "us": med * 1e3,
                                    "p10_us": p10 * 1e3, "p90_us": p90 * 1e3,
                                    "algorithmic_bytes": nb, "GB/s": gbs,
-                                   "frac": gbs / peaks["hbm_gbs"]})
+                                   "frac": gbs / peaks["hbm_gbs"],
+                                   "rotated_us_per_launch": rus,
+                                   "rotated_frac": nb / (rus * 1e-6) / 1e9 / peaks["hbm_gbs"]})
     elif args.workload == "quant":
         # the decode-weight quantizers one at a time
         cfg = synth.Decode()
@@ -624,24 +643,40 @@ def main():
         wl.step()                       # eager warm-up (also sizes the GEMM workspace)
     w4.w4_device_status()
 
-    # The timed steps run as one CUDA graph: K steps, each kernel bracketed by
-    # timing events captured into the graph, so host launch overhead is not in
-    # `value` (the e2e figure below goes through the eager public API instead).
+    # The timed steps run as one CUDA graph of K steps with no event inside, so
+    # neither host launch overhead nor event records are in `value` (the e2e
+    # figure below goes through the eager public API instead).  Two more graphs
+    # of the same K steps, replayed after it, give the breakdown: one with an
+    # event pair around every launch (per-kernel times), one with a single
+    # event pair around each step's decode GEMM launches (the GEMM family).
     def ev():
         return torch.cuda.Event(enable_timing=True, external=True)
 
-    def capture(nsteps, with_events):
-        evs = [{k: (ev(), ev()) for k in wl.kernels} for _ in range(nsteps)] if with_events else None
+    def capture(nsteps, mode):
+        evs = None
+        if mode == "kernel":
+            evs = [{k: (ev(), ev()) for k in wl.kernels} for _ in range(nsteps)]
+        elif mode == "gemm":
+            evs = [(ev(), ev()) for _ in range(nsteps)]
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             for i in range(nsteps):
-                wl.step(evs[i] if evs else None)
+                if mode == "kernel":
+                    wl.step(evs[i])
+                elif mode == "gemm":
+                    wl.step(None, evs[i])
+                else:
+                    wl.step()
         return g, evs
 
-    roll, _ = capture(8, False)
-    timed, evs = capture(args.steps, True)
+    roll, _ = capture(8, None)
+    timed, _ = capture(args.steps, None)
+    timed_k, evs = capture(args.steps, "kernel")
+    timed_g, gevs = capture(args.steps, "gemm")
     for _ in range(max(3, args.warmup)):
         roll.replay()
+    timed_k.replay()
+    timed_g.replay()
     torch.cuda.synchronize()
 
     sampler = ClockSampler(local) if rank == 0 else None
@@ -663,6 +698,10 @@ def main():
     torch.cuda.synchronize()
     barrier(world)
     elapsed_ms = t0.elapsed_time(t1)
+    # the breakdown graphs, under the same load
+    timed_k.replay()
+    timed_g.replay()
+    torch.cuda.synchronize()
     # post-roll for the sampler
     t_end = time.perf_counter() + 0.4
     while time.perf_counter() < t_end:
@@ -690,7 +729,8 @@ def main():
         if k in wl.flops:
             r["tflops"] = wl.flops[k] / (per[k] * 1e-3) / 1e12
         rooflines[k] = r
-    gemm_us = sum(per[k] for k in wl.kernels if k.startswith("gemm")) * 1e3
+    gemm_us = sum(a.elapsed_time(b) for a, b in gevs) / len(gevs) * 1e3
+    gemm_us_per_kernel_sum = sum(per[k] for k in wl.kernels if k.startswith("gemm")) * 1e3
     gemm_bytes = sum(wl.bytes[k] for k in wl.kernels if k.startswith("gemm"))
     # The dominant kernel is the one with the largest share of the step; the four
     # decode GEMM launches (one kernel at four activation heights) count together.
@@ -703,8 +743,9 @@ def main():
                         "frac": gbs / peaks["hbm_gbs"],
                         "traffic": _traffic("gemm_m16", "decode"),
                         "note": "decode GEMM, launches at M = 1, 8, 16, 32 together: "
-                                "algorithmic bytes summed over the four / their summed "
-                                "event time; traffic is the M = 16 launch's"}
+                                "algorithmic bytes summed over the four / the time between "
+                                "one event pair around the four launches; traffic is the "
+                                "M = 16 launch's"}
     else:
         dom_roofline = {k: v for k, v in rooflines[dominant].items()
                         if k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
@@ -740,12 +781,14 @@ def main():
             "rooflines": rooflines,
             "decode_gemm": {"GB/s": gemm_bytes / (gemm_us * 1e-6) / 1e9,
                             "frac": gemm_bytes / (gemm_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
-                            "us_sum_4M": gemm_us},
+                            "us_4M_one_event_pair": gemm_us,
+                            "us_4M_sum_of_per_kernel_events": gemm_us_per_kernel_sum},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": wl.launches_per_step * args.steps,
-            "launch": "timed steps replayed as one CUDA graph (per-kernel events inside)",
+            "launch": "timed steps replayed as one CUDA graph with no events inside; per-kernel "
+                      "and GEMM-family times from two more replays of the same steps with events",
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
