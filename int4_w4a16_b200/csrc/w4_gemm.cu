@@ -94,7 +94,9 @@ struct GemmParams {
     int64_t num_slots;           // MoE
     int64_t a_rows;              // MoE
     int a_row_div;               // MoE
-    int cap_blocks;              // MoE: length of expert_ids (bounds num_post_pad / MT)
+    int cap_blocks;              // MoE: length of expert_ids (bounds num_post_pad / block)
+    int moe_sub;                 // MoE: MT-slot sub-blocks per aligned block (block / MT)
+    int moe_mt;                  // MoE: MT (slots per work item)
     int rows_per_tile;           // R <= 128
     int n_row_tiles;
     int n_tok_tiles;             // dense
@@ -164,12 +166,20 @@ __device__ __forceinline__ bool next_item(ItemIter &I, const GemmParams &p, int 
         tt = 0;
     } else {
         const uint32_t nrt = (uint32_t)p.n_row_tiles;
-        const uint32_t q = I.cur / nrt;
-        rt = (int)(I.cur - q * nrt);
-        tt = (int)q;
+        for (;;) {
+            const uint32_t q = I.cur / nrt;
+            rt = (int)(I.cur - q * nrt);
+            tt = (int)q;
+            I.cur += I.step;
+            // MoE: a sub-block whose first slot is padding is padding throughout
+            // (an expert's run holds its real slots first); every role skips it
+            if (p.sorted_ids == nullptr || p.moe_sub == 1) break;
+            const int32_t first = __ldg(p.sorted_ids + (int64_t)tt * p.moe_mt);
+            if (first >= 0 && first < p.num_slots) break;
+            if (I.cur >= I.end) return false;
+        }
         kb0 = 0;
         kb1 = p.num_kb;
-        I.cur += I.step;
     }
     return true;
 }
@@ -354,7 +364,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
     int num_items;
     if (MOE) {
         const int npp = *p.num_post_pad;
-        const int nblocks = min(max(npp, 0) / MT, p.cap_blocks);
+        const int nblocks = min(max(npp, 0) / MT, p.cap_blocks * p.moe_sub);
         num_items = nblocks * p.n_row_tiles;
     } else {
         num_items = p.n_row_tiles * p.n_tok_tiles;
@@ -374,7 +384,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
             // lane t % 32 of register t / 32, loaded once per work item
             int gather_row[(MT + 31) / 32];
             if (MOE) {
-                expert = __ldg(p.expert_ids + tt);
+                expert = __ldg(p.expert_ids + tt / p.moe_sub);
 #pragma unroll
                 for (int r = 0; r < (MT + 31) / 32; ++r) {
                     const int t = r * 32 + lane;
@@ -461,7 +471,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
             const uint16_t *srow = nullptr;
             if (KB != 256 && valid) {
                 int64_t base = row * gpr;
-                if (MOE) base += (int64_t)__ldg(p.expert_ids + tt) * p.N * gpr;
+                if (MOE) base += (int64_t)__ldg(p.expert_ids + tt / p.moe_sub) * p.N * gpr;
                 srow = p.S + base;
             }
             for (int kb = kb0; kb < kb1; ++kb, ++it) {
@@ -1182,11 +1192,24 @@ extern "C" w4_status w4_moe_w4a16_gemm(const w4_bf16 *A, int a_row_div, const in
                       CU_TENSOR_MAP_SWIZZLE_NONE))
             return W4_ERR_CUDA;
     }
-    const int64_t items_max = (cap / block) * p.n_row_tiles;
+    // 32-slot blocks that the routing fills on average (>= 16 slots per expert)
+    // run as they are.  Otherwise every block size runs on 16-slot work items:
+    // an aligned block of 32 or 64 slots is block / 16 sub-blocks of the same
+    // expert, and sub-blocks that hold only padding are skipped, so a wide
+    // block costs what its real slots need (at decode sizes most of a wide
+    // block is padding).
+    if (block == 32 && num_slots >= 16 * E) {
+        p.moe_mt = 32;
+        p.moe_sub = 1;
+        const int64_t items_max = (cap / 32) * p.n_row_tiles;
+        const int items = (int)std::min<int64_t>(items_max, 1 << 30);
+        return launch_cfg<256, 32, 6, 2, 2, 4, 2, true>(tw, ts, tx, p, items, st);
+    }
+    p.moe_mt = 16;
+    p.moe_sub = block / 16;
+    const int64_t items_max = (cap / 16) * p.n_row_tiles;
     const int items = (int)std::min<int64_t>(items_max, 1 << 30);
-    if (block == 16) return launch_cfg<256, 16, 6, 2, 3, 4, 2, true>(tw, ts, tx, p, items, st);
-    if (block == 32) return launch_cfg<256, 32, 6, 2, 2, 4, 2, true>(tw, ts, tx, p, items, st);
-    return launch_cfg<256, 64, 4, 1, 2, 4, 2, true>(tw, ts, tx, p, items, st);
+    return launch_cfg<256, 16, 6, 2, 3, 4, 2, true>(tw, ts, tx, p, items, st);
 }
 
 // ---------------------------------------------------------------------------

@@ -379,6 +379,16 @@ def test_moe_gemm_down(T, block):
     assert_gemm_close(C, R, f"moe down T={T} block={block}")
 
 
+@pytest.mark.parametrize("T,E,block", [(64, 8, 32), (40, 8, 64), (48, 16, 32)])
+def test_moe_gemm_dense_routing(T, E, block):
+    """Few experts, many slots each: 32-slot blocks that the routing fills
+    (>= 16 slots per expert) run as 32-slot work items; wider or emptier blocks
+    run as 16-slot sub-blocks with the all-padding ones skipped."""
+    C, R, _ = _moe_case(T, block, N=700, K=1024, E=E, seed=7 * T + E)
+    assert not np.any(C == 0x7FC1), "a real slot was left unwritten"
+    assert_gemm_close(C, R, f"moe T={T} E={E} block={block}")
+
+
 def test_moe_gemm_padding_rows_untouched():
     """Slots that no expert owns (routing ids out of range) keep the canary."""
     E, N, K, T, topk, block = 8, 256, 512, 10, 2, 16
