@@ -50,7 +50,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # (profiles/ holds the summaries and commands); an entry is used only while the
 # kernel's source file is unchanged since the capture.
 NCU_TRAFFIC = {
-    ("gemm_m16", "decode"): {"bytes": 28509696 + 0, "file": "w4_gemm.cu", "src": "54b19eef2ee33544"},
+    ("gemm_m16", "decode"): {"bytes": 28512768 + 0, "file": "w4_gemm.cu", "src": "8c6da770ed6d02e8"},
     ("gemm_m1", "decode"): {"bytes": 28345088 + 0, "file": "w4_gemv.cu", "src": "d7c1dfe0481fe22a"},
     ("fake_quant", "decode"): {"bytes": 100675072 + 51477248, "file": "w4_quant.cu", "src": "71486a6e4f64248c"},
     ("ste_backward", "decode"): {"bytes": 100671232 + 50535936, "file": "w4_quant.cu", "src": "71486a6e4f64248c"},
@@ -453,7 +453,7 @@ def run_extra(args):
         W = cfg.weight(dev)
         Wq, S = w4.quantize_pack(W)
         del W
-        for M in cfg.Ms:
+        for M in ([args.m] if args.m else cfg.Ms):
             X = cfg.activations(M, dev)
             Y = torch.empty((M, cfg.N), dtype=torch.bfloat16, device=dev)
             fn = lambda: w4.w4a16_gemm(X, Wq, S, Y)
@@ -481,13 +481,13 @@ def run_extra(args):
         del Wg, Wd
         per_gu = 2 * cfg.inter * cfg.hidden * 9 // 16
         per_dn = cfg.hidden * cfg.inter * 9 // 16
-        for T in cfg.Ts:
+        for T in ([args.m] if args.m else cfg.Ts):
             ids, _ = cfg.routing(T)
             ids_d = ids.to(dev)
             active = len(set(ids.view(-1).tolist()))
             X = cfg.tokens(T, dev)
             H = synth.normal_bf16((T * cfg.topk, cfg.inter), 1.0, 0, 300 + T, dev)
-            for block in cfg.blocks:
+            for block in ([args.block] if args.block else cfg.blocks):
                 s_ids, e_ids, npp = w4.moe_align(ids_d, E, block)
                 C1 = torch.empty((T * cfg.topk, 2 * cfg.inter), dtype=torch.bfloat16, device=dev)
                 C2 = torch.empty((T * cfg.topk, cfg.hidden), dtype=torch.bfloat16, device=dev)
@@ -612,7 +612,10 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--m", type=int, default=0, help="--workload gemv: one activation height")
+    ap.add_argument("--m", type=int, default=0,
+                    help="one size only: the activation height (--workload gemv, prefill) or "
+                         "the token count T (--workload moe)")
+    ap.add_argument("--block", type=int, default=0, help="--workload moe: one block size only")
     ap.add_argument("--workload", default="decode",
                     choices=["decode", "prefill", "moe", "qat", "gemv", "quant"],
                     help="decode is the bench line; the others print their own lines")
