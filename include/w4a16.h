@@ -221,6 +221,65 @@ w4_status w4_moe_w4a16_gemm(const w4_bf16 *A, int a_row_div, const int32_t *Wq,
                             int64_t cap, int block, int64_t num_slots, w4_bf16 *C,
                             int64_t N, int64_t K, int E, void *stream);
 
+/*
+ * ---------------------------------------------------------------------------
+ * MoE layer around the grouped GEMMs.  The pages name the pieces without
+ * defining them: a fused gating kernel (softmax + top-k), a block size chosen
+ * from the token count and the expert histogram, and the fusion of the MoE
+ * operators ([QAT] "moe_align_block_size", "MoE operator deep fusion"; [TAG]
+ * [35]).  The readings below are the plainest ones the pages allow.
+ * ---------------------------------------------------------------------------
+ */
+
+/*
+ * Router gating: softmax over the E logits of each token, then the topk
+ * experts with the largest probability, in descending order, ties to the
+ * lower expert id.  The order is decided on the logits (softmax is strictly
+ * increasing in the logit, so this is the order of the exact probabilities;
+ * no rounding of an exponential decides an id).  The weights are the selected
+ * probabilities, not renormalized over the topk:
+ *     p[t, e] = exp(l[t, e] - max_e l[t, e]) / sum_e exp(l[t, e] - max_e l[t, e])   (FP32)
+ *   logits        in   [T, E] FP32 (finite)
+ *   topk_ids      out  [T, topk] int32
+ *   topk_weights  out  [T, topk] FP32
+ * E in [1, 256], topk in [1, E].  One warp per token.
+ */
+w4_status w4_moe_gate_topk(const float *logits, int64_t T, int E, int topk, int32_t *topk_ids,
+                           float *topk_weights, void *stream);
+
+/*
+ * Block size for w4_moe_align / w4_moe_w4a16_gemm from the routing's average
+ * load per expert (T * topk / E): 16 up to 48 slots per expert, 32 up to 96,
+ * 64 beyond.  The grouped GEMM runs blocks of 32 and 64 as 16-slot sub-blocks
+ * and skips the padding ones, so small blocks cost least at decode sizes
+ * (measured on B200 at T = 16, 64, 256 with 128 experts, top-8: block 16 was
+ * fastest or within 5 %); wider blocks only pay off when they are filled.
+ * Host-only; returns 0 for invalid arguments.
+ */
+int w4_moe_block_size(int64_t T, int topk, int E);
+
+/*
+ * SiLU-gated product between the two grouped GEMMs: for each row s,
+ *     h[s, j] = bf16( silu(g) * u ),  g = gate_up[s, j], u = gate_up[s, F + j],
+ *     silu(x) = x / (1 + exp(-x))   (FP32)
+ *   gate_up   in   [S, 2F] BF16 (the gate rows of the expert weights first)
+ *   h         out  [S, F] BF16
+ * F a multiple of 8; rows are 16-byte aligned.
+ */
+w4_status w4_silu_mul(const w4_bf16 *gate_up, int64_t S, int64_t F, w4_bf16 *h, void *stream);
+
+/*
+ * Weighted top-k combine after the down projection:
+ *     out[t, n] = bf16( sum_{k = 0..topk-1} w[t, k] * D[t * topk + k, n] )
+ * accumulated in FP32 in ascending k, each product rounded before its add.
+ *   D       in   [T * topk, N] BF16 (slot rows, slot = t * topk + k)
+ *   w       in   [T, topk] FP32
+ *   out     out  [T, N] BF16
+ * N a multiple of 8.
+ */
+w4_status w4_moe_combine(const w4_bf16 *D, const float *w, int64_t T, int topk, int64_t N,
+                         w4_bf16 *out, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

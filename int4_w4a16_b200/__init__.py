@@ -27,7 +27,9 @@ __all__ = [
     "W4Error", "lib", "workspace", "w4a16_gemm_workspace_bytes", "w4_version",
     "w4_device_status", "w4_wait_selftest", "w4_fake_quant", "w4_ste_backward",
     "w4_quantize_pack", "w4_dequant", "w4a16_gemm", "w4_moe_capacity", "w4_moe_align",
-    "w4_moe_w4a16_gemm", "fake_quant", "quantize_pack", "dequant", "gemm", "moe_align",
+    "w4_moe_w4a16_gemm", "w4_moe_gate_topk", "w4_moe_block_size", "w4_silu_mul",
+    "w4_moe_combine", "fake_quant", "quantize_pack", "dequant", "gemm", "moe_align",
+    "moe_gate_topk", "silu_mul", "moe_combine",
     "moe_gemm", "FakeInt4STE", "GROUP",
 ]
 
@@ -73,6 +75,9 @@ def lib() -> ctypes.CDLL:
             "w4_moe_align": [_P, _I64, _INT, _INT, _INT, _P, _I64, _P, _P, _P],
             "w4_moe_w4a16_gemm": [_P, _INT, _P, _P, _P, _P, _P, _I64, _INT, _I64, _P, _I64,
                                   _I64, _INT, _P],
+            "w4_moe_gate_topk": [_P, _I64, _INT, _INT, _P, _P, _P],
+            "w4_silu_mul": [_P, _I64, _I64, _P, _P],
+            "w4_moe_combine": [_P, _P, _I64, _INT, _I64, _P, _P],
             "w4_device_status": [_P],
             "w4_wait_selftest": [ctypes.c_uint32, _P],
         }.items():
@@ -83,6 +88,8 @@ def lib() -> ctypes.CDLL:
         L.w4a16_gemm_workspace_bytes.restype = ctypes.c_size_t
         L.w4_moe_capacity.argtypes = [_I64, _INT, _INT, _INT]
         L.w4_moe_capacity.restype = ctypes.c_int64
+        L.w4_moe_block_size.argtypes = [_I64, _INT, _INT]
+        L.w4_moe_block_size.restype = ctypes.c_int
         L.w4_version.restype = ctypes.c_int
         L.w4_last_cuda_error.restype = ctypes.c_int
         L.w4_status_string.argtypes = [_INT]
@@ -239,6 +246,35 @@ def w4_moe_w4a16_gemm(A, a_row_div: int, Wq, S, sorted_ids, expert_ids, num_post
         _stream(stream)))
 
 
+def w4_moe_gate_topk(logits, topk: int, topk_ids, topk_weights, stream=None) -> None:
+    _dtype(logits, torch.float32, "logits")
+    _dtype(topk_ids, torch.int32, "topk_ids")
+    _dtype(topk_weights, torch.float32, "topk_weights")
+    T, E = logits.shape
+    _check("w4_moe_gate_topk", lib().w4_moe_gate_topk(_ptr(logits), T, E, topk, _ptr(topk_ids),
+                                                      _ptr(topk_weights), _stream(stream)))
+
+
+def w4_moe_block_size(T: int, topk: int, E: int) -> int:
+    return int(lib().w4_moe_block_size(T, topk, E))
+
+
+def w4_silu_mul(gate_up, h, stream=None) -> None:
+    _dtype(gate_up, torch.bfloat16, "gate_up")
+    _dtype(h, torch.bfloat16, "h")
+    S, F2 = gate_up.shape
+    _check("w4_silu_mul", lib().w4_silu_mul(_ptr(gate_up), S, F2 // 2, _ptr(h), _stream(stream)))
+
+
+def w4_moe_combine(D, w, out, stream=None) -> None:
+    _dtype(D, torch.bfloat16, "D")
+    _dtype(w, torch.float32, "w")
+    _dtype(out, torch.bfloat16, "out")
+    T, topk = w.shape
+    _check("w4_moe_combine", lib().w4_moe_combine(_ptr(D), _ptr(w), T, topk, D.shape[1],
+                                                  _ptr(out), _stream(stream)))
+
+
 # ---------------------------------------------------------------------------
 # Allocating conveniences (outputs from torch.empty on the input's device)
 # ---------------------------------------------------------------------------
@@ -290,6 +326,27 @@ def moe_gemm(A, a_row_div, Wq, S, sorted_ids, expert_ids, num_post_pad, block, n
     w4_moe_w4a16_gemm(A, a_row_div, Wq, S, sorted_ids, expert_ids, num_post_pad, block,
                       num_slots, C)
     return C
+
+
+def moe_gate_topk(logits: torch.Tensor, topk: int):
+    T = logits.shape[0]
+    ids = torch.empty((T, topk), dtype=torch.int32, device=logits.device)
+    w = torch.empty((T, topk), dtype=torch.float32, device=logits.device)
+    w4_moe_gate_topk(logits, topk, ids, w)
+    return ids, w
+
+
+def silu_mul(gate_up: torch.Tensor) -> torch.Tensor:
+    h = torch.empty((gate_up.shape[0], gate_up.shape[1] // 2), dtype=torch.bfloat16,
+                    device=gate_up.device)
+    w4_silu_mul(gate_up, h)
+    return h
+
+
+def moe_combine(D: torch.Tensor, w: torch.Tensor) -> torch.Tensor:
+    out = torch.empty((w.shape[0], D.shape[1]), dtype=torch.bfloat16, device=D.device)
+    w4_moe_combine(D, w, out)
+    return out
 
 
 class FakeInt4STE(torch.autograd.Function):

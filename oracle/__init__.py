@@ -70,6 +70,8 @@ def load_library(path: str) -> ctypes.CDLL:
     L.w4o_moe_align.argtypes = [_P, _I64, _I64, _I64, _I64, _P, _I64, _P, _P]
     L.w4o_moe_gemm.argtypes = [_P, _I64, _P, _P, _P, _I64, _I64, _I64, _I64,
                                _I64, _P, _P]
+    L.w4o_moe_gate_topk.argtypes = [_P, _I64, _I64, _I64, _P, _P]
+    L.w4o_moe_combine.argtypes = [_P, _P, _I64, _I64, _I64, _P]
     return L
 
 
@@ -254,6 +256,30 @@ def moe_gemm(A: np.ndarray, a_row_div: int, Wdq: np.ndarray, sorted_ids, expert_
                        _ptr(expert_ids), num_post_pad, num_slots, block, N, K,
                        _ptr(C), _ptr(R))
     return C, R
+
+
+def moe_gate_topk(logits: np.ndarray, topk: int):
+    """Router gating: (topk_ids int32 [T, topk], topk_weights float32 [T, topk]).
+    p = softmax(logits) per token in fp32; the topk largest p in descending
+    order, ties to the lower expert id (decided on the logits: the order of the
+    exact p); weights = the selected p, not renormalized."""
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    T, E = logits.shape
+    ids = np.empty((T, topk), np.int32)
+    w = np.empty((T, topk), np.float32)
+    lib().w4o_moe_gate_topk(_ptr(logits), T, E, topk, _ptr(ids), _ptr(w))
+    return ids, w
+
+
+def moe_combine(D: np.ndarray, w: np.ndarray, topk: int) -> np.ndarray:
+    """out[t, n] = bf16(sum_k w[t, k] * D[t*topk + k, n]), fp32, ascending k."""
+    D = _u16(D)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    T = w.shape[0]
+    N = D.shape[1]
+    out = np.empty((T, N), np.uint16)
+    lib().w4o_moe_combine(_ptr(D), _ptr(w), T, topk, N, _ptr(out))
+    return out
 
 
 def silu_mul(gate_up: np.ndarray) -> np.ndarray:

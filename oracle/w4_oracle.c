@@ -383,3 +383,51 @@ void w4o_moe_gemm(const uint16_t *A, int64_t a_row_div, const uint16_t *Wdq,
         }
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* Router gating ([QAT] the fused gating kernel before moe_align; its exact */
+/* rule is silent, read as): p = softmax(logits) per token in fp32, the     */
+/* topk largest p in descending order with ties to the lower expert id,     */
+/* weights = the selected p (not renormalized).  The order is taken on the  */
+/* logits, which is the order of the exact p (exp is strictly increasing).  */
+/* ------------------------------------------------------------------------ */
+void w4o_moe_gate_topk(const float *logits, int64_t T, int64_t E, int64_t topk,
+                       int32_t *topk_ids, float *topk_weights)
+{
+    #pragma omp parallel for
+    for (int64_t t = 0; t < T; ++t) {
+        const float *l = logits + t * E;
+        float mx = l[0];
+        for (int64_t e = 1; e < E; ++e) mx = l[e] > mx ? l[e] : mx;
+        float sum = 0.0f;
+        for (int64_t e = 0; e < E; ++e) sum = sum + expf(l[e] - mx);
+        unsigned char *taken = (unsigned char *)calloc((size_t)E, 1);
+        for (int64_t k = 0; k < topk; ++k) {
+            int64_t best = -1;
+            for (int64_t e = 0; e < E; ++e)        /* strict >: ties keep the lower id */
+                if (!taken[e] && (best < 0 || l[e] > l[best])) best = e;
+            taken[best] = 1;
+            topk_ids[t * topk + k] = (int32_t)best;
+            topk_weights[t * topk + k] = expf(l[best] - mx) / sum;
+        }
+        free(taken);
+    }
+}
+
+/* Weighted top-k combine after the down projection:
+ * out[t, n] = bf16( sum_k w[t, k] * D[t*topk + k, n] ), fp32, ascending k,
+ * each product rounded to fp32 before its add. */
+void w4o_moe_combine(const uint16_t *D, const float *w, int64_t T, int64_t topk,
+                     int64_t N, uint16_t *out)
+{
+    #pragma omp parallel for
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t n = 0; n < N; ++n) {
+            float acc = 0.0f;
+            for (int64_t k = 0; k < topk; ++k) {
+                float prod = w[t * topk + k] * w4o_f32_from_bf16(D[(t * topk + k) * N + n]);
+                acc = acc + prod;
+            }
+            out[t * N + n] = w4o_bf16_from_f32(acc);
+        }
+}

@@ -22,7 +22,8 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for required in ["w4_fake_quant", "w4_ste_backward", "w4_quantize_pack", "w4_dequant",
                      "w4a16_gemm", "w4a16_gemm_workspace_bytes", "w4_moe_align",
-                     "w4_moe_w4a16_gemm", "w4_moe_capacity",
+                     "w4_moe_w4a16_gemm", "w4_moe_capacity", "w4_moe_gate_topk",
+                     "w4_moe_block_size", "w4_silu_mul", "w4_moe_combine",
                      "w4_device_status", "w4_status_string", "w4_version",
                      "w4_last_cuda_error"]:
         assert required in names
@@ -102,3 +103,32 @@ def test_binding_refuses_cpu_tensors():
     W = torch.zeros(4, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         w4.w4_fake_quant(W, torch.empty_like(W))
+
+
+def test_moe_block_size_rule_host_only():
+    L = w4.lib()
+    assert L.w4_moe_block_size(16, 8, 128) == 16       # 1 slot per expert
+    assert L.w4_moe_block_size(768, 8, 128) == 16      # 48: the edge stays 16
+    assert L.w4_moe_block_size(769, 8, 128) == 32
+    assert L.w4_moe_block_size(1536, 8, 128) == 32     # 96
+    assert L.w4_moe_block_size(1537, 8, 128) == 64
+    assert L.w4_moe_block_size(0, 8, 128) == 0
+    assert L.w4_moe_block_size(16, 0, 128) == 0
+
+
+def test_moe_glue_validation_host_only():
+    L = w4.lib()
+    # gating: E out of range, topk > E (twice), T = 0 (nothing to do)
+    assert L.w4_moe_gate_topk(A16, 4, 257, 8, A16, A16, None) == 1
+    assert L.w4_moe_gate_topk(A16, 4, 8, 9, A16, A16, None) == 1
+    assert L.w4_moe_gate_topk(A16, 4, 64, 65, A16, A16, None) == 1
+    assert L.w4_moe_gate_topk(A16, 0, 128, 8, A16, A16, None) == 0
+    # silu_mul: F not a multiple of 8, misaligned, empty
+    assert L.w4_silu_mul(A16, 4, 12, A16, None) == 1
+    assert L.w4_silu_mul(MIS, 4, 16, A16, None) == 1
+    assert L.w4_silu_mul(A16, 0, 16, A16, None) == 0
+    # combine: N not a multiple of 8, topk < 1, misaligned output, empty
+    assert L.w4_moe_combine(A16, A16, 4, 8, 12, A16, None) == 1
+    assert L.w4_moe_combine(A16, A16, 4, 0, 16, A16, None) == 1
+    assert L.w4_moe_combine(A16, A16, 4, 8, 16, MIS, None) == 1
+    assert L.w4_moe_combine(A16, A16, 0, 8, 16, A16, None) == 0

@@ -1,0 +1,101 @@
+"""Parity of the MoE layer glue on the GPU with the CPU oracle, through the C ABI:
+router gating (softmax + top-k), the SiLU-gated product and the weighted top-k
+combine, then one whole MoE layer (gating -> moe_align -> gate_up -> SiLU*up ->
+down -> combine) checked stage by stage."""
+import numpy as np
+import pytest
+import torch
+
+import int4_w4a16_b200 as w4
+import oracle
+import synth
+from synth import bits
+from tests.test_gpu_parity import DEV, _experts, _np_bf16, assert_gemm_close
+
+pytestmark = pytest.mark.gpu
+
+
+def _logits(T, E, seed):
+    return np.random.default_rng(seed).standard_normal((T, E)).astype(np.float32)
+
+
+@pytest.mark.parametrize("T,E,topk", [(1, 128, 8), (16, 128, 8), (256, 128, 8), (1000, 128, 8),
+                                      (37, 8, 1), (64, 33, 33), (9, 256, 32), (5, 1, 1)])
+def test_gate_topk(T, E, topk):
+    logits = _logits(T, E, seed=T * 7 + E)
+    ids, w = w4.moe_gate_topk(torch.from_numpy(logits).to(DEV), topk)
+    w4.w4_device_status()
+    o_ids, o_w = oracle.moe_gate_topk(logits, topk)
+    assert np.array_equal(ids.cpu().numpy(), o_ids)                  # ids bit-exact
+    assert np.allclose(w.cpu().numpy(), o_w, rtol=1e-5, atol=0)     # fp32 exp/sum order
+
+
+def test_gate_topk_ties():
+    """Integer logits: many exact ties, all broken toward the lower expert id."""
+    rng = np.random.default_rng(5)
+    logits = rng.integers(-3, 4, size=(300, 128)).astype(np.float32)
+    ids, w = w4.moe_gate_topk(torch.from_numpy(logits).to(DEV), 8)
+    o_ids, o_w = oracle.moe_gate_topk(logits, 8)
+    assert np.array_equal(ids.cpu().numpy(), o_ids)
+    assert np.allclose(w.cpu().numpy(), o_w, rtol=1e-5, atol=0)
+
+
+@pytest.mark.parametrize("S,F", [(1, 8), (3, 1536), (128, 1536), (2048, 1536), (7, 40)])
+def test_silu_mul(S, F):
+    gu = synth.normal_bf16((S, 2 * F), 2.0, seed=S + F)
+    h = bits(w4.silu_mul(gu.to(DEV)))
+    w4.w4_device_status()
+    want = oracle.silu_mul(bits(gu))
+    # FP32 silu on both sides; CUDA's expf and the host's exp may differ in the
+    # last bit, which can move the BF16 rounding by one unit
+    diff = np.abs(h.astype(np.int32) - want.astype(np.int32))
+    assert diff.max() <= 1
+    assert (diff == 0).mean() >= 0.999
+
+
+@pytest.mark.parametrize("T,topk,N", [(1, 8, 8), (16, 8, 4096), (256, 8, 4096), (5, 3, 40)])
+def test_combine(T, topk, N):
+    D = synth.normal_bf16((T * topk, N), 1.0, seed=T + N)
+    w = np.random.default_rng(T).random((T, topk)).astype(np.float32)
+    out = bits(w4.moe_combine(D.to(DEV), torch.from_numpy(w).to(DEV)))
+    w4.w4_device_status()
+    assert np.array_equal(out, oracle.moe_combine(bits(D), w, topk))   # bit-exact
+
+
+@pytest.mark.parametrize("T", [16, 64])
+def test_moe_layer_stage_by_stage(T):
+    """One MoE decode layer on the GPU, each stage checked against the oracle fed
+    the GPU's previous stage (so stage errors do not compound)."""
+    cfg = synth.MoEDecode()
+    E, topk, hidden, inter = cfg.E, cfg.topk, cfg.hidden, cfg.inter
+    logits = _logits(T, E, seed=1000 + T)
+    X = synth.normal_bf16((T, hidden), 1.0, seed=2000 + T)
+    Wq_g, S_g, Wdq_g = _experts(E, 2 * inter, hidden)
+    Wq_d, S_d, Wdq_d = _experts(E, hidden, inter)
+    block = w4.w4_moe_block_size(T, topk, E)
+    # gating
+    ids, w = w4.moe_gate_topk(torch.from_numpy(logits).to(DEV), topk)
+    o_ids, o_w = oracle.moe_gate_topk(logits, topk)
+    assert np.array_equal(ids.cpu().numpy(), o_ids)
+    # align
+    s_d, e_d, n_d = w4.moe_align(ids, E, block)
+    s_o, e_o, n_o = oracle.moe_align(o_ids, E, block)
+    assert int(n_d.item()) == n_o and np.array_equal(s_d.cpu().numpy(), s_o)
+    # gate_up
+    C1 = w4.moe_gemm(X.to(DEV), topk, torch.from_numpy(Wq_g).to(DEV), _np_bf16(S_g).to(DEV),
+                     s_d, e_d, n_d, block, T * topk)
+    _, R1 = oracle.moe_gemm(bits(X), topk, Wdq_g, s_o, e_o, n_o, T * topk, block)
+    assert_gemm_close(bits(C1), R1, f"layer gate_up T={T}")
+    # SiLU * up on the GPU's gate_up output
+    H = w4.silu_mul(C1)
+    diff = np.abs(bits(H).astype(np.int32) - oracle.silu_mul(bits(C1)).astype(np.int32))
+    assert diff.max() <= 1
+    # down on the GPU's h
+    C2 = w4.moe_gemm(H, 1, torch.from_numpy(Wq_d).to(DEV), _np_bf16(S_d).to(DEV),
+                     s_d, e_d, n_d, block, T * topk)
+    _, R2 = oracle.moe_gemm(bits(H), 1, Wdq_d, s_o, e_o, n_o, T * topk, block)
+    assert_gemm_close(bits(C2), R2, f"layer down T={T}")
+    # combine of the GPU's down output with the GPU's weights
+    out = w4.moe_combine(C2, w)
+    w4.w4_device_status()
+    assert np.array_equal(bits(out), oracle.moe_combine(bits(C2), w.cpu().numpy(), topk))

@@ -39,6 +39,14 @@ MUTANTS = [
     ("moe_align_descending", "for (int64_t i = 0; i < slots; ++i)       /* ascending slot order */",
      "for (int64_t i = slots - 1; i >= 0; --i)",
      [lambda: [pins.test_moe_align_brute_force(s) for s in range(40)]]),
+    ("gate_ties_to_higher_id", "if (!taken[e] && (best < 0 || l[e] > l[best])) best = e;",
+     "if (!taken[e] && (best < 0 || l[e] >= l[best])) best = e;",
+     [pins.test_moe_gate_topk_ties_go_to_lower_id]),
+    ("gate_no_max_shift", "sum = sum + expf(l[e] - mx);", "sum = sum + expf(l[e]);",
+     [lambda: pins.test_moe_gate_topk_brute_force(3, 8, 3, 1)]),
+    ("combine_drops_last_k", "for (int64_t k = 0; k < topk; ++k) {\n                float prod = w[",
+     "for (int64_t k = 0; k + 1 < topk; ++k) {\n                float prod = w[",
+     [pins.test_moe_combine_reference_and_one_hot]),
     ("moe_align_no_pad", "total += (cnt[e] + block - 1) / block * block;", "total += cnt[e];",
      [lambda: [pins.test_moe_align_brute_force(s) for s in range(40)]]),
     # (random fp64 data has no exact ties, so the tie rule of this path is pinned

@@ -344,3 +344,81 @@ def test_moe_gemm_equals_dense_rows():
     for slot in range(T * topk):
         Yd, Rd = oracle.gemm(A[slot // topk:slot // topk + 1], Wdq[flat[slot]])
         assert np.array_equal(C[slot], Yd[0]) and np.array_equal(R[slot], Rd[0])
+
+
+# ---------------------------------------------------------------------------
+# MoE layer glue: gating, SiLU-gated product, weighted combine
+# ---------------------------------------------------------------------------
+
+def _brute_gate(logits, topk):
+    """Independent restatement: sort experts by (-logit, id) with Python's sort,
+    probabilities from a float64 softmax."""
+    ids, ws = [], []
+    for row in logits.astype(np.float64):
+        order = sorted(range(len(row)), key=lambda e: (-row[e], e))[:topk]
+        p = np.exp(row - row.max())
+        p /= p.sum()
+        ids.append(order)
+        ws.append([p[e] for e in order])
+    return np.array(ids, np.int32), np.array(ws)
+
+
+@pytest.mark.parametrize("T,E,topk,seed", [(1, 1, 1, 0), (3, 8, 3, 1), (17, 128, 8, 2),
+                                           (5, 33, 33, 3), (9, 256, 32, 4)])
+def test_moe_gate_topk_brute_force(T, E, topk, seed):
+    logits = np.random.default_rng(seed).standard_normal((T, E)).astype(np.float32)
+    ids, w = oracle.moe_gate_topk(logits, topk)
+    want_ids, want_w = _brute_gate(logits, topk)
+    assert np.array_equal(ids, want_ids)
+    assert np.allclose(w, want_w, rtol=2e-6, atol=0)
+    assert np.all(np.diff(w, axis=1) <= 0)                  # descending
+    if topk == E:
+        assert np.allclose(w.sum(axis=1), 1.0, rtol=1e-5)    # all of the softmax
+
+
+def test_moe_gate_topk_ties_go_to_lower_id():
+    logits = np.array([[1.0, 3.0, 3.0, -2.0, 3.0, 0.5],
+                       [0.0, 0.0, 0.0, 0.0, 0.0, 0.0]], np.float32)
+    ids, w = oracle.moe_gate_topk(logits, 4)
+    assert ids.tolist() == [[1, 2, 4, 0], [0, 1, 2, 3]]
+    assert np.allclose(w[1], 1.0 / 6.0, rtol=1e-6)
+    assert w[0, 0] == w[0, 1] == w[0, 2]
+
+
+def test_moe_gate_topk_shift_invariant():
+    """softmax(l + c) = softmax(l): the same ids, weights within fp32 rounding."""
+    logits = np.random.default_rng(7).standard_normal((6, 64)).astype(np.float32)
+    a_ids, a_w = oracle.moe_gate_topk(logits, 8)
+    b_ids, b_w = oracle.moe_gate_topk(logits + np.float32(40.0), 8)
+    assert np.array_equal(a_ids, b_ids)
+    assert np.allclose(a_w, b_w, rtol=1e-5)
+
+
+def test_moe_combine_reference_and_one_hot():
+    rng = np.random.default_rng(3)
+    T, topk, N = 7, 4, 24
+    D = oracle.f32_to_bf16_bits(rng.standard_normal((T * topk, N)).astype(np.float32))
+    w = rng.random((T, topk)).astype(np.float32)
+    out = oracle.moe_combine(D, w, topk)
+    Df = oracle.bf16_to_f32(D).astype(np.float64).reshape(T, topk, N)
+    ref = np.einsum("tk,tkn->tn", w.astype(np.float64), Df)
+    got = oracle.bf16_to_f32(out).astype(np.float64)
+    assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-6)   # BF16 rounding
+    # one-hot weights pick a slot row exactly
+    w1 = np.zeros((T, topk), np.float32)
+    w1[np.arange(T), np.arange(T) % topk] = 1.0
+    out1 = oracle.moe_combine(D, w1, topk)
+    assert np.array_equal(out1, D.reshape(T, topk, N)[np.arange(T), np.arange(T) % topk])
+
+
+def test_silu_mul_closed_forms():
+    g = np.array([0.0, 1.0, -1.0, 30.0, -30.0, 2.0], np.float32)
+    u = np.array([5.0, 2.0, 2.0, 1.0, 1.0, 0.0], np.float32)
+    gu = oracle.f32_to_bf16_bits(np.concatenate([g, u])[None, :])
+    h = oracle.bf16_to_f32(oracle.silu_mul(gu))[0].astype(np.float64)
+    gd, ud = g.astype(np.float64), u.astype(np.float64)
+    want = gd / (1.0 + np.exp(-gd)) * ud          # silu(g) * u in float64
+    assert h[0] == 0.0 and h[5] == 0.0            # silu(0) = 0; u = 0
+    assert h[3] == 30.0                           # silu(x) -> x for large x
+    assert abs(h[4]) < 1e-11                      # silu(x) -> 0 for very negative x
+    assert np.all(np.abs(h - want) <= 2.0 ** -8 * np.abs(want))   # one BF16 rounding
