@@ -2,7 +2,7 @@
 """Benchmark of the INT4 W4A16 hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode|prefill|moe|qat]
+                    [--workload decode|prefill|moe|moe_layer|qat|gemv|quant]
 
 Default workload: the decode GEMV sweep -- W[12288, 4096] BF16 ~ N(0, 0.02^2)
 with 0.1 % x20 outliers, group 32, activations X[M, 4096] ~ N(0, 1) for
@@ -511,6 +511,64 @@ def run_extra(args):
                     "gate_up_frac": b_gu / (t_gu * 1e-3) / 1e9 / peaks["hbm_gbs"],
                     "down_us": t_dn * 1e3, "down_GB/s": b_dn / (t_dn * 1e-3) / 1e9,
                     "down_frac": b_dn / (t_dn * 1e-3) / 1e9 / peaks["hbm_gbs"]})
+    elif args.workload == "moe_layer":
+        # one whole MoE decode layer on the GPU: gating -> moe_align -> gate_up ->
+        # SiLU * up -> down -> weighted combine, block size from the library's rule
+        cfg = synth.MoEDecode()
+        E, topk, hid, inter = cfg.E, cfg.topk, cfg.hidden, cfg.inter
+        Wg = cfg.gate_up_weight(dev)
+        Wd = cfg.down_weight(dev)
+        Wq_g = torch.empty((E, 2 * inter, hid // 8), dtype=torch.int32, device=dev)
+        S_g = torch.empty((E, 2 * inter, hid // 32), dtype=torch.bfloat16, device=dev)
+        Wq_d = torch.empty((E, hid, inter // 8), dtype=torch.int32, device=dev)
+        S_d = torch.empty((E, hid, inter // 32), dtype=torch.bfloat16, device=dev)
+        for e in range(E):
+            w4.w4_quantize_pack(Wg[e], Wq_g[e], S_g[e])
+            w4.w4_quantize_pack(Wd[e], Wq_d[e], S_d[e])
+        del Wg, Wd
+        per_expert = (2 * inter * hid + hid * inter) * 9 // 16
+        for T in ([args.m] if args.m else cfg.Ts):
+            slots = T * topk
+            block = w4.w4_moe_block_size(T, topk, E)
+            logits = cfg.logits(T, dev)
+            X = cfg.tokens(T, dev)
+            ids = torch.empty((T, topk), dtype=torch.int32, device=dev)
+            wts = torch.empty((T, topk), dtype=torch.float32, device=dev)
+            cap = w4.w4_moe_capacity(T, topk, E, block)
+            s_ids = torch.empty(cap, dtype=torch.int32, device=dev)
+            e_ids = torch.empty(cap // block, dtype=torch.int32, device=dev)
+            npp = torch.empty(4, dtype=torch.int32, device=dev)[:1]
+            C1 = torch.empty((slots, 2 * inter), dtype=torch.bfloat16, device=dev)
+            H = torch.empty((slots, inter), dtype=torch.bfloat16, device=dev)
+            C2 = torch.empty((slots, hid), dtype=torch.bfloat16, device=dev)
+            out_t = torch.empty((T, hid), dtype=torch.bfloat16, device=dev)
+            steps = [
+                ("gate_topk", lambda: w4.w4_moe_gate_topk(logits, topk, ids, wts)),
+                ("moe_align", lambda: w4.w4_moe_align(ids, E, block, s_ids, e_ids, npp)),
+                ("gate_up", lambda: w4.w4_moe_w4a16_gemm(X, topk, Wq_g, S_g, s_ids, e_ids, npp,
+                                                         block, slots, C1)),
+                ("silu_mul", lambda: w4.w4_silu_mul(C1, H)),
+                ("down", lambda: w4.w4_moe_w4a16_gemm(H, 1, Wq_d, S_d, s_ids, e_ids, npp, block,
+                                                      slots, C2)),
+                ("combine", lambda: w4.w4_moe_combine(C2, wts, out_t)),
+            ]
+            layer = lambda: [f() for _, f in steps]
+            layer()
+            torch.cuda.synchronize()
+            active = int(torch.unique(ids).numel())
+            lmed, lp10, lp90 = _time_kernel(layer, reps, flush)
+            per = {}
+            for name, f in steps:
+                per[name] = _time_kernel(f, max(5, reps // 2), flush)[0] * 1e3
+            act_bytes = (2 * T * hid + 4 * T * E + 8 * slots + 2 * slots * 2 * inter * 2 +
+                         2 * slots * inter * 2 + 2 * slots * hid * 2 + 2 * T * hid)
+            nb = active * per_expert + act_bytes
+            gbs = nb / (lmed * 1e-3) / 1e9
+            out["results"].append({"T": T, "block": block, "active_experts": active,
+                                   "layer_us": lmed * 1e3, "p10_us": lp10 * 1e3,
+                                   "p90_us": lp90 * 1e3, "algorithmic_bytes": nb,
+                                   "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"],
+                                   "per_kernel_us": per})
     elif args.workload == "gemv":
         # the decode GEMM alone, one activation height at a time (--m picks one)
         cfg = synth.Decode()
@@ -617,7 +675,7 @@ def main():
                          "the token count T (--workload moe)")
     ap.add_argument("--block", type=int, default=0, help="--workload moe: one block size only")
     ap.add_argument("--workload", default="decode",
-                    choices=["decode", "prefill", "moe", "qat", "gemv", "quant"],
+                    choices=["decode", "prefill", "moe", "moe_layer", "qat", "gemv", "quant"],
                     help="decode is the bench line; the others print their own lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=512)

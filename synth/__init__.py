@@ -61,6 +61,12 @@ def laplace_bf16(shape, b: float, seed: int, index: int = 0, device="cpu") -> to
     return x.to(torch.bfloat16)
 
 
+def router_logits(T: int, E: int, seed: int, index: int = 0, device="cpu"):
+    """Router logits ~ N(0, 1), float32 [T, E] (the input of the gating kernel)."""
+    g = _gen(seed, index, "cpu")
+    return torch.randn((T, E), generator=g, dtype=torch.float32).to(device)
+
+
 def routing(T: int, E: int, topk: int, seed: int, index: int = 0):
     """Router logits ~ N(0,1) [T, E] -> softmax -> top-k (ties to lower id).
     Returns (topk_ids int32 [T, topk], topk_weights float32 [T, topk]) on CPU."""
@@ -152,6 +158,9 @@ class MoEDecode:
 
     def routing(self, T: int):
         return routing(T, self.E, self.topk, self.seed, 200 + T)
+
+    def logits(self, T: int, device="cpu"):
+        return router_logits(T, self.E, self.seed, 200 + T, device)
 
 
 @dataclass(frozen=True)
