@@ -552,22 +552,32 @@ def run_extra(args):
                                                       slots, C2)),
                 ("combine", lambda: w4.w4_moe_combine(C2, wts, out_t)),
             ]
+            fused = [steps[0], steps[1],
+                     ("gate_up_silu", lambda: w4.w4_moe_w4a16_gemm_silu(
+                         X, topk, Wq_g, S_g, s_ids, e_ids, npp, block, slots, H)),
+                     steps[4], steps[5]]
             layer = lambda: [f() for _, f in steps]
+            layer_fused = lambda: [f() for _, f in fused]
             layer()
+            layer_fused()
             torch.cuda.synchronize()
             active = int(torch.unique(ids).numel())
             lmed, lp10, lp90 = _time_kernel(layer, reps, flush)
+            fmed = _time_kernel(layer_fused, reps, flush)[0]
             per = {}
-            for name, f in steps:
+            for name, f in steps + [fused[2]]:
                 per[name] = _time_kernel(f, max(5, reps // 2), flush)[0] * 1e3
             act_bytes = (2 * T * hid + 4 * T * E + 8 * slots + 2 * slots * 2 * inter * 2 +
                          2 * slots * inter * 2 + 2 * slots * hid * 2 + 2 * T * hid)
             nb = active * per_expert + act_bytes
             gbs = nb / (lmed * 1e-3) / 1e9
+            nb_fused = nb - 2 * slots * 2 * inter * 2 - 2 * slots * inter     # no gate_up round trip
             out["results"].append({"T": T, "block": block, "active_experts": active,
                                    "layer_us": lmed * 1e3, "p10_us": lp10 * 1e3,
                                    "p90_us": lp90 * 1e3, "algorithmic_bytes": nb,
                                    "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"],
+                                   "layer_fused_us": fmed * 1e3,
+                                   "fused_frac": nb_fused / (fmed * 1e-3) / 1e9 / peaks["hbm_gbs"],
                                    "per_kernel_us": per})
     elif args.workload == "gemv":
         # the decode GEMM alone, one activation height at a time (--m picks one)

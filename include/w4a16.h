@@ -222,6 +222,23 @@ w4_status w4_moe_w4a16_gemm(const w4_bf16 *A, int a_row_div, const int32_t *Wq,
                             int64_t N, int64_t K, int E, void *stream);
 
 /*
+ * Grouped W4A16 GEMM for the gate_up projection with the SiLU-gated product
+ * fused into its epilogue ([QAT] "MoE operator deep fusion"): for every real
+ * slot of every aligned block (as in w4_moe_w4a16_gemm), with the slot's FP32
+ * sums g = A.dq(W_e)[j]^T and u = A.dq(W_e)[F + j]^T,
+ *     H[slot, j] = bf16( silu(g) * u ),  silu(x) = x / (1 + exp(-x))   (FP32)
+ * i.e. w4_silu_mul applied to the unrounded gate_up sums, without writing them.
+ *   Wq, S   in   [E, 2F, K/8] int32, [E, 2F, K/32] BF16: rows 0..F-1 gate, F..2F-1 up
+ *   H       out  [num_slots, F] BF16; rows of padding slots are never written
+ * Other arguments and constraints as in w4_moe_w4a16_gemm.
+ */
+w4_status w4_moe_w4a16_gemm_silu(const w4_bf16 *A, int a_row_div, const int32_t *Wq,
+                                 const w4_bf16 *S, const int32_t *sorted_ids,
+                                 const int32_t *expert_ids, const int32_t *num_post_pad,
+                                 int64_t cap, int block, int64_t num_slots, w4_bf16 *H,
+                                 int64_t F, int64_t K, int E, void *stream);
+
+/*
  * ---------------------------------------------------------------------------
  * MoE layer around the grouped GEMMs.  The pages name the pieces without
  * defining them: a fused gating kernel (softmax + top-k), a block size chosen

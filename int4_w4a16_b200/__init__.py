@@ -27,7 +27,8 @@ __all__ = [
     "W4Error", "lib", "workspace", "w4a16_gemm_workspace_bytes", "w4_version",
     "w4_device_status", "w4_wait_selftest", "w4_fake_quant", "w4_ste_backward",
     "w4_quantize_pack", "w4_dequant", "w4a16_gemm", "w4_moe_capacity", "w4_moe_align",
-    "w4_moe_w4a16_gemm", "w4_moe_gate_topk", "w4_moe_block_size", "w4_silu_mul",
+    "w4_moe_w4a16_gemm", "w4_moe_w4a16_gemm_silu", "w4_moe_gate_topk", "w4_moe_block_size",
+    "w4_silu_mul", "moe_gemm_silu",
     "w4_moe_combine", "fake_quant", "quantize_pack", "dequant", "gemm", "moe_align",
     "moe_gate_topk", "silu_mul", "moe_combine",
     "moe_gemm", "FakeInt4STE", "GROUP",
@@ -75,6 +76,8 @@ def lib() -> ctypes.CDLL:
             "w4_moe_align": [_P, _I64, _INT, _INT, _INT, _P, _I64, _P, _P, _P],
             "w4_moe_w4a16_gemm": [_P, _INT, _P, _P, _P, _P, _P, _I64, _INT, _I64, _P, _I64,
                                   _I64, _INT, _P],
+            "w4_moe_w4a16_gemm_silu": [_P, _INT, _P, _P, _P, _P, _P, _I64, _INT, _I64, _P,
+                                       _I64, _I64, _INT, _P],
             "w4_moe_gate_topk": [_P, _I64, _INT, _INT, _P, _P, _P],
             "w4_silu_mul": [_P, _I64, _I64, _P, _P],
             "w4_moe_combine": [_P, _P, _I64, _INT, _I64, _P, _P],
@@ -246,6 +249,16 @@ def w4_moe_w4a16_gemm(A, a_row_div: int, Wq, S, sorted_ids, expert_ids, num_post
         _stream(stream)))
 
 
+def w4_moe_w4a16_gemm_silu(A, a_row_div: int, Wq, S, sorted_ids, expert_ids, num_post_pad,
+                           block: int, num_slots: int, H, stream=None) -> None:
+    """gate_up grouped GEMM with SiLU*up fused: Wq [E, 2F, K/8]; H [num_slots, F]."""
+    E, N2, K8 = Wq.shape
+    _check("w4_moe_w4a16_gemm_silu", lib().w4_moe_w4a16_gemm_silu(
+        _ptr(A), a_row_div, _ptr(Wq), _ptr(S), _ptr(sorted_ids), _ptr(expert_ids),
+        _ptr(num_post_pad), sorted_ids.numel(), block, num_slots, _ptr(H), N2 // 2, K8 * 8, E,
+        _stream(stream)))
+
+
 def w4_moe_gate_topk(logits, topk: int, topk_ids, topk_weights, stream=None) -> None:
     _dtype(logits, torch.float32, "logits")
     _dtype(topk_ids, torch.int32, "topk_ids")
@@ -326,6 +339,15 @@ def moe_gemm(A, a_row_div, Wq, S, sorted_ids, expert_ids, num_post_pad, block, n
     w4_moe_w4a16_gemm(A, a_row_div, Wq, S, sorted_ids, expert_ids, num_post_pad, block,
                       num_slots, C)
     return C
+
+
+def moe_gemm_silu(A, a_row_div, Wq, S, sorted_ids, expert_ids, num_post_pad, block, num_slots,
+                  H=None):
+    if H is None:
+        H = torch.empty((num_slots, Wq.shape[1] // 2), dtype=torch.bfloat16, device=A.device)
+    w4_moe_w4a16_gemm_silu(A, a_row_div, Wq, S, sorted_ids, expert_ids, num_post_pad, block,
+                           num_slots, H)
+    return H
 
 
 def moe_gate_topk(logits: torch.Tensor, topk: int):

@@ -97,6 +97,9 @@ struct GemmParams {
     int cap_blocks;              // MoE: length of expert_ids (bounds num_post_pad / block)
     int moe_sub;                 // MoE: MT-slot sub-blocks per aligned block (block / MT)
     int moe_mt;                  // MoE: MT (slots per work item)
+    int silu_inter;              // MoE gate_up with SiLU*up fused: the intermediate
+                                 // size F (weights [E, 2F, K]; Y = H [num_slots, F]);
+                                 // 0 = plain grouped GEMM
     int rows_per_tile;           // R <= 128
     int n_row_tiles;
     int n_tok_tiles;             // dense
@@ -304,6 +307,10 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
     constexpr uint32_t kIdesc = idesc_bf16_f32(128, MT);
 
     extern __shared__ uint8_t smem_raw[];
+    // MoE gate_up with SiLU*up: the up rows' sums of one 16-column chunk, handed
+    // from the epilogue warps of lane quarters 2-3 to those of 0-1
+    __shared__ __align__(16) float xchg[MOE ? 64 * 16 : 4];
+    __shared__ __align__(8) uint64_t xchg_bar[2];     // [0] written, [1] read
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -344,6 +351,10 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
             mbar_init(accempty_bar(d), 128u);
         }
         mbar_init(mmadone_bar, (uint32_t)NSPLIT);
+        if (MOE) {
+            mbar_init(smem_u32(&xchg_bar[0]), 2u);
+            mbar_init(smem_u32(&xchg_bar[1]), 2u);
+        }
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tm_w);
@@ -410,7 +421,19 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                     const uint32_t sbytes = (KB == 256) ? (uint32_t)R * 16u : 0u;
                     const uint32_t xbytes = MOE ? 0u : (uint32_t)L::kXBytes;
                     mbar_arrive_expect_tx(full_bar(s), wbytes + sbytes + xbytes);
-                    if (MOE) {
+                    if (MOE && p.silu_inter > 0) {
+                        // SiLU*up tile: rows 0-63 are gate rows rt*64 + i, rows
+                        // 64-127 the matching up rows F + rt*64 + i (64-row boxes)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int grow = h * p.silu_inter + rt * 64;
+                            tma_load_3d(w_stage(s) + (uint32_t)(64 * h) * (KB / 2), &tm_w,
+                                        full_bar(s), kb * kWords, grow, expert);
+                            if (KB == 256)
+                                tma_load_3d(s_stage(s) + (uint32_t)(64 * h) * 16u, &tm_s,
+                                            full_bar(s), kb * 8, grow, expert);
+                        }
+                    } else if (MOE) {
                         tma_load_3d(w_stage(s), &tm_w, full_bar(s), kb * kWords, row0, expert);
                         if (KB == 256)
                             tma_load_3d(s_stage(s), &tm_s, full_bar(s), kb * 8, row0, expert);
@@ -626,6 +649,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
         const int lrow = q4 * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
         uint32_t it = 0, acc_it = 0;
+        uint32_t xchg_count = 0;                    // SiLU*up hand-overs so far
         bool ok = true;
         ItemIter I = make_iter(p, num_items);
         int rt, tt, kb0, kb1;
@@ -741,6 +765,44 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                                make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
                                            __uint_as_float(v[4 * q + 2]),
                                            __uint_as_float(v[4 * q + 3])));
+                    continue;
+                }
+                if (MOE && p.silu_inter > 0) {
+                    // h = bf16(silu(g) * u): lane quarters 0-1 hold the gate rows,
+                    // 2-3 the up rows of the same 64 output columns; the up values
+                    // cross through shared memory (bounded mbarrier hand-over)
+                    const uint32_t xc = xchg_count++;
+                    float *xrow = xchg + ((q4 & 1) * 32 + lane) * 16;
+                    if (q4 >= 2) {
+                        if (xc > 0 && !warp_wait(smem_u32(&xchg_bar[1]), (xc - 1) & 1u,
+                                                 abort_flag, kPollSleepNs))
+                            break;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            reinterpret_cast<float4 *>(xrow)[q] = make_float4(
+                                __uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(smem_u32(&xchg_bar[0]));
+                    } else {
+                        if (!warp_wait(smem_u32(&xchg_bar[0]), xc & 1u, abort_flag, kPollSleepNs))
+                            break;
+                        const int64_t hcol = (int64_t)rt * 64 + q4 * 32 + lane;
+#pragma unroll
+                        for (int jj = 0; jj < 16; ++jj) {
+                            const float g = __uint_as_float(v[jj]);
+                            const float u = xrow[jj];
+                            const int slot = __ldg(p.sorted_ids + (int64_t)tt * MT + c0 + jj);
+                            if (hcol < p.silu_inter && slot >= 0 && slot < p.num_slots) {
+                                const __nv_bfloat16 h =
+                                    __float2bfloat16_rn((g / (1.0f + expf(-g))) * u);
+                                p.Y[(int64_t)slot * p.silu_inter + hcol] =
+                                    *reinterpret_cast<const uint16_t *>(&h);
+                            }
+                        }
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(smem_u32(&xchg_bar[1]));
+                    }
                     continue;
                 }
 #pragma unroll
@@ -1137,14 +1199,19 @@ extern "C" int64_t w4_moe_capacity(int64_t T, int topk, int E, int block) {
     return (cap + block - 1) / block * block;
 }
 
-extern "C" w4_status w4_moe_w4a16_gemm(const w4_bf16 *A, int a_row_div, const int32_t *Wq,
-                                       const w4_bf16 *S, const int32_t *sorted_ids,
-                                       const int32_t *expert_ids, const int32_t *num_post_pad,
-                                       int64_t cap, int block, int64_t num_slots, w4_bf16 *C,
-                                       int64_t N, int64_t K, int E, void *stream) {
+namespace w4 {
+namespace {
+
+// Grouped GEMM launch shared by the plain entry (silu_inter = 0: Y = C
+// [num_slots, N]) and the SiLU*up entry (silu_inter = F, N = 2F: Y = H
+// [num_slots, F]).
+w4_status moe_launch(const w4_bf16 *A, int a_row_div, const int32_t *Wq, const w4_bf16 *S,
+                     const int32_t *sorted_ids, const int32_t *expert_ids,
+                     const int32_t *num_post_pad, int64_t cap, int block, int64_t num_slots,
+                     w4_bf16 *Y, int64_t N, int64_t K, int E, int64_t silu_inter, void *stream) {
     if (!w4host::aligned16(A) || !w4host::aligned16(Wq) || !w4host::aligned16(S) ||
         !w4host::aligned16(sorted_ids) || !w4host::aligned16(expert_ids) ||
-        !w4host::aligned16(num_post_pad) || !w4host::aligned16(C))
+        !w4host::aligned16(num_post_pad) || !w4host::aligned16(Y))
         return W4_ERR_INVALID_ARG;
     if (a_row_div <= 0 || N <= 0 || K <= 0 || (K % 32) != 0 || E <= 0 || num_slots < 0 ||
         cap < 0 || block <= 0 || (cap % block) != 0)
@@ -1156,7 +1223,7 @@ extern "C" w4_status w4_moe_w4a16_gemm(const w4_bf16 *A, int a_row_div, const in
 
     GemmParams p = {};
     p.S = reinterpret_cast<const uint16_t *>(S);
-    p.Y = reinterpret_cast<uint16_t *>(C);
+    p.Y = reinterpret_cast<uint16_t *>(Y);
     p.A = reinterpret_cast<const uint16_t *>(A);
     p.sorted_ids = sorted_ids;
     p.expert_ids = expert_ids;
@@ -1167,19 +1234,22 @@ extern "C" w4_status w4_moe_w4a16_gemm(const w4_bf16 *A, int a_row_div, const in
     p.num_slots = num_slots;
     p.a_row_div = a_row_div;
     p.a_rows = (num_slots + a_row_div - 1) / a_row_div;
-    if (cap / block > (1 << 30)) return W4_ERR_UNSUPPORTED;
+    if (cap / block > (1 << 30) || silu_inter > (1 << 28)) return W4_ERR_UNSUPPORTED;
     p.cap_blocks = (int)(cap / block);
     p.rows_per_tile = 128;
-    p.n_row_tiles = ceil_div_i(N, 128);
+    p.silu_inter = (int)silu_inter;
+    // a SiLU*up tile covers 64 output columns (64 gate + 64 up rows)
+    p.n_row_tiles = silu_inter > 0 ? ceil_div_i(silu_inter, 64) : ceil_div_i(N, 128);
     p.n_tok_tiles = 0;
     p.num_kb = ceil_div_i(K, 256);
+    const cuuint32_t box_rows = silu_inter > 0 ? 64u : 128u;
 
     CUtensorMap tw, ts, tx;
     memset(&tx, 0, sizeof tx);
     {
         cuuint64_t dims[3] = {(cuuint64_t)(K / 8), (cuuint64_t)N, (cuuint64_t)E};
         cuuint64_t strides[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N * (K / 2)};
-        cuuint32_t box[3] = {32u, 128u, 1u};
+        cuuint32_t box[3] = {32u, box_rows, 1u};
         if (!make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_INT32, 3, Wq, dims, strides, box,
                       CU_TENSOR_MAP_SWIZZLE_128B))
             return W4_ERR_CUDA;
@@ -1187,7 +1257,7 @@ extern "C" w4_status w4_moe_w4a16_gemm(const w4_bf16 *A, int a_row_div, const in
     {
         cuuint64_t dims[3] = {(cuuint64_t)(K / 32), (cuuint64_t)N, (cuuint64_t)E};
         cuuint64_t strides[2] = {(cuuint64_t)(K / 16), (cuuint64_t)N * (K / 16)};
-        cuuint32_t box[3] = {8u, 128u, 1u};
+        cuuint32_t box[3] = {8u, box_rows, 1u};
         if (!make_map(&ts, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, S, dims, strides, box,
                       CU_TENSOR_MAP_SWIZZLE_NONE))
             return W4_ERR_CUDA;
@@ -1210,6 +1280,29 @@ extern "C" w4_status w4_moe_w4a16_gemm(const w4_bf16 *A, int a_row_div, const in
     const int64_t items_max = (cap / 16) * p.n_row_tiles;
     const int items = (int)std::min<int64_t>(items_max, 1 << 30);
     return launch_cfg<256, 16, 6, 2, 3, 4, 2, true>(tw, ts, tx, p, items, st);
+}
+
+}  // namespace
+}  // namespace w4
+
+extern "C" w4_status w4_moe_w4a16_gemm(const w4_bf16 *A, int a_row_div, const int32_t *Wq,
+                                       const w4_bf16 *S, const int32_t *sorted_ids,
+                                       const int32_t *expert_ids, const int32_t *num_post_pad,
+                                       int64_t cap, int block, int64_t num_slots, w4_bf16 *C,
+                                       int64_t N, int64_t K, int E, void *stream) {
+    return w4::moe_launch(A, a_row_div, Wq, S, sorted_ids, expert_ids, num_post_pad, cap, block,
+                          num_slots, C, N, K, E, 0, stream);
+}
+
+extern "C" w4_status w4_moe_w4a16_gemm_silu(const w4_bf16 *A, int a_row_div, const int32_t *Wq,
+                                            const w4_bf16 *S, const int32_t *sorted_ids,
+                                            const int32_t *expert_ids,
+                                            const int32_t *num_post_pad, int64_t cap, int block,
+                                            int64_t num_slots, w4_bf16 *H, int64_t F, int64_t K,
+                                            int E, void *stream) {
+    if (F <= 0) return W4_ERR_INVALID_ARG;
+    return w4::moe_launch(A, a_row_div, Wq, S, sorted_ids, expert_ids, num_post_pad, cap, block,
+                          num_slots, H, 2 * F, K, E, F, stream);
 }
 
 // ---------------------------------------------------------------------------

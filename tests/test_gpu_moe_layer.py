@@ -99,3 +99,37 @@ def test_moe_layer_stage_by_stage(T):
     out = w4.moe_combine(C2, w)
     w4.w4_device_status()
     assert np.array_equal(bits(out), oracle.moe_combine(bits(C2), w.cpu().numpy(), topk))
+
+
+def _silu_ref(R, F):
+    """h = silu(g) * u from the oracle's FP32 gate_up sums (float64 evaluation)."""
+    g, u = R[:, :F].astype(np.float64), R[:, F:].astype(np.float64)
+    return (g / (1.0 + np.exp(-g)) * u).astype(np.float32)
+
+
+@pytest.mark.parametrize("T,E,F,K,block", [(16, 128, 1536, 4096, 16), (64, 128, 1536, 4096, 64),
+                                            (40, 8, 100, 1024, 16), (64, 8, 96, 512, 32)])
+def test_moe_gate_up_silu_fused(T, E, F, K, block):
+    """gate_up with SiLU*up in the epilogue against silu(g) * u of the oracle's FP32
+    sums (the fused path never rounds g and u to BF16), and against the unfused
+    chain (gate_up GEMM, then w4_silu_mul), which differs by that one rounding."""
+    topk = 8
+    logits = _logits(T, E, seed=50 + T + F)
+    ids, w = w4.moe_gate_topk(torch.from_numpy(logits).to(DEV), topk)
+    X = synth.normal_bf16((T, K), 1.0, seed=60 + T)
+    Wq, S, Wdq = _experts(E, 2 * F, K)
+    s_d, e_d, n_d = w4.moe_align(ids, E, block)
+    canary = torch.full((T * topk, F), 0x7FC1, dtype=torch.int16).view(torch.bfloat16).to(DEV)
+    Wq_d, S_d = torch.from_numpy(Wq).to(DEV), _np_bf16(S).to(DEV)
+    H = w4.moe_gemm_silu(X.to(DEV), topk, Wq_d, S_d, s_d, e_d, n_d, block, T * topk, H=canary)
+    w4.w4_device_status()
+    Hb = bits(H)
+    assert not np.any(Hb == 0x7FC1), "a real slot was left unwritten"
+    o_ids, _ = oracle.moe_gate_topk(logits, topk)
+    s_o, e_o, n_o = oracle.moe_align(o_ids, E, block)
+    _, R = oracle.moe_gemm(bits(X), topk, Wdq, s_o, e_o, n_o, T * topk, block)
+    assert_gemm_close(Hb, _silu_ref(R, F), f"fused silu T={T} F={F}")
+    if F % 8 == 0:          # w4_silu_mul takes F in multiples of 8
+        C1 = w4.moe_gemm(X.to(DEV), topk, Wq_d, S_d, s_d, e_d, n_d, block, T * topk)
+        H2 = bits(w4.silu_mul(C1))
+        assert_gemm_close(H2, _silu_ref(R, F), f"unfused silu T={T} F={F}")
