@@ -178,6 +178,23 @@ w4_status w4a16_gemm_noalloc(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 
                              w4_bf16 *Y, int64_t M, int64_t N, int64_t K, int group,
                              void *stream);
 
+/*
+ * QAT forward GEMM with the fake quantization fused into the weight prologue
+ * (the training-side counterpart of w4a16_gemm; INT4 QAT blog, fake
+ * quantization in the forward pass; reportify.cn "量化感知训练" [8][16][62]):
+ *     Y[m, n] = sum_k X[m, k] * Wdq[n, k],   Wdq = w4_fake_quant(W)  (group 32)
+ * FP32 accumulation, one BF16 rounding, without ever writing Wdq: every
+ * 128 x 64 tile of W is quantized and dequantized in registers (the exact
+ * arithmetic of w4_fake_quant) on its way to the tensor cores.  The backward
+ * pass is the plain BF16 GEMMs of the straight-through estimator (dX = dY.Wdq,
+ * dW = dY^T.X), outside this library.
+ *   X   in   [M, K] BF16;  W  in  [N, K] BF16 (the master weights);  Y  out  [M, N] BF16
+ * K a multiple of 64 (W4_ERR_UNSUPPORTED otherwise; of 32: W4_ERR_INVALID_ARG);
+ * group must be 32; 16-byte aligned, contiguous rows.
+ */
+w4_status w4_qat_gemm(const w4_bf16 *X, const w4_bf16 *W, w4_bf16 *Y, int64_t M, int64_t N,
+                      int64_t K, int group, void *stream);
+
 /* Padded capacity the caller must provide for w4_moe_align's sorted_ids:
  * T*topk + E*(block-1), rounded up to a multiple of block.  Host-only. */
 int64_t w4_moe_capacity(int64_t T, int topk, int E, int block);

@@ -28,7 +28,7 @@ __all__ = [
     "w4_device_status", "w4_wait_selftest", "w4_fake_quant", "w4_ste_backward",
     "w4_quantize_pack", "w4_dequant", "w4a16_gemm", "w4_moe_capacity", "w4_moe_align",
     "w4_moe_w4a16_gemm", "w4_moe_w4a16_gemm_silu", "w4_moe_gate_topk", "w4_moe_block_size",
-    "w4_silu_mul", "moe_gemm_silu",
+    "w4_silu_mul", "moe_gemm_silu", "w4_qat_gemm", "qat_gemm",
     "w4_moe_combine", "fake_quant", "quantize_pack", "dequant", "gemm", "moe_align",
     "moe_gate_topk", "silu_mul", "moe_combine",
     "moe_gemm", "FakeInt4STE", "GROUP",
@@ -79,6 +79,7 @@ def lib() -> ctypes.CDLL:
             "w4_moe_w4a16_gemm_silu": [_P, _INT, _P, _P, _P, _P, _P, _I64, _INT, _I64, _P,
                                        _I64, _I64, _INT, _P],
             "w4_moe_gate_topk": [_P, _I64, _INT, _INT, _P, _P, _P],
+            "w4_qat_gemm": [_P, _P, _P, _I64, _I64, _I64, _INT, _P],
             "w4_silu_mul": [_P, _I64, _I64, _P, _P],
             "w4_moe_combine": [_P, _P, _I64, _INT, _I64, _P, _P],
             "w4_device_status": [_P],
@@ -259,6 +260,17 @@ def w4_moe_w4a16_gemm_silu(A, a_row_div: int, Wq, S, sorted_ids, expert_ids, num
         _stream(stream)))
 
 
+def w4_qat_gemm(X, W, Y, group: int = GROUP, stream=None) -> None:
+    """Y = X . fake_quant(W)^T, the QDQ fused into the GEMM's weight prologue."""
+    _dtype(X, torch.bfloat16, "X")
+    _dtype(W, torch.bfloat16, "W")
+    _dtype(Y, torch.bfloat16, "Y")
+    M, K = X.shape
+    N = W.shape[0]
+    _check("w4_qat_gemm", lib().w4_qat_gemm(_ptr(X), _ptr(W), _ptr(Y), M, N, K, group,
+                                            _stream(stream)))
+
+
 def w4_moe_gate_topk(logits, topk: int, topk_ids, topk_weights, stream=None) -> None:
     _dtype(logits, torch.float32, "logits")
     _dtype(topk_ids, torch.int32, "topk_ids")
@@ -348,6 +360,12 @@ def moe_gemm_silu(A, a_row_div, Wq, S, sorted_ids, expert_ids, num_post_pad, blo
     w4_moe_w4a16_gemm_silu(A, a_row_div, Wq, S, sorted_ids, expert_ids, num_post_pad, block,
                            num_slots, H)
     return H
+
+
+def qat_gemm(X: torch.Tensor, W: torch.Tensor) -> torch.Tensor:
+    Y = torch.empty((X.shape[0], W.shape[0]), dtype=torch.bfloat16, device=X.device)
+    w4_qat_gemm(X, W, Y)
+    return Y
 
 
 def moe_gate_topk(logits: torch.Tensor, topk: int):

@@ -44,6 +44,7 @@
 #include <type_traits>
 
 #include "w4_common.cuh"
+#include "w4_qdq.cuh"
 
 namespace w4 {
 namespace {
@@ -205,9 +206,10 @@ __device__ __forceinline__ int unit_owner(uint32_t x, const GemmParams &p) {
 }
 
 // Shared-memory layout, all offsets from a 1024-aligned base.
-template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT>
+template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT, bool BF16W = false>
 struct Layout {
-    static constexpr int kWBytes = 128 * KB / 2;            // packed tile, up to 128 rows
+    // weight tile of up to 128 rows: packed INT4 words, or BF16 weights (QAT)
+    static constexpr int kWBytes = BF16W ? 128 * KB * 2 : 128 * KB / 2;
     static constexpr int kSBytes = (KB == 256) ? 128 * 16 : 0;
     static constexpr int kXSub = MT * 128;                  // one 64-wide K slice
     static constexpr int kXBytes = (KB / 64) * kXSub;
@@ -282,12 +284,13 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 // issuer / accumulator u % NSPLIT, and the epilogue adds the accumulators in
 // a fixed order.
 template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT, int NDQ, bool MOE,
-          bool WGL>
+          bool WGL, bool QAT>
 __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
     w4a16_tc_kernel(const __grid_constant__ CUtensorMap tm_w,
                     const __grid_constant__ CUtensorMap tm_s,
                     const __grid_constant__ CUtensorMap tm_x, const GemmParams p) {
-    using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE, NSPLIT>;
+    using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE, NSPLIT, QAT>;
+    static_assert(!QAT || (KB == 64 && !MOE), "QAT: 64-wide k-blocks of dense BF16 weights");
     constexpr int kWords = KB / 8;             // packed words per row per k-block
     constexpr int kAStageCols = KB / 2;        // TMEM columns per A stage
     constexpr int kAccCols = NSPLIT * MT;      // TMEM columns per work item accumulator
@@ -417,7 +420,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                     break;
                 }
                 if (lane == 0) {
-                    const uint32_t wbytes = (uint32_t)R * (KB / 2);
+                    const uint32_t wbytes = QAT ? (uint32_t)R * KB * 2u : (uint32_t)R * (KB / 2);
                     const uint32_t sbytes = (KB == 256) ? (uint32_t)R * 16u : 0u;
                     const uint32_t xbytes = MOE ? 0u : (uint32_t)L::kXBytes;
                     mbar_arrive_expect_tx(full_bar(s), wbytes + sbytes + xbytes);
@@ -438,7 +441,8 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                         if (KB == 256)
                             tma_load_3d(s_stage(s), &tm_s, full_bar(s), kb * 8, row0, expert);
                     } else {
-                        tma_load_2d(w_stage(s), &tm_w, full_bar(s), kb * kWords, row0);
+                        tma_load_2d(w_stage(s), &tm_w, full_bar(s), QAT ? kb * KB : kb * kWords,
+                                    row0);
                         if (KB == 256) tma_load_2d(s_stage(s), &tm_s, full_bar(s), kb * 8, row0);
 #pragma unroll
                         for (int u = 0; u < KB / 64; ++u)
@@ -501,6 +505,41 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                 if (it % NDQ != grp) continue;
                 const int s = it % NSTAGE;
                 const int a = it % NASTAGE;
+                if constexpr (QAT) {
+                    // QAT forward: the row's 64 BF16 weights (two groups of 32,
+                    // 128-byte swizzled line) go through the exact group QDQ of the
+                    // quantizers, straight into this k-block's A columns
+                    if (!warp_wait(full_bar(s), (it / NSTAGE) & 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    uint32_t v[2][16], o[32];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 x = lds128(w_stage(s) + swz((uint32_t)(lrow * 128 + c * 16), 128));
+                        v[c >> 2][4 * (c & 3)] = x.x;
+                        v[c >> 2][4 * (c & 3) + 1] = x.y;
+                        v[c >> 2][4 * (c & 3) + 2] = x.z;
+                        v[c >> 2][4 * (c & 3) + 3] = x.w;
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t og[16];
+                        qdq::fake_quant_group(v[h], og);
+#pragma unroll
+                        for (int z = 0; z < 16; ++z) o[16 * h + z] = og[z];
+                    }
+                    if (!warp_wait(aempty_bar(a), ((it / NASTAGE) & 1u) ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    tmem_st_x32(tmem_base + lane_addr + (uint32_t)(kABase + a * kAStageCols), o);
+                    tmem_wait_st();
+                    tc_fence_before_sync();
+                    mbar_arrive(afull_bar(a));
+                    continue;
+                }
                 static_assert(KB == 256 || G == 2, "direct-load scales: one chunk pair per k-block");
                 uint32_t sc[G];
                 if (KB != 256) {
@@ -961,11 +1000,11 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
 // ---------------------------------------------------------------------------
 
 template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT, int NDQ, bool MOE,
-          bool WGL = false>
+          bool WGL = false, bool QAT = false>
 w4_status launch_cfg(const CUtensorMap &tw, const CUtensorMap &ts, const CUtensorMap &tx,
                      const GemmParams &p, int num_items_max, cudaStream_t stream) {
-    using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE, NSPLIT>;
-    auto kern = w4a16_tc_kernel<KB, MT, NSTAGE, NACC, NASTAGE, NSPLIT, NDQ, MOE, WGL>;
+    using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE, NSPLIT, QAT>;
+    auto kern = w4a16_tc_kernel<KB, MT, NSTAGE, NACC, NASTAGE, NSPLIT, NDQ, MOE, WGL, QAT>;
     // At least half of the SM's shared memory, so one CTA (and one TMEM
     // allocation of 512 columns) per SM.
     const int smem = std::max(L::kAlloc, 120 * 1024);
@@ -1191,6 +1230,52 @@ extern "C" w4_status w4a16_gemm(const w4_bf16 *X, const int32_t *Wq, const w4_bf
     if (items > (1 << 30)) return W4_ERR_UNSUPPORTED;
     if (mt == 64) return launch_cfg<64, 64, 8, 1, 8, 4, 2, false>(tw, ts, tx, p, (int)items, st);
     return launch_cfg<64, 256, 6, 1, 8, 1, 2, false>(tw, ts, tx, p, (int)items, st);
+}
+
+extern "C" w4_status w4_qat_gemm(const w4_bf16 *X, const w4_bf16 *W, w4_bf16 *Y, int64_t M,
+                                 int64_t N, int64_t K, int group, void *stream) {
+    if (group != 32) return W4_ERR_UNSUPPORTED;
+    if (M < 0 || N < 0 || K <= 0 || (K % 32) != 0) return W4_ERR_INVALID_ARG;
+    if (!w4host::aligned16(X) || !w4host::aligned16(W) || !w4host::aligned16(Y))
+        return W4_ERR_INVALID_ARG;
+    if ((K % 64) != 0) return W4_ERR_UNSUPPORTED;
+    if (M == 0 || N == 0) return W4_OK;
+    if (N > (1 << 30) || M > (1 << 30) || K > (1 << 24)) return W4_ERR_UNSUPPORTED;
+    cudaStream_t st = (cudaStream_t)stream;
+    GemmParams p = {};
+    p.Y = reinterpret_cast<uint16_t *>(Y);
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    const int mt = M <= 64 ? 64 : 256;
+    p.rows_per_tile = 128;
+    p.n_row_tiles = ceil_div_i(N, 128);
+    p.n_tok_tiles = ceil_div_i(M, mt);
+    p.num_kb = (int)(K / 64);
+    CUtensorMap tw, ts, tx;
+    memset(&ts, 0, sizeof ts);
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+        cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+        cuuint32_t box[2] = {64u, (cuuint32_t)mt};
+        if (!make_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+            return W4_ERR_CUDA;
+    }
+    {
+        // BF16 weights [N, K]: 64-wide K boxes (128-byte lines) of 128 rows
+        cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)N};
+        cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+        cuuint32_t box[2] = {64u, 128u};
+        if (!make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+            return W4_ERR_CUDA;
+    }
+    const int64_t items = (int64_t)p.n_row_tiles * p.n_tok_tiles;
+    if (items > (1 << 30)) return W4_ERR_UNSUPPORTED;
+    if (mt == 64)
+        return launch_cfg<64, 64, 8, 1, 8, 4, 2, false, false, true>(tw, ts, tx, p, (int)items, st);
+    return launch_cfg<64, 256, 4, 1, 8, 1, 2, false, false, true>(tw, ts, tx, p, (int)items, st);
 }
 
 extern "C" int64_t w4_moe_capacity(int64_t T, int topk, int E, int block) {

@@ -1,0 +1,84 @@
+"""Parity of the QAT forward GEMM (fake quantization fused into the weight
+prologue, w4_qat_gemm) with the CPU oracle: Y = X . fake_quant(W)^T, where the
+oracle materializes fake_quant(W) and multiplies; the GPU never writes it."""
+import numpy as np
+import pytest
+import torch
+
+import int4_w4a16_b200 as w4
+import oracle
+import synth
+from synth import bits
+from tests.test_gpu_parity import DEV, _np_bf16, assert_gemm_close
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(M, N, K, seed, outliers=0.001):
+    W = synth.normal_bf16((N, K), 0.02, seed=seed, outlier_frac=outliers)
+    X = synth.normal_bf16((M, K), 1.0, seed=seed + 1)
+    Y = bits(w4.qat_gemm(X.to(DEV), W.to(DEV)))
+    w4.w4_device_status()
+    Wdq, _ = oracle.fake_quant(bits(W))
+    _, R = oracle.gemm(bits(X), Wdq)
+    return Y, R
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 1, 64), (5, 100, 128), (64, 300, 640), (65, 257, 256),
+                                   (300, 1000, 1024), (512, 1024, 2048), (3, 129, 4096)])
+def test_qat_gemm_shapes(M, N, K):
+    Y, R = _case(M, N, K, seed=M + N + K)
+    assert_gemm_close(Y, R, f"qat M={M} N={N} K={K}")
+
+
+def test_qat_gemm_one_hot_exact_with_edge_groups():
+    """X = identity rows: Y[m, n] = fake_quant(W)[n, m] bit for bit, on weights
+    with zero groups, subnormal-scale groups and huge values (the exact
+    division path of the in-prologue QDQ) next to ordinary ones."""
+    N, K = 200, 256
+    W = synth.normal_bf16((N, K), 0.02, seed=9, outlier_frac=0.01).clone()
+    W[3, 0:32] = 0.0                                        # amax 0 -> s = +0
+    W[4, 32:64] = 1e-39                                     # subnormal scale
+    W[5, 64:96] = torch.linspace(-3e30, 3e30, 32).to(torch.bfloat16)   # huge
+    W[6, 96:128] = torch.tensor([0.5 * (i % 3 - 1) for i in range(32)]).to(torch.bfloat16)  # ties
+    Wd = W.to(DEV)
+    Wdq, _ = oracle.fake_quant(bits(W))
+    for m0 in range(0, K, 64):
+        X = torch.zeros((64, K), dtype=torch.bfloat16)
+        X[torch.arange(64), m0 + torch.arange(64)] = 1.0
+        Y = bits(w4.qat_gemm(X.to(DEV), Wd))
+        want = Wdq[:, m0:m0 + 64].T
+        if not np.array_equal(Y, want):
+            bad = np.argwhere(Y != want)
+            raise AssertionError(f"one-hot mismatch at m0={m0}: {bad[:8].tolist()}")
+    w4.w4_device_status()
+
+
+def test_qat_gemm_layer_shape_sampled():
+    """A QAT-stack layer shape (W[12288, 4096]) at 2048 tokens; the oracle checks
+    16 rows of Y spread over M (every weight group enters every checked element)."""
+    N, K, M = 12288, 4096, 2048
+    W = synth.normal_bf16((N, K), 0.02, seed=0, index=1, device=DEV, outlier_frac=0.001)
+    X = synth.normal_bf16((M, K), 1.0, seed=0, index=2, device=DEV)
+    Y = w4.qat_gemm(X, W)
+    w4.w4_device_status()
+    rows = torch.linspace(0, M - 1, 16).long()
+    Wdq, _ = oracle.fake_quant(bits(W.cpu()))
+    _, R = oracle.gemm(bits(X[rows].cpu()), Wdq)
+    assert_gemm_close(bits(Y[rows]), R, "qat layer sampled")
+
+
+def test_qat_gemm_matches_fake_quant_then_gemm():
+    """The fused path and the unfused one (w4_fake_quant, then the same product
+    from the materialized Wdq through the oracle) agree within GEMM tolerance,
+    and the fused path is deterministic."""
+    M, N, K = 128, 512, 1024
+    W = synth.normal_bf16((N, K), 0.02, seed=4)
+    X = synth.normal_bf16((M, K), 1.0, seed=5)
+    Xd, Wd = X.to(DEV), W.to(DEV)
+    Y1 = bits(w4.qat_gemm(Xd, Wd))
+    Y2 = bits(w4.qat_gemm(Xd, Wd))
+    assert np.array_equal(Y1, Y2)
+    Wdq_gpu = bits(w4.fake_quant(Wd))
+    _, R = oracle.gemm(bits(X), Wdq_gpu)
+    assert_gemm_close(Y1, R, "fused vs materialized")
