@@ -2,7 +2,7 @@
 """Benchmark of the INT4 W4A16 hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode|prefill|moe|moe_layer|qat|gemv|quant]
+                    [--workload decode|prefill|moe|moe_layer|qat|qat_gemm|gemv|quant]
 
 Default workload: the decode GEMV sweep -- W[12288, 4096] BF16 ~ N(0, 0.02^2)
 with 0.1 % x20 outliers, group 32, activations X[M, 4096] ~ N(0, 1) for
@@ -579,6 +579,30 @@ def run_extra(args):
                                    "layer_fused_us": fmed * 1e3,
                                    "fused_frac": nb_fused / (fmed * 1e-3) / 1e9 / peaks["hbm_gbs"],
                                    "per_kernel_us": per})
+    elif args.workload == "qat_gemm":
+        # QAT forward GEMM on a layer of the QAT stack (W[12288, 4096]) with the
+        # fake quantization fused into the weight prologue, beside the unfused
+        # chain (w4_fake_quant, then a cuBLAS BF16 GEMM on the materialized Wdq)
+        cfg = synth.QATStack()
+        N, K = cfg.shapes[0]
+        W = cfg.weight(0, 0, dev)
+        Wdq = torch.empty_like(W)
+        for M in ([args.m] if args.m else (2048, 8192)):
+            X = synth.normal_bf16((M, K), 1.0, 0, 400 + M, dev)
+            Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            fused = lambda: w4.w4_qat_gemm(X, W, Y)
+            unfused = lambda: (w4.w4_fake_quant(W, Wdq), torch.matmul(X, Wdq.t(), out=Y))
+            for f in (fused, unfused):
+                f()
+            med, p10, p90 = _time_kernel(fused, reps, flush)
+            umed = _time_kernel(unfused, reps, flush)[0]
+            fl = 2.0 * M * N * K
+            tf = fl / (med * 1e-3) / 1e12
+            out["results"].append({"M": M, "N": N, "K": K, "ms": med, "p10": p10, "p90": p90,
+                                   "TFLOP/s": tf, "frac_bf16_burst": tf / peaks["bf16_tflops"],
+                                   "frac_bf16_sustained": tf / peaks["bf16_tflops_sustained"],
+                                   "unfused_ms": umed,
+                                   "unfused": "w4_fake_quant + torch.matmul (cuBLAS BF16)"})
     elif args.workload == "gemv":
         # the decode GEMM alone, one activation height at a time (--m picks one)
         cfg = synth.Decode()
@@ -685,7 +709,8 @@ def main():
                          "the token count T (--workload moe)")
     ap.add_argument("--block", type=int, default=0, help="--workload moe: one block size only")
     ap.add_argument("--workload", default="decode",
-                    choices=["decode", "prefill", "moe", "moe_layer", "qat", "gemv", "quant"],
+                    choices=["decode", "prefill", "moe", "moe_layer", "qat", "qat_gemm", "gemv",
+                             "quant"],
                     help="decode is the bench line; the others print their own lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=512)

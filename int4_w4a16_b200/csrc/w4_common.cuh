@@ -123,6 +123,30 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
     }
 }
 
+// Non-blocking test of the phase with the given parity (acquire on success).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait of a single thread on the critical path (the MMA issuer): a short spin
+// of non-blocking tests, whose latency is well below that of a suspending
+// try_wait when the phase is already complete, then the bounded wait above.
+constexpr int kSpinTests = 64;
+__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity,
+                                               volatile int *abort_flag) {
+    for (int i = 0; i < kSpinTests; ++i)
+        if (mbar_test(bar, parity)) return true;
+    return mbar_wait(bar, parity, abort_flag);
+}
+
 // ---------------------------------------------------------------------------
 // Proxy fences
 // ---------------------------------------------------------------------------

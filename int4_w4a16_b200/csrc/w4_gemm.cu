@@ -54,9 +54,10 @@ namespace {
 // k-blocks only) kPermWarps warps that reorder the activation chunks, then
 // 4 epilogue warps (each drains the accumulators of its TMEM lane quarter),
 // then NSPLIT MMA issuer warps: lane 0 of issuer i issues every NSPLIT-th
-// 16-wide K step into accumulator i.  A thread issues a small tcgen05.mma only
-// about every 110 cycles (issue latency, not the tensor core), so small-N
-// tiles need several issuers to keep up with HBM.
+// 16-wide K step into accumulator i.  A thread issues a tcgen05.mma only about
+// every 100 cycles (issue latency, not the tensor core), and each k-block adds
+// a barrier poll and two commits, so small-N tiles need several issuers to
+// keep up with HBM.
 __host__ __device__ constexpr int perm_warps(int kb) { return kb == 256 ? 2 : 0; }
 __host__ __device__ constexpr int gemm_threads(int ndq, int kb, int nsplit, bool wgl) {
     return wgl ? 128 * (ndq + 4) : 32 * (1 + 4 * ndq + perm_warps(kb) + 4 + nsplit);
@@ -701,25 +702,24 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                 }
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(d * kAccCols + ji * MT);
-                for (int kb = kb0; kb < kb1; ++kb, ++it) {
-                    const int s = it % NSTAGE;
-                    const int a = it % NASTAGE;
-                    // the stage's loads landed (with 256-wide k-blocks the A slot's
-                    // barrier also covers the activation reorder, which itself
-                    // waited for the loads)
-                    if (!kXPerm && !warp_wait(full_bar(s), (it / NSTAGE) & 1u, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    if (!warp_wait(afull_bar(a), (it / NASTAGE) & 1u, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after_sync();
-                    if (lane == 0) {
+                // Lane 0 alone polls and issues: a warp-wide wait adds a vote to
+                // every poll, and each poll sits on the issue path between two
+                // k-blocks' MMAs.  The issuer waits only for the A slot: the
+                // threads that arrive on it (the dequant group, plus the
+                // activation-reorder warps with 256-wide k-blocks) each waited
+                // for the stage's loads first, so the acquire of the A slot's
+                // phase also orders the loaded tiles before these MMAs.
+                if (lane == 0) {
+                    for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                        const int s = it % NSTAGE;
+                        const int a = it % NASTAGE;
+                        if (!mbar_wait_spin(afull_bar(a), (it / NASTAGE) & 1u, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after_sync();
                         if (MOE) fence_proxy_async_smem();   // cp.async (generic proxy) -> MMA
-                        const uint32_t a_tmem =
-                            tmem_base + (uint32_t)(kABase + a * kAStageCols);
+                        const uint32_t a_tmem = tmem_base + (uint32_t)(kABase + a * kAStageCols);
 #pragma unroll
                         for (int u = ji; u < KB / 16; u += NSPLIT) {
                             const uint32_t baddr =
@@ -730,8 +730,11 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                         tc_commit(empty_bar(s));
                         tc_commit(aempty_bar(a));
                     }
-                    __syncwarp();
+                } else {
+                    it += (uint32_t)(kb1 - kb0);
                 }
+                ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+                it = __shfl_sync(0xFFFFFFFFu, it, 0);
                 if (!ok) break;
                 if (lane == 0) tc_commit(accfull_bar(d));
                 __syncwarp();

@@ -117,22 +117,51 @@ __device__ __forceinline__ uint4 dequant8_fast(const float (&c)[8], float s, flo
 }
 
 
+// Packed pairs of fp32 (sm_100 f32x2 arithmetic: one instruction per two
+// lanes of an IEEE fma / add, each rounded to nearest even as the scalar form).
+__device__ __forceinline__ uint64_t f2_splat(float x) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(x));
+    return r;
+}
+// The two BF16 halves of a word, widened exactly: {low half, high half}.
+__device__ __forceinline__ uint64_t f2_from_bf16x2(uint32_t w) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(w << 16), "r"(w & 0xFFFF0000u));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// Both lanes rounded to BF16 (nearest even), low lane into the low half.
+__device__ __forceinline__ uint32_t f2_to_bf16x2(uint64_t d) {
+    uint32_t r;
+    asm("{\n\t.reg .f32 lo, hi;\n\tmov.b64 {lo, hi}, %1;\n\tcvt.rn.bf16x2.f32 %0, hi, lo;\n\t}"
+        : "=r"(r)
+        : "l"(d));
+    return r;
+}
+
 // One group of 32 BF16 values (16 words, natural order) -> the 16 BF16x2 words
 // of bf16_rne(q * s), natural order; exact for every finite input (the slow
 // path divides in IEEE fp32 for zero, subnormal or huge scales).
 __device__ __forceinline__ void fake_quant_group(const uint32_t (&v)[16], uint32_t (&o)[16]) {
     const GroupScale gs = make_scale(group_amax_bits(v));
     if (gs.mode == 1 && gs.s <= 1.2676506e30f) {
-        const float neg_cs = -kMagic * gs.s;
+        // code_fast and dequant8_fast's arithmetic, two weights per instruction
+        const uint64_t r2 = f2_splat(gs.r), snap2 = f2_splat(kSnap), toint2 = f2_splat(kToInt);
+        const uint64_t s2 = f2_splat(gs.s), ncs2 = f2_splat(-kMagic * gs.s);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            float cd[8];
-            codes8_fast(make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]), gs.r, cd);
-            const uint4 d = dequant8_fast(cd, gs.s, neg_cs);
-            o[4 * c] = d.x;
-            o[4 * c + 1] = d.y;
-            o[4 * c + 2] = d.z;
-            o[4 * c + 3] = d.w;
+        for (int j = 0; j < 16; ++j) {
+            const uint64_t c = f2_add(f2_fma(f2_from_bf16x2(v[j]), r2, snap2), toint2);
+            o[j] = f2_to_bf16x2(f2_fma(c, s2, ncs2));
         }
     } else {
         const float s = gs.s;
