@@ -56,6 +56,9 @@ def load_library(path: str) -> ctypes.CDLL:
     L.w4o_quantize.argtypes = [_P, _I64, _I64, _I64, _P, _P]
     L.w4o_fake_quant.argtypes = [_P, _I64, _I64, _I64, _P, _P]
     L.w4o_ste_backward.argtypes = [_P, _I64, _P]
+    L.w4o_pack8_u.restype = ctypes.c_int32
+    L.w4o_pack8_u.argtypes = [_P]
+    L.w4o_unpack8_u.argtypes = [ctypes.c_int32, _P]
     L.w4o_pack8.restype = ctypes.c_int32
     L.w4o_pack8.argtypes = [_P]
     L.w4o_unpack8.argtypes = [ctypes.c_int32, _P]
@@ -66,6 +69,9 @@ def load_library(path: str) -> ctypes.CDLL:
     L.w4o_symmetric_quantize_f64.argtypes = [_P, _I64, _I64, ctypes.c_int, _P, _P]
     L.w4o_gemm.argtypes = [_P, _P, _I64, _I64, _I64, _P, _P]
     L.w4o_w4a16_gemm.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _P]
+    L.w4o_quantize_zp.argtypes = [_P, _I64, _I64, _I64, _P, _P, _P]
+    L.w4o_quantize_pack_zp.argtypes = [_P, _I64, _I64, _I64, _P, _P, _P]
+    L.w4o_dequant_zp.argtypes = [_P, _P, _P, _I64, _I64, _I64, _P]
     L.w4o_moe_align.restype = ctypes.c_int
     L.w4o_moe_align.argtypes = [_P, _I64, _I64, _I64, _I64, _P, _I64, _P, _P]
     L.w4o_moe_gemm.argtypes = [_P, _I64, _P, _P, _P, _I64, _I64, _I64, _I64,
@@ -176,6 +182,64 @@ def dequant(Wq: np.ndarray, S: np.ndarray, group: int = 32) -> np.ndarray:
     Wdq = np.empty((rows, K), np.uint16)
     lib().w4o_dequant(_ptr(Wq), _ptr(S), rows, K, group, _ptr(Wdq))
     return Wdq
+
+
+# ---- asymmetric (zero-point) quantization ---------------------------------
+
+def quantize_zp(W: np.ndarray, group: int = 32):
+    """(q uint8 [rows, K] in [0, 15], S bf16-bits [rows, K/group], Z uint8 [rows, K/group])."""
+    W = _u16(W)
+    rows, K = W.shape
+    q = np.empty((rows, K), np.uint8)
+    S = np.empty((rows, K // group), np.uint16)
+    Z = np.empty((rows, K // group), np.uint8)
+    lib().w4o_quantize_zp(_ptr(W), rows, K, group, _ptr(q), _ptr(S), _ptr(Z))
+    return q, S, Z
+
+
+def pack_u(q: np.ndarray) -> np.ndarray:
+    """Unsigned codes in [0, 15] (last dim a multiple of 8) -> int32 words."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    flat = q.reshape(-1, 8)
+    words = np.array([lib().w4o_pack8_u(_ptr(np.ascontiguousarray(r))) for r in flat], np.int32)
+    return words.reshape(q.shape[:-1] + (q.shape[-1] // 8,))
+
+
+def unpack_u(words: np.ndarray) -> np.ndarray:
+    words = np.ascontiguousarray(words, dtype=np.int32)
+    out = np.empty(words.size * 8, np.uint8)
+    for j, w in enumerate(words.reshape(-1)):
+        buf = np.empty(8, np.uint8)
+        lib().w4o_unpack8_u(ctypes.c_int32(int(w)), _ptr(buf))
+        out[8 * j:8 * j + 8] = buf
+    return out.reshape(words.shape[:-1] + (words.shape[-1] * 8,))
+
+
+def quantize_pack_zp(W: np.ndarray, group: int = 32):
+    """(Wq int32 [rows, K/8], S bf16-bits [rows, K/group], Z uint8 [rows, K/group])."""
+    W = _u16(W)
+    rows, K = W.shape
+    Wq = np.empty((rows, K // 8), np.int32)
+    S = np.empty((rows, K // group), np.uint16)
+    Z = np.empty((rows, K // group), np.uint8)
+    lib().w4o_quantize_pack_zp(_ptr(W), rows, K, group, _ptr(Wq), _ptr(S), _ptr(Z))
+    return Wq, S, Z
+
+
+def dequant_zp(Wq: np.ndarray, S: np.ndarray, Z: np.ndarray, group: int = 32) -> np.ndarray:
+    Wq = np.ascontiguousarray(Wq, dtype=np.int32)
+    S = _u16(S)
+    Z = np.ascontiguousarray(Z, dtype=np.uint8)
+    rows, K = Wq.shape[0], Wq.shape[1] * 8
+    Wdq = np.empty((rows, K), np.uint16)
+    lib().w4o_dequant_zp(_ptr(Wq), _ptr(S), _ptr(Z), rows, K, group, _ptr(Wdq))
+    return Wdq
+
+
+def w4a16_gemm_zp(X: np.ndarray, Wq: np.ndarray, S: np.ndarray, Z: np.ndarray,
+                  group: int = 32, want_r: bool = True):
+    """Y = X · dequant_zp(Wq, S, Z)^T, by the plain GEMM definition."""
+    return gemm(X, dequant_zp(Wq, S, Z, group), want_r)
 
 
 def symmetric_quantize_f64(x: np.ndarray, qmax: int, group: int | None = None):

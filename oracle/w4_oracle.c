@@ -249,6 +249,127 @@ void w4o_dequant(const int32_t *Wq, const uint16_t *S, int64_t rows, int64_t K,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Group-32 asymmetric (zero-point) INT4 quantization: the affine map of     */
+/* [BAS] §2.1 (q = clamp(round(x / s) + z, q_min, q_max), x^ = (q - z) * s)  */
+/* with the asymmetric scale and zero point of [BAS] §2.3                    */
+/* (s = (x_max - x_min) / (q_max - q_min), z = clamp(round(q_min - x_min/s)))*/
+/* over the unsigned INT4 range q_min = 0, q_max = 15.  x_max and x_min are  */
+/* the group's own extremes; the scale is stored in BF16 like the symmetric  */
+/* one, the zero point as one byte per group.  A group with s == 0 (all      */
+/* values equal) gets q = z = 0.                                             */
+/* ------------------------------------------------------------------------ */
+
+static uint16_t quantize_one_group_zp(const uint16_t *w, int64_t n, uint8_t *q,
+                                      uint8_t *z_out)
+{
+    /* step 1: the group's extremes, on the BF16 values */
+    float xmax = w4o_f32_from_bf16(w[0]), xmin = xmax;
+    for (int64_t i = 1; i < n; ++i) {
+        float x = w4o_f32_from_bf16(w[i]);
+        if (x > xmax) xmax = x;
+        if (x < xmin) xmin = x;
+    }
+    /* step 2: s = (x_max - x_min) / 15 in IEEE fp32, stored as BF16 */
+    volatile float fifteen = 15.0f;
+    float range = xmax - xmin;
+    float s32 = range / fifteen;
+    uint16_t s_bits = w4o_bf16_from_f32(s32);
+    const float s = w4o_f32_from_bf16(s_bits);
+    if (s == 0.0f) {
+        for (int64_t i = 0; i < n; ++i) q[i] = 0;
+        *z_out = 0;
+        return s_bits;
+    }
+    /* step 3: z = clamp(round_half_even(0 - x_min / s), 0, 15) */
+    float zf = nearbyintf(0.0f - xmin / s);
+    if (zf < 0.0f) zf = 0.0f;
+    if (zf > 15.0f) zf = 15.0f;
+    /* step 4: q = clamp(round_half_even(x / s) + z, 0, 15) */
+    for (int64_t i = 0; i < n; ++i) {
+        float y = w4o_f32_from_bf16(w[i]) / s;      /* IEEE fp32 quotient */
+        float v = nearbyintf(y) + zf;
+        if (v < 0.0f) v = 0.0f;
+        if (v > 15.0f) v = 15.0f;
+        q[i] = (uint8_t)v;
+    }
+    *z_out = (uint8_t)zf;
+    return s_bits;
+}
+
+/* q[rows*K] codes in [0, 15], S[rows*(K/group)] BF16 scales, Z zero points. */
+void w4o_quantize_zp(const uint16_t *W, int64_t rows, int64_t K, int64_t group,
+                     uint8_t *q, uint16_t *S, uint8_t *Z)
+{
+    int64_t gpr = K / group;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t g = 0; g < gpr; ++g) {
+            int64_t base = r * K + g * group;
+            S[r * gpr + g] = quantize_one_group_zp(W + base, group, q + base, Z + r * gpr + g);
+        }
+}
+
+/* Dequantized value of one code: bf16_rne((q - z) * s), +0.0 for q == z.
+ * (q - z) * s is exact in fp32 (4 x 8 significant bits); the BF16 rounding
+ * is the one step that can round. */
+static uint16_t dequant_one_zp(uint8_t q, uint8_t z, uint16_t s_bits)
+{
+    float s = w4o_f32_from_bf16(s_bits);
+    float v = (float)((int)q - (int)z) * s;
+    if (v == 0.0f) v = 0.0f;
+    return w4o_bf16_from_f32(v);
+}
+
+/* Eight unsigned codes <-> one word, element i at bits [4i, 4i+3]. */
+int32_t w4o_pack8_u(const uint8_t *q8)
+{
+    uint32_t word = 0;
+    for (int i = 0; i < 8; ++i)
+        word |= (uint32_t)(q8[i] & 0xFu) << (4 * i);
+    return (int32_t)word;
+}
+
+void w4o_unpack8_u(int32_t word, uint8_t *q8)
+{
+    uint32_t u = (uint32_t)word;
+    for (int i = 0; i < 8; ++i) q8[i] = (uint8_t)((u >> (4 * i)) & 0xFu);
+}
+
+/* Export: Wq[rows*(K/8)] packed unsigned codes, S BF16 scales, Z zero points. */
+void w4o_quantize_pack_zp(const uint16_t *W, int64_t rows, int64_t K, int64_t group,
+                          int32_t *Wq, uint16_t *S, uint8_t *Z)
+{
+    int64_t gpr = K / group;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        uint8_t *qrow = (uint8_t *)malloc((size_t)K);
+        for (int64_t g = 0; g < gpr; ++g)
+            S[r * gpr + g] = quantize_one_group_zp(W + r * K + g * group, group,
+                                                   qrow + g * group, Z + r * gpr + g);
+        for (int64_t j = 0; j < K / 8; ++j) Wq[r * (K / 8) + j] = w4o_pack8_u(qrow + 8 * j);
+        free(qrow);
+    }
+}
+
+void w4o_dequant_zp(const int32_t *Wq, const uint16_t *S, const uint8_t *Z, int64_t rows,
+                    int64_t K, int64_t group, uint16_t *Wdq)
+{
+    int64_t gpr = K / group;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        uint8_t q8[8];
+        for (int64_t j = 0; j < K / 8; ++j) {
+            w4o_unpack8_u(Wq[r * (K / 8) + j], q8);
+            for (int i = 0; i < 8; ++i) {
+                int64_t k = 8 * j + i;
+                int64_t g = r * gpr + k / group;
+                Wdq[r * K + k] = dequant_one_zp(q8[i], Z[g], S[g]);
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
 /* Generic symmetric quantizer of [BAS] §2.2 / §6.1, in fp64, with the scale */
 /* left unrounded: s = max|x| / qmax per group, q = clip(round(x/s)).       */
 /* Used to reproduce the page's worked INT8 example.                         */

@@ -49,6 +49,21 @@ MUTANTS = [
      [pins.test_moe_combine_reference_and_one_hot]),
     ("moe_align_no_pad", "total += (cnt[e] + block - 1) / block * block;", "total += cnt[e];",
      [lambda: [pins.test_moe_align_brute_force(s) for s in range(40)]]),
+    ("zp_sign_flipped", "float zf = nearbyintf(0.0f - xmin / s);", "float zf = nearbyintf(xmin / s);",
+     [lambda: pins.test_zp_exact_ramps(-5, 1)]),
+    ("zp_dequant_adds_z", "float v = (float)((int)q - (int)z) * s;", "float v = (float)((int)q + (int)z) * s;",
+     [lambda: pins.test_zp_exact_ramps(-5, 1)]),
+    ("zp_no_upper_z_clamp", "if (zf > 15.0f) zf = 15.0f;", "",
+     [pins.test_zp_brute_force_codes_and_zero_points]),
+    ("zp_no_lower_z_clamp", "if (zf < 0.0f) zf = 0.0f;", "",
+     [pins.test_zp_brute_force_codes_and_zero_points]),
+    ("zp_range_is_max", "float range = xmax - xmin;", "float range = xmax;",
+     [lambda: pins.test_zp_exact_ramps(-5, 1)]),
+    ("zp_round_half_away", "float v = nearbyintf(y) + zf;", "float v = roundf(y) + zf;",
+     [pins.test_zp_brute_force_codes_and_zero_points]),
+    ("zp_pack_high_first", "word |= (uint32_t)(q8[i] & 0xFu) << (4 * i);",
+     "word |= (uint32_t)(q8[i] & 0xFu) << (4 * (7 - i));",
+     [pins.test_zp_pack_examples]),
     # (random fp64 data has no exact ties, so the tie rule of this path is pinned
     # by group A through the INT4 path, not by the printed example)
     ("p4_scale_off_by_one", "double s = amax / (double)qmax;",
@@ -86,3 +101,5 @@ def test_unmutated_copy_passes(tmp_path, monkeypatch):
     pins.test_hand_groups("group_B")
     pins.test_pack_examples()
     pins.test_gemm_one_hot_is_exact()
+    pins.test_zp_exact_ramps(-5, 1)
+    pins.test_zp_pack_examples()

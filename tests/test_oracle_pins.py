@@ -422,3 +422,106 @@ def test_silu_mul_closed_forms():
     assert h[3] == 30.0                           # silu(x) -> x for large x
     assert abs(h[4]) < 1e-11                      # silu(x) -> 0 for very negative x
     assert np.all(np.abs(h - want) <= 2.0 ** -8 * np.abs(want))   # one BF16 rounding
+
+
+# ---------------------------------------------------------------------------
+# Asymmetric (zero-point) groups: the affine map of the quantization tutorial
+# (§2.1) with the asymmetric scale and zero point of its §2.3, unsigned INT4
+# codes [0, 15].  Pinned by exact ramps, by brute force over the 16 codes in
+# exact rational arithmetic, and by the tutorial's |x^ - x| <= s/2 bound (§2.4).
+# ---------------------------------------------------------------------------
+
+def _zp_group(values, exact=True):
+    bits = np.array([fraction_to_bf16_bits(Fraction(v)) for v in values], np.uint16)
+    if exact:
+        assert [bf16_bits_to_fraction(int(b)) for b in bits] == [Fraction(v) for v in values]
+    return bits.reshape(1, -1)
+
+
+@pytest.mark.parametrize("lo,step", [(0, 1), (-5, 1), (-15, 1), (-7, Fraction(1, 64)),
+                                     (-3, 4), (0, Fraction(3, 8))])
+def test_zp_exact_ramps(lo, step):
+    # values lo*step ... (lo+15)*step, twice: x_max - x_min = 15 step, so s = step,
+    # z = -lo, every code q = i and x^ = x exactly
+    vals = [Fraction(lo + i) * step for i in range(16)] * 2
+    q, S, Z = oracle.quantize_zp(_zp_group(vals))
+    assert bf16_bits_to_fraction(int(S[0, 0])) == Fraction(step)
+    assert int(Z[0, 0]) == -lo
+    assert q[0].tolist() == list(range(16)) * 2
+    Wq, S2, Z2 = oracle.quantize_pack_zp(_zp_group(vals))
+    back = [bf16_bits_to_fraction(int(b)) for b in oracle.dequant_zp(Wq, S2, Z2)[0]]
+    assert back == vals
+
+
+def _brute_zp(vals, s, z):
+    """Codes by brute force: the nearest of (c - z) * s, c in [0, 15], to each x,
+    ties to the even c - z; exact rationals."""
+    out = []
+    for x in vals:
+        best = None
+        for c in range(16):
+            d = abs(x - (c - z) * s)
+            key = (d, (c - z) % 2)
+            if best is None or key < best[0]:
+                best = (key, c)
+        out.append(best[1])
+    return out
+
+
+def test_zp_brute_force_codes_and_zero_points():
+    rng = random.Random(7)
+    for trial in range(300):
+        kind = trial % 5
+        if kind == 0:      # straddles zero
+            vals = [Fraction(rng.randint(-200, 200), 64) for _ in range(32)]
+        elif kind == 1:    # all positive: z clamps at 0, top codes clamp at 15
+            vals = [Fraction(rng.randint(40, 300), 32) for _ in range(32)]
+        elif kind == 2:    # all negative: z clamps at 15
+            vals = [Fraction(-rng.randint(40, 300), 32) for _ in range(32)]
+        elif kind == 3:    # wide dynamic range
+            vals = [Fraction(rng.choice([-1, 1]) * rng.randint(1, 255), 2 ** rng.randint(0, 12))
+                    for _ in range(32)]
+        else:              # few distinct values, many ties
+            vals = [Fraction(rng.randint(-8, 8), 4) for _ in range(32)]
+        bits = _zp_group(vals, exact=False)     # rounded to BF16, then read back
+        vals = [bf16_bits_to_fraction(int(b)) for b in bits[0]]
+        q, S, Z = oracle.quantize_zp(bits)
+        s = bf16_bits_to_fraction(int(S[0, 0]))
+        rng_x = max(vals) - min(vals)
+        if rng_x == 0:
+            assert s == 0 and int(Z[0, 0]) == 0 and q.max() == 0
+            continue
+        # s is the BF16 nearest (within half a BF16 ulp, plus the fp32 step) to range / 15
+        assert abs(s - rng_x / 15) <= s / 256 + s / 2 ** 20, (trial, s, rng_x)
+        # z: the integer in [0, 15] nearest to -x_min / s, ties to even
+        zt = -min(vals) / s
+        zc = min(range(16), key=lambda c: (abs(c - zt), c % 2))
+        assert int(Z[0, 0]) == zc, (trial, zt)
+        assert q[0].tolist() == _brute_zp(vals, s, zc), trial
+        # the group's minimum maps to code 0 whenever z is not clamped
+        if 0 <= round_half_even(zt) <= 15:
+            assert q[0][vals.index(min(vals))] == 0
+
+
+def test_zp_error_bound_half_step():
+    rng = np.random.default_rng(11)
+    x = (rng.standard_normal((64, 256)) * 0.05 + rng.uniform(-0.05, 0.05, (64, 1))).astype(np.float32)
+    W = oracle.f32_to_bf16_bits(x)
+    Wq, S, Z = oracle.quantize_pack_zp(W)
+    back = oracle.bf16_to_f32(oracle.dequant_zp(Wq, S, Z)).astype(np.float64)
+    xv = oracle.bf16_to_f32(W).astype(np.float64)
+    s = np.repeat(oracle.bf16_to_f32(S).astype(np.float64), 32, axis=1)
+    z = np.repeat(Z.astype(np.int64), 32, axis=1)
+    unclamped = (np.rint(xv / s) + z >= 0) & (np.rint(xv / s) + z <= 15)
+    assert unclamped.mean() > 0.99
+    # |x^ - x| <= s / 2, plus the BF16 rounding of (q - z) * s (half an ulp, 2^-8 relative)
+    err = np.abs(back - xv)
+    assert np.all(err[unclamped] <= s[unclamped] / 2 + np.abs(back[unclamped]) * 2.0 ** -8 + 1e-30)
+
+
+def test_zp_pack_examples():
+    assert oracle.pack_u(np.arange(8, dtype=np.uint8))[0] == 0x76543210
+    w = oracle.pack_u(np.arange(8, 16, dtype=np.uint8))[0]
+    assert (int(w) & 0xFFFFFFFF) == 0xFEDCBA98
+    words = np.array([0x76543210, np.int32(-0x01234568)], np.int32)     # 0xFEDCBA98
+    assert oracle.unpack_u(words).tolist() == list(range(16))
