@@ -2,7 +2,7 @@
 """Benchmark of the INT4 W4A16 hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode|prefill|moe|moe_layer|qat|qat_gemm|gemv|quant]
+                    [--workload decode|prefill|moe|moe_layer|qat|qat_gemm|gemv|quant|zp]
 
 Default workload: the decode GEMV sweep -- W[12288, 4096] BF16 ~ N(0, 0.02^2)
 with 0.1 % x20 outliers, group 32, activations X[M, 4096] ~ N(0, 1) for
@@ -579,6 +579,44 @@ def run_extra(args):
                                    "layer_fused_us": fmed * 1e3,
                                    "fused_frac": nb_fused / (fmed * 1e-3) / 1e9 / peaks["hbm_gbs"],
                                    "per_kernel_us": per})
+    elif args.workload == "zp":
+        # asymmetric (zero-point) groups: quantizer on the decode sweep's weights
+        # (W[12288, 4096]), then the GEMM on that shape at decode and prefill
+        # token counts, the symmetric path beside it
+        cfg = synth.Decode()
+        W = cfg.weight(dev)
+        n = W.numel()
+        Wq = torch.empty((cfg.N, cfg.K // 8), dtype=torch.int32, device=dev)
+        S = torch.empty((cfg.N, cfg.K // 32), dtype=torch.bfloat16, device=dev)
+        Z = torch.empty((cfg.N, cfg.K // 32), dtype=torch.uint8, device=dev)
+        fq = lambda: w4.w4_quantize_pack_zp(W, Wq, S, Z)
+        for _ in range(3):
+            fq()
+        med, p10, p90 = _time_kernel(fq, reps, flush)
+        bpe = 2.0 + 0.5 + 3.0 / 32          # W read; codes, scale and zero point written
+        gbs = n * bpe / (med * 1e-3) / 1e9
+        out["results"].append({"kernel": "quantize_pack_zp", "elements": n, "us": med * 1e3,
+                               "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"]})
+        Wq_s, S_s = w4.quantize_pack(W)
+        del W
+        for M in ([args.m] if args.m else (1, 16, 512, 2048)):
+            X = synth.normal_bf16((M, cfg.K), 1.0, 0, 500 + M, dev)
+            Y = torch.empty((M, cfg.N), dtype=torch.bfloat16, device=dev)
+            fz = lambda: w4.w4a16_gemm_zp(X, Wq, S, Z, Y)
+            fs = lambda: w4.w4a16_gemm(X, Wq_s, S_s, Y)
+            for f in (fz, fs):
+                for _ in range(3):
+                    f()
+            med, p10, p90 = _time_kernel(fz, reps, flush)
+            smed = _time_kernel(fs, reps, flush)[0]
+            byts = cfg.N * cfg.K * (0.5 + 3.0 / 32) + 2.0 * M * (cfg.K + cfg.N)
+            fl = 2.0 * M * cfg.N * cfg.K
+            out["results"].append({"kernel": "w4a16_gemm_zp", "M": M, "N": cfg.N, "K": cfg.K,
+                                   "us": med * 1e3, "GB/s": byts / (med * 1e-3) / 1e9,
+                                   "frac_hbm": byts / (med * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                   "TFLOP/s": fl / (med * 1e-3) / 1e12,
+                                   "frac_bf16_burst": fl / (med * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                                   "symmetric_us": smed * 1e3})
     elif args.workload == "qat_gemm":
         # QAT forward GEMM on a layer of the QAT stack (W[12288, 4096]) with the
         # fake quantization fused into the weight prologue, beside the unfused
@@ -710,7 +748,7 @@ def main():
     ap.add_argument("--block", type=int, default=0, help="--workload moe: one block size only")
     ap.add_argument("--workload", default="decode",
                     choices=["decode", "prefill", "moe", "moe_layer", "qat", "qat_gemm", "gemv",
-                             "quant"],
+                             "quant", "zp"],
                     help="decode is the bench line; the others print their own lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=512)

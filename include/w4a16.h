@@ -195,6 +195,40 @@ w4_status w4a16_gemm_noalloc(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 
 w4_status w4_qat_gemm(const w4_bf16 *X, const w4_bf16 *W, w4_bf16 *Y, int64_t M, int64_t N,
                       int64_t K, int group, void *stream);
 
+/*
+ * Asymmetric (zero-point) groups -- [BAS] §2.1 (affine map q = clamp(round(x/s)
+ * + z, q_min, q_max), x^ = (q - z) * s) and §2.3 (s = (x_max - x_min) /
+ * (q_max - q_min), z = clamp(round(q_min - x_min / s))), over the unsigned INT4
+ * range q_min = 0, q_max = 15 of the GPTQ / AWQ formats (P1: "compatible with
+ * GPTQ and AWQ").  Per group of 32 along K:
+ *   s = bf16_rne(fl32(fl32(x_max - x_min) / 15)),
+ *   z = clamp(rint_even(0 - fl32(x_min / s)), 0, 15),
+ *   q = clamp(rint_even(fl32(x / s)) + z, 0, 15);  q = z = 0 when s == 0,
+ *   x^ = bf16_rne((q - z) * s).
+ *   W    in   [rows, K] BF16
+ *   Wq   out  [rows, K/8] int32, low-nibble-first unsigned codes
+ *   S    out  [rows, K/32] BF16 scales
+ *   Z    out  [rows, K/32] uint8 zero points in [0, 15]
+ * Same argument rules as w4_quantize_pack (Z: any alignment, not NULL).
+ */
+w4_status w4_quantize_pack_zp(const w4_bf16 *W, int32_t *Wq, w4_bf16 *S, uint8_t *Z,
+                              int64_t rows, int64_t K, int group, void *stream);
+
+/* Unpack + dequantize asymmetric groups: Wdq = bf16_rne((q - Z) * S). */
+w4_status w4_dequant_zp(const int32_t *Wq, const w4_bf16 *S, const uint8_t *Z, w4_bf16 *Wdq,
+                        int64_t rows, int64_t K, int group, void *stream);
+
+/*
+ * W4A16 GEMM on asymmetric groups: Y[M, N] = X[M, K] . dequant_zp(Wq, S, Z)^T,
+ * fp32 accumulation, BF16 output (the zero point is subtracted in the same
+ * register unpack as w4a16_gemm's constant bias, no extra instruction).  Every M
+ * runs the tensor-memory kernel with 64-wide k-blocks (no warp-level decode
+ * kernel for this format).  K a multiple of 32; group 32; X, Wq, S, Y 16-byte
+ * aligned; Z not NULL.  Device pointers; the call is asynchronous on `stream`.
+ */
+w4_status w4a16_gemm_zp(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S, const uint8_t *Z,
+                        w4_bf16 *Y, int64_t M, int64_t N, int64_t K, int group, void *stream);
+
 /* Padded capacity the caller must provide for w4_moe_align's sorted_ids:
  * T*topk + E*(block-1), rounded up to a multiple of block.  Host-only. */
 int64_t w4_moe_capacity(int64_t T, int topk, int E, int block);

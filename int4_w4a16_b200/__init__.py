@@ -29,6 +29,8 @@ __all__ = [
     "w4_quantize_pack", "w4_dequant", "w4a16_gemm", "w4_moe_capacity", "w4_moe_align",
     "w4_moe_w4a16_gemm", "w4_moe_w4a16_gemm_silu", "w4_moe_gate_topk", "w4_moe_block_size",
     "w4_silu_mul", "moe_gemm_silu", "w4_qat_gemm", "qat_gemm",
+    "w4_quantize_pack_zp", "w4_dequant_zp", "w4a16_gemm_zp", "quantize_pack_zp", "dequant_zp",
+    "gemm_zp",
     "w4_moe_combine", "fake_quant", "quantize_pack", "dequant", "gemm", "moe_align",
     "moe_gate_topk", "silu_mul", "moe_combine",
     "moe_gemm", "FakeInt4STE", "GROUP",
@@ -80,6 +82,9 @@ def lib() -> ctypes.CDLL:
                                        _I64, _I64, _INT, _P],
             "w4_moe_gate_topk": [_P, _I64, _INT, _INT, _P, _P, _P],
             "w4_qat_gemm": [_P, _P, _P, _I64, _I64, _I64, _INT, _P],
+            "w4_quantize_pack_zp": [_P, _P, _P, _P, _I64, _I64, _INT, _P],
+            "w4_dequant_zp": [_P, _P, _P, _P, _I64, _I64, _INT, _P],
+            "w4a16_gemm_zp": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _INT, _P],
             "w4_silu_mul": [_P, _I64, _I64, _P, _P],
             "w4_moe_combine": [_P, _P, _I64, _INT, _I64, _P, _P],
             "w4_device_status": [_P],
@@ -271,6 +276,37 @@ def w4_qat_gemm(X, W, Y, group: int = GROUP, stream=None) -> None:
                                             _stream(stream)))
 
 
+def w4_quantize_pack_zp(W, Wq, S, Z, group: int = GROUP, stream=None) -> None:
+    """Asymmetric groups: unsigned codes Wq, BF16 scales S, uint8 zero points Z."""
+    _dtype(W, torch.bfloat16, "W")
+    _dtype(Wq, torch.int32, "Wq")
+    _dtype(S, torch.bfloat16, "S")
+    _dtype(Z, torch.uint8, "Z")
+    rows, K = W.shape
+    _check("w4_quantize_pack_zp", lib().w4_quantize_pack_zp(_ptr(W), _ptr(Wq), _ptr(S), _ptr(Z),
+                                                            rows, K, group, _stream(stream)))
+
+
+def w4_dequant_zp(Wq, S, Z, Wdq, group: int = GROUP, stream=None) -> None:
+    _dtype(Wq, torch.int32, "Wq")
+    _dtype(Z, torch.uint8, "Z")
+    rows, K = Wdq.shape
+    _check("w4_dequant_zp", lib().w4_dequant_zp(_ptr(Wq), _ptr(S), _ptr(Z), _ptr(Wdq), rows, K,
+                                                group, _stream(stream)))
+
+
+def w4a16_gemm_zp(X, Wq, S, Z, Y, group: int = GROUP, stream=None) -> None:
+    _dtype(X, torch.bfloat16, "X")
+    _dtype(Wq, torch.int32, "Wq")
+    _dtype(S, torch.bfloat16, "S")
+    _dtype(Z, torch.uint8, "Z")
+    _dtype(Y, torch.bfloat16, "Y")
+    M, K = X.shape
+    N = Wq.shape[0]
+    _check("w4a16_gemm_zp", lib().w4a16_gemm_zp(_ptr(X), _ptr(Wq), _ptr(S), _ptr(Z), _ptr(Y),
+                                                M, N, K, group, _stream(stream)))
+
+
 def w4_moe_gate_topk(logits, topk: int, topk_ids, topk_weights, stream=None) -> None:
     _dtype(logits, torch.float32, "logits")
     _dtype(topk_ids, torch.int32, "topk_ids")
@@ -325,6 +361,28 @@ def dequant(Wq: torch.Tensor, S: torch.Tensor) -> torch.Tensor:
     Wdq = torch.empty((rows, K8 * 8), dtype=torch.bfloat16, device=Wq.device)
     w4_dequant(Wq, S, Wdq)
     return Wdq
+
+
+def quantize_pack_zp(W: torch.Tensor):
+    rows, K = W.shape
+    Wq = torch.empty((rows, K // 8), dtype=torch.int32, device=W.device)
+    S = torch.empty((rows, K // GROUP), dtype=torch.bfloat16, device=W.device)
+    Z = torch.empty((rows, K // GROUP), dtype=torch.uint8, device=W.device)
+    w4_quantize_pack_zp(W, Wq, S, Z)
+    return Wq, S, Z
+
+
+def dequant_zp(Wq: torch.Tensor, S: torch.Tensor, Z: torch.Tensor) -> torch.Tensor:
+    rows, K8 = Wq.shape
+    Wdq = torch.empty((rows, K8 * 8), dtype=torch.bfloat16, device=Wq.device)
+    w4_dequant_zp(Wq, S, Z, Wdq)
+    return Wdq
+
+
+def gemm_zp(X: torch.Tensor, Wq: torch.Tensor, S: torch.Tensor, Z: torch.Tensor) -> torch.Tensor:
+    Y = torch.empty((X.shape[0], Wq.shape[0]), dtype=torch.bfloat16, device=X.device)
+    w4a16_gemm_zp(X, Wq, S, Z, Y)
+    return Y
 
 
 def gemm(X: torch.Tensor, Wq: torch.Tensor, S: torch.Tensor, ws="auto") -> torch.Tensor:

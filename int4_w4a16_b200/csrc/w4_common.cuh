@@ -386,6 +386,36 @@ __device__ __forceinline__ void dequant_word(uint32_t w, uint32_t s2, uint32_t (
     }
 }
 
+// Unsigned codes with a zero point (asymmetric groups): OR-ing a nibble into
+// BF16 128.0 (0x4300) gives 128 + q exactly; subtracting zb2 = (128 + z, 128 + z)
+// leaves q - z exactly (|q - z| <= 15), and one multiply by the scale rounds
+// (q - z) * s to BF16.  Same instruction count as dequant_word, natural order.
+__device__ __forceinline__ void dequant_word_zp(uint32_t w, uint32_t s2, uint32_t zb2,
+                                                uint32_t (&out)[4]) {
+    const uint32_t m = 0x000F000Fu, x = 0x43004300u;
+    uint32_t t0 = lop3_and_xor(w, m, x);          // codes 0, 4
+    uint32_t t1 = lop3_and_xor(w >> 4, m, x);     // codes 1, 5
+    uint32_t t2 = lop3_and_xor(w >> 8, m, x);     // codes 2, 6
+    uint32_t t3 = lop3_and_xor(w >> 12, m, x);    // codes 3, 7
+    uint32_t in[4] = {__byte_perm(t0, t1, 0x5410), __byte_perm(t2, t3, 0x5410),
+                      __byte_perm(t0, t1, 0x7632), __byte_perm(t2, t3, 0x7632)};
+    const __nv_bfloat162 zb = *reinterpret_cast<const __nv_bfloat162 *>(&zb2);
+    const __nv_bfloat162 sc = *reinterpret_cast<const __nv_bfloat162 *>(&s2);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162 *>(&in[j]);
+        v = __hsub2(v, zb);
+        v = __hmul2(v, sc);
+        out[j] = *reinterpret_cast<uint32_t *>(&v);
+    }
+}
+
+// (128 + z) in both BF16 halves, z in [0, 15]: bits 0x4300 | z.
+__device__ __forceinline__ uint32_t zp_bias2(uint32_t z) {
+    const uint32_t h = 0x4300u | (z & 0xFu);
+    return h | (h << 16);
+}
+
 // Same unpack without the pairing permutes: out[j] = (q_j * s, q_{j+4} * s).
 // Used with activations whose 8-element chunks are stored in the matching order
 // [x0, x4, x1, x5, x2, x6, x3, x7] (see permute_chunk8), which leaves the

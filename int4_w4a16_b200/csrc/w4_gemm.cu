@@ -87,6 +87,7 @@ constexpr int kTmemCols = 512;
 
 struct GemmParams {
     const uint16_t *S;           // scales (direct loads when KB < 256)
+    const uint8_t *Z;            // zero points of asymmetric groups (ZP), one byte per group
     uint16_t *Y;                 // dense: Y [M, N]; MoE: C [num_slots, N]
     const uint16_t *A;           // MoE: activation rows [a_rows, K]
     const int32_t *sorted_ids;   // MoE
@@ -285,13 +286,14 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 // issuer / accumulator u % NSPLIT, and the epilogue adds the accumulators in
 // a fixed order.
 template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT, int NDQ, bool MOE,
-          bool WGL, bool QAT>
+          bool WGL, bool QAT, bool ZP>
 __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
     w4a16_tc_kernel(const __grid_constant__ CUtensorMap tm_w,
                     const __grid_constant__ CUtensorMap tm_s,
                     const __grid_constant__ CUtensorMap tm_x, const GemmParams p) {
     using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE, NSPLIT, QAT>;
     static_assert(!QAT || (KB == 64 && !MOE), "QAT: 64-wide k-blocks of dense BF16 weights");
+    static_assert(!ZP || (KB == 64 && !MOE && !QAT), "zero points: dense 64-wide k-blocks");
     constexpr int kWords = KB / 8;             // packed words per row per k-block
     constexpr int kAStageCols = KB / 2;        // TMEM columns per A stage
     constexpr int kAccCols = NSPLIT * MT;      // TMEM columns per work item accumulator
@@ -502,6 +504,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                 if (MOE) base += (int64_t)__ldg(p.expert_ids + tt / p.moe_sub) * p.N * gpr;
                 srow = p.S + base;
             }
+            const uint8_t *zrow = (ZP && srow != nullptr) ? p.Z + (srow - p.S) : nullptr;
             for (int kb = kb0; kb < kb1; ++kb, ++it) {
                 if (it % NDQ != grp) continue;
                 const int s = it % NSTAGE;
@@ -542,14 +545,17 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                     continue;
                 }
                 static_assert(KB == 256 || G == 2, "direct-load scales: one chunk pair per k-block");
-                uint32_t sc[G];
+                uint32_t sc[G], zb[G];
                 if (KB != 256) {
-                    // scales of this k-block (direct loads when the tile has no TMA scales)
+                    // scales (and zero points) of this k-block (direct loads when the
+                    // tile has no TMA scales)
 #pragma unroll
                     for (int j = 0; j < G; ++j) {
                         const int64_t gi = (int64_t)kb * G + j;
                         const uint16_t v = (srow != nullptr && gi < gpr) ? __ldg(srow + gi) : 0;
                         sc[j] = bf16x2_splat(v);
+                        if (ZP)
+                            zb[j] = zp_bias2((zrow != nullptr && gi < gpr) ? __ldg(zrow + gi) : 0u);
                     }
                 }
                 if (!warp_wait(full_bar(s), (it / NSTAGE) & 1u, abort_flag)) {
@@ -586,6 +592,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                         for (int q = 0; q < 4; ++q) {
                             uint32_t t4[4];
                             if (kXPerm) dequant_word_k8perm(ws[q], scp[jj], t4);
+                            else if (ZP) dequant_word_zp(ws[q], scp[jj], zb[jj], t4);
                             else dequant_word(ws[q], scp[jj], t4);
 #pragma unroll
                             for (int z = 0; z < 4; ++z) o[jj * 16 + q * 4 + z] = t4[z];
@@ -1003,11 +1010,11 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
 // ---------------------------------------------------------------------------
 
 template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT, int NDQ, bool MOE,
-          bool WGL = false, bool QAT = false>
+          bool WGL = false, bool QAT = false, bool ZP = false>
 w4_status launch_cfg(const CUtensorMap &tw, const CUtensorMap &ts, const CUtensorMap &tx,
                      const GemmParams &p, int num_items_max, cudaStream_t stream) {
     using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE, NSPLIT, QAT>;
-    auto kern = w4a16_tc_kernel<KB, MT, NSTAGE, NACC, NASTAGE, NSPLIT, NDQ, MOE, WGL, QAT>;
+    auto kern = w4a16_tc_kernel<KB, MT, NSTAGE, NACC, NASTAGE, NSPLIT, NDQ, MOE, WGL, QAT, ZP>;
     // At least half of the SM's shared memory, so one CTA (and one TMEM
     // allocation of 512 columns) per SM.
     const int smem = std::max(L::kAlloc, 120 * 1024);
@@ -1279,6 +1286,58 @@ extern "C" w4_status w4_qat_gemm(const w4_bf16 *X, const w4_bf16 *W, w4_bf16 *Y,
     if (mt == 64)
         return launch_cfg<64, 64, 8, 1, 8, 4, 2, false, false, true>(tw, ts, tx, p, (int)items, st);
     return launch_cfg<64, 256, 4, 1, 8, 1, 2, false, false, true>(tw, ts, tx, p, (int)items, st);
+}
+
+extern "C" w4_status w4a16_gemm_zp(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S,
+                                   const uint8_t *Z, w4_bf16 *Y, int64_t M, int64_t N, int64_t K,
+                                   int group, void *stream) {
+    if (group != 32) return W4_ERR_UNSUPPORTED;
+    if (M < 0 || N < 0 || K <= 0 || (K % 32) != 0) return W4_ERR_INVALID_ARG;
+    if (!w4host::aligned16(X) || !w4host::aligned16(Wq) || !w4host::aligned16(S) ||
+        !w4host::aligned16(Y) || Z == nullptr)
+        return W4_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return W4_OK;
+    if (N > (1 << 30) || M > (1 << 30) || K > (1 << 24)) return W4_ERR_UNSUPPORTED;
+    cudaStream_t st = (cudaStream_t)stream;
+    GemmParams p = {};
+    p.S = reinterpret_cast<const uint16_t *>(S);
+    p.Z = Z;
+    p.Y = reinterpret_cast<uint16_t *>(Y);
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    // every M: 128-row tiles, 64-wide K blocks, scales and zero points read
+    // directly by the dequant warps
+    const int mt = M <= 64 ? 64 : 256;
+    p.rows_per_tile = 128;
+    p.n_row_tiles = ceil_div_i(N, 128);
+    p.n_tok_tiles = ceil_div_i(M, mt);
+    p.num_kb = ceil_div_i(K, 64);
+    CUtensorMap tw, ts, tx;
+    memset(&ts, 0, sizeof ts);
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+        cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+        cuuint32_t box[2] = {64u, (cuuint32_t)mt};
+        if (!make_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+            return W4_ERR_CUDA;
+    }
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)(K / 8), (cuuint64_t)N};
+        cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+        cuuint32_t box[2] = {8u, 128u};
+        if (!make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_INT32, 2, Wq, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_32B))
+            return W4_ERR_CUDA;
+    }
+    const int64_t items = (int64_t)p.n_row_tiles * p.n_tok_tiles;
+    if (items > (1 << 30)) return W4_ERR_UNSUPPORTED;
+    if (mt == 64)
+        return launch_cfg<64, 64, 8, 1, 8, 4, 2, false, false, false, true>(tw, ts, tx, p,
+                                                                           (int)items, st);
+    return launch_cfg<64, 256, 6, 1, 8, 1, 2, false, false, false, true>(tw, ts, tx, p,
+                                                                        (int)items, st);
 }
 
 extern "C" int64_t w4_moe_capacity(int64_t T, int topk, int E, int block) {

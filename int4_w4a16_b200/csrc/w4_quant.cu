@@ -283,6 +283,89 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint4 *__restri
     }
 }
 
+// ---- asymmetric (zero-point) groups: the affine map of the quantization
+// tutorial (§2.1) with its asymmetric scale and zero point (§2.3) over the
+// unsigned INT4 range [0, 15]:
+//   s = bf16_rne(fl32(fl32(x_max - x_min) / 15)),
+//   z = clamp(rint_even(0 - fl32(x_min / s)), 0, 15),
+//   q = clamp(rint_even(fl32(x / s)) + z, 0, 15),   q = z = 0 when s == 0.
+// The quotients are IEEE divisions: x / s is not bounded by the group's
+// range here (a narrow group far from zero has |x / s| up to ~3840), so the
+// reciprocal-and-snap rounding of the symmetric path does not carry over.
+
+__device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t bf16x2_min(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("min.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// One thread per group of 32 weights: Wq (4 words), S, Z.
+template <bool V8>
+__global__ void __launch_bounds__(kThreads, kQuantBlocksPerSm)
+    quant_zp_kernel(const uint32_t *__restrict__ W, uint4 *__restrict__ Wq,
+                    uint16_t *__restrict__ S, uint8_t *__restrict__ Z, int64_t ngroups) {
+    const int64_t T = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < ngroups; g += T) {
+        uint32_t v[16];
+        load_group<V8>(W + 16 * g, v);
+        uint32_t mx = v[0], mn = v[0];
+#pragma unroll
+        for (int j = 1; j < 16; ++j) {
+            mx = bf16x2_max(mx, v[j]);
+            mn = bf16x2_min(mn, v[j]);
+        }
+        const float xmax = fmaxf(lo_f(mx), hi_f(mx));
+        const float xmin = fminf(lo_f(mn), hi_f(mn));
+        const float s32 = __fdiv_rn(__fsub_rn(xmax, xmin), 15.0f);
+        const __nv_bfloat16 sb = __float2bfloat16_rn(s32);
+        const float s = __bfloat162float(sb);
+        uint32_t words[4] = {0u, 0u, 0u, 0u};
+        float zf = 0.0f;
+        if (s != 0.0f) {
+            zf = fminf(fmaxf(rintf(__fsub_rn(0.0f, __fdiv_rn(xmin, s))), 0.0f), 15.0f);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float x2[2] = {lo_f(v[j]), hi_f(v[j])};
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float c = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(x2[h], s)), zf), 0.0f), 15.0f);
+                    const int i = 2 * j + h;               // element of the group
+                    words[i >> 3] |= (uint32_t)c << (4 * (i & 7));
+                }
+            }
+        }
+        __stcs(Wq + g, make_uint4(words[0], words[1], words[2], words[3]));
+        S[g] = *reinterpret_cast<const uint16_t *>(&sb);
+        Z[g] = (uint8_t)zf;
+    }
+}
+
+// One thread = one group: 4 words of unsigned codes, its scale and zero point.
+__global__ void __launch_bounds__(kThreads) dequant_zp_kernel(const uint4 *__restrict__ Wq,
+                                                              const uint16_t *__restrict__ S,
+                                                              const uint8_t *__restrict__ Z,
+                                                              uint4 *__restrict__ Wdq,
+                                                              int64_t ngroups) {
+    const int64_t T = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < ngroups; g += T) {
+        const uint4 w = __ldcs(Wq + g);
+        const uint32_t s2 = bf16x2_splat(S[g]);
+        const uint32_t zb2 = zp_bias2(Z[g]);
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint32_t o[4];
+            dequant_word_zp(ws[j], s2, zb2, o);
+            __stcs(Wdq + 4 * g + j, make_uint4(o[0], o[1], o[2], o[3]));
+        }
+    }
+}
+
 bool aligned32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 // One CTA per kThreads * per_thread work items: the streaming kernels run each
@@ -379,6 +462,38 @@ extern "C" w4_status w4_dequant(const int32_t *Wq, const w4_bf16 *S, w4_bf16 *Wd
     if (ngroups == 0) return W4_OK;
     dequant_kernel<<<grid_for(ngroups, 1), kThreads, 0, (cudaStream_t)stream>>>(
         reinterpret_cast<const uint4 *>(Wq), reinterpret_cast<const uint16_t *>(S),
+        reinterpret_cast<uint4 *>(Wdq), ngroups);
+    return w4host::launch_status();
+}
+
+extern "C" w4_status w4_quantize_pack_zp(const w4_bf16 *W, int32_t *Wq, w4_bf16 *S, uint8_t *Z,
+                                         int64_t rows, int64_t K, int group, void *stream) {
+    w4_status st = check_quant_args(W, Wq, rows, K, group);
+    if (st != W4_OK) return st;
+    if (!w4host::aligned16(S) || Z == nullptr) return W4_ERR_INVALID_ARG;
+    const int64_t ngroups = rows * K / 32;
+    if (ngroups == 0) return W4_OK;
+    const int grid = grid_for(ngroups, 1);
+    const uint32_t *w = reinterpret_cast<const uint32_t *>(W);
+    uint4 *q = reinterpret_cast<uint4 *>(Wq);
+    uint16_t *s = reinterpret_cast<uint16_t *>(S);
+    if (aligned32(W))
+        quant_zp_kernel<true><<<grid, kThreads, 0, (cudaStream_t)stream>>>(w, q, s, Z, ngroups);
+    else
+        quant_zp_kernel<false><<<grid, kThreads, 0, (cudaStream_t)stream>>>(w, q, s, Z, ngroups);
+    return w4host::launch_status();
+}
+
+extern "C" w4_status w4_dequant_zp(const int32_t *Wq, const w4_bf16 *S, const uint8_t *Z,
+                                   w4_bf16 *Wdq, int64_t rows, int64_t K, int group,
+                                   void *stream) {
+    w4_status st = check_quant_args(Wq, Wdq, rows, K, group);
+    if (st != W4_OK) return st;
+    if (!w4host::aligned16(S) || Z == nullptr) return W4_ERR_INVALID_ARG;
+    const int64_t ngroups = rows * K / 32;
+    if (ngroups == 0) return W4_OK;
+    dequant_zp_kernel<<<grid_for(ngroups, 1), kThreads, 0, (cudaStream_t)stream>>>(
+        reinterpret_cast<const uint4 *>(Wq), reinterpret_cast<const uint16_t *>(S), Z,
         reinterpret_cast<uint4 *>(Wdq), ngroups);
     return w4host::launch_status();
 }

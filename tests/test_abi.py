@@ -24,7 +24,8 @@ def test_header_declares_the_boundary():
                      "w4a16_gemm", "w4a16_gemm_workspace_bytes", "w4_moe_align",
                      "w4_moe_w4a16_gemm", "w4_moe_capacity", "w4_moe_gate_topk",
                      "w4_moe_block_size", "w4_silu_mul", "w4_moe_combine", "w4_qat_gemm",
-                     "w4_moe_w4a16_gemm_silu",
+                     "w4_moe_w4a16_gemm_silu", "w4_quantize_pack_zp", "w4_dequant_zp",
+                     "w4a16_gemm_zp",
                      "w4_device_status", "w4_status_string", "w4_version",
                      "w4_last_cuda_error"]:
         assert required in names
@@ -142,3 +143,19 @@ def test_qat_gemm_validation_host_only():
     assert L.w4_qat_gemm(A16, A16, A16, 4, 8, 96, 32, None) == 2      # K % 64 != 0
     assert L.w4_qat_gemm(MIS, A16, A16, 4, 8, 64, 32, None) == 1      # misaligned X
     assert L.w4_qat_gemm(A16, A16, A16, 0, 8, 64, 32, None) == 0      # empty: no launch
+
+
+def test_zero_point_validation_host_only():
+    L = w4.lib()
+    assert L.w4_quantize_pack_zp(A16, A16, A16, A16, 4, 64, 64, None) == 2     # group != 32
+    assert L.w4_quantize_pack_zp(A16, A16, A16, A16, 4, 48, 32, None) == 1     # K % 32 != 0
+    assert L.w4_quantize_pack_zp(A16, A16, A16, None, 4, 64, 32, None) == 1    # Z missing
+    assert L.w4_quantize_pack_zp(MIS, A16, A16, A16, 4, 64, 32, None) == 1     # misaligned W
+    assert L.w4_quantize_pack_zp(A16, A16, A16, A16, 0, 64, 32, None) == 0     # empty
+    assert L.w4_dequant_zp(A16, A16, None, A16, 4, 64, 32, None) == 1
+    assert L.w4_dequant_zp(A16, A16, A16, A16, 0, 64, 32, None) == 0
+    assert L.w4a16_gemm_zp(A16, A16, A16, A16, A16, 4, 8, 64, 64, None) == 2   # group != 32
+    assert L.w4a16_gemm_zp(A16, A16, A16, A16, A16, 4, 8, 48, 32, None) == 1   # K % 32 != 0
+    assert L.w4a16_gemm_zp(A16, A16, A16, None, A16, 4, 8, 64, 32, None) == 1  # Z missing
+    assert L.w4a16_gemm_zp(A16, A16, A16, A16, MIS, 4, 8, 64, 32, None) == 1   # misaligned Y
+    assert L.w4a16_gemm_zp(A16, A16, A16, A16, A16, 0, 8, 64, 32, None) == 0   # empty

@@ -1,0 +1,99 @@
+"""Parity of the asymmetric (zero-point) group path with the CPU oracle: the
+quantizer and dequant bit for bit, the W4A16 GEMM on zero-point groups within
+the GEMM tolerance and bit for bit on one-hot activations (quantization
+tutorial §2.1 affine map, §2.3 asymmetric scale and zero point)."""
+import numpy as np
+import pytest
+import torch
+
+import int4_w4a16_b200 as w4
+import oracle
+import synth
+from synth import bits
+from tests.test_gpu_parity import DEV, assert_gemm_close
+
+pytestmark = pytest.mark.gpu
+
+
+def _edge_weights(N, K, seed):
+    """Ordinary groups next to each special case of the asymmetric map."""
+    W = synth.normal_bf16((N, K), 0.02, seed=seed, outlier_frac=0.01).clone()
+    if N > 8 and K >= 256:
+        W[0, 0:32] = 0.0                                                # s = 0
+        W[1, 32:64] = 0.75                                              # constant: s = 0
+        W[2, 64:96] = torch.linspace(1.0, 2.0, 32).to(torch.bfloat16)   # all positive: z -> 0
+        W[3, 96:128] = torch.linspace(-2.0, -1.0, 32).to(torch.bfloat16)  # all negative: z -> 15
+        W[4, 128:160] = torch.tensor([float(i % 16 - 5) for i in range(32)]).to(torch.bfloat16)
+        W[5, 160:192] = torch.linspace(100.0, 100.5, 32).to(torch.bfloat16)  # narrow, far from 0
+        W[6, 192:224] = 1e-39 * torch.linspace(-1, 1, 32).to(torch.bfloat16)  # subnormal range
+        W[7, 224:256] = torch.tensor([0.25 * (i % 7 - 3) for i in range(32)]).to(torch.bfloat16)
+    return W
+
+
+@pytest.mark.parametrize("rows,K", [(1, 32), (9, 256), (300, 640), (1000, 4096), (4097, 256)])
+def test_quantize_pack_zp_bit_exact(rows, K):
+    W = _edge_weights(rows, K, seed=rows + K)
+    Wq, S, Z = w4.quantize_pack_zp(W.to(DEV))
+    w4.w4_device_status()
+    oWq, oS, oZ = oracle.quantize_pack_zp(bits(W))
+    assert np.array_equal(Wq.cpu().numpy(), oWq)
+    assert np.array_equal(bits(S), oS)
+    assert np.array_equal(Z.cpu().numpy(), oZ)
+    Wdq = bits(w4.dequant_zp(Wq, S, Z))
+    assert np.array_equal(Wdq, oracle.dequant_zp(oWq, oS, oZ))
+
+
+def test_quantize_pack_zp_layer_shape():
+    """The prefill layer's weights (18432 x 7168): every output compared."""
+    W = synth.normal_bf16((18432, 7168), 0.02, seed=3, outlier_frac=0.001)
+    Wq, S, Z = w4.quantize_pack_zp(W.to(DEV))
+    oWq, oS, oZ = oracle.quantize_pack_zp(bits(W))
+    assert np.array_equal(Wq.cpu().numpy(), oWq)
+    assert np.array_equal(bits(S), oS)
+    assert np.array_equal(Z.cpu().numpy(), oZ)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 1, 64), (1, 300, 4096), (5, 100, 128), (64, 300, 640),
+                                   (65, 257, 256), (300, 1000, 1024), (512, 1024, 2048),
+                                   (3, 129, 96)])
+def test_gemm_zp_shapes(M, N, K):
+    W = _edge_weights(N, K, seed=M + N + K)
+    X = synth.normal_bf16((M, K), 1.0, seed=M + 7)
+    oWq, oS, oZ = oracle.quantize_pack_zp(bits(W))
+    Y = bits(w4.gemm_zp(X.to(DEV), torch.from_numpy(oWq).to(DEV),
+                        torch.from_numpy(oS.view(np.int16)).view(torch.bfloat16).to(DEV),
+                        torch.from_numpy(oZ).to(DEV)))
+    w4.w4_device_status()
+    _, R = oracle.w4a16_gemm_zp(bits(X), oWq, oS, oZ)
+    assert_gemm_close(Y, R, f"zp M={M} N={N} K={K}")
+
+
+def test_gemm_zp_one_hot_exact():
+    """X = identity rows: Y[m, n] = dequant_zp(W)[n, m] bit for bit."""
+    N, K = 200, 256
+    W = _edge_weights(N, K, seed=21)
+    Wq, S, Z = w4.quantize_pack_zp(W.to(DEV))
+    Wdq = oracle.dequant_zp(Wq.cpu().numpy(), bits(S), Z.cpu().numpy())
+    for m0 in range(0, K, 64):
+        X = torch.zeros((64, K), dtype=torch.bfloat16)
+        X[torch.arange(64), m0 + torch.arange(64)] = 1.0
+        Y = bits(w4.gemm_zp(X.to(DEV), Wq, S, Z))
+        want = Wdq[:, m0:m0 + 64].T
+        if not np.array_equal(Y, want):
+            bad = np.argwhere(Y != want)
+            raise AssertionError(f"one-hot mismatch at m0={m0}: {bad[:8].tolist()}")
+    w4.w4_device_status()
+
+
+def test_gemm_zp_layer_sampled():
+    """The prefill layer's weights (N = 18432, K = 7168) at M = 16; every 97th
+    output row against the oracle's GEMM on the same codes."""
+    N, K, M = 18432, 7168, 16
+    W = synth.normal_bf16((N, K), 0.02, seed=5, outlier_frac=0.001)
+    X = synth.normal_bf16((M, K), 1.0, seed=6)
+    Wq, S, Z = w4.quantize_pack_zp(W.to(DEV))
+    Y = bits(w4.gemm_zp(X.to(DEV), Wq, S, Z))
+    rows = np.arange(0, N, 97)
+    _, R = oracle.w4a16_gemm_zp(bits(X), Wq.cpu().numpy()[rows], bits(S)[rows],
+                                Z.cpu().numpy()[rows])
+    assert_gemm_close(Y[:, rows], R, "zp layer")
