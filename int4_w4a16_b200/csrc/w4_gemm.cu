@@ -325,6 +325,14 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
     auto empty_bar = [&](int s) { return bar0 + 8u * (NSTAGE + s); };
     auto afull_bar = [&](int a) { return bar0 + 8u * (2 * NSTAGE + a); };
     auto aempty_bar = [&](int a) { return bar0 + 8u * (2 * NSTAGE + NASTAGE + a); };
+    // As many A slots as stages: k-block it uses stage and A slot it % NSTAGE,
+    // both freed by the completion of its MMAs, so one commit (to the stage's
+    // "empty" barrier) releases both, and the dequant warps wait on that one.
+    constexpr bool kOneRelease = (NSTAGE == NASTAGE);
+    auto aslot_free_bar = [&](uint32_t it) {
+        return kOneRelease ? empty_bar((int)(it % NSTAGE)) : aempty_bar((int)(it % NASTAGE));
+    };
+    auto aslot_free_parity = [&](uint32_t it) { return ((it / NASTAGE) & 1u) ^ 1u; };
     auto accfull_bar = [&](int d) { return bar0 + 8u * (2 * NSTAGE + 2 * NASTAGE + d); };
     auto accempty_bar = [&](int d) {
         return bar0 + 8u * (2 * NSTAGE + 2 * NASTAGE + NACC + d);
@@ -533,7 +541,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
 #pragma unroll
                         for (int z = 0; z < 16; ++z) o[16 * h + z] = og[z];
                     }
-                    if (!warp_wait(aempty_bar(a), ((it / NASTAGE) & 1u) ^ 1u, abort_flag)) {
+                    if (!warp_wait(aslot_free_bar(it), aslot_free_parity(it), abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -608,7 +616,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                 load_pair(0, cur);
                 uint32_t o[2][32];
                 unpack_pair(cur, load_scales(0), o[0]);
-                if (!warp_wait(aempty_bar(a), ((it / NASTAGE) & 1u) ^ 1u, abort_flag)) {
+                if (!warp_wait(aslot_free_bar(it), aslot_free_parity(it), abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -677,7 +685,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                 // Waiting for the slot to be free first keeps this arrival in the
                 // slot's current phase (these warps may run ahead of the dequant).
                 const int a = it % NASTAGE;
-                if (!warp_wait(aempty_bar(a), ((it / NASTAGE) & 1u) ^ 1u, abort_flag, kSleepAhead)) {
+                if (!warp_wait(aslot_free_bar(it), aslot_free_parity(it), abort_flag, kSleepAhead)) {
                     ok = false;
                     break;
                 }
@@ -735,7 +743,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                                       (kb > kb0 || u >= NSPLIT) ? 1u : 0u);
                         }
                         tc_commit(empty_bar(s));
-                        tc_commit(aempty_bar(a));
+                        if (!kOneRelease) tc_commit(aempty_bar(a));
                     }
                 } else {
                     it += (uint32_t)(kb1 - kb0);
@@ -1239,7 +1247,7 @@ extern "C" w4_status w4a16_gemm(const w4_bf16 *X, const int32_t *Wq, const w4_bf
     const int64_t items = (int64_t)p.n_row_tiles * p.n_tok_tiles;
     if (items > (1 << 30)) return W4_ERR_UNSUPPORTED;
     if (mt == 64) return launch_cfg<64, 64, 8, 1, 8, 4, 2, false>(tw, ts, tx, p, (int)items, st);
-    return launch_cfg<64, 256, 6, 1, 8, 1, 2, false>(tw, ts, tx, p, (int)items, st);
+    return launch_cfg<64, 256, 6, 1, 6, 1, 2, false>(tw, ts, tx, p, (int)items, st);
 }
 
 extern "C" w4_status w4_qat_gemm(const w4_bf16 *X, const w4_bf16 *W, w4_bf16 *Y, int64_t M,
@@ -1285,7 +1293,7 @@ extern "C" w4_status w4_qat_gemm(const w4_bf16 *X, const w4_bf16 *W, w4_bf16 *Y,
     if (items > (1 << 30)) return W4_ERR_UNSUPPORTED;
     if (mt == 64)
         return launch_cfg<64, 64, 8, 1, 8, 4, 2, false, false, true>(tw, ts, tx, p, (int)items, st);
-    return launch_cfg<64, 256, 4, 1, 8, 1, 2, false, false, true>(tw, ts, tx, p, (int)items, st);
+    return launch_cfg<64, 256, 4, 1, 4, 1, 2, false, false, true>(tw, ts, tx, p, (int)items, st);
 }
 
 extern "C" w4_status w4a16_gemm_zp(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S,
@@ -1336,7 +1344,7 @@ extern "C" w4_status w4a16_gemm_zp(const w4_bf16 *X, const int32_t *Wq, const w4
     if (mt == 64)
         return launch_cfg<64, 64, 8, 1, 8, 4, 2, false, false, false, true>(tw, ts, tx, p,
                                                                            (int)items, st);
-    return launch_cfg<64, 256, 6, 1, 8, 1, 2, false, false, false, true>(tw, ts, tx, p,
+    return launch_cfg<64, 256, 6, 1, 6, 1, 2, false, false, false, true>(tw, ts, tx, p,
                                                                         (int)items, st);
 }
 
