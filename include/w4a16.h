@@ -221,10 +221,11 @@ w4_status w4_dequant_zp(const int32_t *Wq, const w4_bf16 *S, const uint8_t *Z, w
 /*
  * W4A16 GEMM on asymmetric groups: Y[M, N] = X[M, K] . dequant_zp(Wq, S, Z)^T,
  * fp32 accumulation, BF16 output (the zero point is subtracted in the same
- * register unpack as w4a16_gemm's constant bias, no extra instruction).  Every M
- * runs the tensor-memory kernel with 64-wide k-blocks (no warp-level decode
- * kernel for this format).  K a multiple of 32; group 32; X, Wq, S, Y 16-byte
- * aligned; Z not NULL.  Device pointers; the call is asynchronous on `stream`.
+ * register unpack as w4a16_gemm's constant bias, no extra instruction).  1..8
+ * rows with K % 512 == 0 and a 16-byte-aligned Z take the warp-level decode
+ * kernel; every other shape the tensor-memory kernel with 64-wide k-blocks.
+ * K a multiple of 32; group 32; X, Wq, S, Y 16-byte aligned; Z not NULL.
+ * Device pointers; the call is asynchronous on `stream`.
  */
 w4_status w4a16_gemm_zp(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S, const uint8_t *Z,
                         w4_bf16 *Y, int64_t M, int64_t N, int64_t K, int group, void *stream);

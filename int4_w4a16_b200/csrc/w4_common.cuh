@@ -438,6 +438,26 @@ __device__ __forceinline__ void dequant_word_k8perm(uint32_t w, uint32_t s2, uin
     }
 }
 
+// dequant_word_k8perm for unsigned codes with a zero point (zb2 = zp_bias2(z)).
+__device__ __forceinline__ void dequant_word_k8perm_zp(uint32_t w, uint32_t s2, uint32_t zb2,
+                                                       uint32_t (&out)[4]) {
+    const uint32_t m = 0x000F000Fu, x = 0x43004300u;
+    uint32_t in[4];
+    in[0] = lop3_and_xor(w, m, x);          // codes 0, 4
+    in[1] = lop3_and_xor(w >> 4, m, x);     // codes 1, 5
+    in[2] = lop3_and_xor(w >> 8, m, x);     // codes 2, 6
+    in[3] = lop3_and_xor(w >> 12, m, x);    // codes 3, 7
+    const __nv_bfloat162 zb = *reinterpret_cast<const __nv_bfloat162 *>(&zb2);
+    const __nv_bfloat162 sc = *reinterpret_cast<const __nv_bfloat162 *>(&s2);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162 *>(&in[j]);
+        v = __hsub2(v, zb);
+        v = __hmul2(v, sc);
+        out[j] = *reinterpret_cast<uint32_t *>(&v);
+    }
+}
+
 // 8 BF16 values [x0..x7] (16 bytes) -> [x0, x4, x1, x5, x2, x6, x3, x7].
 __device__ __forceinline__ uint4 permute_chunk8(uint4 v) {
     uint4 o;
@@ -470,6 +490,11 @@ cudaError_t gemv_device_status(unsigned int *flag);
 bool gemv_supported(int64_t M, int64_t N, int64_t K);
 w4_status gemv_launch(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S, w4_bf16 *Y,
                       int64_t M, int64_t N, int64_t K, void *stream);
+// The same for zero-point groups (unsigned codes, Z one byte per group); also
+// needs K % 512 == 0 (whole 16-byte lines of zero points per row) and a
+// 16-byte-aligned Z, W4_ERR_UNSUPPORTED otherwise.
+w4_status gemv_launch_zp(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S, const uint8_t *Z,
+                         w4_bf16 *Y, int64_t M, int64_t N, int64_t K, void *stream);
 
 inline bool aligned16(const void *p) {
     return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0;

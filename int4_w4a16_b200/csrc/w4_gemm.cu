@@ -1306,6 +1306,12 @@ extern "C" w4_status w4a16_gemm_zp(const w4_bf16 *X, const int32_t *Wq, const w4
         return W4_ERR_INVALID_ARG;
     if (M == 0 || N == 0) return W4_OK;
     if (N > (1 << 30) || M > (1 << 30) || K > (1 << 24)) return W4_ERR_UNSUPPORTED;
+    // 1..8 activation rows: the warp-level MMA kernel (w4_gemv.cu) when K and
+    // Z suit its TMA boxes
+    if (w4host::gemv_supported(M, N, K)) {
+        const w4_status gs = w4host::gemv_launch_zp(X, Wq, S, Z, Y, M, N, K, stream);
+        if (gs != W4_ERR_UNSUPPORTED) return gs;
+    }
     cudaStream_t st = (cudaStream_t)stream;
     GemmParams p = {};
     p.S = reinterpret_cast<const uint16_t *>(S);

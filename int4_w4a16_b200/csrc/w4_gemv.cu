@@ -50,7 +50,7 @@ constexpr int kGvThreads = 32 * (kGvWarps + 1);       // + the reduction warp
 constexpr int kGvKW = 128;                            // K of one warp chunk (4 groups)
 constexpr int kGvWPT = 4;                             // packed words per lane, row and chunk
 
-template <int NT, int RT>
+template <int NT, int RT, bool ZP = false>
 struct GvCfg {
     static constexpr int MT = 8 * NT;                 // token columns (MMA N = 8 per tile)
     static constexpr int TPW = 1;                     // 16-row tiles per warp and stage
@@ -59,16 +59,21 @@ struct GvCfg {
     static constexpr int WBYTES = KCW * ROWS * 64;    // packed words of a stage
     static constexpr int SKB = KCW / 2;               // 256-wide K blocks of scales per stage
     static constexpr int SBYTES = SKB * ROWS * 16;    // scales of a stage
+    // zero points (ZP): 16-byte lines of 16 groups (512 of K) per row
+    static constexpr int ZKB = KCW / 4;               // 512-wide K blocks per stage
+    static constexpr int ZBYTES = ZP ? ZKB * ROWS * 16 : 0;
     static constexpr int NSTAGE = WBYTES >= 32768 ? 4 : 6;
     static_assert(NT == 1 || NT == 2, "at most 16 token columns per launch");
     static constexpr int PROWS = 16 * TPW;            // rows of one warp's partial tile
     static constexpr int TS = PROWS + 4;              // floats per token row (bank spread)
     static constexpr int RED_FLOATS = kGvWarps * MT * TS;      // one partial buffer
     static constexpr int NRED = 4;
-    static constexpr int FIXED_BYTES = 1024 + NSTAGE * (WBYTES + SBYTES) + NRED * RED_FLOATS * 4;
+    static constexpr int FIXED_BYTES =
+        1024 + NSTAGE * (WBYTES + SBYTES + ZBYTES) + NRED * RED_FLOATS * 4;
     static_assert(WBYTES % 1024 == 0 && SBYTES % 128 == 0, "slot alignment");
     static_assert((ROWS * 64) % 512 == 0, "64-byte swizzle atoms");
     static_assert(KCW % 2 == 0, "chunk pairs share a scale block");
+    static_assert(!ZP || KCW % 4 == 0, "chunk quads share a zero-point line");
 };
 
 struct GemvParams {
@@ -148,8 +153,8 @@ __device__ __forceinline__ uint32_t gv_word_off(int r, int j, int t) {
 //   chunk * 128 + 32 j + 8 t + (0..7), scale group j of the chunk;
 //   MMA step 2 j uses code pairs (0,4), (1,5); step 2 j + 1 uses (2,6), (3,7),
 // matching the B fragments built by permute_chunk8 from the same 8 activations.
-template <int NT, int TPW>
-__device__ __forceinline__ void gv_stage_math(uint32_t wblk, uint32_t sblk, int tile0, int g,
+template <int NT, int TPW, bool ZP = false>
+__device__ __forceinline__ void gv_stage_math(uint32_t wblk, uint32_t sblk, uint32_t zblk, int tile0, int g,
                                               int t, const uint4 (&xf)[NT][kGvWPT],
                                               float (&acc)[TPW][NT][4]) {
     // words j even / odd accumulate into two chains (half the dependent MMA
@@ -175,11 +180,19 @@ __device__ __forceinline__ void gv_stage_math(uint32_t wblk, uint32_t sblk, int 
                                  __byte_perm(sg.y, 0, 0x1010), __byte_perm(sg.y, 0, 0x3232)};
         const uint32_t shv[4] = {__byte_perm(sh.x, 0, 0x1010), __byte_perm(sh.x, 0, 0x3232),
                                  __byte_perm(sh.y, 0, 0x1010), __byte_perm(sh.y, 0, 0x3232)};
+        // zero points of groups 0..3 (one byte each) for rows rg and rh
+        const uint32_t zg = ZP ? gv_lds32(zblk + (uint32_t)rg * 16) : 0u;
+        const uint32_t zh = ZP ? gv_lds32(zblk + (uint32_t)rh * 16) : 0u;
 #pragma unroll
         for (int j = 0; j < kGvWPT; ++j) {
             uint32_t pg[4], ph[4];
-            dequant_word_k8perm(wg[j], sgv[j], pg);
-            dequant_word_k8perm(wh[j], shv[j], ph);
+            if (ZP) {
+                dequant_word_k8perm_zp(wg[j], sgv[j], zp_bias2(zg >> (8 * j)), pg);
+                dequant_word_k8perm_zp(wh[j], shv[j], zp_bias2(zh >> (8 * j)), ph);
+            } else {
+                dequant_word_k8perm(wg[j], sgv[j], pg);
+                dequant_word_k8perm(wh[j], shv[j], ph);
+            }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 float (&d)[4] = (j & 1) ? acc2[u][nt] : acc[u][nt];
@@ -196,11 +209,11 @@ __device__ __forceinline__ void gv_stage_math(uint32_t wblk, uint32_t sblk, int 
             for (int e = 0; e < 4; ++e) acc[u][nt][e] += acc2[u][nt][e];
 }
 
-template <int NT, int RT>
+template <int NT, int RT, bool ZP>
 __global__ void __launch_bounds__(kGvThreads, 1)
     w4a16_gemv_kernel(const __grid_constant__ CUtensorMap tw, const __grid_constant__ CUtensorMap ts,
-                      const GemvParams p) {
-    using C = GvCfg<NT, RT>;
+                      const __grid_constant__ CUtensorMap tz, const GemvParams p) {
+    using C = GvCfg<NT, RT, ZP>;
     extern __shared__ __align__(1024) uint8_t gv_smem[];
     __shared__ __align__(8) uint64_t full_bar[C::NSTAGE];       // stage landed (TMA bytes)
     __shared__ __align__(8) uint64_t red_full[C::NRED];         // partials of a stage written
@@ -213,7 +226,8 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     const uint32_t base = (raw + 1023u) & ~1023u;
     const uint32_t sm_w = base;
     const uint32_t sm_s = sm_w + C::NSTAGE * C::WBYTES;
-    const uint32_t sm_red = sm_s + C::NSTAGE * C::SBYTES;
+    const uint32_t sm_z = sm_s + C::NSTAGE * C::SBYTES;     // ZP only
+    const uint32_t sm_red = sm_z + C::NSTAGE * C::ZBYTES;
     float *red = reinterpret_cast<float *>(gv_smem + (sm_red - raw));
     float *rowsum = red + C::NRED * C::RED_FLOATS;    // [MT][acc_rows], passes > 1 only
 
@@ -230,13 +244,16 @@ __global__ void __launch_bounds__(kGvThreads, 1)
         const int slot = s % C::NSTAGE, pass = s / nrb, rb = s % nrb;
         const uint32_t fb = smem_u32(&full_bar[slot]);
         slot_last[slot] = s;
-        mbar_arrive_expect_tx(fb, (uint32_t)(C::WBYTES + C::SBYTES));
+        mbar_arrive_expect_tx(fb, (uint32_t)(C::WBYTES + C::SBYTES + C::ZBYTES));
         tma_load_3d(sm_w + slot * C::WBYTES, &tw, fb, 0, row0 + rb * C::ROWS, pass * C::KCW);
         tma_load_3d(sm_s + slot * C::SBYTES, &ts, fb, 0, row0 + rb * C::ROWS, pass * C::SKB);
+        if (ZP)
+            tma_load_3d(sm_z + slot * C::ZBYTES, &tz, fb, 0, row0 + rb * C::ROWS, pass * C::ZKB);
     };
     if (threadIdx.x == 0) {
         tma_prefetch_desc(&tw);
         tma_prefetch_desc(&ts);
+        if (ZP) tma_prefetch_desc(&tz);
         for (int i = 0; i < C::NSTAGE; ++i) {
             mbar_init(smem_u32(&full_bar[i]), 1u);
             slot_done[i] = 0u;
@@ -340,7 +357,9 @@ __global__ void __launch_bounds__(kGvThreads, 1)
                     const uint32_t wblk = sm_w + slot * C::WBYTES + cw * (C::ROWS * 64);
                     const uint32_t sblk =
                         sm_s + slot * C::SBYTES + (cw >> 1) * (C::ROWS * 16) + (cw & 1) * 8;
-                    gv_stage_math<NT, C::TPW>(wblk, sblk, rt * C::TPW, g, tig, xf, acc);
+                    const uint32_t zblk =
+                        sm_z + slot * C::ZBYTES + (cw >> 2) * (C::ROWS * 16) + (cw & 3) * 4;
+                    gv_stage_math<NT, C::TPW, ZP>(wblk, sblk, zblk, rt * C::TPW, g, tig, xf, acc);
                 }
                 // The math has consumed this warp's reads of the slot; the last
                 // warp done with it (the counter only grows: 16 arrivals per use)
@@ -388,10 +407,10 @@ __global__ void __launch_bounds__(kGvThreads, 1)
 // Host side
 // ---------------------------------------------------------------------------
 
-template <int NT, int RT>
-w4_status gv_launch(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S, w4_bf16 *Y, int M,
-                    int N, int K, cudaStream_t stream) {
-    using C = GvCfg<NT, RT>;
+template <int NT, int RT, bool ZP = false>
+w4_status gv_launch(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S, const uint8_t *Z,
+                    w4_bf16 *Y, int M, int N, int K, cudaStream_t stream) {
+    using C = GvCfg<NT, RT, ZP>;
     const int sms = w4host::num_sms();
     GemvParams p = {};
     p.X = reinterpret_cast<const uint16_t *>(X);
@@ -409,7 +428,7 @@ w4_status gv_launch(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S, w4_bf
     const size_t smem = (size_t)C::FIXED_BYTES + (size_t)p.acc_rows * C::MT * 4;
     if (smem > 225 * 1024) return W4_ERR_UNSUPPORTED;
 
-    CUtensorMap tw, ts;
+    CUtensorMap tw, ts, tz;
     {
         // packed words as [K / 128 chunks][N rows][16 words]; the chunk stride
         // (one 64-byte line) is smaller than the row stride
@@ -429,7 +448,18 @@ w4_status gv_launch(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S, w4_bf
                                  dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
             return W4_ERR_CUDA;
     }
-    auto kern = w4a16_gemv_kernel<NT, RT>;
+    if (ZP) {
+        // zero points as [K / 512 blocks][N rows][16 groups], one byte each
+        cuuint64_t dims[3] = {16u, (cuuint64_t)N, (cuuint64_t)(K / 512)};
+        cuuint64_t strides[2] = {(cuuint64_t)K / 32, 16u};
+        cuuint32_t box[3] = {16u, (cuuint32_t)C::ROWS, (cuuint32_t)C::ZKB};
+        if (w4host::encode_tiled(&tz, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(Z),
+                                 dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
+            return W4_ERR_CUDA;
+    } else {
+        tz = ts;                                     // not read
+    }
+    auto kern = w4a16_gemv_kernel<NT, RT, ZP>;
     static size_t configured = 0;
     if (smem > configured) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
@@ -437,7 +467,7 @@ w4_status gv_launch(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S, w4_bf
             return w4host::launch_status();
         configured = smem;
     }
-    kern<<<p.ctas, kGvThreads, smem, stream>>>(tw, ts, p);
+    kern<<<p.ctas, kGvThreads, smem, stream>>>(tw, ts, tz, p);
     return w4host::launch_status();
 }
 
@@ -459,8 +489,19 @@ w4_status w4host::gemv_launch(const w4_bf16 *X, const int32_t *Wq, const w4_bf16
     cudaStream_t st = (cudaStream_t)stream;
     const int m = (int)M, n = (int)N, k = (int)K;
     // short K (at most 8 chunks of 128): two row tiles of warps per stage
-    return k / kGvKW <= 8 ? gv_launch<1, 2>(X, Wq, S, Y, m, n, k, st)
-                          : gv_launch<1, 1>(X, Wq, S, Y, m, n, k, st);
+    return k / kGvKW <= 8 ? gv_launch<1, 2>(X, Wq, S, nullptr, Y, m, n, k, st)
+                          : gv_launch<1, 1>(X, Wq, S, nullptr, Y, m, n, k, st);
+}
+
+w4_status w4host::gemv_launch_zp(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S,
+                                 const uint8_t *Z, w4_bf16 *Y, int64_t M, int64_t N, int64_t K,
+                                 void *stream) {
+    using namespace w4;
+    if (!gemv_supported(M, N, K) || (K % 512) != 0 || !aligned16(Z)) return W4_ERR_UNSUPPORTED;
+    cudaStream_t st = (cudaStream_t)stream;
+    const int m = (int)M, n = (int)N, k = (int)K;
+    return k / kGvKW <= 8 ? gv_launch<1, 2, true>(X, Wq, S, Z, Y, m, n, k, st)
+                          : gv_launch<1, 1, true>(X, Wq, S, Z, Y, m, n, k, st);
 }
 
 cudaError_t w4host::gemv_device_status(unsigned int *flag) {

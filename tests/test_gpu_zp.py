@@ -97,3 +97,51 @@ def test_gemm_zp_layer_sampled():
     _, R = oracle.w4a16_gemm_zp(bits(X), Wq.cpu().numpy()[rows], bits(S)[rows],
                                 Z.cpu().numpy()[rows])
     assert_gemm_close(Y[:, rows], R, "zp layer")
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 333, 512), (3, 257, 1024), (8, 1000, 4096),
+                                   (5, 64, 4608), (8, 129, 2560), (2, 12288, 4096)])
+def test_gemm_zp_decode_kernel(M, N, K):
+    """1..8 rows with K % 512 == 0 take the warp-level MMA kernel (zero points by
+    TMA beside the scales); one to three passes over K, ragged N."""
+    W = _edge_weights(N, K, seed=M * 7 + N + K)
+    X = synth.normal_bf16((M, K), 1.0, seed=M + 11)
+    Wq, S, Z = w4.quantize_pack_zp(W.to(DEV))
+    Y = bits(w4.gemm_zp(X.to(DEV), Wq, S, Z))
+    w4.w4_device_status()
+    _, R = oracle.w4a16_gemm_zp(bits(X), Wq.cpu().numpy(), bits(S), Z.cpu().numpy())
+    assert_gemm_close(Y, R, f"zp decode M={M} N={N} K={K}")
+
+
+def test_gemm_zp_decode_kernel_one_hot_exact():
+    """X = 8 identity rows through the warp-level kernel: Y[m, n] =
+    dequant_zp(W)[n, m] bit for bit."""
+    N, K = 300, 1024
+    W = _edge_weights(N, K, seed=33)
+    Wq, S, Z = w4.quantize_pack_zp(W.to(DEV))
+    Wdq = oracle.dequant_zp(Wq.cpu().numpy(), bits(S), Z.cpu().numpy())
+    for m0 in range(0, K, 8 * 16):
+        X = torch.zeros((8, K), dtype=torch.bfloat16)
+        X[torch.arange(8), m0 + torch.arange(8)] = 1.0
+        Y = bits(w4.gemm_zp(X.to(DEV), Wq, S, Z))
+        want = Wdq[:, m0:m0 + 8].T
+        if not np.array_equal(Y, want):
+            bad = np.argwhere(Y != want)
+            raise AssertionError(f"one-hot mismatch at m0={m0}: {bad[:8].tolist()}")
+    w4.w4_device_status()
+
+
+def test_gemm_zp_unaligned_zero_points_take_the_tensor_memory_kernel():
+    """Zero points not 16-byte aligned: the decode kernel declines, the
+    tensor-memory kernel computes the same product."""
+    N, K, M = 200, 1024, 4
+    W = _edge_weights(N, K, seed=44)
+    X = synth.normal_bf16((M, K), 1.0, seed=45)
+    Wq, S, Z = w4.quantize_pack_zp(W.to(DEV))
+    Zbuf = torch.empty(Z.numel() + 16, dtype=torch.uint8, device=DEV)
+    Zoff = Zbuf[1:1 + Z.numel()].view(Z.shape)
+    Zoff.copy_(Z)
+    Y = bits(w4.gemm_zp(X.to(DEV), Wq, S, Zoff))
+    w4.w4_device_status()
+    _, R = oracle.w4a16_gemm_zp(bits(X), Wq.cpu().numpy(), bits(S), Z.cpu().numpy())
+    assert_gemm_close(Y, R, "zp unaligned Z")
