@@ -33,7 +33,7 @@
  *          §6.1 numpy symmetric quantizer and its printed output,
  *          §6.2 torch.round rounds half to even.
  *
- * Readings where the sources are silent (each is listed in the design doc):
+ * Readings where the sources are silent:
  *   - groups are 32 contiguous elements along K (the reduction dim) of a
  *     row-major [rows, K] BF16 matrix ([TAG] [11] "1x32");
  *   - s32 = fl32(amax / 7) in IEEE fp32, then s = bf16_rne(s32) is the

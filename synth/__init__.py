@@ -5,7 +5,7 @@ tensors) and by ``bench.py``.  This module holds input generation only: random
 draws, casts to BF16 and the workload shapes.  It contains none of the method's
 arithmetic (no scale, rounding, packing, GEMM or alignment).
 
-Recipes (stated again in the design doc):
+Recipes:
   * values are drawn in fp32 and cast to BF16 with round-to-nearest-even
     (``Tensor.to(torch.bfloat16)``);
   * every tensor has its own generator seeded with ``seed * 1000 + index``;
