@@ -284,19 +284,28 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 
 // NSPLIT: MMA issuers = accumulators per work item; 16-wide K step u goes to
 // issuer / accumulator u % NSPLIT, and the epilogue adds the accumulators in
-// a fixed order.
+// a fixed order.  SPLITN: the NSPLIT issuers split the tile's tokens instead
+// (issuer i: columns [i MT/NSPLIT, (i+1) MT/NSPLIT) of the one accumulator,
+// every K step), so NSPLIT threads issue into one accumulator in parallel:
+// one thread issues a tcgen05.mma only about every 100 cycles, and with a
+// barrier poll and a commit per k-block a single issuer cannot keep up with
+// the tensor core on N = 256 tiles.
 template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT, int NDQ, bool MOE,
-          bool WGL, bool QAT, bool ZP>
+          bool WGL, bool QAT, bool ZP, bool SPLITN>
 __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
     w4a16_tc_kernel(const __grid_constant__ CUtensorMap tm_w,
                     const __grid_constant__ CUtensorMap tm_s,
                     const __grid_constant__ CUtensorMap tm_x, const GemmParams p) {
-    using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE, NSPLIT, QAT>;
+    constexpr int kAccSets = SPLITN ? 1 : NSPLIT;   // accumulators per work item
+    using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE, kAccSets, QAT>;
     static_assert(!QAT || (KB == 64 && !MOE), "QAT: 64-wide k-blocks of dense BF16 weights");
+    static_assert(!SPLITN || (KB == 64 && !MOE && !WGL && MT % (16 * NSPLIT) == 0),
+                  "token-split issuers: dense 64-wide k-blocks, N per issuer a multiple of 16");
     static_assert(!ZP || (KB == 64 && !MOE && !QAT), "zero points: dense 64-wide k-blocks");
     constexpr int kWords = KB / 8;             // packed words per row per k-block
     constexpr int kAStageCols = KB / 2;        // TMEM columns per A stage
-    constexpr int kAccCols = NSPLIT * MT;      // TMEM columns per work item accumulator
+    constexpr int kAccCols = kAccSets * MT;    // TMEM columns per work item accumulator
+    constexpr int kNPer = SPLITN ? MT / NSPLIT : MT;   // MMA N of one issuer
     constexpr int kABase = NACC * kAccCols;    // first A column
     constexpr int kDqWarps = 4 * NDQ;
     constexpr int kPermWarps = perm_warps(KB);
@@ -310,7 +319,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
     // 256-wide k-blocks (decode / MoE, few activation rows per tile): reorder the
     // activation chunks in shared memory instead of pairing the unpacked codes.
     constexpr bool kXPerm = (KB == 256);
-    constexpr uint32_t kIdesc = idesc_bf16_f32(128, MT);
+    constexpr uint32_t kIdesc = idesc_bf16_f32(128, kNPer);
 
     extern __shared__ uint8_t smem_raw[];
     // MoE gate_up with SiLU*up: the up rows' sums of one 16-column chunk, handed
@@ -716,7 +725,8 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                     break;
                 }
                 tc_fence_after_sync();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(d * kAccCols + ji * MT);
+                const uint32_t d_tmem =
+                    tmem_base + (uint32_t)(d * kAccCols + (SPLITN ? ji * kNPer : ji * MT));
                 // Lane 0 alone polls and issues: a warp-wide wait adds a vote to
                 // every poll, and each poll sits on the issue path between two
                 // k-blocks' MMAs.  The issuer waits only for the A slot: the
@@ -735,12 +745,16 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                         tc_fence_after_sync();
                         if (MOE) fence_proxy_async_smem();   // cp.async (generic proxy) -> MMA
                         const uint32_t a_tmem = tmem_base + (uint32_t)(kABase + a * kAStageCols);
+                        // SPLITN: this issuer's tokens start kNPer rows (128 B each,
+                        // whole 1024-byte swizzle atoms) into the activation tile
+                        constexpr int kU0Step = SPLITN ? 1 : NSPLIT;
+                        const uint32_t xrow = SPLITN ? (uint32_t)(ji * kNPer * 128) : 0u;
 #pragma unroll
-                        for (int u = ji; u < KB / 16; u += NSPLIT) {
+                        for (int u = SPLITN ? 0 : ji; u < KB / 16; u += kU0Step) {
                             const uint32_t baddr =
-                                x_stage(s) + (u >> 2) * L::kXSub + (u & 3) * 32;
+                                x_stage(s) + (u >> 2) * L::kXSub + (u & 3) * 32 + xrow;
                             tc_mma_ts(d_tmem, a_tmem + u * 8, smem_desc_k_sw128(baddr), kIdesc,
-                                      (kb > kb0 || u >= NSPLIT) ? 1u : 0u);
+                                      (kb > kb0 || u >= kU0Step) ? 1u : 0u);
                         }
                         tc_commit(empty_bar(s));
                         if (!kOneRelease) tc_commit(aempty_bar(a));
@@ -790,9 +804,9 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                 // all NSPLIT accumulator loads in flight, one wait, then the sum in
                 // accumulator order (two at a time, to bound the registers)
                 uint32_t v[16];
-                constexpr int kLd = NSPLIT < 2 ? NSPLIT : 2;
+                constexpr int kLd = kAccSets < 2 ? kAccSets : 2;
 #pragma unroll
-                for (int sp0 = 0; sp0 < NSPLIT; sp0 += kLd) {
+                for (int sp0 = 0; sp0 < kAccSets; sp0 += kLd) {
                     uint32_t w2[kLd][16];
 #pragma unroll
                     for (int sp = 0; sp < kLd; ++sp)
@@ -1018,11 +1032,12 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
 // ---------------------------------------------------------------------------
 
 template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT, int NDQ, bool MOE,
-          bool WGL = false, bool QAT = false, bool ZP = false>
+          bool WGL = false, bool QAT = false, bool ZP = false, bool SPLITN = false>
 w4_status launch_cfg(const CUtensorMap &tw, const CUtensorMap &ts, const CUtensorMap &tx,
                      const GemmParams &p, int num_items_max, cudaStream_t stream) {
-    using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE, NSPLIT, QAT>;
-    auto kern = w4a16_tc_kernel<KB, MT, NSTAGE, NACC, NASTAGE, NSPLIT, NDQ, MOE, WGL, QAT, ZP>;
+    using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE, (SPLITN ? 1 : NSPLIT), QAT>;
+    auto kern =
+        w4a16_tc_kernel<KB, MT, NSTAGE, NACC, NASTAGE, NSPLIT, NDQ, MOE, WGL, QAT, ZP, SPLITN>;
     // At least half of the SM's shared memory, so one CTA (and one TMEM
     // allocation of 512 columns) per SM.
     const int smem = std::max(L::kAlloc, 120 * 1024);
@@ -1247,7 +1262,9 @@ extern "C" w4_status w4a16_gemm(const w4_bf16 *X, const int32_t *Wq, const w4_bf
     const int64_t items = (int64_t)p.n_row_tiles * p.n_tok_tiles;
     if (items > (1 << 30)) return W4_ERR_UNSUPPORTED;
     if (mt == 64) return launch_cfg<64, 64, 8, 1, 8, 4, 2, false>(tw, ts, tx, p, (int)items, st);
-    return launch_cfg<64, 256, 6, 1, 6, 1, 2, false>(tw, ts, tx, p, (int)items, st);
+    // two issuers, 128 tokens each (measured: 2-4 % faster than one; four were slower)
+    return launch_cfg<64, 256, 6, 1, 6, 2, 2, false, false, false, false, true>(tw, ts, tx, p,
+                                                                               (int)items, st);
 }
 
 extern "C" w4_status w4_qat_gemm(const w4_bf16 *X, const w4_bf16 *W, w4_bf16 *Y, int64_t M,
@@ -1293,6 +1310,7 @@ extern "C" w4_status w4_qat_gemm(const w4_bf16 *X, const w4_bf16 *W, w4_bf16 *Y,
     if (items > (1 << 30)) return W4_ERR_UNSUPPORTED;
     if (mt == 64)
         return launch_cfg<64, 64, 8, 1, 8, 4, 2, false, false, true>(tw, ts, tx, p, (int)items, st);
+    // one issuer: with the QDQ prologue, more issuers measured no faster
     return launch_cfg<64, 256, 4, 1, 4, 1, 2, false, false, true>(tw, ts, tx, p, (int)items, st);
 }
 
@@ -1350,8 +1368,8 @@ extern "C" w4_status w4a16_gemm_zp(const w4_bf16 *X, const int32_t *Wq, const w4
     if (mt == 64)
         return launch_cfg<64, 64, 8, 1, 8, 4, 2, false, false, false, true>(tw, ts, tx, p,
                                                                            (int)items, st);
-    return launch_cfg<64, 256, 6, 1, 6, 1, 2, false, false, false, true>(tw, ts, tx, p,
-                                                                        (int)items, st);
+    return launch_cfg<64, 256, 6, 1, 6, 2, 2, false, false, false, true, true>(tw, ts, tx, p,
+                                                                              (int)items, st);
 }
 
 extern "C" int64_t w4_moe_capacity(int64_t T, int topk, int E, int block) {
