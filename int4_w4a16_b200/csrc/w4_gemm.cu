@@ -6,6 +6,10 @@
 // dq(W)[n, k] = bf16_rne(q[n, k] * S[n, k/32]), FP32 accumulation, one BF16
 // rounding of the result.  The MoE variant runs the same product per aligned
 // block of slots with the block's expert weights and gathered activation rows.
+// Two more weight prologues share the tile: BF16 weights through the exact
+// group QDQ of the quantizers (QAT forward, Y = X . fake_quant(W)^T), and
+// unsigned codes with a zero point per group, dq = bf16_rne((q - z) * s)
+// (quantization tutorial §2.1 / §2.3).
 //
 // Design (B200-first; the pages' Marlin kernel targets H-series mma.sync and
 // is prior art only):
@@ -20,16 +24,18 @@
 //    which keeps the shared-memory traffic of a decode step at the packed
 //    bytes plus the activations;
 //  * with 256-wide k-blocks a register pair holds codes (j, j + 4) of a packed
-//    word, which saves the PRMT that natural order needs; the MMA issuers
-//    reorder their activation chunks in shared memory to match, overlapped
-//    with the unpacking of the same stage;
+//    word, which saves the PRMT that natural order needs; two activation-
+//    reorder warps permute the activation chunks in shared memory to match,
+//    overlapped with the unpacking of the same stage;
 //  * activations arrive by TMA in the canonical K-major 128-byte-swizzled
 //    layout (dense), or by cp.async row gathers into the same layout (MoE);
 //  * warp specialization: warp 0 = loads + TMEM allocation, then groups of
-//    four dequant warps that take turns over the k-blocks, then four MMA +
-//    epilogue warps (several MMA issuers, each into its own accumulator,
-//    because one thread issues a small tcgen05.mma only every ~100 cycles),
-//    with mbarrier rings between the roles;
+//    four dequant warps that take turns over the k-blocks, then four epilogue
+//    warps and the MMA issuers (several where one thread cannot keep up: it
+//    issues a tcgen05.mma only every ~100 cycles; each issuer owns its own
+//    accumulator and every NSPLIT-th K step, or, for the 256-token tiles, its
+//    own token range of one accumulator at every K step), with mbarrier rings
+//    between the roles;
 //  * persistent CTAs (one per SM) walk a static list of work items.  A decode
 //    GEMM given a workspace splits the (row tile, k-block) units evenly over
 //    the SMs (stream-K); the last CTA to finish a row tile adds the parked
