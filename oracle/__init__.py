@@ -72,6 +72,18 @@ def load_library(path: str) -> ctypes.CDLL:
     L.w4o_quantize_zp.argtypes = [_P, _I64, _I64, _I64, _P, _P, _P]
     L.w4o_quantize_pack_zp.argtypes = [_P, _I64, _I64, _I64, _P, _P, _P]
     L.w4o_dequant_zp.argtypes = [_P, _P, _P, _I64, _I64, _I64, _P]
+    L.w4o_e2m1_value.restype = ctypes.c_double
+    L.w4o_e2m1_value.argtypes = [ctypes.c_uint8]
+    L.w4o_e2m1_encode.restype = ctypes.c_uint8
+    L.w4o_e2m1_encode.argtypes = [ctypes.c_double]
+    L.w4o_e4m3_value.restype = ctypes.c_double
+    L.w4o_e4m3_value.argtypes = [ctypes.c_uint8]
+    L.w4o_e4m3_encode.restype = ctypes.c_uint8
+    L.w4o_e4m3_encode.argtypes = [ctypes.c_double]
+    L.w4o_quantize_mxfp4.argtypes = [_P, _I64, _I64, _P, _P]
+    L.w4o_dequant_mxfp4.argtypes = [_P, _P, _I64, _I64, _P]
+    L.w4o_quantize_nvfp4.argtypes = [_P, _I64, _I64, _P, _P, _P]
+    L.w4o_dequant_nvfp4.argtypes = [_P, _P, ctypes.c_float, _I64, _I64, _P]
     L.w4o_moe_align.restype = ctypes.c_int
     L.w4o_moe_align.argtypes = [_P, _I64, _I64, _I64, _I64, _P, _I64, _P, _P]
     L.w4o_moe_gemm.argtypes = [_P, _I64, _P, _P, _P, _I64, _I64, _I64, _I64,
@@ -240,6 +252,63 @@ def w4a16_gemm_zp(X: np.ndarray, Wq: np.ndarray, S: np.ndarray, Z: np.ndarray,
                   group: int = 32, want_r: bool = True):
     """Y = X · dequant_zp(Wq, S, Z)^T, by the plain GEMM definition."""
     return gemm(X, dequant_zp(Wq, S, Z, group), want_r)
+
+
+# ---- micro-scaled FP4 (MXFP4: 32 per E8M0 scale; NVFP4: 16 per E4M3 scale) ---
+
+def e2m1_value(code: int) -> float:
+    return float(lib().w4o_e2m1_value(code))
+
+
+def e2m1_encode(v: float) -> int:
+    return int(lib().w4o_e2m1_encode(float(v)))
+
+
+def e4m3_value(code: int) -> float:
+    return float(lib().w4o_e4m3_value(code))
+
+
+def e4m3_encode(v: float) -> int:
+    return int(lib().w4o_e4m3_encode(float(v)))
+
+
+def quantize_mxfp4(W: np.ndarray):
+    """(q uint8 E2M1 codes [rows, K], E uint8 biased exponents [rows, K/32])."""
+    W = _u16(W)
+    rows, K = W.shape
+    q = np.empty((rows, K), np.uint8)
+    E = np.empty((rows, K // 32), np.uint8)
+    lib().w4o_quantize_mxfp4(_ptr(W), rows, K, _ptr(q), _ptr(E))
+    return q, E
+
+
+def dequant_mxfp4(q: np.ndarray, E: np.ndarray) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    E = np.ascontiguousarray(E, dtype=np.uint8)
+    rows, K = q.shape
+    Wdq = np.empty((rows, K), np.uint16)
+    lib().w4o_dequant_mxfp4(_ptr(q), _ptr(E), rows, K, _ptr(Wdq))
+    return Wdq
+
+
+def quantize_nvfp4(W: np.ndarray):
+    """(q uint8 E2M1 codes [rows, K], S uint8 E4M3 scales [rows, K/16], g float)."""
+    W = _u16(W)
+    rows, K = W.shape
+    q = np.empty((rows, K), np.uint8)
+    S = np.empty((rows, K // 16), np.uint8)
+    g = np.zeros(1, np.float32)
+    lib().w4o_quantize_nvfp4(_ptr(W), rows, K, _ptr(q), _ptr(S), _ptr(g))
+    return q, S, float(g[0])
+
+
+def dequant_nvfp4(q: np.ndarray, S: np.ndarray, g: float) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    S = np.ascontiguousarray(S, dtype=np.uint8)
+    rows, K = q.shape
+    Wdq = np.empty((rows, K), np.uint16)
+    lib().w4o_dequant_nvfp4(_ptr(q), _ptr(S), ctypes.c_float(g), rows, K, _ptr(Wdq))
+    return Wdq
 
 
 def symmetric_quantize_f64(x: np.ndarray, qmax: int, group: int | None = None):

@@ -370,6 +370,160 @@ void w4o_dequant_zp(const int32_t *Wq, const uint16_t *S, const uint8_t *Z, int6
 }
 
 /* ------------------------------------------------------------------------ */
+/* Micro-scaled 4-bit floating point (the MR-GPTQ / QuTLASS summary page:    */
+/* MXFP4 shares one scale per 32 elements, 4.25 bits per element, so an      */
+/* 8-bit power-of-two scale; NVFP4 shares one per 16 elements).  The element */
+/* format is the 4-bit float E2M1 (1 sign, 2 exponent bits with bias 1, 1     */
+/* mantissa bit; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6; no inf or NaN).      */
+/* Readings where the page is silent:                                        */
+/*   - element rounding: nearest E2M1 value, ties to the even code (mantissa  */
+/*     bit 0), magnitudes above 6 saturate to 6, zero is +0;                  */
+/*   - MXFP4: scale 2^e with e = floor(log2(amax)) - 2 (2 = the exponent of   */
+/*     E2M1's largest value), clamped to [-127, 127], stored as e + 127; an   */
+/*     all-zero group stores e = 0;                                          */
+/*   - NVFP4: an FP8 E4M3 group scale (bias 7, largest 448) under one fp32    */
+/*     per-tensor scale g = fl32(amax_tensor / (6 * 448)) (g = 1 for an all-  */
+/*     zero tensor); the group scale is amax_group / (6 g) rounded to E4M3    */
+/*     (nearest, ties to the even code, saturating at 448); elements divide   */
+/*     by s * g; a group whose scale rounds to 0 stores zeros;               */
+/*   - dequantized value: bf16_rne(fl32(fl32(value(q) * s) * g)) (MXFP4:       */
+/*     value(q) * 2^e, exact, then BF16).                                    */
+/* Quotients are taken in fp64: a BF16 value over a 4- or 8-bit significand */
+/* (times the fp32 g) is either exactly on a rounding midpoint or at least    */
+/* 2^-32 relative away from it, far above the fp64 rounding error.           */
+/* ------------------------------------------------------------------------ */
+
+static const double kE2M1[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+double w4o_e2m1_value(uint8_t code)
+{
+    double v = kE2M1[code & 7u];
+    return (code & 8u) ? -v : v;
+}
+
+/* Nearest-even rounding of v onto a sorted table of n non-negative values
+ * (index order = code order), saturating at the last entry. */
+static int round_to_table(double a, const double *tab, int n)
+{
+    if (a >= tab[n - 1]) return n - 1;
+    int i = 0;
+    while (i + 1 < n && tab[i + 1] <= a) ++i;       /* tab[i] <= a < tab[i+1] */
+    if (a == tab[i]) return i;
+    double lo = a - tab[i], hi = tab[i + 1] - a;
+    if (lo < hi) return i;
+    if (hi < lo) return i + 1;
+    return (i % 2 == 0) ? i : i + 1;                 /* tie: the even code */
+}
+
+uint8_t w4o_e2m1_encode(double v)
+{
+    int c = round_to_table(fabs(v), kE2M1, 8);
+    return (uint8_t)((c != 0 && v < 0.0) ? (c | 8) : c);
+}
+
+/* E4M3: code = e << 3 | m (positive half; 0x7F is NaN and never produced). */
+double w4o_e4m3_value(uint8_t code)
+{
+    int e = (code >> 3) & 15, m = code & 7;
+    double v = (e == 0) ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+    return (code & 0x80u) ? -v : v;
+}
+
+uint8_t w4o_e4m3_encode(double v)      /* v >= 0 */
+{
+    static double tab[127];
+    static int init = 0;
+    if (!init) {
+        for (int c = 0; c < 127; ++c) tab[c] = w4o_e4m3_value((uint8_t)c);
+        init = 1;
+    }
+    return (uint8_t)round_to_table(v, tab, 127);
+}
+
+void w4o_quantize_mxfp4(const uint16_t *W, int64_t rows, int64_t K, uint8_t *q, uint8_t *E)
+{
+    int64_t gpr = K / 32;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t g = 0; g < gpr; ++g) {
+            const uint16_t *w = W + r * K + g * 32;
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i) {
+                double a = fabs((double)w4o_f32_from_bf16(w[i]));
+                if (a > amax) amax = a;
+            }
+            int e = 0;
+            if (amax > 0.0) {
+                int ex;
+                frexp(amax, &ex);                  /* amax = f * 2^ex, f in [0.5, 1) */
+                e = (ex - 1) - 2;                  /* floor(log2(amax)) - 2 */
+                if (e < -127) e = -127;
+                if (e > 127) e = 127;
+            }
+            E[r * gpr + g] = (uint8_t)(e + 127);
+            for (int i = 0; i < 32; ++i)
+                q[r * K + g * 32 + i] =
+                    amax > 0.0 ? w4o_e2m1_encode(ldexp((double)w4o_f32_from_bf16(w[i]), -e)) : 0;
+        }
+}
+
+void w4o_dequant_mxfp4(const uint8_t *q, const uint8_t *E, int64_t rows, int64_t K,
+                       uint16_t *Wdq)
+{
+    int64_t gpr = K / 32;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t k = 0; k < K; ++k) {
+            double v = ldexp(w4o_e2m1_value(q[r * K + k]), (int)E[r * gpr + k / 32] - 127);
+            float f = (float)v;                      /* exact: 2 bits times a power of two */
+            if (f == 0.0f) f = 0.0f;
+            Wdq[r * K + k] = w4o_bf16_from_f32(f);
+        }
+}
+
+void w4o_quantize_nvfp4(const uint16_t *W, int64_t rows, int64_t K, uint8_t *q, uint8_t *S,
+                        float *g_out)
+{
+    double amax_t = 0.0;
+    for (int64_t i = 0; i < rows * K; ++i) {
+        double a = fabs((double)w4o_f32_from_bf16(W[i]));
+        if (a > amax_t) amax_t = a;
+    }
+    volatile float denom = 2688.0f;                  /* 6 * 448 */
+    float g = amax_t > 0.0 ? (float)amax_t / denom : 1.0f;
+    if (g == 0.0f) g = 1.0f;
+    *g_out = g;
+    int64_t gpr = K / 16;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < gpr; ++j) {
+            const uint16_t *w = W + r * K + j * 16;
+            double amax = 0.0;
+            for (int i = 0; i < 16; ++i) {
+                double a = fabs((double)w4o_f32_from_bf16(w[i]));
+                if (a > amax) amax = a;
+            }
+            uint8_t sc = w4o_e4m3_encode(amax / (6.0 * (double)g));
+            S[r * gpr + j] = sc;
+            double step = w4o_e4m3_value(sc) * (double)g;
+            for (int i = 0; i < 16; ++i)
+                q[r * K + j * 16 + i] =
+                    step > 0.0 ? w4o_e2m1_encode((double)w4o_f32_from_bf16(w[i]) / step) : 0;
+        }
+}
+
+void w4o_dequant_nvfp4(const uint8_t *q, const uint8_t *S, float g, int64_t rows, int64_t K,
+                       uint16_t *Wdq)
+{
+    int64_t gpr = K / 16;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t k = 0; k < K; ++k) {
+            float qs = (float)(w4o_e2m1_value(q[r * K + k]) *
+                               w4o_e4m3_value(S[r * gpr + k / 16]));   /* exact */
+            float f = qs * g;
+            if (f == 0.0f) f = 0.0f;
+            Wdq[r * K + k] = w4o_bf16_from_f32(f);
+        }
+}
+
+/* ------------------------------------------------------------------------ */
 /* Generic symmetric quantizer of [BAS] §2.2 / §6.1, in fp64, with the scale */
 /* left unrounded: s = max|x| / qmax per group, q = clip(round(x/s)).       */
 /* Used to reproduce the page's worked INT8 example.                         */

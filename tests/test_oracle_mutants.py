@@ -64,6 +64,16 @@ MUTANTS = [
     ("zp_pack_high_first", "word |= (uint32_t)(q8[i] & 0xFu) << (4 * i);",
      "word |= (uint32_t)(q8[i] & 0xFu) << (4 * (7 - i));",
      [pins.test_zp_pack_examples]),
+    ("fp4_ties_up", "return (i % 2 == 0) ? i : i + 1;                 /* tie: the even code */",
+     "return i + 1;", [pins.test_e2m1_table_and_rounding]),
+    ("fp4_no_saturation", "if (a >= tab[n - 1]) return n - 1;", "if (a > 1e30) return n - 1;",
+     [pins.test_e2m1_table_and_rounding]),
+    ("mxfp4_exponent_off_by_one", "e = (ex - 1) - 2;                  /* floor(log2(amax)) - 2 */",
+     "e = (ex - 1) - 1;", [pins.test_mxfp4_brute_force]),
+    ("nvfp4_scale_over_7", "uint8_t sc = w4o_e4m3_encode(amax / (6.0 * (double)g));",
+     "uint8_t sc = w4o_e4m3_encode(amax / (7.0 * (double)g));", [pins.test_nvfp4_brute_force]),
+    ("e4m3_bias_8", "ldexp(1.0 + (double)m / 8.0, e - 7);", "ldexp(1.0 + (double)m / 8.0, e - 8);",
+     [pins.test_e4m3_table_and_rounding]),
     # (random fp64 data has no exact ties, so the tie rule of this path is pinned
     # by group A through the INT4 path, not by the printed example)
     ("p4_scale_off_by_one", "double s = amax / (double)qmax;",

@@ -525,3 +525,117 @@ def test_zp_pack_examples():
     assert (int(w) & 0xFFFFFFFF) == 0xFEDCBA98
     words = np.array([0x76543210, np.int32(-0x01234568)], np.int32)     # 0xFEDCBA98
     assert oracle.unpack_u(words).tolist() == list(range(16))
+
+
+# ---------------------------------------------------------------------------
+# Micro-scaled FP4 (the MR-GPTQ / QuTLASS summary page: MXFP4 with one scale
+# per 32 elements, NVFP4 with one per 16).  The element and scale formats are
+# decoded here from their bit-field definitions (sign, exponent with bias,
+# mantissa), independently of the oracle's tables; codes are checked by brute
+# force over every code in exact rationals.
+# ---------------------------------------------------------------------------
+
+def _minifloat(code: int, ebits: int, mbits: int, bias: int) -> Fraction:
+    sign = -1 if code >> (ebits + mbits) & 1 else 1
+    e = (code >> mbits) & ((1 << ebits) - 1)
+    m = code & ((1 << mbits) - 1)
+    if e == 0:
+        return sign * Fraction(m, 1 << mbits) * Fraction(2) ** (1 - bias)
+    return sign * (1 + Fraction(m, 1 << mbits)) * Fraction(2) ** (e - bias)
+
+
+def _e2m1(c):
+    return _minifloat(c, 2, 1, 1)
+
+
+def _e4m3(c):
+    return _minifloat(c, 4, 3, 7)
+
+
+def _nearest_code(x: Fraction, codes, value):
+    """Nearest representable value to x among codes, ties to the even code; a
+    zero result takes the positive code."""
+    best = None
+    for c in codes:
+        key = (abs(x - value(c)), c & 1, c)
+        if best is None or key < best[0]:
+            best = (key, c)
+    return best[1]
+
+
+def test_e2m1_table_and_rounding():
+    for c in range(16):
+        assert Fraction(oracle.e2m1_value(c)) == _e2m1(c)
+    assert [float(_e2m1(c)) for c in range(8)] == [0, 0.5, 1, 1.5, 2, 3, 4, 6]
+    rng = random.Random(3)
+    pts = [Fraction(k, 8) for k in range(-64, 65)] + [Fraction(rng.randint(-900, 900), 97) for _ in range(300)]
+    for x in pts:
+        want = _nearest_code(x, [c for c in range(16) if c != 8], _e2m1)
+        assert oracle.e2m1_encode(float(x)) == want, x
+    # midpoints go to the even code; magnitudes above 6 saturate
+    assert [oracle.e2m1_encode(v) for v in (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 7.0, 100.0)] == \
+        [0, 2, 2, 4, 4, 6, 6, 7, 7]
+
+
+def test_e4m3_table_and_rounding():
+    for c in range(127):
+        assert Fraction(oracle.e4m3_value(c)) == _e4m3(c), c
+    assert oracle.e4m3_value(126) == 448.0 and oracle.e4m3_value(1) == 2.0 ** -9
+    rng = random.Random(5)
+    for _ in range(2000):
+        x = Fraction(rng.randint(1, 1 << 20), 1 << rng.randint(0, 40))
+        want = _nearest_code(x, range(127), _e4m3)
+        assert oracle.e4m3_encode(float(x)) == want, x
+    assert oracle.e4m3_encode(1000.0) == 126             # saturates at 448
+    assert oracle.e4m3_encode(2.0 ** -11) == 0            # below half the smallest step: 0
+
+
+def test_mxfp4_brute_force():
+    rng = random.Random(13)
+    for trial in range(120):
+        scale = Fraction(2) ** rng.randint(-20, 10)
+        vals = [scale * Fraction(rng.randint(-4000, 4000), 512) for _ in range(32)]
+        if trial % 10 == 0:
+            vals = [Fraction(0)] * 32
+        bits = np.array([fraction_to_bf16_bits(v) for v in vals], np.uint16).reshape(1, -1)
+        xs = [bf16_bits_to_fraction(int(b)) for b in bits[0]]
+        q, E = oracle.quantize_mxfp4(bits)
+        amax = max(abs(x) for x in xs)
+        if amax == 0:
+            assert int(E[0, 0]) == 127 and q.max() == 0
+            continue
+        e = 0
+        while Fraction(2) ** e > amax:
+            e -= 1
+        while Fraction(2) ** (e + 1) <= amax:
+            e += 1
+        assert int(E[0, 0]) == e - 2 + 127, trial
+        X = Fraction(2) ** (e - 2)
+        for i, x in enumerate(xs):
+            want = _nearest_code(x / X, [c for c in range(16) if c != 8], _e2m1)
+            assert int(q[0, i]) == want, (trial, i)
+        # dequant: value * 2^e, exact, then BF16
+        back = oracle.dequant_mxfp4(q, E)[0]
+        assert [bf16_bits_to_fraction(int(b)) for b in back] == \
+            [bf16_bits_to_fraction(fraction_to_bf16_bits(_e2m1(int(c)) * X)) for c in q[0]]
+
+
+def test_nvfp4_brute_force():
+    rng = np.random.default_rng(17)
+    x = (rng.standard_normal((6, 64)) * np.exp(rng.uniform(-3, 3, (6, 4))).repeat(16, axis=1)).astype(np.float32)
+    W = oracle.f32_to_bf16_bits(x)
+    q, S, g = oracle.quantize_nvfp4(W)
+    xs = [[bf16_bits_to_fraction(int(b)) for b in row] for row in W]
+    amax_t = max(abs(v) for row in xs for v in row)
+    assert np.float32(g) == np.float32(np.float32(float(amax_t)) / np.float32(2688.0))
+    gF = Fraction(float(np.float32(g)))
+    for r in range(W.shape[0]):
+        for j in range(W.shape[1] // 16):
+            grp = xs[r][16 * j:16 * j + 16]
+            amax = max(abs(v) for v in grp)
+            sc = _nearest_code(amax / (6 * gF), range(127), _e4m3)
+            assert int(S[r, j]) == sc, (r, j)
+            step = _e4m3(sc) * gF
+            for i, v in enumerate(grp):
+                want = 0 if step == 0 else _nearest_code(v / step, [c for c in range(16) if c != 8], _e2m1)
+                assert int(q[r, 16 * j + i]) == want, (r, j, i)
