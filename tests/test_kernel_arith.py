@@ -59,3 +59,38 @@ def test_snap_rounding_matches_ieee_quotient(rel):
         # the code is the low byte of the float's bits
         low = (c.view(np.uint32) & 0xFF).astype(np.uint8).view(np.int8)
         assert np.array_equal(low.astype(np.float64), ref)
+
+
+def _bf16_rne(x64: np.ndarray) -> np.ndarray:
+    """Round float64 values (exact results of a BF16 pair operation) to BF16,
+    ties to even, as packed BF16 arithmetic does; returned as float64."""
+    f = x64.astype(np.float32)          # exact here: the inputs below have <= 24 bits
+    return oracle.bf16_to_f32(oracle.f32_to_bf16_bits(f)).astype(np.float64)
+
+
+def test_zero_point_unpack_identity():
+    """The zero-point unpack: OR-ing a nibble into BF16 128.0 gives 128 + q,
+    subtracting 128 + z leaves q - z exactly, one multiply by the BF16 scale
+    rounds (q - z) * s once, which is the oracle's dequantized value, for
+    every code, every zero point and a spread of scales (normal, subnormal,
+    large)."""
+    q = np.arange(16)
+    z = np.arange(16)
+    qq, zz = np.meshgrid(q, z, indexing="ij")
+    lhs_bits = (0x4300 | qq).astype(np.uint16)
+    rhs_bits = (0x4300 | zz).astype(np.uint16)
+    lhs = oracle.bf16_to_f32(lhs_bits).astype(np.float64)
+    rhs = oracle.bf16_to_f32(rhs_bits).astype(np.float64)
+    assert np.array_equal(lhs, 128.0 + qq) and np.array_equal(rhs, 128.0 + zz)
+    diff = _bf16_rne(lhs - rhs)
+    assert np.array_equal(diff, (qq - zz).astype(np.float64))
+    rng = np.random.default_rng(1)
+    s_bits = np.concatenate([rng.integers(0x0001, 0x7E80, 400), [0x0001, 0x0080, 0x3F80, 0x7E80]])
+    for sb in s_bits.astype(np.uint16):
+        s = float(oracle.bf16_to_f32(np.array([sb], np.uint16))[0])
+        got = _bf16_rne(diff * s)
+        # the oracle's value: bf16_rne of the exact product (q - z) * s
+        want = np.array([[float(oracle.bf16_to_f32(np.array(
+            [oracle.bf16_from_f32_scalar(float(np.float32((a - b) * s)))], np.uint16))[0])
+            for b in z] for a in q])
+        assert np.array_equal(got, want), hex(int(sb))
