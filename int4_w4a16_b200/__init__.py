@@ -133,6 +133,21 @@ def _dtype(t: torch.Tensor, dt: torch.dtype, what: str) -> None:
         raise TypeError(f"{what} must be {dt}, got {t.dtype}")
 
 
+def _arg(t: torch.Tensor, dt: torch.dtype, shape: tuple, what: str) -> None:
+    """dtype and exact shape: the C side sizes its bulk copies from the
+    integer arguments alone, so a smaller buffer would be read or written
+    past its end on the device."""
+    _dtype(t, dt, what)
+    if tuple(t.shape) != tuple(int(d) for d in shape):
+        raise ValueError(f"{what} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _group_cols(K: int, group: int, what: str) -> int:
+    if group <= 0 or K % group:
+        raise ValueError(f"{what}: K = {K} is not a multiple of the group size {group}")
+    return K // group
+
+
 # ---------------------------------------------------------------------------
 # C-ABI calls (same names as include/w4a16.h)
 # ---------------------------------------------------------------------------
@@ -154,8 +169,10 @@ def w4_wait_selftest(limit_us: int, stream=None) -> None:
 
 def w4_fake_quant(W, Wdq, S=None, group: int = GROUP, stream=None) -> None:
     _dtype(W, torch.bfloat16, "W")
-    _dtype(Wdq, torch.bfloat16, "Wdq")
     rows, K = W.shape
+    _arg(Wdq, torch.bfloat16, (rows, K), "Wdq")
+    if S is not None:
+        _arg(S, torch.bfloat16, (rows, _group_cols(K, group, "w4_fake_quant")), "S")
     _check("w4_fake_quant", lib().w4_fake_quant(_ptr(W), _ptr(Wdq), _ptr(S), rows, K, group,
                                                 _stream(stream)))
 
@@ -163,22 +180,26 @@ def w4_fake_quant(W, Wdq, S=None, group: int = GROUP, stream=None) -> None:
 def w4_ste_backward(dWdq, dW, stream=None) -> None:
     _dtype(dWdq, torch.bfloat16, "dWdq")
     _dtype(dW, torch.bfloat16, "dW")
+    if dW.numel() != dWdq.numel():
+        raise ValueError("dW and dWdq must have the same number of elements")
     _check("w4_ste_backward", lib().w4_ste_backward(_ptr(dWdq), _ptr(dW), dWdq.numel(),
                                                     _stream(stream)))
 
 
 def w4_quantize_pack(W, Wq, S, group: int = GROUP, stream=None) -> None:
     _dtype(W, torch.bfloat16, "W")
-    _dtype(Wq, torch.int32, "Wq")
-    _dtype(S, torch.bfloat16, "S")
     rows, K = W.shape
+    _arg(Wq, torch.int32, (rows, K // 8), "Wq")
+    _arg(S, torch.bfloat16, (rows, _group_cols(K, group, "w4_quantize_pack")), "S")
     _check("w4_quantize_pack", lib().w4_quantize_pack(_ptr(W), _ptr(Wq), _ptr(S), rows, K,
                                                       group, _stream(stream)))
 
 
 def w4_dequant(Wq, S, Wdq, group: int = GROUP, stream=None) -> None:
-    _dtype(Wq, torch.int32, "Wq")
+    _dtype(Wdq, torch.bfloat16, "Wdq")
     rows, K = Wdq.shape
+    _arg(Wq, torch.int32, (rows, K // 8), "Wq")
+    _arg(S, torch.bfloat16, (rows, _group_cols(K, group, "w4_dequant")), "S")
     _check("w4_dequant", lib().w4_dequant(_ptr(Wq), _ptr(S), _ptr(Wdq), rows, K, group,
                                           _stream(stream)))
 
@@ -197,6 +218,18 @@ def workspace(device, nbytes: int) -> torch.Tensor:
     return t
 
 
+def _gemm_args(X, Wq, S, Y, group: int, fn: str):
+    """X [M, K] bf16, Wq [N, K/8] int32, S [N, K/group] bf16, Y [M, N] bf16."""
+    _dtype(X, torch.bfloat16, "X")
+    _dtype(Wq, torch.int32, "Wq")
+    M, K = X.shape
+    N = Wq.shape[0]
+    _arg(Wq, torch.int32, (N, K // 8), "Wq")
+    _arg(S, torch.bfloat16, (N, _group_cols(K, group, fn)), "S")
+    _arg(Y, torch.bfloat16, (M, N), "Y")
+    return M, K, N
+
+
 def w4a16_gemm_workspace_bytes(M: int, N: int, K: int) -> int:
     return int(lib().w4a16_gemm_workspace_bytes(M, N, K))
 
@@ -204,12 +237,7 @@ def w4a16_gemm_workspace_bytes(M: int, N: int, K: int) -> int:
 def w4a16_gemm(X, Wq, S, Y, group: int = GROUP, ws="auto", stream=None) -> None:
     """ws: "auto" (the module's zeroed per-device buffer), None (unsplit
     schedule), or a zeroed uint8 CUDA tensor."""
-    _dtype(X, torch.bfloat16, "X")
-    _dtype(Wq, torch.int32, "Wq")
-    M, K = X.shape
-    N = Wq.shape[0]
-    if Wq.shape[1] * 8 != K or tuple(Y.shape) != (M, N):
-        raise ValueError("shape mismatch")
+    M, K, N = _gemm_args(X, Wq, S, Y, group, "w4a16_gemm")
     if isinstance(ws, str):
         need = w4a16_gemm_workspace_bytes(M, N, K)
         ws = workspace(X.device, need) if need > 0 else None
@@ -222,12 +250,7 @@ def w4a16_gemm_noalloc(X, Wq, S, Y, group: int = GROUP, stream=None) -> None:
     """w4a16_gemm without any workspace argument or allocation: the library uses
     a fixed 8 MiB scratch array of its own per device (see include/w4a16.h for
     who needs this and its limits)."""
-    _dtype(X, torch.bfloat16, "X")
-    _dtype(Wq, torch.int32, "Wq")
-    M, K = X.shape
-    N = Wq.shape[0]
-    if Wq.shape[1] * 8 != K or tuple(Y.shape) != (M, N):
-        raise ValueError("shape mismatch")
+    M, K, N = _gemm_args(X, Wq, S, Y, group, "w4a16_gemm_noalloc")
     _check("w4a16_gemm_noalloc", lib().w4a16_gemm_noalloc(_ptr(X), _ptr(Wq), _ptr(S), _ptr(Y),
                                                           M, N, K, group, _stream(stream)))
 
@@ -240,15 +263,38 @@ def w4_moe_align(topk_ids, E: int, block: int, sorted_ids, expert_ids, num_post_
                  stream=None) -> None:
     _dtype(topk_ids, torch.int32, "topk_ids")
     T, topk = topk_ids.shape
+    _dtype(sorted_ids, torch.int32, "sorted_ids")
+    cap = sorted_ids.numel()
+    _arg(expert_ids, torch.int32, (cap // block if block > 0 else 0,), "expert_ids")
+    _arg(num_post_pad, torch.int32, (1,), "num_post_pad")
     _check("w4_moe_align", lib().w4_moe_align(_ptr(topk_ids), T, topk, E, block,
                                               _ptr(sorted_ids), sorted_ids.numel(),
                                               _ptr(expert_ids), _ptr(num_post_pad),
                                               _stream(stream)))
 
 
+def _moe_args(A, a_row_div, S, sorted_ids, expert_ids, num_post_pad, block, num_slots, E, N,
+              K, fn):
+    _dtype(A, torch.bfloat16, "A")
+    if A.dim() != 2 or A.shape[1] != K:
+        raise ValueError(f"A must be [rows, {K}], got {tuple(A.shape)}")
+    if a_row_div <= 0 or A.shape[0] * a_row_div < num_slots:
+        raise ValueError(f"A has {A.shape[0]} rows; slot / {a_row_div} must index them for "
+                         f"{num_slots} slots")
+    _arg(S, torch.bfloat16, (E, N, _group_cols(K, GROUP, fn)), "S")
+    _dtype(sorted_ids, torch.int32, "sorted_ids")
+    _arg(expert_ids, torch.int32, (sorted_ids.numel() // block if block > 0 else 0,),
+         "expert_ids")
+    _arg(num_post_pad, torch.int32, (1,), "num_post_pad")
+
+
 def w4_moe_w4a16_gemm(A, a_row_div: int, Wq, S, sorted_ids, expert_ids, num_post_pad,
                       block: int, num_slots: int, C, stream=None) -> None:
+    _dtype(Wq, torch.int32, "Wq")
     E, N, K8 = Wq.shape
+    _moe_args(A, a_row_div, S, sorted_ids, expert_ids, num_post_pad, block, num_slots, E, N,
+              K8 * 8, "w4_moe_w4a16_gemm")
+    _arg(C, torch.bfloat16, (num_slots, N), "C")
     _check("w4_moe_w4a16_gemm", lib().w4_moe_w4a16_gemm(
         _ptr(A), a_row_div, _ptr(Wq), _ptr(S), _ptr(sorted_ids), _ptr(expert_ids),
         _ptr(num_post_pad), sorted_ids.numel(), block, num_slots, _ptr(C), N, K8 * 8, E,
@@ -258,7 +304,11 @@ def w4_moe_w4a16_gemm(A, a_row_div: int, Wq, S, sorted_ids, expert_ids, num_post
 def w4_moe_w4a16_gemm_silu(A, a_row_div: int, Wq, S, sorted_ids, expert_ids, num_post_pad,
                            block: int, num_slots: int, H, stream=None) -> None:
     """gate_up grouped GEMM with SiLU*up fused: Wq [E, 2F, K/8]; H [num_slots, F]."""
+    _dtype(Wq, torch.int32, "Wq")
     E, N2, K8 = Wq.shape
+    _moe_args(A, a_row_div, S, sorted_ids, expert_ids, num_post_pad, block, num_slots, E, N2,
+              K8 * 8, "w4_moe_w4a16_gemm_silu")
+    _arg(H, torch.bfloat16, (num_slots, N2 // 2), "H")
     _check("w4_moe_w4a16_gemm_silu", lib().w4_moe_w4a16_gemm_silu(
         _ptr(A), a_row_div, _ptr(Wq), _ptr(S), _ptr(sorted_ids), _ptr(expert_ids),
         _ptr(num_post_pad), sorted_ids.numel(), block, num_slots, _ptr(H), N2 // 2, K8 * 8, E,
@@ -268,10 +318,11 @@ def w4_moe_w4a16_gemm_silu(A, a_row_div: int, Wq, S, sorted_ids, expert_ids, num
 def w4_qat_gemm(X, W, Y, group: int = GROUP, stream=None) -> None:
     """Y = X . fake_quant(W)^T, the QDQ fused into the GEMM's weight prologue."""
     _dtype(X, torch.bfloat16, "X")
-    _dtype(W, torch.bfloat16, "W")
-    _dtype(Y, torch.bfloat16, "Y")
     M, K = X.shape
+    _dtype(W, torch.bfloat16, "W")
     N = W.shape[0]
+    _arg(W, torch.bfloat16, (N, K), "W")
+    _arg(Y, torch.bfloat16, (M, N), "Y")
     _check("w4_qat_gemm", lib().w4_qat_gemm(_ptr(X), _ptr(W), _ptr(Y), M, N, K, group,
                                             _stream(stream)))
 
@@ -279,39 +330,38 @@ def w4_qat_gemm(X, W, Y, group: int = GROUP, stream=None) -> None:
 def w4_quantize_pack_zp(W, Wq, S, Z, group: int = GROUP, stream=None) -> None:
     """Asymmetric groups: unsigned codes Wq, BF16 scales S, uint8 zero points Z."""
     _dtype(W, torch.bfloat16, "W")
-    _dtype(Wq, torch.int32, "Wq")
-    _dtype(S, torch.bfloat16, "S")
-    _dtype(Z, torch.uint8, "Z")
     rows, K = W.shape
+    G = _group_cols(K, group, "w4_quantize_pack_zp")
+    _arg(Wq, torch.int32, (rows, K // 8), "Wq")
+    _arg(S, torch.bfloat16, (rows, G), "S")
+    _arg(Z, torch.uint8, (rows, G), "Z")
     _check("w4_quantize_pack_zp", lib().w4_quantize_pack_zp(_ptr(W), _ptr(Wq), _ptr(S), _ptr(Z),
                                                             rows, K, group, _stream(stream)))
 
 
 def w4_dequant_zp(Wq, S, Z, Wdq, group: int = GROUP, stream=None) -> None:
-    _dtype(Wq, torch.int32, "Wq")
-    _dtype(Z, torch.uint8, "Z")
+    _dtype(Wdq, torch.bfloat16, "Wdq")
     rows, K = Wdq.shape
+    G = _group_cols(K, group, "w4_dequant_zp")
+    _arg(Wq, torch.int32, (rows, K // 8), "Wq")
+    _arg(S, torch.bfloat16, (rows, G), "S")
+    _arg(Z, torch.uint8, (rows, G), "Z")
     _check("w4_dequant_zp", lib().w4_dequant_zp(_ptr(Wq), _ptr(S), _ptr(Z), _ptr(Wdq), rows, K,
                                                 group, _stream(stream)))
 
 
 def w4a16_gemm_zp(X, Wq, S, Z, Y, group: int = GROUP, stream=None) -> None:
-    _dtype(X, torch.bfloat16, "X")
-    _dtype(Wq, torch.int32, "Wq")
-    _dtype(S, torch.bfloat16, "S")
-    _dtype(Z, torch.uint8, "Z")
-    _dtype(Y, torch.bfloat16, "Y")
-    M, K = X.shape
-    N = Wq.shape[0]
+    M, K, N = _gemm_args(X, Wq, S, Y, group, "w4a16_gemm_zp")
+    _arg(Z, torch.uint8, (N, K // group), "Z")
     _check("w4a16_gemm_zp", lib().w4a16_gemm_zp(_ptr(X), _ptr(Wq), _ptr(S), _ptr(Z), _ptr(Y),
                                                 M, N, K, group, _stream(stream)))
 
 
 def w4_moe_gate_topk(logits, topk: int, topk_ids, topk_weights, stream=None) -> None:
     _dtype(logits, torch.float32, "logits")
-    _dtype(topk_ids, torch.int32, "topk_ids")
-    _dtype(topk_weights, torch.float32, "topk_weights")
     T, E = logits.shape
+    _arg(topk_ids, torch.int32, (T, topk), "topk_ids")
+    _arg(topk_weights, torch.float32, (T, topk), "topk_weights")
     _check("w4_moe_gate_topk", lib().w4_moe_gate_topk(_ptr(logits), T, E, topk, _ptr(topk_ids),
                                                       _ptr(topk_weights), _stream(stream)))
 
@@ -322,16 +372,17 @@ def w4_moe_block_size(T: int, topk: int, E: int) -> int:
 
 def w4_silu_mul(gate_up, h, stream=None) -> None:
     _dtype(gate_up, torch.bfloat16, "gate_up")
-    _dtype(h, torch.bfloat16, "h")
     S, F2 = gate_up.shape
+    _arg(h, torch.bfloat16, (S, F2 // 2), "h")
     _check("w4_silu_mul", lib().w4_silu_mul(_ptr(gate_up), S, F2 // 2, _ptr(h), _stream(stream)))
 
 
 def w4_moe_combine(D, w, out, stream=None) -> None:
-    _dtype(D, torch.bfloat16, "D")
     _dtype(w, torch.float32, "w")
-    _dtype(out, torch.bfloat16, "out")
     T, topk = w.shape
+    _dtype(D, torch.bfloat16, "D")
+    _arg(D, torch.bfloat16, (T * topk, D.shape[1]), "D")
+    _arg(out, torch.bfloat16, (T, D.shape[1]), "out")
     _check("w4_moe_combine", lib().w4_moe_combine(_ptr(D), _ptr(w), T, topk, D.shape[1],
                                                   _ptr(out), _stream(stream)))
 

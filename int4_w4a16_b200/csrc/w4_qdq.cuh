@@ -42,7 +42,7 @@ __device__ __forceinline__ uint32_t group_amax_bits(const uint32_t (&v)[16]) {
 
 struct GroupScale {
     float s;        // the stored BF16 scale, widened
-    float r;        // rcp_rn(s) on the fast path
+    float r;        // rcp.approx(s) on the fast path (relative error <= 2^-23)
     uint16_t bits;  // BF16 bits of s
     int mode;       // 0: s == 0, 1: normal s (fast path), 2: subnormal s
 };
@@ -150,8 +150,12 @@ __device__ __forceinline__ uint32_t f2_to_bf16x2(uint64_t d) {
 }
 
 // One group of 32 BF16 values (16 words, natural order) -> the 16 BF16x2 words
-// of bf16_rne(q * s), natural order; exact for every finite input (the slow
-// path divides in IEEE fp32 for zero, subnormal or huge scales).
+// of bf16_rne(q * s), natural order; exact for every finite input.  The fast
+// path needs no clamp: a normal BF16 scale is within 2^-9 of amax / 7, so
+// |w / s| <= 7.03.  The slow path (zero, subnormal or huge scale) divides in
+// IEEE fp32 and clamps to [-8, 7]: a subnormal scale has 1..7 significant
+// bits, so there amax / s reaches 8 and more (amax bits 0x001F: s = 4 * 2^-133,
+// 31/4 = 7.75 -> 7; a negative group of that size gives -8).
 __device__ __forceinline__ void fake_quant_group(const uint32_t (&v)[16], uint32_t (&o)[16]) {
     const GroupScale gs = make_scale(group_amax_bits(v));
     if (gs.mode == 1 && gs.s <= 1.2676506e30f) {
@@ -171,7 +175,11 @@ __device__ __forceinline__ void fake_quant_group(const uint32_t (&v)[16], uint32
             float d[2];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const float q = (s == 0.0f) ? 0.0f : (float)__float2int_rn(__fdiv_rn(xs[h], s));
+                // A subnormal s carries as few as one significant bit, so
+                // |w / s| can exceed 7.5 here: the clamp to [-8, 7] fires.
+                const float q = (s == 0.0f)
+                                    ? 0.0f
+                                    : fminf(fmaxf((float)__float2int_rn(__fdiv_rn(xs[h], s)), -8.0f), 7.0f);
                 d[h] = __fmul_rn(q, s);                       // exact
             }
             __nv_bfloat162 hh = __floats2bfloat162_rn(d[0], d[1]);

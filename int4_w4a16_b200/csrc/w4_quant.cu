@@ -34,8 +34,12 @@
 //    brings it to 1.5 * 2^23.  Snapping maps exact ties onto the half-integer
 //    and keeps every other quotient strictly on its own side, so the result
 //    equals rint_half_even(y).  The code is then the low byte of the float's
-//    bits (bits = 0x4B400000 + q).  Scales below 2^-126 (subnormal) take the
-//    plain IEEE-division path.
+//    bits (bits = 0x4B400000 + q).  The fast path needs no clamp: a normal
+//    BF16 scale is within 2^-9 of amax / 7, so |y| <= 7.03.  Scales below
+//    2^-126 (subnormal) take the plain IEEE-division path, which clamps to
+//    [-8, 7]: such a scale has 1..7 significant bits, so amax / s can round to
+//    8 or more there (amax bits 0x001F give s = 4 * 2^-133 and 7.75), and a
+//    negative group then gets code -8.
 #include <algorithm>
 
 #include "w4_common.cuh"
@@ -59,7 +63,11 @@ __device__ __forceinline__ void item_slow(uint4 v, float s, uint32_t *Wq, uint4 
         const float xs[2] = {lo_f(w[j]), hi_f(w[j])};
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            const float q = (s == 0.0f) ? 0.0f : (float)__float2int_rn(__fdiv_rn(xs[h], s));
+            // clamp to [-8, 7]: with a subnormal s (1..7 significant bits)
+            // the quotient can round past the INT4 range
+            const float q = (s == 0.0f)
+                                ? 0.0f
+                                : fminf(fmaxf((float)__float2int_rn(__fdiv_rn(xs[h], s)), -8.0f), 7.0f);
             c[2 * j + h] = __fadd_rn(q, kMagic);
         }
     }

@@ -159,3 +159,48 @@ def test_zero_point_validation_host_only():
     assert L.w4a16_gemm_zp(A16, A16, A16, None, A16, 4, 8, 64, 32, None) == 1  # Z missing
     assert L.w4a16_gemm_zp(A16, A16, A16, A16, MIS, 4, 8, 64, 32, None) == 1   # misaligned Y
     assert L.w4a16_gemm_zp(A16, A16, A16, A16, A16, 0, 8, 64, 32, None) == 0   # empty
+
+
+def _t(shape, dtype):
+    import torch
+    return torch.zeros(shape, dtype=dtype)
+
+
+@pytest.mark.parametrize("case", ["S_dtype", "S_short", "Y_dtype", "Y_shape", "Wq_cols"])
+def test_gemm_binding_checks_every_operand(case):
+    """The binding rejects a wrongly typed or sized operand before any pointer
+    reaches the library: the C side sizes its bulk copies from M, N and K
+    alone, so a short S would be read past its end on the device."""
+    import torch
+    M, N, K = 4, 64, 256
+    X, Wq = _t((M, K), torch.bfloat16), _t((N, K // 8), torch.int32)
+    S, Y = _t((N, K // 32), torch.bfloat16), _t((M, N), torch.bfloat16)
+    if case == "S_dtype":
+        S = _t((N, K // 32), torch.float32)
+    elif case == "S_short":
+        S = _t((N, K // 64), torch.bfloat16)
+    elif case == "Y_dtype":
+        Y = _t((M, N), torch.float32)
+    elif case == "Y_shape":
+        Y = _t((M, N - 1), torch.bfloat16)
+    else:
+        Wq = _t((N, K // 16), torch.int32)
+    for fn in (w4.w4a16_gemm, w4.w4a16_gemm_noalloc):
+        with pytest.raises((TypeError, ValueError)) as ei:
+            fn(X, Wq, S, Y)
+        assert "CUDA tensors" not in str(ei.value), "checked only at the pointer"
+
+
+def test_quantizer_bindings_check_output_shapes():
+    import torch
+    W = _t((8, 64), torch.bfloat16)
+    with pytest.raises(ValueError):
+        w4.w4_quantize_pack(W, _t((8, 8), torch.int32), _t((8, 1), torch.bfloat16))
+    with pytest.raises(ValueError):
+        w4.w4_fake_quant(W, _t((8, 64), torch.bfloat16), _t((8, 3), torch.bfloat16))
+    with pytest.raises(TypeError):
+        w4.w4_dequant(_t((8, 8), torch.int32), _t((8, 2), torch.float16), _t((8, 64), torch.bfloat16))
+    with pytest.raises(ValueError):
+        w4.w4a16_gemm_zp(_t((2, 64), torch.bfloat16), _t((8, 8), torch.int32),
+                         _t((8, 2), torch.bfloat16), _t((8, 1), torch.uint8),
+                         _t((2, 8), torch.bfloat16))

@@ -107,6 +107,43 @@ def test_quantizers_edge_scales():
     _check_quantizers(W)
 
 
+def _subnormal_scale_groups() -> np.ndarray:
+    """Groups whose BF16 scale is subnormal (amax below 7 * 2^-126): there the
+    scale carries 1..7 significant bits, so |w / s| reaches 8 and more and the
+    clamp to [-8, 7] decides the code ("量化基础" §1.3, INT4 = [-8, 7])."""
+    g = []
+    ramp = np.arange(32, dtype=np.uint16)
+    g.append(ramp)                                   # +0x0000 .. +0x001F
+    g.append(ramp | 0x8000)                          # -0x0000 .. -0x001F
+    t = np.zeros(32, np.uint16); t[0] = 0x000A; g.append(t)      # s = 2^-133, w/s = 10
+    t = np.zeros(32, np.uint16); t[17] = 0x800A; g.append(t)
+    # every positive subnormal amax heads a ramp of both signs, and its negation
+    for a in range(0x0001, 0x0080):
+        v = np.linspace(a, 0, 32).round().astype(np.uint16)
+        v[1::2] |= 0x8000
+        v[0] = a
+        g.append(v)
+        g.append(v ^ 0x8000)
+    return np.stack(g)
+
+
+def test_quantizers_subnormal_scales_clamp():
+    G = _subnormal_scale_groups()
+    # the groups really reach past the INT4 range before the clamp
+    w = (G.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    _, S = oracle.quantize(G)
+    s = (S.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        y = np.where(s > 0, w / np.where(s > 0, s, 1.0), 0.0)
+    assert np.rint(y).max() >= 8 and np.rint(y).min() <= -9
+    q, _ = oracle.quantize(G)
+    assert q.max() == 7 and q.min() == -8
+    _check_quantizers(_np_bf16(G))
+    # the same groups as rows of a wider matrix (several groups per row)
+    rows = G.shape[0] // 8
+    _check_quantizers(_np_bf16(G[: rows * 8].reshape(rows, 256)))
+
+
 def test_quantizers_decode_weight_full():
     _check_quantizers(synth.Decode().weight())
 

@@ -54,6 +54,27 @@ def test_qat_gemm_one_hot_exact_with_edge_groups():
     w4.w4_device_status()
 
 
+def test_qat_gemm_one_hot_subnormal_scales():
+    """One-hot X on groups with subnormal scales, where the clamp to [-8, 7]
+    fires: the in-prologue QDQ gives fake_quant(W) bit for bit."""
+    from tests.test_gpu_parity import _subnormal_scale_groups
+    G = _subnormal_scale_groups()
+    rows = G.shape[0] // 8
+    Wb = np.ascontiguousarray(G[: rows * 8].reshape(rows, 256))
+    Wdq, _ = oracle.fake_quant(Wb)
+    Wd = _np_bf16(Wb).to(DEV)
+    K = 256
+    for m0 in range(0, K, 64):
+        X = torch.zeros((64, K), dtype=torch.bfloat16)
+        X[torch.arange(64), m0 + torch.arange(64)] = 1.0
+        Y = bits(w4.qat_gemm(X.to(DEV), Wd))
+        want = Wdq[:, m0:m0 + 64].T
+        if not np.array_equal(Y, want):
+            bad = np.argwhere(Y != want)
+            raise AssertionError(f"one-hot mismatch at m0={m0}: {bad[:8].tolist()}")
+    w4.w4_device_status()
+
+
 def test_qat_gemm_layer_shape_sampled():
     """A QAT-stack layer shape (W[12288, 4096]) at 2048 tokens; the oracle checks
     16 rows of Y spread over M (every weight group enters every checked element)."""
