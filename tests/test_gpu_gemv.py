@@ -3,10 +3,11 @@ ABI.  1..8 activation rows with K a multiple of 256 take the warp-level MMA
 kernel (w4_gemv.cu); the other shapes here run the tensor-memory kernel at the
 same sizes.
 
-Shapes cover every launch configuration of the warp-level kernel: one and two
-row groups of warps per stage (short K); one and several passes of the warps
-over K, with a partly idle last pass; ragged N (not a multiple of 16 or of 4,
-fewer rows than one stage, fewer rows than CTAs)."""
+Shapes cover every launch configuration of the warp-level kernel: one and
+several passes of the warps over K (4096 each), with a partly idle last pass;
+row ranges of one to six 16-row tiles per CTA, including ones whose stages
+outnumber the ring's slots (refills) and more CTAs than SMs; ragged N (not a
+multiple of 16 or of 4, fewer rows than one tile, fewer rows than CTAs)."""
 import numpy as np
 import pytest
 import torch
@@ -26,6 +27,9 @@ pytestmark = pytest.mark.gpu
     (9, 5, 256), (16, 333, 1024), (12, 1000, 1536), (15, 2049, 2048), (16, 260, 4352),
     (10, 300, 7168), (17, 50, 256), (24, 777, 1024), (31, 2049, 1536), (32, 129, 4352),
     (20, 300, 7168), (32, 64, 4096),
+    (2, 9472, 8192),      # 4 tiles x 2 passes per CTA: slots refilled from the ring
+    (3, 20000, 512),      # more CTAs than SMs (24 row quads each at most)
+    (1, 14212, 256),      # just past one wave of 96-row CTAs
 ])
 def test_gemv_shapes(M, N, K):
     X, Wq, S, Y = _gemm_case(M, N, K, seed=M * 31 + N + K)
