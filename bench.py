@@ -35,6 +35,7 @@ import sys
 import tempfile
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -333,6 +334,144 @@ def time_oracle(target_s: float = 15.0, rows: int = 1024, target_1t_s: float = 8
             "cpu_model": _cpu_model()}
 
 
+def _timed_both(fn, budget_s, budget_1t_s):
+    """Seconds per call of fn on all oracle threads and on one thread (each the
+    mean over as many calls as fit the budget, after one warm call)."""
+    import oracle
+
+    def timed(budget):
+        t0 = time.perf_counter()
+        fn()
+        one = time.perf_counter() - t0
+        reps = max(1, int(budget / max(one, 1e-3)))
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            fn()
+        return (time.perf_counter() - t0) / reps, reps
+
+    cores = oracle.get_threads()
+    dt, reps = timed(budget_s)
+    oracle.set_threads(1)
+    try:
+        dt1, reps1 = timed(budget_1t_s)
+    finally:
+        oracle.set_threads(cores)
+    return dt, reps, dt1, reps1, cores
+
+
+def time_oracle_configs(budget_s: float = 3.0, budget_1t_s: float = 2.0, device="cpu"):
+    """The CPU oracle on the other configs, bounded samples, all host cores and
+    one thread (a reported baseline, not a target).  The large inputs are
+    generated on `device` (the same bytes the GPU runs use) and copied to the
+    host before any timing."""
+    import oracle
+    res = {}
+    # tiny layer: the whole hot path on W[1024, 1024], X[4, 1024]
+    cfg = synth.TinyLayer()
+    W, X = synth.bits(cfg.weight()), synth.bits(cfg.activations())
+    G = synth.bits(synth.normal_bf16((cfg.N, cfg.K), 1e-3, 0, 5))
+
+    def tiny():
+        oracle.fake_quant(W)
+        oracle.ste_backward(G)
+        Wq, S = oracle.quantize_pack(W)
+        oracle.w4a16_gemm(X, Wq, S, want_r=False)
+    nk = cfg.N * cfg.K
+    nb = 4 * nk + 4 * nk + (2 * nk + nk // 2 + nk // 16) + (nk // 2 + nk // 16 + 2 * X.size +
+                                                            2 * cfg.M * cfg.N)
+    dt, reps, dt1, reps1, cores = _timed_both(tiny, budget_s, budget_1t_s)
+    res["tiny_layer"] = {"value": nb / dt / 1e9, "value_1_thread": nb / dt1 / 1e9,
+                         "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"the whole config: fake_quant + STE + quantize_pack + "
+                                   f"GEMM (M={cfg.M}) on W[{cfg.N},{cfg.K}]; {reps} / {reps1} "
+                                   "timed passes"}
+    # prefill at M = 512: the GEMM on 4 rows of X spread over M (every weight
+    # group enters every row), throughput extrapolated to the full M
+    pcfg = synth.Prefill()
+    Wp = synth.bits(pcfg.weight(device))
+    Wq, S = oracle.quantize_pack(Wp)
+    del Wp
+    Xp = synth.bits(pcfg.activations(512, device))
+    rows = np.linspace(0, 511, 4).astype(np.int64)
+    Xs = np.ascontiguousarray(Xp[rows])
+    dt, reps, dt1, reps1, cores = _timed_both(
+        lambda: oracle.w4a16_gemm(Xs, Wq, S, want_r=False), budget_s, budget_1t_s)
+    fl = 2.0 * len(rows) * pcfg.N * pcfg.K
+    res["prefill_m512"] = {"value": fl / dt / 1e12, "value_1_thread": fl / dt1 / 1e12,
+                           "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                           "extrapolated": True,
+                           "sample": f"W4A16 GEMM of {len(rows)} of the 512 rows of X (evenly spaced) "
+                                     f"with the full W[{pcfg.N},{pcfg.K}]; the rate holds "
+                                     f"for all 512 rows (time scales linearly in M); "
+                                     f"{reps} / {reps1} timed calls"}
+    del Wq, S
+    # MoE decode, block 16: moe_align + both grouped GEMMs for 4 of the 16 tokens
+    # with the routing folded onto 8 of the 128 experts (the per-slot work, one
+    # expert's weights per routed token, is the same)
+    mcfg = synth.MoEDecode()
+    E8, T = 8, 4
+    ids, _ = mcfg.routing(16)
+    ids = ids[:T]
+    ids8 = (ids.numpy() % E8).astype(np.int32)
+    hid, inter, topk = mcfg.hidden, mcfg.inter, mcfg.topk
+    Wg = synth.normal_bf16((E8, 2 * inter, hid), 0.02, 0, 11, device).cpu()
+    Wd = synth.normal_bf16((E8, hid, inter), 0.02, 0, 12, device).cpu()
+    Wg_dq = np.stack([oracle.fake_quant(synth.bits(Wg[e]))[0] for e in range(E8)])
+    Wd_dq = np.stack([oracle.fake_quant(synth.bits(Wd[e]))[0] for e in range(E8)])
+    del Wg, Wd
+    A = synth.bits(mcfg.tokens(T))
+    Hs = synth.bits(synth.normal_bf16((T * topk, inter), 1.0, 0, 13))
+
+    def moe():
+        s_ids, e_ids, npp = oracle.moe_align(ids8, E8, 16)
+        oracle.moe_gemm(A, topk, Wg_dq, s_ids, e_ids, npp, T * topk, 16, want_r=False)
+        oracle.moe_gemm(Hs, 1, Wd_dq, s_ids, e_ids, npp, T * topk, 16, want_r=False)
+    dt, reps, dt1, reps1, cores = _timed_both(moe, budget_s, budget_1t_s)
+    nb = E8 * (2 * inter * hid + hid * inter) * 9 // 16 + A.nbytes + Hs.nbytes + \
+        2 * T * topk * (2 * inter + hid)
+    res["moe_t16"] = {"value": nb / dt / 1e9, "value_1_thread": nb / dt1 / 1e9,
+                      "unit": "GB/s", "cores": cores, "kind": "oracle",
+                      "sample": f"moe_align + gate_up + down for {T} of the T=16 tokens, "
+                                f"top-{topk}, block 16, "
+                                f"with the routing folded onto {E8} of the 128 experts "
+                                f"(bytes: those experts' packed weights + activations); "
+                                f"{reps} / {reps1} timed passes"}
+    return res
+
+
+def _clocked(local, fn):
+    """fn() with the clocks sampled around it; returns (fn's result, clocks)."""
+    smp = ClockSampler(local)
+    smp.start()
+    try:
+        r = fn()
+    finally:
+        clocks = smp.stop()
+    return r, clocks
+
+
+def run_config_extras(w4, dev, local, peaks):
+    """The other configs' headline figures, measured in the default run with
+    their own clock records: prefill GEMM at M = 2048, one MoE decode layer at
+    T = 64, the 48-layer QAT weight pass."""
+    l2 = torch.zeros(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    flush = lambda: _flush_l2(l2)
+    out = {}
+    r, c = _clocked(local, lambda: bench_prefill(w4, dev, peaks, [2048], 20, flush))
+    out["prefill"] = {**r[0], "clocks": c,
+                      "l2": "256 MB buffer read before every timed launch; median of 20"}
+    torch.cuda.empty_cache()
+    r, c = _clocked(local, lambda: bench_moe_layer(w4, dev, peaks, [64], 20, flush))
+    out["moe_layer"] = {**r[0], "clocks": c,
+                        "l2": "256 MB buffer read before every timed layer; median of 20"}
+    torch.cuda.empty_cache()
+    r, c = _clocked(local, lambda: bench_qat_pass(w4, dev, peaks, 3, flush))
+    out["qat_pass"] = {"kernels": {x["kernel"]: x for x in r}, "clocks": c,
+                       "l2": "each pass reads 9.7 GB (inputs far larger than L2); median of 3"}
+    torch.cuda.empty_cache()
+    return out
+
+
 # ---------------------------------------------------------------------------
 # Main
 # ---------------------------------------------------------------------------
@@ -437,6 +576,143 @@ def _time_kernel(fn, reps, flush):
     return ts[len(ts) // 2], ts[len(ts) // 10], ts[(9 * len(ts)) // 10]
 
 
+def bench_prefill(w4, dev, peaks, Ms, reps, flush):
+    """Prefill GEMM (W[18432, 7168] Laplace(0, 0.015), group 32) at each M."""
+    cfg = synth.Prefill()
+    W = cfg.weight(dev)
+    Wq, S = w4.quantize_pack(W)
+    del W
+    res = []
+    for M in Ms:
+        X = cfg.activations(M, dev)
+        Y = torch.empty((M, cfg.N), dtype=torch.bfloat16, device=dev)
+        fn = lambda: w4.w4a16_gemm(X, Wq, S, Y)
+        for _ in range(3):
+            fn()
+        med, p10, p90 = _time_kernel(fn, reps, flush)
+        fl = 2.0 * M * cfg.N * cfg.K
+        tf = fl / (med * 1e-3) / 1e12
+        res.append({"M": M, "N": cfg.N, "K": cfg.K, "ms": med, "p10": p10,
+                    "p90": p90, "TFLOP/s": tf,
+                    "frac_bf16_burst": tf / peaks["bf16_tflops"],
+                    "frac_bf16_sustained": tf / peaks["bf16_tflops_sustained"]})
+        del X, Y
+    return res
+
+
+def bench_moe_layer(w4, dev, peaks, Ts, reps, flush):
+    """One whole MoE decode layer on the GPU (128 experts, top-8, hidden 4096,
+    intermediate 1536): gating -> moe_align -> gate_up -> SiLU * up -> down ->
+    weighted combine, block size from the library's rule."""
+    cfg = synth.MoEDecode()
+    E, topk, hid, inter = cfg.E, cfg.topk, cfg.hidden, cfg.inter
+    Wg = cfg.gate_up_weight(dev)
+    Wd = cfg.down_weight(dev)
+    Wq_g = torch.empty((E, 2 * inter, hid // 8), dtype=torch.int32, device=dev)
+    S_g = torch.empty((E, 2 * inter, hid // 32), dtype=torch.bfloat16, device=dev)
+    Wq_d = torch.empty((E, hid, inter // 8), dtype=torch.int32, device=dev)
+    S_d = torch.empty((E, hid, inter // 32), dtype=torch.bfloat16, device=dev)
+    for e in range(E):
+        w4.w4_quantize_pack(Wg[e], Wq_g[e], S_g[e])
+        w4.w4_quantize_pack(Wd[e], Wq_d[e], S_d[e])
+    del Wg, Wd
+    per_expert = (2 * inter * hid + hid * inter) * 9 // 16
+    res = []
+    for T in Ts:
+        slots = T * topk
+        block = w4.w4_moe_block_size(T, topk, E)
+        logits = cfg.logits(T, dev)
+        X = cfg.tokens(T, dev)
+        ids = torch.empty((T, topk), dtype=torch.int32, device=dev)
+        wts = torch.empty((T, topk), dtype=torch.float32, device=dev)
+        cap = w4.w4_moe_capacity(T, topk, E, block)
+        s_ids = torch.empty(cap, dtype=torch.int32, device=dev)
+        e_ids = torch.empty(cap // block, dtype=torch.int32, device=dev)
+        npp = torch.empty(4, dtype=torch.int32, device=dev)[:1]
+        C1 = torch.empty((slots, 2 * inter), dtype=torch.bfloat16, device=dev)
+        H = torch.empty((slots, inter), dtype=torch.bfloat16, device=dev)
+        C2 = torch.empty((slots, hid), dtype=torch.bfloat16, device=dev)
+        out_t = torch.empty((T, hid), dtype=torch.bfloat16, device=dev)
+        steps = [
+            ("gate_topk", lambda: w4.w4_moe_gate_topk(logits, topk, ids, wts)),
+            ("moe_align", lambda: w4.w4_moe_align(ids, E, block, s_ids, e_ids, npp)),
+            ("gate_up", lambda: w4.w4_moe_w4a16_gemm(X, topk, Wq_g, S_g, s_ids, e_ids, npp,
+                                                     block, slots, C1)),
+            ("silu_mul", lambda: w4.w4_silu_mul(C1, H)),
+            ("down", lambda: w4.w4_moe_w4a16_gemm(H, 1, Wq_d, S_d, s_ids, e_ids, npp, block,
+                                                  slots, C2)),
+            ("combine", lambda: w4.w4_moe_combine(C2, wts, out_t)),
+        ]
+        fused = [steps[0], steps[1],
+                 ("gate_up_silu", lambda: w4.w4_moe_w4a16_gemm_silu(
+                     X, topk, Wq_g, S_g, s_ids, e_ids, npp, block, slots, H)),
+                 steps[4], steps[5]]
+        layer = lambda: [f() for _, f in steps]
+        layer_fused = lambda: [f() for _, f in fused]
+        layer()
+        layer_fused()
+        torch.cuda.synchronize()
+        active = int(torch.unique(ids).numel())
+        lmed, lp10, lp90 = _time_kernel(layer, reps, flush)
+        fmed = _time_kernel(layer_fused, reps, flush)[0]
+        per = {}
+        for name, f in steps + [fused[2]]:
+            per[name] = _time_kernel(f, max(5, reps // 2), flush)[0] * 1e3
+        act_bytes = (2 * T * hid + 4 * T * E + 8 * slots + 2 * slots * 2 * inter * 2 +
+                     2 * slots * inter * 2 + 2 * slots * hid * 2 + 2 * T * hid)
+        nb = active * per_expert + act_bytes
+        gbs = nb / (lmed * 1e-3) / 1e9
+        nb_fused = nb - 2 * slots * 2 * inter * 2 - 2 * slots * inter     # no gate_up round trip
+        res.append({"T": T, "block": block, "active_experts": active,
+                    "layer_us": lmed * 1e3, "p10_us": lp10 * 1e3,
+                    "p90_us": lp90 * 1e3, "algorithmic_bytes": nb,
+                    "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"],
+                    "layer_fused_us": fmed * 1e3,
+                    "fused_frac": nb_fused / (fmed * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                    "per_kernel_us": per})
+    return res
+
+
+def bench_qat_pass(w4, dev, peaks, reps, flush):
+    """The QAT weight pass over the 48-layer stack (96 matrices, 4.83 G
+    elements): fake_quant, STE into a separate buffer, quantize_pack, each over
+    all matrices back to back."""
+    cfg = synth.QATStack()
+    mats = []
+    for layer in range(cfg.layers):
+        for which in range(2):
+            W = cfg.weight(layer, which, dev)
+            G = cfg.grad(layer, which, dev)
+            rows, K = W.shape
+            mats.append((W, G, torch.empty_like(W), torch.empty_like(W),
+                         torch.empty((rows, K // 8), dtype=torch.int32, device=dev),
+                         torch.empty((rows, K // 32), dtype=torch.bfloat16, device=dev)))
+    n = cfg.elements
+
+    def fq():
+        for (W, G, Wdq, dW, Wq, S) in mats:
+            w4.w4_fake_quant(W, Wdq)
+
+    def ste():
+        for (W, G, Wdq, dW, Wq, S) in mats:
+            w4.w4_ste_backward(G, dW)
+
+    def qp():
+        for (W, G, Wdq, dW, Wq, S) in mats:
+            w4.w4_quantize_pack(W, Wq, S)
+
+    res = []
+    for name, f, bpe in (("fake_quant", fq, 4.0), ("ste_backward", ste, 4.0),
+                         ("quantize_pack", qp, 2.5625)):
+        f()
+        med, p10, p90 = _time_kernel(f, reps, flush)
+        gbs = n * bpe / (med * 1e-3) / 1e9
+        res.append({"kernel": name, "elements": n, "ms": med, "GB/s": gbs,
+                    "frac": gbs / peaks["hbm_gbs"]})
+    del mats
+    return res
+
+
 def run_extra(args):
     import int4_w4a16_b200 as w4
     dev = torch.device("cuda", 0)
@@ -449,23 +725,8 @@ def run_extra(args):
     out = {"workload": args.workload, "peaks": peaks, "l2": "256 MB buffer read before "
            "every timed launch", "reps": reps, "results": []}
     if args.workload == "prefill":
-        cfg = synth.Prefill()
-        W = cfg.weight(dev)
-        Wq, S = w4.quantize_pack(W)
-        del W
-        for M in ([args.m] if args.m else cfg.Ms):
-            X = cfg.activations(M, dev)
-            Y = torch.empty((M, cfg.N), dtype=torch.bfloat16, device=dev)
-            fn = lambda: w4.w4a16_gemm(X, Wq, S, Y)
-            for _ in range(3):
-                fn()
-            med, p10, p90 = _time_kernel(fn, reps, flush)
-            fl = 2.0 * M * cfg.N * cfg.K
-            tf = fl / (med * 1e-3) / 1e12
-            out["results"].append({"M": M, "N": cfg.N, "K": cfg.K, "ms": med, "p10": p10,
-                                   "p90": p90, "TFLOP/s": tf,
-                                   "frac_bf16_burst": tf / peaks["bf16_tflops"],
-                                   "frac_bf16_sustained": tf / peaks["bf16_tflops_sustained"]})
+        out["results"] += bench_prefill(w4, dev, peaks, [args.m] if args.m else synth.Prefill().Ms,
+                                        reps, flush)
     elif args.workload == "moe":
         cfg = synth.MoEDecode()
         Wg = cfg.gate_up_weight(dev)
@@ -512,73 +773,8 @@ def run_extra(args):
                     "down_us": t_dn * 1e3, "down_GB/s": b_dn / (t_dn * 1e-3) / 1e9,
                     "down_frac": b_dn / (t_dn * 1e-3) / 1e9 / peaks["hbm_gbs"]})
     elif args.workload == "moe_layer":
-        # one whole MoE decode layer on the GPU: gating -> moe_align -> gate_up ->
-        # SiLU * up -> down -> weighted combine, block size from the library's rule
-        cfg = synth.MoEDecode()
-        E, topk, hid, inter = cfg.E, cfg.topk, cfg.hidden, cfg.inter
-        Wg = cfg.gate_up_weight(dev)
-        Wd = cfg.down_weight(dev)
-        Wq_g = torch.empty((E, 2 * inter, hid // 8), dtype=torch.int32, device=dev)
-        S_g = torch.empty((E, 2 * inter, hid // 32), dtype=torch.bfloat16, device=dev)
-        Wq_d = torch.empty((E, hid, inter // 8), dtype=torch.int32, device=dev)
-        S_d = torch.empty((E, hid, inter // 32), dtype=torch.bfloat16, device=dev)
-        for e in range(E):
-            w4.w4_quantize_pack(Wg[e], Wq_g[e], S_g[e])
-            w4.w4_quantize_pack(Wd[e], Wq_d[e], S_d[e])
-        del Wg, Wd
-        per_expert = (2 * inter * hid + hid * inter) * 9 // 16
-        for T in ([args.m] if args.m else cfg.Ts):
-            slots = T * topk
-            block = w4.w4_moe_block_size(T, topk, E)
-            logits = cfg.logits(T, dev)
-            X = cfg.tokens(T, dev)
-            ids = torch.empty((T, topk), dtype=torch.int32, device=dev)
-            wts = torch.empty((T, topk), dtype=torch.float32, device=dev)
-            cap = w4.w4_moe_capacity(T, topk, E, block)
-            s_ids = torch.empty(cap, dtype=torch.int32, device=dev)
-            e_ids = torch.empty(cap // block, dtype=torch.int32, device=dev)
-            npp = torch.empty(4, dtype=torch.int32, device=dev)[:1]
-            C1 = torch.empty((slots, 2 * inter), dtype=torch.bfloat16, device=dev)
-            H = torch.empty((slots, inter), dtype=torch.bfloat16, device=dev)
-            C2 = torch.empty((slots, hid), dtype=torch.bfloat16, device=dev)
-            out_t = torch.empty((T, hid), dtype=torch.bfloat16, device=dev)
-            steps = [
-                ("gate_topk", lambda: w4.w4_moe_gate_topk(logits, topk, ids, wts)),
-                ("moe_align", lambda: w4.w4_moe_align(ids, E, block, s_ids, e_ids, npp)),
-                ("gate_up", lambda: w4.w4_moe_w4a16_gemm(X, topk, Wq_g, S_g, s_ids, e_ids, npp,
-                                                         block, slots, C1)),
-                ("silu_mul", lambda: w4.w4_silu_mul(C1, H)),
-                ("down", lambda: w4.w4_moe_w4a16_gemm(H, 1, Wq_d, S_d, s_ids, e_ids, npp, block,
-                                                      slots, C2)),
-                ("combine", lambda: w4.w4_moe_combine(C2, wts, out_t)),
-            ]
-            fused = [steps[0], steps[1],
-                     ("gate_up_silu", lambda: w4.w4_moe_w4a16_gemm_silu(
-                         X, topk, Wq_g, S_g, s_ids, e_ids, npp, block, slots, H)),
-                     steps[4], steps[5]]
-            layer = lambda: [f() for _, f in steps]
-            layer_fused = lambda: [f() for _, f in fused]
-            layer()
-            layer_fused()
-            torch.cuda.synchronize()
-            active = int(torch.unique(ids).numel())
-            lmed, lp10, lp90 = _time_kernel(layer, reps, flush)
-            fmed = _time_kernel(layer_fused, reps, flush)[0]
-            per = {}
-            for name, f in steps + [fused[2]]:
-                per[name] = _time_kernel(f, max(5, reps // 2), flush)[0] * 1e3
-            act_bytes = (2 * T * hid + 4 * T * E + 8 * slots + 2 * slots * 2 * inter * 2 +
-                         2 * slots * inter * 2 + 2 * slots * hid * 2 + 2 * T * hid)
-            nb = active * per_expert + act_bytes
-            gbs = nb / (lmed * 1e-3) / 1e9
-            nb_fused = nb - 2 * slots * 2 * inter * 2 - 2 * slots * inter     # no gate_up round trip
-            out["results"].append({"T": T, "block": block, "active_experts": active,
-                                   "layer_us": lmed * 1e3, "p10_us": lp10 * 1e3,
-                                   "p90_us": lp90 * 1e3, "algorithmic_bytes": nb,
-                                   "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"],
-                                   "layer_fused_us": fmed * 1e3,
-                                   "fused_frac": nb_fused / (fmed * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                                   "per_kernel_us": per})
+        out["results"] += bench_moe_layer(w4, dev, peaks,
+                                          [args.m] if args.m else synth.MoEDecode().Ts, reps, flush)
     elif args.workload == "zp":
         # asymmetric (zero-point) groups: quantizer on the decode sweep's weights
         # (W[12288, 4096]), then the GEMM on that shape at decode and prefill
@@ -692,37 +888,7 @@ def run_extra(args):
             out["results"].append({"kernel": name, "elements": n, "us": med * 1e3,
                                    "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"]})
     elif args.workload == "qat":
-        cfg = synth.QATStack()
-        mats = []
-        for layer in range(cfg.layers):
-            for which in range(2):
-                W = cfg.weight(layer, which, dev)
-                G = cfg.grad(layer, which, dev)
-                rows, K = W.shape
-                mats.append((W, G, torch.empty_like(W), torch.empty_like(W),
-                             torch.empty((rows, K // 8), dtype=torch.int32, device=dev),
-                             torch.empty((rows, K // 32), dtype=torch.bfloat16, device=dev)))
-        n = cfg.elements
-
-        def fq():
-            for (W, G, Wdq, dW, Wq, S) in mats:
-                w4.w4_fake_quant(W, Wdq)
-
-        def ste():
-            for (W, G, Wdq, dW, Wq, S) in mats:
-                w4.w4_ste_backward(G, dW)
-
-        def qp():
-            for (W, G, Wdq, dW, Wq, S) in mats:
-                w4.w4_quantize_pack(W, Wq, S)
-
-        for name, f, bpe in (("fake_quant", fq, 4.0), ("ste_backward", ste, 4.0),
-                             ("quantize_pack", qp, 2.5625)):
-            f()
-            med, p10, p90 = _time_kernel(f, max(3, reps // 10), flush)
-            gbs = n * bpe / (med * 1e-3) / 1e9
-            out["results"].append({"kernel": name, "elements": n, "ms": med, "GB/s": gbs,
-                                   "frac": gbs / peaks["hbm_gbs"]})
+        out["results"] += bench_qat_pass(w4, dev, peaks, max(3, reps // 10), flush)
     w4.w4_device_status()
     print(json.dumps(out), flush=True)
     return 0
@@ -751,6 +917,8 @@ def main():
                              "quant", "zp"],
                     help="decode is the bench line; the others print their own lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other configs' blocks (prefill, MoE layer, QAT pass)")
     ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--e2e-steps", type=int, default=5)
     args = ap.parse_args()
@@ -899,10 +1067,21 @@ def main():
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.e2e_steps
     e2e_value = world * wl.step_bytes / (e2e_ms * 1e-3) / 1e9
+    launches = wl.launches_per_step * args.steps
+    config = wl.config()
 
     cpu = None
+    cpu_configs = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = time_oracle()
+        cpu_configs = time_oracle_configs(device=dev)
+
+    extras = {}
+    if world == 1 and not args.no_extras:
+        del wl, roll, timed, timed_k, timed_g
+        torch.cuda.empty_cache()
+        extras = run_config_extras(w4, dev, local, peaks)
+        w4.w4_device_status()
 
     if rank == 0:
         line = {
@@ -910,7 +1089,7 @@ def main():
             "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16", "data": "synthetic", "config": wl.config(),
+            "dtype": "bf16", "data": "synthetic", "config": config,
             "roofline": {"kernel": dominant, **dom_roofline, "peak_source": peaks["source"]},
             "rooflines": rooflines,
             "decode_gemm": {"GB/s": gemm_bytes / (gemm_us * 1e-6) / 1e9,
@@ -918,9 +1097,11 @@ def main():
                             "us_4M_one_event_pair": gemm_us,
                             "us_4M_sum_of_per_kernel_events": gemm_us_per_kernel_sum},
             "cpu_baseline": cpu,
+            "cpu_baseline_configs": cpu_configs,
+            **extras,
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": wl.launches_per_step * args.steps,
+            "gpu_launches": launches,
             "launch": "timed steps replayed as one CUDA graph with no events inside; per-kernel "
                       "and GEMM-family times from two more replays of the same steps with events",
             "clocks": clocks,

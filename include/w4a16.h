@@ -172,6 +172,11 @@ size_t w4a16_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *     must start at zero (asynchronously, on `stream`), and calls that may
  *     overlap on the GPU (different streams) race on it and must be serialized
  *     by the caller.
+ *   - The device address found at the first call is kept for the life of the
+ *     process: it assumes the device's primary context is not reset
+ *     (cudaDeviceReset) in between.
+ *   - Shapes that w4a16_gemm runs without a split (1..8 rows with K a multiple
+ *     of 256, or shapes too small to split) use no scratch and touch nothing.
  * Arguments as in w4a16_gemm.
  */
 w4_status w4a16_gemm_noalloc(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S,

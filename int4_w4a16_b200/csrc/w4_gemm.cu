@@ -1543,6 +1543,9 @@ extern "C" w4_status w4a16_gemm_noalloc(const w4_bf16 *X, const int32_t *Wq, con
     if (group != 32) return W4_ERR_UNSUPPORTED;
     if (M < 0 || N < 0 || K <= 0 || (K % 32) != 0) return W4_ERR_INVALID_ARG;
     if (M == 0 || N == 0) return W4_OK;
+    // Shapes the warp-level decode kernel takes need no scratch at all.
+    if (w4host::gemv_supported(M, N, K))
+        return w4a16_gemm(X, Wq, S, Y, M, N, K, group, nullptr, 0, stream);
     // The scratch this shape's schedule needs must fit the fixed array.
     SplitPlan sp;
     size_t need = 0, zero_bytes = 0;

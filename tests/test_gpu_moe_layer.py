@@ -62,7 +62,7 @@ def test_combine(T, topk, N):
     assert np.array_equal(out, oracle.moe_combine(bits(D), w, topk))   # bit-exact
 
 
-@pytest.mark.parametrize("T", [16, 64])
+@pytest.mark.parametrize("T", [16, 64, 256])
 def test_moe_layer_stage_by_stage(T):
     """One MoE decode layer on the GPU, each stage checked against the oracle fed
     the GPU's previous stage (so stage errors do not compound)."""

@@ -403,14 +403,15 @@ def _moe_case(T, block, N, K, E=128, topk=8, seed=0, down=False):
     return bits(C), R, ids
 
 
-@pytest.mark.parametrize("T,block", [(16, 16), (16, 32), (16, 64), (64, 16), (64, 64)])
+@pytest.mark.parametrize("T,block", [(16, 16), (16, 32), (16, 64), (64, 16), (64, 32), (64, 64),
+                                     (256, 16), (256, 32)])
 def test_moe_gemm_gate_up(T, block):
     C, R, _ = _moe_case(T, block, N=3072, K=4096, seed=T)
     assert not np.any(C == 0x7FC1), "a real slot was left unwritten"
     assert_gemm_close(C, R, f"moe gate_up T={T} block={block}")
 
 
-@pytest.mark.parametrize("T,block", [(16, 16), (64, 32)])
+@pytest.mark.parametrize("T,block", [(16, 16), (64, 32), (256, 16), (256, 32)])
 def test_moe_gemm_down(T, block):
     C, R, _ = _moe_case(T, block, N=4096, K=1536, seed=100 + T, down=True)
     assert_gemm_close(C, R, f"moe down T={T} block={block}")

@@ -20,9 +20,9 @@ pytestmark = pytest.mark.gpu
 REL_TOL = 1e-2
 
 
-def _close(y_bits, ref_bits, what):
+def _close_to_oracle(y_bits, R, what):
     y = (y_bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-    r = (ref_bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    r = R.astype(np.float64)
     scale = np.abs(r).max()
     err = np.abs(y - r)
     assert err.max() <= REL_TOL * scale, what
@@ -31,9 +31,15 @@ def _close(y_bits, ref_bits, what):
 
 @pytest.mark.parametrize("M", [1, 16, 32])
 def test_noalloc_matches_workspace_entry_point_twice(M):
+    """Two calls in a row give the very bits of w4a16_gemm with a caller
+    workspace: both run the same schedule and add the split's partial sums in
+    the same fixed order, so a wrongly zeroed counter in the shared array would
+    show as a difference.  M = 16 and 32 run the split (scratch in use); M = 1
+    the warp-level kernel, which needs none.  M = 16 is also checked against
+    the oracle's FP32-accumulated product."""
     L = w4.lib()
     cfg = synth.Decode()
-    Wq_h, S_h = oracle.quantize_pack(bits(cfg.weight()))
+    Wq_h, S_h = _decode_weight()
     dev = "cuda"
     Wq = torch.from_numpy(Wq_h).to(dev)
     S = torch.from_numpy(S_h.view(np.int16)).view(torch.bfloat16).to(dev)
@@ -41,6 +47,7 @@ def test_noalloc_matches_workspace_entry_point_twice(M):
     N, K = cfg.N, cfg.K
     stream = torch.cuda.current_stream().cuda_stream
     need = L.w4a16_gemm_workspace_bytes(M, N, K)
+    assert (need > 0) == (M > 8), "the split schedule (scratch) is what M > 8 exercises"
     ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
     Y_ref = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     rc = L.w4a16_gemm(X.data_ptr(), Wq.data_ptr(), S.data_ptr(), Y_ref.data_ptr(), M, N, K, 32,
@@ -52,8 +59,20 @@ def test_noalloc_matches_workspace_entry_point_twice(M):
                                   M, N, K, 32, stream)
         assert rc == 0, f"call {call}: status {rc}"
         torch.cuda.synchronize()
-        _close(bits(Y), bits(Y_ref), f"M={M} call {call}")
+        assert np.array_equal(bits(Y), bits(Y_ref)), f"M={M} call {call}: not the same bits"
     assert L.w4_device_status(stream) == 0
+    if M == 16:
+        _, R = oracle.w4a16_gemm(bits(X), Wq_h, S_h)
+        _close_to_oracle(bits(Y), R, f"M={M} against the oracle")
+
+
+_DECODE = {}
+
+
+def _decode_weight():
+    if "w" not in _DECODE:
+        _DECODE["w"] = oracle.quantize_pack(bits(synth.Decode().weight()))
+    return _DECODE["w"]
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
