@@ -205,24 +205,62 @@ class DecodeWorkload:
         if gemm_ev is not None:
             gemm_ev[1].record()
 
-    def e2e_step(self, host):
-        """Same pass through the public API from pinned host buffers, with the
-        step's inputs copied in and its results copied out."""
+    def e2e_run(self, host, nsteps, start_ev, end_ev):
+        """nsteps passes through the public API from pinned host buffers, with
+        every step's inputs copied in and its results copied out, pipelined the
+        way a serving loop runs: step i + 1's host-to-device copies (one
+        stream) and step i - 1's device-to-host copies (another) overlap step
+        i's kernels, on two device buffer sets.  start_ev / end_ev bracket all
+        of it on the current stream."""
         w4 = self.w4
-        W = host["W"].to(self.W[0].device, non_blocking=True)
-        G = host["G"].to(self.W[0].device, non_blocking=True)
-        Xs = {M: host["X"][M].to(self.W[0].device, non_blocking=True) for M in self.Ms}
-        w4.w4_fake_quant(W, self.Wdq)
-        w4.w4_ste_backward(G, self.dW)
-        w4.w4_quantize_pack(W, self.Wq, self.S)
-        for M in self.Ms:
-            w4.w4a16_gemm(Xs[M], self.Wq, self.S, self.Y[M])
-        host["Wdq"].copy_(self.Wdq, non_blocking=True)
-        host["dW"].copy_(self.dW, non_blocking=True)
-        host["Wq"].copy_(self.Wq, non_blocking=True)
-        host["S"].copy_(self.S, non_blocking=True)
-        for M in self.Ms:
-            host["Y"][M].copy_(self.Y[M], non_blocking=True)
+        dev = self.W[0].device
+        comp = torch.cuda.current_stream()
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        if not hasattr(self, "_e2e_bufs"):
+            mk = lambda t: torch.empty_like(t)
+            self._e2e_bufs = [{"W": mk(self.W[0]), "G": mk(self.G[0]),
+                               "X": {M: mk(self.X[M]) for M in self.Ms},
+                               "Wdq": mk(self.Wdq), "dW": mk(self.dW), "Wq": mk(self.Wq),
+                               "S": mk(self.S), "Y": {M: mk(self.Y[M]) for M in self.Ms}}
+                              for _ in range(2)]
+        bufs = self._e2e_bufs
+        in_ready = [torch.cuda.Event() for _ in range(2)]
+        comp_done = [torch.cuda.Event() for _ in range(2)]
+        out_done = [torch.cuda.Event() for _ in range(2)]
+        start_ev.record(comp)
+        s_in.wait_event(start_ev)
+        s_out.wait_event(start_ev)
+        for i in range(nsteps):
+            b = bufs[i % 2]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(comp_done[i % 2])        # step i - 2 read these inputs
+                b["W"].copy_(host["W"], non_blocking=True)
+                b["G"].copy_(host["G"], non_blocking=True)
+                for M in self.Ms:
+                    b["X"][M].copy_(host["X"][M], non_blocking=True)
+                in_ready[i % 2].record(s_in)
+            comp.wait_event(in_ready[i % 2])
+            if i >= 2:
+                comp.wait_event(out_done[i % 2])             # step i - 2's results copied out
+            w4.w4_fake_quant(b["W"], b["Wdq"])
+            w4.w4_ste_backward(b["G"], b["dW"])
+            w4.w4_quantize_pack(b["W"], b["Wq"], b["S"])
+            for M in self.Ms:
+                w4.w4a16_gemm(b["X"][M], b["Wq"], b["S"], b["Y"][M])
+            comp_done[i % 2].record(comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(comp_done[i % 2])
+                host["Wdq"].copy_(b["Wdq"], non_blocking=True)
+                host["dW"].copy_(b["dW"], non_blocking=True)
+                host["Wq"].copy_(b["Wq"], non_blocking=True)
+                host["S"].copy_(b["S"], non_blocking=True)
+                for M in self.Ms:
+                    host["Y"][M].copy_(b["Y"][M], non_blocking=True)
+                out_done[i % 2].record(s_out)
+        comp.wait_stream(s_in)
+        comp.wait_stream(s_out)
+        end_ev.record(comp)
 
     def host_buffers(self):
         pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
@@ -469,6 +507,14 @@ def run_config_extras(w4, dev, local, peaks):
     out["qat_pass"] = {"kernels": {x["kernel"]: x for x in r}, "clocks": c,
                        "l2": "each pass reads 9.7 GB (inputs far larger than L2); median of 3"}
     torch.cuda.empty_cache()
+    r, c = _clocked(local, lambda: bench_qat_gemm(w4, dev, peaks, [2048], 10, flush))
+    out["qat_gemm"] = {**r[0], "clocks": c,
+                       "l2": "256 MB buffer read before every timed launch; median of 10"}
+    torch.cuda.empty_cache()
+    r, c = _clocked(local, lambda: bench_fp4(w4, dev, peaks, 10, flush))
+    out["fp4"] = {**r, "clocks": c,
+                  "l2": "256 MB buffer read before every timed launch; median of 10"}
+    torch.cuda.empty_cache()
     return out
 
 
@@ -647,16 +693,23 @@ def bench_moe_layer(w4, dev, peaks, Ts, reps, flush):
                  ("gate_up_silu", lambda: w4.w4_moe_w4a16_gemm_silu(
                      X, topk, Wq_g, S_g, s_ids, e_ids, npp, block, slots, H)),
                  steps[4], steps[5]]
+        cnt = torch.zeros(w4.w4_moe_combine_counter_bytes(T, hid), dtype=torch.uint8, device=dev)
+        down_comb = ("down_combine", lambda: w4.w4_moe_w4a16_gemm_combine(
+            H, Wq_d, S_d, s_ids, e_ids, npp, block, wts, C2, cnt, out_t))
+        combined = steps[:4] + [down_comb]
         layer = lambda: [f() for _, f in steps]
         layer_fused = lambda: [f() for _, f in fused]
+        layer_comb = lambda: [f() for _, f in combined]
         layer()
         layer_fused()
+        layer_comb()
         torch.cuda.synchronize()
         active = int(torch.unique(ids).numel())
         lmed, lp10, lp90 = _time_kernel(layer, reps, flush)
         fmed = _time_kernel(layer_fused, reps, flush)[0]
+        cmed = _time_kernel(layer_comb, reps, flush)[0]
         per = {}
-        for name, f in steps + [fused[2]]:
+        for name, f in steps + [fused[2], down_comb]:
             per[name] = _time_kernel(f, max(5, reps // 2), flush)[0] * 1e3
         act_bytes = (2 * T * hid + 4 * T * E + 8 * slots + 2 * slots * 2 * inter * 2 +
                      2 * slots * inter * 2 + 2 * slots * hid * 2 + 2 * T * hid)
@@ -669,6 +722,8 @@ def bench_moe_layer(w4, dev, peaks, Ts, reps, flush):
                     "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"],
                     "layer_fused_us": fmed * 1e3,
                     "fused_frac": nb_fused / (fmed * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                    "layer_combine_fused_us": cmed * 1e3,
+                    "combine_fused_frac": nb / (cmed * 1e-3) / 1e9 / peaks["hbm_gbs"],
                     "per_kernel_us": per})
     return res
 
@@ -713,6 +768,91 @@ def bench_qat_pass(w4, dev, peaks, reps, flush):
     return res
 
 
+def bench_qat_gemm(w4, dev, peaks, Ms, reps, flush):
+    """QAT GEMMs on a layer of the QAT stack (W[12288, 4096]) with the fake
+    quantization fused into the weight prologue -- forward Y = X . Wdq^T and
+    input gradient dX = dY . Wdq -- beside the unfused chain (w4_fake_quant,
+    then a cuBLAS BF16 GEMM on the materialized Wdq)."""
+    cfg = synth.QATStack()
+    N, K = cfg.shapes[0]
+    W = cfg.weight(0, 0, dev)
+    Wdq = torch.empty_like(W)
+    res = []
+    for M in Ms:
+        X = synth.normal_bf16((M, K), 1.0, 0, 400 + M, dev)
+        dY = synth.normal_bf16((M, N), 1.0, 0, 500 + M, dev)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+        runs = {
+            "forward_fused": lambda: w4.w4_qat_gemm(X, W, Y),
+            "forward_unfused": lambda: (w4.w4_fake_quant(W, Wdq), torch.matmul(X, Wdq.t(), out=Y)),
+            "dx_fused": lambda: w4.w4_qat_gemm_dx(dY, W, dX),
+            "dx_unfused": lambda: (w4.w4_fake_quant(W, Wdq), torch.matmul(dY, Wdq, out=dX)),
+        }
+        fl = 2.0 * M * N * K
+        r = {"M": M, "N": N, "K": K,
+             "unfused": "w4_fake_quant + torch.matmul (cuBLAS BF16) on the materialized Wdq"}
+        for name, f in runs.items():
+            for _ in range(3):
+                f()
+            med, p10, p90 = _time_kernel(f, reps, flush)
+            tf = fl / (med * 1e-3) / 1e12
+            r[name] = {"ms": med, "p10": p10, "p90": p90, "TFLOP/s": tf,
+                       "frac_bf16_burst": tf / peaks["bf16_tflops"]}
+        res.append(r)
+        del X, dY, Y, dX
+    return res
+
+
+def bench_fp4(w4, dev, peaks, reps, flush):
+    """Micro-scaled FP4 weights (MXFP4 and NVFP4) on the decode layer's shape
+    W[12288, 4096]: the W4A16 GEMM at M = 1 (GB/s of packed codes + scales +
+    activations + output) and M = 2048 (TFLOP/s), and the quantizers (GB/s of
+    BF16 in + codes and scales out)."""
+    cfg = synth.Decode()
+    W = cfg.weight(dev)
+    N, K = cfg.N, cfg.K
+    mx = w4.quantize_pack_mxfp4(W)
+    nv = w4.quantize_pack_nvfp4(W)
+    g = float(nv[2].item())
+    res = {}
+    for fmt, Wq, sc, run in (
+            ("mxfp4", mx[0], mx[1], lambda X, Y: w4.w4a16_gemm_mxfp4(X, mx[0], mx[1], Y)),
+            ("nvfp4", nv[0], nv[1], lambda X, Y: w4.w4a16_gemm_nvfp4(X, nv[0], nv[1], g, Y))):
+        r = {}
+        for M in (1, 2048):
+            X = cfg.activations(M, dev) if M <= 64 else synth.normal_bf16((M, K), 1.0, 0, 600, dev)
+            Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            f = lambda: run(X, Y)
+            for _ in range(3):
+                f()
+            med, p10, p90 = _time_kernel(f, reps, flush)
+            nb = Wq.nbytes + sc.nbytes + X.nbytes + Y.nbytes
+            gbs = nb / (med * 1e-3) / 1e9
+            tf = 2.0 * M * N * K / (med * 1e-3) / 1e12
+            r[f"gemm_m{M}"] = {"us": med * 1e3, "p10_us": p10 * 1e3, "p90_us": p90 * 1e3,
+                               "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"], "TFLOP/s": tf,
+                               "frac_bf16_burst": tf / peaks["bf16_tflops"]}
+            del X, Y
+        Wq2, sc2 = torch.empty_like(Wq), torch.empty_like(sc)
+        gd = torch.empty(1, dtype=torch.float32, device=dev)
+        if fmt == "mxfp4":
+            qf = lambda: w4.w4_quantize_pack_mxfp4(W, Wq2, sc2)
+        else:
+            qf = lambda: (w4.w4_nvfp4_tensor_scale(W, gd), w4.w4_quantize_pack_nvfp4(W, gd, Wq2, sc2))
+        for _ in range(3):
+            qf()
+        med, _, _ = _time_kernel(qf, reps, flush)
+        nb = W.nbytes + Wq.nbytes + sc.nbytes + (W.nbytes if fmt == "nvfp4" else 0)
+        r["quantize_pack"] = {"us": med * 1e3, "GB/s": nb / (med * 1e-3) / 1e9,
+                              "frac_hbm": nb / (med * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                              "bytes": "BF16 W in, codes + scales out" +
+                                       (" (+ W read once more for the tensor amax)"
+                                        if fmt == "nvfp4" else "")}
+        res[fmt] = r
+    return res
+
+
 def run_extra(args):
     import int4_w4a16_b200 as w4
     dev = torch.device("cuda", 0)
@@ -743,9 +883,10 @@ def run_extra(args):
         per_gu = 2 * cfg.inter * cfg.hidden * 9 // 16
         per_dn = cfg.hidden * cfg.inter * 9 // 16
         for T in ([args.m] if args.m else cfg.Ts):
-            ids, _ = cfg.routing(T)
+            ids, _ = cfg.routing(T, args.skew)
             ids_d = ids.to(dev)
             active = len(set(ids.view(-1).tolist()))
+            hist = torch.bincount(ids.view(-1).long(), minlength=E)
             X = cfg.tokens(T, dev)
             H = synth.normal_bf16((T * cfg.topk, cfg.inter), 1.0, 0, 300 + T, dev)
             for block in ([args.block] if args.block else cfg.blocks):
@@ -766,7 +907,8 @@ def run_extra(args):
                 b_gu = active * per_gu + X.nbytes + C1.nbytes
                 b_dn = active * per_dn + H.nbytes + C2.nbytes
                 out["results"].append({
-                    "T": T, "block": block, "active_experts": active, "padded_slots": npad,
+                    "T": T, "block": block, "skew": args.skew, "active_experts": active,
+                    "max_expert_slots": int(hist.max()), "padded_slots": npad,
                     "moe_align_us": t_al * 1e3,
                     "gate_up_us": t_gu * 1e3, "gate_up_GB/s": b_gu / (t_gu * 1e-3) / 1e9,
                     "gate_up_frac": b_gu / (t_gu * 1e-3) / 1e9 / peaks["hbm_gbs"],
@@ -814,29 +956,10 @@ def run_extra(args):
                                    "frac_bf16_burst": fl / (med * 1e-3) / 1e12 / peaks["bf16_tflops"],
                                    "symmetric_us": smed * 1e3})
     elif args.workload == "qat_gemm":
-        # QAT forward GEMM on a layer of the QAT stack (W[12288, 4096]) with the
-        # fake quantization fused into the weight prologue, beside the unfused
-        # chain (w4_fake_quant, then a cuBLAS BF16 GEMM on the materialized Wdq)
-        cfg = synth.QATStack()
-        N, K = cfg.shapes[0]
-        W = cfg.weight(0, 0, dev)
-        Wdq = torch.empty_like(W)
-        for M in ([args.m] if args.m else (2048, 8192)):
-            X = synth.normal_bf16((M, K), 1.0, 0, 400 + M, dev)
-            Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-            fused = lambda: w4.w4_qat_gemm(X, W, Y)
-            unfused = lambda: (w4.w4_fake_quant(W, Wdq), torch.matmul(X, Wdq.t(), out=Y))
-            for f in (fused, unfused):
-                f()
-            med, p10, p90 = _time_kernel(fused, reps, flush)
-            umed = _time_kernel(unfused, reps, flush)[0]
-            fl = 2.0 * M * N * K
-            tf = fl / (med * 1e-3) / 1e12
-            out["results"].append({"M": M, "N": N, "K": K, "ms": med, "p10": p10, "p90": p90,
-                                   "TFLOP/s": tf, "frac_bf16_burst": tf / peaks["bf16_tflops"],
-                                   "frac_bf16_sustained": tf / peaks["bf16_tflops_sustained"],
-                                   "unfused_ms": umed,
-                                   "unfused": "w4_fake_quant + torch.matmul (cuBLAS BF16)"})
+        out["results"] += bench_qat_gemm(w4, dev, peaks, [args.m] if args.m else [2048, 8192],
+                                         reps, flush)
+    elif args.workload == "fp4":
+        out["results"].append(bench_fp4(w4, dev, peaks, reps, flush))
     elif args.workload == "gemv":
         # the decode GEMM alone, one activation height at a time (--m picks one)
         cfg = synth.Decode()
@@ -912,15 +1035,17 @@ def main():
                     help="one size only: the activation height (--workload gemv, prefill) or "
                          "the token count T (--workload moe)")
     ap.add_argument("--block", type=int, default=0, help="--workload moe: one block size only")
+    ap.add_argument("--skew", type=float, default=0.0,
+                    help="--workload moe: Zipf-like routing skew (0 = uniform logits)")
     ap.add_argument("--workload", default="decode",
                     choices=["decode", "prefill", "moe", "moe_layer", "qat", "qat_gemm", "gemv",
-                             "quant", "zp"],
+                             "quant", "zp", "fp4"],
                     help="decode is the bench line; the others print their own lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the other configs' blocks (prefill, MoE layer, QAT pass)")
     ap.add_argument("--ref-rows", type=int, default=512)
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=8)
     args = ap.parse_args()
 
     if args.impl == "reference":
@@ -1054,16 +1179,12 @@ def main():
 
     # end to end through the public API, from pinned host memory
     host, h2d, d2h = wl.host_buffers()
-    for _ in range(2):
-        wl.e2e_step(host)
-    torch.cuda.synchronize()
-    barrier(world)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
-        wl.e2e_step(host)
-    e1.record(stream)
+    wl.e2e_run(host, 2, e0, e1)                         # warm-up
+    torch.cuda.synchronize()
+    barrier(world)
+    wl.e2e_run(host, args.e2e_steps, e0, e1)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.e2e_steps
     e2e_value = world * wl.step_bytes / (e2e_ms * 1e-3) / 1e9
@@ -1100,7 +1221,11 @@ def main():
             "cpu_baseline_configs": cpu_configs,
             **extras,
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                    "steps": args.e2e_steps,
+                    "pipelining": "step i+1's host-to-device copies and step i-1's "
+                                  "device-to-host copies on their own streams, overlapping "
+                                  "step i's kernels (two device buffer sets)"},
             "gpu_launches": launches,
             "launch": "timed steps replayed as one CUDA graph with no events inside; per-kernel "
                       "and GEMM-family times from two more replays of the same steps with events",

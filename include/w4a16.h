@@ -16,6 +16,9 @@
  *   [BAS] "量化基础：从 FP32 到 INT4 的压缩艺术": §1.3 (INT4 range [-8, 7],
  *         BF16 1+8+7 bits), §2.2 (s = max|x| / q_max, q = clamp(round(x/s))),
  *         §2.4 (|x_hat - x| <= s/2), §6.2 (round half to even).
+ *   [FP4] MR-GPTQ / QuTLASS FP4 summary page (NVFP4 / MXFP4 on Blackwell):
+ *         MXFP4 = one shared power-of-two scale per 32 values (4.25 bits per
+ *         value), NVFP4 = one FP8 scale per 16 values.
  *
  * Data formats (all row-major, all buffers owned by the caller):
  *   W    [rows, K]        BF16 weights (w4_bf16 = raw BF16 bits), K contiguous.
@@ -138,8 +141,10 @@ w4_status w4_dequant(const int32_t *Wq, const w4_bf16 *S, w4_bf16 *Wdq,
  *        per SM).  NULL, or fewer bytes than w4a16_gemm_workspace_bytes(M, N, K)
  *        reports, selects the unsplit schedule instead (same results).  The
  *        workspace must be all zero before its first use; every call leaves
- *        its counters at zero again.  Calls that may overlap on the GPU must
- *        not share a workspace.  After W4_ERR_TIMEOUT, zero it again.
+ *        its counters (the first 4 KB, whatever the shape) at zero again, so
+ *        one workspace serves any sequence of shapes.  Calls that may overlap
+ *        on the GPU must not share a workspace.  After W4_ERR_TIMEOUT, zero it
+ *        again.
  * Any M >= 1, N >= 1.  Y may not alias an input.
  */
 w4_status w4a16_gemm(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S,
@@ -191,14 +196,31 @@ w4_status w4a16_gemm_noalloc(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 
  * FP32 accumulation, one BF16 rounding, without ever writing Wdq: every
  * 128 x 64 tile of W is quantized and dequantized in registers (the exact
  * arithmetic of w4_fake_quant) on its way to the tensor cores.  The backward
- * pass is the plain BF16 GEMMs of the straight-through estimator (dX = dY.Wdq,
- * dW = dY^T.X), outside this library.
+ * pass of the straight-through estimator is dX = dY.Wdq (w4_qat_gemm_dx, below,
+ * with the same fusion) and dW = dY^T.X (a plain BF16 GEMM that needs no
+ * quantized weight, outside this library).
  *   X   in   [M, K] BF16;  W  in  [N, K] BF16 (the master weights);  Y  out  [M, N] BF16
  * K a multiple of 64 (W4_ERR_UNSUPPORTED otherwise; of 32: W4_ERR_INVALID_ARG);
  * group must be 32; 16-byte aligned, contiguous rows.
  */
 w4_status w4_qat_gemm(const w4_bf16 *X, const w4_bf16 *W, w4_bf16 *Y, int64_t M, int64_t N,
                       int64_t K, int group, void *stream);
+
+/*
+ * QAT input gradient with the same fusion -- [QAT] fake quantization with a
+ * straight-through estimator, [TAG] [8][9] (the backward pass through the fake-
+ * quantized weight uses Wdq itself):
+ *     dX[m, k] = sum_n dY[m, n] * Wdq[n, k],   Wdq = w4_fake_quant(W)  (group 32)
+ * FP32 accumulation, one BF16 rounding, without writing Wdq: each 64 x 128
+ * tile of W goes through the group QDQ in registers and is stored transposed
+ * in shared memory as the A operand of tcgen05 BF16 MMAs (output rows = K).
+ *   dY  in   [M, N] BF16;  W  in  [N, K] BF16 (the master weights);  dX  out  [M, K] BF16
+ * K a multiple of 64 and N a multiple of 8 (W4_ERR_UNSUPPORTED otherwise; K
+ * not a multiple of 32: W4_ERR_INVALID_ARG); group must be 32; 16-byte
+ * aligned, contiguous rows.  N == 0 writes dX = 0.
+ */
+w4_status w4_qat_gemm_dx(const w4_bf16 *dY, const w4_bf16 *W, w4_bf16 *dX, int64_t M, int64_t N,
+                         int64_t K, int group, void *stream);
 
 /*
  * Asymmetric (zero-point) groups -- [BAS] §2.1 (affine map q = clamp(round(x/s)
@@ -234,6 +256,57 @@ w4_status w4_dequant_zp(const int32_t *Wq, const w4_bf16 *S, const uint8_t *Z, w
  */
 w4_status w4a16_gemm_zp(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S, const uint8_t *Z,
                         w4_bf16 *Y, int64_t M, int64_t N, int64_t K, int group, void *stream);
+
+/*
+ * ---------------------------------------------------------------------------
+ * Micro-scaled FP4 weight groups -- [FP4] (MXFP4: groups of 32 with a power-of-
+ * two scale; NVFP4: groups of 16 with an FP8 E4M3 scale); the activations stay
+ * BF16, as in every W4A16 call.  The element is E2M1 (magnitudes 0, 0.5, 1,
+ * 1.5, 2, 3, 4, 6; code = sign << 3 | magnitude index).  The page gives the
+ * group sizes and scale types; the rest is read plainly:
+ *   element code = nearest E2M1 value of w / step, ties to the even code,
+ *                  saturating at 6, zero coded as +0;
+ *   MXFP4 step   = 2^e, e = floor(log2 amax) - 2 clamped to [-127, 127],
+ *                  stored as E = e + 127 (E8M0); all-zero group: E = 127;
+ *   NVFP4 step   = e4m3(amax_group / (6 g)) * g, g = fl32(amax_tensor / 2688)
+ *                  (1 for an all-zero tensor), E4M3 rounding nearest-even and
+ *                  saturating at 448; a zero group scale stores zero codes;
+ *   dequantized  = bf16_rne(fl32(fl32(value * s) * g))  (MXFP4: g = 1), +0.0
+ *                  for a zero.
+ *   Wq   [rows, K/8]  int32, eight 4-bit codes per word, low nibble first
+ *   E    [rows, K/32] uint8 E8M0 exponents (MXFP4); 255 is not a valid scale
+ *   S    [rows, K/16] uint8 E4M3 scales (NVFP4); 0x7F / 0xFF are not valid
+ *   g    FP32 tensor scale (NVFP4)
+ * K a positive multiple of 32; W, Wq, Wdq, X, Y 16-byte aligned; E, S any
+ * alignment, not NULL.
+ */
+w4_status w4_quantize_pack_mxfp4(const w4_bf16 *W, int32_t *Wq, uint8_t *E, int64_t rows,
+                                 int64_t K, void *stream);
+w4_status w4_dequant_mxfp4(const int32_t *Wq, const uint8_t *E, w4_bf16 *Wdq, int64_t rows,
+                           int64_t K, void *stream);
+/* NVFP4 tensor scale of W[n] into *g (device float, 4-byte aligned):
+ * g = fl32(max|W| / 2688), or 1 when W is all zero.  W 4-byte aligned. */
+w4_status w4_nvfp4_tensor_scale(const w4_bf16 *W, int64_t n, float *g, void *stream);
+/* NVFP4 codes and group scales of W under the tensor scale *g (device float,
+ * as written by w4_nvfp4_tensor_scale). */
+w4_status w4_quantize_pack_nvfp4(const w4_bf16 *W, const float *g, int32_t *Wq, uint8_t *S,
+                                 int64_t rows, int64_t K, void *stream);
+/* g is passed by value (host float). */
+w4_status w4_dequant_nvfp4(const int32_t *Wq, const uint8_t *S, float g, w4_bf16 *Wdq,
+                           int64_t rows, int64_t K, void *stream);
+/*
+ * W4A16 GEMM on FP4 weight groups: Y[M, N] = X[M, K] . Wdq^T with Wdq the
+ * dequantized FP4 weights above, FP32 accumulation, one BF16 rounding.  The
+ * codes are unpacked in registers (hardware E2M1 -> FP16 conversion, exact
+ * FP32 scaling, BF16 rounding) and stored into tensor memory as the A
+ * operand of tcgen05 BF16 MMAs, as in w4a16_gemm_zp's kernel.
+ *   X in [M, K] BF16;  Wq in [N, K/8];  E in [N, K/32] / S in [N, K/16];
+ *   Y out [M, N] BF16.  Device pointers; asynchronous on `stream`.
+ */
+w4_status w4a16_gemm_mxfp4(const w4_bf16 *X, const int32_t *Wq, const uint8_t *E, w4_bf16 *Y,
+                           int64_t M, int64_t N, int64_t K, void *stream);
+w4_status w4a16_gemm_nvfp4(const w4_bf16 *X, const int32_t *Wq, const uint8_t *S, float g,
+                           w4_bf16 *Y, int64_t M, int64_t N, int64_t K, void *stream);
 
 /* Padded capacity the caller must provide for w4_moe_align's sorted_ids:
  * T*topk + E*(block-1), rounded up to a multiple of block.  Host-only. */
@@ -353,6 +426,34 @@ w4_status w4_silu_mul(const w4_bf16 *gate_up, int64_t S, int64_t F, w4_bf16 *h, 
  */
 w4_status w4_moe_combine(const w4_bf16 *D, const float *w, int64_t T, int topk, int64_t N,
                          w4_bf16 *out, void *stream);
+
+/*
+ * Down projection with the weighted top-k combine fused into its epilogue
+ * ([QAT] "MoE operator deep fusion"): w4_moe_w4a16_gemm with a_row_div = 1 and
+ * num_slots = T * topk, writing C as that call does, and in the same kernel
+ *     out[t, n] = bf16( sum_{k ascending} w[t, k] * C[t * topk + k, n] )
+ * with w4_moe_combine's arithmetic (every product and sum rounded once, FP32),
+ * so out is bit for bit what w4_moe_combine gives on this C.  The last work
+ * item to finish a token's rows does the sum: an arrival counter per (token,
+ * 128-row tile, 32-row quarter) in `counters` decides which, so the result does
+ * not depend on the order in which work items finish.
+ *   w         in   [T, topk] FP32 routing weights (device)
+ *   counters  in/out  w4_moe_combine_counter_bytes(T, N) bytes (device, 16-byte
+ *                  aligned), all zero before the first call; every call leaves
+ *                  them zero again (zero them again after W4_ERR_TIMEOUT)
+ *   out       out  [T, N] BF16
+ * Every slot must be routed to an expert in [0, E) (w4_moe_gate_topk's ids
+ * are): a token with a skipped slot never completes and its out row is not
+ * written.  Other arguments and constraints as in w4_moe_w4a16_gemm; topk in
+ * [1, 64].
+ */
+size_t w4_moe_combine_counter_bytes(int64_t T, int64_t N);
+w4_status w4_moe_w4a16_gemm_combine(const w4_bf16 *A, const int32_t *Wq, const w4_bf16 *S,
+                                    const int32_t *sorted_ids, const int32_t *expert_ids,
+                                    const int32_t *num_post_pad, int64_t cap, int block,
+                                    int topk, const float *w, w4_bf16 *C, unsigned int *counters,
+                                    w4_bf16 *out, int64_t T, int64_t N, int64_t K, int E,
+                                    void *stream);
 
 #ifdef __cplusplus
 }

@@ -28,10 +28,15 @@ __all__ = [
     "w4_device_status", "w4_wait_selftest", "w4_fake_quant", "w4_ste_backward",
     "w4_quantize_pack", "w4_dequant", "w4a16_gemm", "w4_moe_capacity", "w4_moe_align",
     "w4_moe_w4a16_gemm", "w4_moe_w4a16_gemm_silu", "w4_moe_gate_topk", "w4_moe_block_size",
-    "w4_silu_mul", "moe_gemm_silu", "w4_qat_gemm", "qat_gemm",
+    "w4_silu_mul", "moe_gemm_silu", "w4_qat_gemm", "qat_gemm", "w4_qat_gemm_dx", "qat_gemm_dx",
     "w4_quantize_pack_zp", "w4_dequant_zp", "w4a16_gemm_zp", "quantize_pack_zp", "dequant_zp",
     "gemm_zp",
-    "w4_moe_combine", "fake_quant", "quantize_pack", "dequant", "gemm", "moe_align",
+    "w4_quantize_pack_mxfp4", "w4_dequant_mxfp4", "w4_nvfp4_tensor_scale",
+    "w4_quantize_pack_nvfp4", "w4_dequant_nvfp4", "w4a16_gemm_mxfp4", "w4a16_gemm_nvfp4",
+    "quantize_pack_mxfp4", "dequant_mxfp4", "gemm_mxfp4", "quantize_pack_nvfp4",
+    "dequant_nvfp4", "gemm_nvfp4",
+    "w4_moe_combine", "w4_moe_combine_counter_bytes", "w4_moe_w4a16_gemm_combine",
+    "moe_gemm_combine", "fake_quant", "quantize_pack", "dequant", "gemm", "moe_align",
     "moe_gate_topk", "silu_mul", "moe_combine",
     "moe_gemm", "FakeInt4STE", "GROUP",
 ]
@@ -82,11 +87,21 @@ def lib() -> ctypes.CDLL:
                                        _I64, _I64, _INT, _P],
             "w4_moe_gate_topk": [_P, _I64, _INT, _INT, _P, _P, _P],
             "w4_qat_gemm": [_P, _P, _P, _I64, _I64, _I64, _INT, _P],
+            "w4_qat_gemm_dx": [_P, _P, _P, _I64, _I64, _I64, _INT, _P],
             "w4_quantize_pack_zp": [_P, _P, _P, _P, _I64, _I64, _INT, _P],
             "w4_dequant_zp": [_P, _P, _P, _P, _I64, _I64, _INT, _P],
             "w4a16_gemm_zp": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _INT, _P],
+            "w4_quantize_pack_mxfp4": [_P, _P, _P, _I64, _I64, _P],
+            "w4_dequant_mxfp4": [_P, _P, _P, _I64, _I64, _P],
+            "w4_nvfp4_tensor_scale": [_P, _I64, _P, _P],
+            "w4_quantize_pack_nvfp4": [_P, _P, _P, _P, _I64, _I64, _P],
+            "w4_dequant_nvfp4": [_P, _P, ctypes.c_float, _P, _I64, _I64, _P],
+            "w4a16_gemm_mxfp4": [_P, _P, _P, _P, _I64, _I64, _I64, _P],
+            "w4a16_gemm_nvfp4": [_P, _P, _P, ctypes.c_float, _P, _I64, _I64, _I64, _P],
             "w4_silu_mul": [_P, _I64, _I64, _P, _P],
             "w4_moe_combine": [_P, _P, _I64, _INT, _I64, _P, _P],
+            "w4_moe_w4a16_gemm_combine": [_P, _P, _P, _P, _P, _P, _I64, _INT, _INT, _P, _P, _P,
+                                          _P, _I64, _I64, _I64, _INT, _P],
             "w4_device_status": [_P],
             "w4_wait_selftest": [ctypes.c_uint32, _P],
         }.items():
@@ -98,6 +113,8 @@ def lib() -> ctypes.CDLL:
         L.w4_moe_capacity.argtypes = [_I64, _INT, _INT, _INT]
         L.w4_moe_capacity.restype = ctypes.c_int64
         L.w4_moe_block_size.argtypes = [_I64, _INT, _INT]
+        L.w4_moe_combine_counter_bytes.argtypes = [_I64, _I64]
+        L.w4_moe_combine_counter_bytes.restype = ctypes.c_size_t
         L.w4_moe_block_size.restype = ctypes.c_int
         L.w4_version.restype = ctypes.c_int
         L.w4_last_cuda_error.restype = ctypes.c_int
@@ -301,6 +318,33 @@ def w4_moe_w4a16_gemm(A, a_row_div: int, Wq, S, sorted_ids, expert_ids, num_post
         _stream(stream)))
 
 
+def w4_moe_combine_counter_bytes(T: int, N: int) -> int:
+    return int(lib().w4_moe_combine_counter_bytes(T, N))
+
+
+def w4_moe_w4a16_gemm_combine(A, Wq, S, sorted_ids, expert_ids, num_post_pad, block: int, w,
+                              C, counters, out, stream=None) -> None:
+    """Down projection with the weighted top-k combine fused: A [T*topk, K], w
+    [T, topk] fp32, C [T*topk, N], counters uint8 (zeroed, w4_moe_combine_counter_bytes),
+    out [T, N]."""
+    _dtype(Wq, torch.int32, "Wq")
+    E, N, K8 = Wq.shape
+    _dtype(w, torch.float32, "w")
+    T, topk = w.shape
+    num_slots = T * topk
+    _moe_args(A, 1, S, sorted_ids, expert_ids, num_post_pad, block, num_slots, E, N, K8 * 8,
+              "w4_moe_w4a16_gemm_combine")
+    _arg(C, torch.bfloat16, (num_slots, N), "C")
+    _arg(out, torch.bfloat16, (T, N), "out")
+    _dtype(counters, torch.uint8, "counters")
+    if counters.numel() < w4_moe_combine_counter_bytes(T, N):
+        raise ValueError("counters is smaller than w4_moe_combine_counter_bytes(T, N)")
+    _check("w4_moe_w4a16_gemm_combine", lib().w4_moe_w4a16_gemm_combine(
+        _ptr(A), _ptr(Wq), _ptr(S), _ptr(sorted_ids), _ptr(expert_ids), _ptr(num_post_pad),
+        sorted_ids.numel(), block, topk, _ptr(w), _ptr(C), _ptr(counters), _ptr(out), T, N,
+        K8 * 8, E, _stream(stream)))
+
+
 def w4_moe_w4a16_gemm_silu(A, a_row_div: int, Wq, S, sorted_ids, expert_ids, num_post_pad,
                            block: int, num_slots: int, H, stream=None) -> None:
     """gate_up grouped GEMM with SiLU*up fused: Wq [E, 2F, K/8]; H [num_slots, F]."""
@@ -325,6 +369,18 @@ def w4_qat_gemm(X, W, Y, group: int = GROUP, stream=None) -> None:
     _arg(Y, torch.bfloat16, (M, N), "Y")
     _check("w4_qat_gemm", lib().w4_qat_gemm(_ptr(X), _ptr(W), _ptr(Y), M, N, K, group,
                                             _stream(stream)))
+
+
+def w4_qat_gemm_dx(dY, W, dX, group: int = GROUP, stream=None) -> None:
+    """dX = dY . fake_quant(W), the QDQ fused into the GEMM's weight prologue."""
+    _dtype(dY, torch.bfloat16, "dY")
+    M, N = dY.shape
+    _dtype(W, torch.bfloat16, "W")
+    K = W.shape[1]
+    _arg(W, torch.bfloat16, (N, K), "W")
+    _arg(dX, torch.bfloat16, (M, K), "dX")
+    _check("w4_qat_gemm_dx", lib().w4_qat_gemm_dx(_ptr(dY), _ptr(W), _ptr(dX), M, N, K, group,
+                                                  _stream(stream)))
 
 
 def w4_quantize_pack_zp(W, Wq, S, Z, group: int = GROUP, stream=None) -> None:
@@ -355,6 +411,88 @@ def w4a16_gemm_zp(X, Wq, S, Z, Y, group: int = GROUP, stream=None) -> None:
     _arg(Z, torch.uint8, (N, K // group), "Z")
     _check("w4a16_gemm_zp", lib().w4a16_gemm_zp(_ptr(X), _ptr(Wq), _ptr(S), _ptr(Z), _ptr(Y),
                                                 M, N, K, group, _stream(stream)))
+
+
+def _fp4_cols(K: int, what: str) -> None:
+    if K <= 0 or K % 32:
+        raise ValueError(f"{what}: K = {K} is not a positive multiple of 32")
+
+
+def w4_quantize_pack_mxfp4(W, Wq, E, stream=None) -> None:
+    """MXFP4: E2M1 codes Wq [rows, K/8] int32 and E8M0 exponents E [rows, K/32] uint8."""
+    _dtype(W, torch.bfloat16, "W")
+    rows, K = W.shape
+    _fp4_cols(K, "w4_quantize_pack_mxfp4")
+    _arg(Wq, torch.int32, (rows, K // 8), "Wq")
+    _arg(E, torch.uint8, (rows, K // 32), "E")
+    _check("w4_quantize_pack_mxfp4", lib().w4_quantize_pack_mxfp4(_ptr(W), _ptr(Wq), _ptr(E),
+                                                                  rows, K, _stream(stream)))
+
+
+def w4_dequant_mxfp4(Wq, E, Wdq, stream=None) -> None:
+    _dtype(Wdq, torch.bfloat16, "Wdq")
+    rows, K = Wdq.shape
+    _fp4_cols(K, "w4_dequant_mxfp4")
+    _arg(Wq, torch.int32, (rows, K // 8), "Wq")
+    _arg(E, torch.uint8, (rows, K // 32), "E")
+    _check("w4_dequant_mxfp4", lib().w4_dequant_mxfp4(_ptr(Wq), _ptr(E), _ptr(Wdq), rows, K,
+                                                      _stream(stream)))
+
+
+def w4_nvfp4_tensor_scale(W, g, stream=None) -> None:
+    """g: a one-element float32 CUDA tensor, set to fl32(max|W| / 2688) (1 if W == 0)."""
+    _dtype(W, torch.bfloat16, "W")
+    _arg(g, torch.float32, (1,), "g")
+    _check("w4_nvfp4_tensor_scale", lib().w4_nvfp4_tensor_scale(_ptr(W), W.numel(), _ptr(g),
+                                                                _stream(stream)))
+
+
+def w4_quantize_pack_nvfp4(W, g, Wq, S, stream=None) -> None:
+    """NVFP4 under the device tensor scale g: codes Wq [rows, K/8], E4M3 scales S [rows, K/16]."""
+    _dtype(W, torch.bfloat16, "W")
+    rows, K = W.shape
+    _fp4_cols(K, "w4_quantize_pack_nvfp4")
+    _arg(g, torch.float32, (1,), "g")
+    _arg(Wq, torch.int32, (rows, K // 8), "Wq")
+    _arg(S, torch.uint8, (rows, K // 16), "S")
+    _check("w4_quantize_pack_nvfp4", lib().w4_quantize_pack_nvfp4(_ptr(W), _ptr(g), _ptr(Wq),
+                                                                  _ptr(S), rows, K,
+                                                                  _stream(stream)))
+
+
+def w4_dequant_nvfp4(Wq, S, g: float, Wdq, stream=None) -> None:
+    _dtype(Wdq, torch.bfloat16, "Wdq")
+    rows, K = Wdq.shape
+    _fp4_cols(K, "w4_dequant_nvfp4")
+    _arg(Wq, torch.int32, (rows, K // 8), "Wq")
+    _arg(S, torch.uint8, (rows, K // 16), "S")
+    _check("w4_dequant_nvfp4", lib().w4_dequant_nvfp4(_ptr(Wq), _ptr(S), float(g), _ptr(Wdq),
+                                                      rows, K, _stream(stream)))
+
+
+def _fp4_gemm_args(X, Wq, Y, what: str):
+    _dtype(X, torch.bfloat16, "X")
+    M, K = X.shape
+    _fp4_cols(K, what)
+    _dtype(Wq, torch.int32, "Wq")
+    N = Wq.shape[0]
+    _arg(Wq, torch.int32, (N, K // 8), "Wq")
+    _arg(Y, torch.bfloat16, (M, N), "Y")
+    return M, K, N
+
+
+def w4a16_gemm_mxfp4(X, Wq, E, Y, stream=None) -> None:
+    M, K, N = _fp4_gemm_args(X, Wq, Y, "w4a16_gemm_mxfp4")
+    _arg(E, torch.uint8, (N, K // 32), "E")
+    _check("w4a16_gemm_mxfp4", lib().w4a16_gemm_mxfp4(_ptr(X), _ptr(Wq), _ptr(E), _ptr(Y), M, N,
+                                                      K, _stream(stream)))
+
+
+def w4a16_gemm_nvfp4(X, Wq, S, g: float, Y, stream=None) -> None:
+    M, K, N = _fp4_gemm_args(X, Wq, Y, "w4a16_gemm_nvfp4")
+    _arg(S, torch.uint8, (N, K // 16), "S")
+    _check("w4a16_gemm_nvfp4", lib().w4a16_gemm_nvfp4(_ptr(X), _ptr(Wq), _ptr(S), float(g),
+                                                      _ptr(Y), M, N, K, _stream(stream)))
 
 
 def w4_moe_gate_topk(logits, topk: int, topk_ids, topk_weights, stream=None) -> None:
@@ -436,6 +574,51 @@ def gemm_zp(X: torch.Tensor, Wq: torch.Tensor, S: torch.Tensor, Z: torch.Tensor)
     return Y
 
 
+def quantize_pack_mxfp4(W: torch.Tensor):
+    rows, K = W.shape
+    Wq = torch.empty((rows, K // 8), dtype=torch.int32, device=W.device)
+    E = torch.empty((rows, K // 32), dtype=torch.uint8, device=W.device)
+    w4_quantize_pack_mxfp4(W, Wq, E)
+    return Wq, E
+
+
+def dequant_mxfp4(Wq: torch.Tensor, E: torch.Tensor) -> torch.Tensor:
+    rows, K8 = Wq.shape
+    Wdq = torch.empty((rows, K8 * 8), dtype=torch.bfloat16, device=Wq.device)
+    w4_dequant_mxfp4(Wq, E, Wdq)
+    return Wdq
+
+
+def gemm_mxfp4(X: torch.Tensor, Wq: torch.Tensor, E: torch.Tensor) -> torch.Tensor:
+    Y = torch.empty((X.shape[0], Wq.shape[0]), dtype=torch.bfloat16, device=X.device)
+    w4a16_gemm_mxfp4(X, Wq, E, Y)
+    return Y
+
+
+def quantize_pack_nvfp4(W: torch.Tensor):
+    """Returns (Wq, S, g) with g a one-element float32 device tensor."""
+    rows, K = W.shape
+    g = torch.empty((1,), dtype=torch.float32, device=W.device)
+    Wq = torch.empty((rows, K // 8), dtype=torch.int32, device=W.device)
+    S = torch.empty((rows, K // 16), dtype=torch.uint8, device=W.device)
+    w4_nvfp4_tensor_scale(W, g)
+    w4_quantize_pack_nvfp4(W, g, Wq, S)
+    return Wq, S, g
+
+
+def dequant_nvfp4(Wq: torch.Tensor, S: torch.Tensor, g: float) -> torch.Tensor:
+    rows, K8 = Wq.shape
+    Wdq = torch.empty((rows, K8 * 8), dtype=torch.bfloat16, device=Wq.device)
+    w4_dequant_nvfp4(Wq, S, g, Wdq)
+    return Wdq
+
+
+def gemm_nvfp4(X: torch.Tensor, Wq: torch.Tensor, S: torch.Tensor, g: float) -> torch.Tensor:
+    Y = torch.empty((X.shape[0], Wq.shape[0]), dtype=torch.bfloat16, device=X.device)
+    w4a16_gemm_nvfp4(X, Wq, S, g, Y)
+    return Y
+
+
 def gemm(X: torch.Tensor, Wq: torch.Tensor, S: torch.Tensor, ws="auto") -> torch.Tensor:
     Y = torch.empty((X.shape[0], Wq.shape[0]), dtype=torch.bfloat16, device=X.device)
     w4a16_gemm(X, Wq, S, Y, ws=ws)
@@ -462,6 +645,19 @@ def moe_gemm(A, a_row_div, Wq, S, sorted_ids, expert_ids, num_post_pad, block, n
     return C
 
 
+def moe_gemm_combine(H, Wq, S, sorted_ids, expert_ids, num_post_pad, block, w, counters,
+                     C=None, out=None):
+    """Returns (C, out): the down projection's slot rows and their weighted combine."""
+    T, topk = w.shape
+    if C is None:
+        C = torch.empty((T * topk, Wq.shape[1]), dtype=torch.bfloat16, device=H.device)
+    if out is None:
+        out = torch.empty((T, Wq.shape[1]), dtype=torch.bfloat16, device=H.device)
+    w4_moe_w4a16_gemm_combine(H, Wq, S, sorted_ids, expert_ids, num_post_pad, block, w, C,
+                              counters, out)
+    return C, out
+
+
 def moe_gemm_silu(A, a_row_div, Wq, S, sorted_ids, expert_ids, num_post_pad, block, num_slots,
                   H=None):
     if H is None:
@@ -475,6 +671,12 @@ def qat_gemm(X: torch.Tensor, W: torch.Tensor) -> torch.Tensor:
     Y = torch.empty((X.shape[0], W.shape[0]), dtype=torch.bfloat16, device=X.device)
     w4_qat_gemm(X, W, Y)
     return Y
+
+
+def qat_gemm_dx(dY: torch.Tensor, W: torch.Tensor) -> torch.Tensor:
+    dX = torch.empty((dY.shape[0], W.shape[1]), dtype=torch.bfloat16, device=dY.device)
+    w4_qat_gemm_dx(dY, W, dX)
+    return dX
 
 
 def moe_gate_topk(logits: torch.Tensor, topk: int):

@@ -254,6 +254,17 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
         : "memory");
 }
 
+// D (TMEM) (+)= A (shared memory, descriptor) * B (shared memory, descriptor).
+__device__ __forceinline__ void tc_mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // The barrier receives one arrival when all previously issued tcgen05.mma of
 // this thread have completed.
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
@@ -470,6 +481,85 @@ __device__ __forceinline__ uint4 permute_chunk8(uint4 v) {
 
 __device__ __forceinline__ uint32_t bf16x2_splat(uint16_t s) {
     return (uint32_t)s | ((uint32_t)s << 16);
+}
+
+// ---------------------------------------------------------------------------
+// Micro-scaled FP4 (MR-GPTQ / QuTLASS FP4 summary: MXFP4 = 32 E2M1 values per
+// power-of-two scale, NVFP4 = 16 per E4M3 scale under an FP32 tensor scale).
+// Codes are packed like the INT4 codes: eight per int32, element i at bits
+// [4i, 4i+3]; an E2M1 code is sign (bit 3), two exponent bits, one mantissa
+// bit: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+// ---------------------------------------------------------------------------
+// Two E2M1 codes (bits 0..3 and 4..7 of b) -> their values in FP32 (exact,
+// through the hardware E2M1 -> FP16 conversion).
+__device__ __forceinline__ void e2m1x2_to_f32(uint32_t b, float &lo, float &hi) {
+    uint32_t h;
+    asm("{.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+        : "=r"(h)
+        : "r"(b));
+    float a, c;
+    asm("{.reg .f16 l, u;\n\tmov.b32 {l, u}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, u;\n\t}"
+        : "=f"(a), "=f"(c)
+        : "r"(h));
+    lo = a;
+    hi = c;
+}
+
+// An E4M3 byte (sign, 4 exponent bits with bias 7, 3 mantissa bits) -> FP32
+// (exact, through the hardware E4M3 -> FP16 conversion).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
+    uint32_t h;
+    asm("{.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
+        : "=r"(h)
+        : "r"(b & 0xFFu));
+    float a;
+    asm("{.reg .f16 l, u;\n\tmov.b32 {l, u}, %1;\n\tcvt.f32.f16 %0, l;\n\t}" : "=f"(a) : "r"(h));
+    return a;
+}
+
+// 2^(E - 127) for a biased E8M0 exponent E in [0, 254] (E = 0: 2^-127, subnormal).
+__device__ __forceinline__ float e8m0_to_f32(uint32_t E) {
+    return __uint_as_float(E == 0u ? 0x00400000u : (E << 23));
+}
+
+__device__ __forceinline__ float fma_rn_f32(float a, float b, float c) {
+    float d;
+    asm("fma.rn.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t f32x2_to_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// MXFP4: one packed word (8 codes) with the group's scale s = 2^(E - 127) ->
+// four BF16x2 words of bf16_rne(value * s), natural order (out[j] = codes 2j,
+// 2j + 1).  value * s is exact (a 2-bit significand times a power of two);
+// the fused + 0 turns -0 into +0.
+__device__ __forceinline__ void dequant_word_mxfp4(uint32_t w, float s, uint32_t (&out)[4]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float a, b;
+        e2m1x2_to_f32(w >> (8 * j), a, b);
+        out[j] = f32x2_to_bf16x2(fma_rn_f32(a, s, 0.0f), fma_rn_f32(b, s, 0.0f));
+    }
+}
+
+// NVFP4: one packed word with the group's E4M3 scale s8 (as FP32) and the
+// tensor scale g -> bf16_rne(fl32(value * s8) * g): value * s8 is exact (2 and
+// 4 significant bits), the product with g rounds once in FP32 (the added +0
+// turns a product that underflows to -0 into +0), then BF16.
+__device__ __forceinline__ void dequant_word_nvfp4(uint32_t w, float s8, float g,
+                                                   uint32_t (&out)[4]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float a, b;
+        e2m1x2_to_f32(w >> (8 * j), a, b);
+        out[j] = f32x2_to_bf16x2(__fadd_rn(__fmul_rn(fma_rn_f32(a, s8, 0.0f), g), 0.0f),
+                                 __fadd_rn(__fmul_rn(fma_rn_f32(b, s8, 0.0f), g), 0.0f));
+    }
 }
 
 }  // namespace w4

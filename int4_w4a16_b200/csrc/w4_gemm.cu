@@ -9,7 +9,10 @@
 // Two more weight prologues share the tile: BF16 weights through the exact
 // group QDQ of the quantizers (QAT forward, Y = X . fake_quant(W)^T), and
 // unsigned codes with a zero point per group, dq = bf16_rne((q - z) * s)
-// (quantization tutorial §2.1 / §2.3).
+// (quantization tutorial §2.1 / §2.3), and micro-scaled FP4 codes (MR-GPTQ /
+// QuTLASS FP4 summary: MXFP4, E2M1 with a power-of-two scale per 32; NVFP4,
+// E2M1 with an E4M3 scale per 16 under an FP32 tensor scale), which keep the
+// activations in BF16.
 //
 // Design (B200-first; the pages' Marlin kernel targets H-series mma.sync and
 // is prior art only):
@@ -93,7 +96,9 @@ constexpr int kTmemCols = 512;
 
 struct GemmParams {
     const uint16_t *S;           // scales (direct loads when KB < 256)
-    const uint8_t *Z;            // zero points of asymmetric groups (ZP), one byte per group
+    const uint8_t *Z;            // zero points of asymmetric groups (ZP), one byte per group;
+                                 // FP4: the group scale bytes (E8M0 or E4M3)
+    float fp4_g;                 // NVFP4: the FP32 tensor scale
     uint16_t *Y;                 // dense: Y [M, N]; MoE: C [num_slots, N]
     const uint16_t *A;           // MoE: activation rows [a_rows, K]
     const int32_t *sorted_ids;   // MoE
@@ -106,6 +111,13 @@ struct GemmParams {
     int cap_blocks;              // MoE: length of expert_ids (bounds num_post_pad / block)
     int moe_sub;                 // MoE: MT-slot sub-blocks per aligned block (block / MT)
     int moe_mt;                  // MoE: MT (slots per work item)
+    // MoE down projection with the weighted top-k combine fused: out [T, N] =
+    // sum_k w[t, k] * C[t * topk + k, :], done by the last work item to finish
+    // a token's row tile (arrival counters per token, row tile, lane quarter)
+    const float *comb_w;         // [T, topk] FP32 routing weights
+    uint16_t *comb_out;          // [T, N] BF16; nullptr: no combine
+    unsigned int *comb_cnt;      // [T][n_row_tiles][4], zero between calls
+    int topk;
     int silu_inter;              // MoE gate_up with SiLU*up fused: the intermediate
                                  // size F (weights [E, 2F, K]; Y = H [num_slots, F]);
                                  // 0 = plain grouped GEMM
@@ -214,7 +226,8 @@ __device__ __forceinline__ int unit_owner(uint32_t x, const GemmParams &p) {
 }
 
 // Shared-memory layout, all offsets from a 1024-aligned base.
-template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT, bool BF16W = false>
+template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT, bool BF16W = false,
+          bool SMEM_A = false>
 struct Layout {
     // weight tile of up to 128 rows: packed INT4 words, or BF16 weights (QAT)
     static constexpr int kWBytes = BF16W ? 128 * KB * 2 : 128 * KB / 2;
@@ -222,7 +235,11 @@ struct Layout {
     static constexpr int kXSub = MT * 128;                  // one 64-wide K slice
     static constexpr int kXBytes = (KB / 64) * kXSub;
     static constexpr int kStage = kWBytes + kSBytes + kXBytes;
-    static constexpr int kBarOff = NSTAGE * kStage;
+    // A operand in shared memory (QAT input gradient): NASTAGE BF16 tiles of
+    // 128 rows x KB, K-major, 128-byte swizzle
+    static constexpr int kAOff = NSTAGE * kStage;
+    static constexpr int kASlot = 128 * KB * 2;
+    static constexpr int kBarOff = kAOff + (SMEM_A ? NASTAGE * kASlot : 0);
     static constexpr int kNumBars = 2 * NSTAGE + 2 * NASTAGE + 2 * NACC + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kBytes = kMiscOff + 16;
@@ -245,6 +262,10 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
     uint32_t v;
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
     return v;
+}
+
+__device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ uint2 lds64(uint32_t addr) {
@@ -297,17 +318,26 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 // barrier poll and a commit per k-block a single issuer cannot keep up with
 // the tensor core on N = 256 tiles.
 template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT, int NDQ, bool MOE,
-          bool WGL, bool QAT, bool ZP, bool SPLITN>
+          bool WGL, int QAT, bool ZP, bool SPLITN, int FP4>
 __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
     w4a16_tc_kernel(const __grid_constant__ CUtensorMap tm_w,
                     const __grid_constant__ CUtensorMap tm_s,
                     const __grid_constant__ CUtensorMap tm_x, const GemmParams p) {
     constexpr int kAccSets = SPLITN ? 1 : NSPLIT;   // accumulators per work item
-    using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE, kAccSets, QAT>;
-    static_assert(!QAT || (KB == 64 && !MOE), "QAT: 64-wide k-blocks of dense BF16 weights");
+    // QAT = 1: forward (fake quantization of W in the weight prologue, A in
+    // TMEM); QAT = 2: input gradient dX = dY . fake_quant(W), A = fake_quant(W)^T
+    // tile in shared memory
+    constexpr bool kQdx = (QAT == 2);
+    using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE, kAccSets, (QAT != 0), kQdx>;
+    static_assert(!QAT || (KB == 64 && !MOE && QAT <= 2),
+                  "QAT: 64-wide k-blocks of dense BF16 weights");
+    static_assert(!kQdx || NSTAGE == NASTAGE, "QAT input gradient: one release per k-block");
     static_assert(!SPLITN || (KB == 64 && !MOE && !WGL && MT % (16 * NSPLIT) == 0),
                   "token-split issuers: dense 64-wide k-blocks, N per issuer a multiple of 16");
     static_assert(!ZP || (KB == 64 && !MOE && !QAT), "zero points: dense 64-wide k-blocks");
+    // FP4 = 1: MXFP4 (a scale byte per 32 codes), 2: NVFP4 (a scale byte per 16)
+    static_assert(FP4 == 0 || (KB == 64 && !MOE && !QAT && !ZP && FP4 <= 2),
+                  "FP4 codes: dense 64-wide k-blocks");
     constexpr int kWords = KB / 8;             // packed words per row per k-block
     constexpr int kAStageCols = KB / 2;        // TMEM columns per A stage
     constexpr int kAccCols = kAccSets * MT;    // TMEM columns per work item accumulator
@@ -361,6 +391,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
     auto x_stage = [&](int s) {
         return sbase + (uint32_t)(s * L::kStage + L::kWBytes + L::kSBytes);
     };
+    auto a_smem = [&](int a) { return sbase + (uint32_t)(L::kAOff + a * L::kASlot); };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -466,6 +497,13 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                         tma_load_3d(w_stage(s), &tm_w, full_bar(s), kb * kWords, row0, expert);
                         if (KB == 256)
                             tma_load_3d(s_stage(s), &tm_s, full_bar(s), kb * 8, row0, expert);
+                    } else if (kQdx) {
+                        // W [N, K] as two 64 x 64 boxes: K (output rows) row0 ..
+                        // row0 + 127, N (the contraction) kb * 64 .. + 63
+                        tma_load_2d(w_stage(s), &tm_w, full_bar(s), row0, kb * KB);
+                        tma_load_2d(w_stage(s) + L::kWBytes / 2, &tm_w, full_bar(s), row0 + 64,
+                                    kb * KB);
+                        tma_load_2d(x_stage(s), &tm_x, full_bar(s), kb * KB, tt * MT);
                     } else {
                         tma_load_2d(w_stage(s), &tm_w, full_bar(s), QAT ? kb * KB : kb * kWords,
                                     row0);
@@ -522,17 +560,64 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
             const int64_t row = (int64_t)rt * R + lrow;
             const bool valid = lrow < R && row < p.N;
             const uint16_t *srow = nullptr;
-            if (KB != 256 && valid) {
+            if (KB != 256 && FP4 == 0 && valid) {
                 int64_t base = row * gpr;
                 if (MOE) base += (int64_t)__ldg(p.expert_ids + tt / p.moe_sub) * p.N * gpr;
                 srow = p.S + base;
             }
             const uint8_t *zrow = (ZP && srow != nullptr) ? p.Z + (srow - p.S) : nullptr;
+            // FP4: the row's scale bytes, one per 32 (MX) or 16 (NV) codes
+            constexpr int kFpg = FP4 == 2 ? 4 : 2;       // scale bytes per k-block
+            const int64_t fgpr = (FP4 == 2) ? p.K / 16 : gpr;
+            const uint8_t *frow = (FP4 != 0 && valid) ? p.Z + row * fgpr : nullptr;
             for (int kb = kb0; kb < kb1; ++kb, ++it) {
                 if (it % NDQ != grp) continue;
                 const int s = it % NSTAGE;
                 const int a = it % NASTAGE;
-                if constexpr (QAT) {
+                if constexpr (kQdx) {
+                    // QAT input gradient: warp q4 takes output rows (K) 32 q4 ..
+                    // 32 q4 + 31 of the tile, lane the contraction rows n, n + 1
+                    // (n = 2 lane) of the k-block: the two groups of 32 go through
+                    // the exact group QDQ, and the results are written transposed,
+                    // as the K-major A tile [128 K rows][64 N] (128-byte swizzle)
+                    if (!warp_wait(full_bar(s), (it / NSTAGE) & 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t src = w_stage(s) + (uint32_t)((q4 >> 1) * (L::kWBytes / 2));
+                    uint32_t v[2][16], o[2][16];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const uint4 x = lds128(
+                                src + swz((uint32_t)((2 * lane + h) * 128 + ((q4 & 1) * 4 + c) * 16),
+                                          128));
+                            v[h][4 * c] = x.x;
+                            v[h][4 * c + 1] = x.y;
+                            v[h][4 * c + 2] = x.z;
+                            v[h][4 * c + 3] = x.w;
+                        }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) qdq::fake_quant_group(v[h], o[h]);
+                    if (!warp_wait(aslot_free_bar(it), aslot_free_parity(it), abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t dst = a_smem(a);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const uint32_t k0 = (uint32_t)(32 * q4 + 2 * i);
+                        sts32(dst + swz(k0 * 128u + 4u * (uint32_t)lane, 128),
+                              __byte_perm(o[0][i], o[1][i], 0x5410));
+                        sts32(dst + swz((k0 + 1u) * 128u + 4u * (uint32_t)lane, 128),
+                              __byte_perm(o[0][i], o[1][i], 0x7632));
+                    }
+                    fence_proxy_async_smem();       // generic writes -> tensor-core reads
+                    mbar_arrive(afull_bar(a));
+                    continue;
+                }
+                if constexpr (QAT == 1) {
                     // QAT forward: the row's 64 BF16 weights (two groups of 32,
                     // 128-byte swizzled line) go through the exact group QDQ of the
                     // quantizers, straight into this k-block's A columns
@@ -568,8 +653,17 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                     continue;
                 }
                 static_assert(KB == 256 || G == 2, "direct-load scales: one chunk pair per k-block");
-                uint32_t sc[G], zb[G];
-                if (KB != 256) {
+                uint32_t sc[G] = {}, zb[G] = {};
+                float fs[kFpg];
+                if constexpr (FP4 != 0) {
+                    // the k-block's FP4 group scales as FP32 (exact conversions)
+#pragma unroll
+                    for (int j = 0; j < kFpg; ++j) {
+                        const int64_t gi = (int64_t)kb * kFpg + j;
+                        const uint32_t b = (frow != nullptr && gi < fgpr) ? __ldg(frow + gi) : 0u;
+                        fs[j] = FP4 == 1 ? e8m0_to_f32(b) : e4m3_to_f32(b);
+                    }
+                } else if (KB != 256) {
                     // scales (and zero points) of this k-block (direct loads when the
                     // tile has no TMA scales)
 #pragma unroll
@@ -615,6 +709,10 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                         for (int q = 0; q < 4; ++q) {
                             uint32_t t4[4];
                             if (kXPerm) dequant_word_k8perm(ws[q], scp[jj], t4);
+                            else if (FP4 == 1) dequant_word_mxfp4(ws[q], fs[jj], t4);
+                            else if (FP4 == 2)
+                                dequant_word_nvfp4(ws[q], fs[(2 * jj + (q >> 1)) % kFpg], p.fp4_g,
+                                                   t4);
                             else if (ZP) dequant_word_zp(ws[q], scp[jj], zb[jj], t4);
                             else dequant_word(ws[q], scp[jj], t4);
 #pragma unroll
@@ -759,8 +857,13 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                         for (int u = SPLITN ? 0 : ji; u < KB / 16; u += kU0Step) {
                             const uint32_t baddr =
                                 x_stage(s) + (u >> 2) * L::kXSub + (u & 3) * 32 + xrow;
-                            tc_mma_ts(d_tmem, a_tmem + u * 8, smem_desc_k_sw128(baddr), kIdesc,
-                                      (kb > kb0 || u >= kU0Step) ? 1u : 0u);
+                            const uint32_t acc_flag = (kb > kb0 || u >= kU0Step) ? 1u : 0u;
+                            if (kQdx)
+                                tc_mma_ss(d_tmem, smem_desc_k_sw128(a_smem(a) + (u & 3) * 32),
+                                          smem_desc_k_sw128(baddr), kIdesc, acc_flag);
+                            else
+                                tc_mma_ts(d_tmem, a_tmem + u * 8, smem_desc_k_sw128(baddr), kIdesc,
+                                          acc_flag);
                         }
                         tc_commit(empty_bar(s));
                         if (!kOneRelease) tc_commit(aempty_bar(a));
@@ -896,6 +999,52 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                     if (valid && out_row >= 0) {
                         const __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(v[jj]));
                         p.Y[out_row * p.N + row] = *reinterpret_cast<const uint16_t *>(&h);
+                    }
+                }
+                if (MOE && p.comb_out != nullptr) {
+                    // Fused combine.  Lane j < 16 counts column c0 + j's slot in
+                    // for its token (this warp's 32 rows of the row tile); the
+                    // lane that brings a token's count to topk has seen every
+                    // slot row of it written, and the warp then sums them in
+                    // ascending k -- the arithmetic of w4_moe_combine, so the
+                    // result does not depend on which work item came last.
+                    // One GPU-scope fence by lane 0 after __syncwarp releases all
+                    // lanes' C stores before the (relaxed) count updates; a
+                    // warp that sees a count complete fences again (acquire)
+                    // before reading the other slot rows.
+                    __syncwarp();
+                    if (lane == 0) __threadfence();
+                    __syncwarp();
+                    int slot = -1;
+                    if (lane < 16) {
+                        slot = __ldg(p.sorted_ids + (int64_t)tt * MT + c0 + lane);
+                        if (slot < 0 || slot >= p.num_slots) slot = -1;
+                    }
+                    bool last = false;
+                    if (slot >= 0) {
+                        unsigned int *cnt_t =
+                            p.comb_cnt + ((int64_t)(slot / p.topk) * p.n_row_tiles + rt) * 4 + q4;
+                        last = atomicAdd(cnt_t, 1u) == (unsigned int)(p.topk - 1);
+                    }
+                    unsigned int todo = __ballot_sync(0xFFFFFFFFu, last);
+                    if (todo != 0u) __threadfence();
+                    __syncwarp();
+                    while (todo != 0u) {
+                        const int j = __ffs(todo) - 1;
+                        todo &= todo - 1u;
+                        const int64_t t = __shfl_sync(0xFFFFFFFFu, slot, j) / p.topk;
+                        if (valid) {
+                            float acc = 0.0f;
+                            for (int k = 0; k < p.topk; ++k) {
+                                const float wk = __ldg(p.comb_w + t * p.topk + k);
+                                const uint16_t d = __ldcg(p.Y + (t * p.topk + k) * p.N + row);
+                                acc = __fadd_rn(acc, __fmul_rn(wk, __uint_as_float((uint32_t)d << 16)));
+                            }
+                            const __nv_bfloat16 h = __float2bfloat16_rn(acc);
+                            p.comb_out[t * p.N + row] = *reinterpret_cast<const uint16_t *>(&h);
+                        }
+                        if (lane == j)
+                            p.comb_cnt[(t * p.n_row_tiles + rt) * 4 + q4] = 0u;   // next call
                     }
                 }
             }
@@ -1038,12 +1187,12 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
 // ---------------------------------------------------------------------------
 
 template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT, int NDQ, bool MOE,
-          bool WGL = false, bool QAT = false, bool ZP = false, bool SPLITN = false>
+          bool WGL = false, int QAT = 0, bool ZP = false, bool SPLITN = false, int FP4 = 0>
 w4_status launch_cfg(const CUtensorMap &tw, const CUtensorMap &ts, const CUtensorMap &tx,
                      const GemmParams &p, int num_items_max, cudaStream_t stream) {
-    using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE, (SPLITN ? 1 : NSPLIT), QAT>;
+    using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE, (SPLITN ? 1 : NSPLIT), (QAT != 0), (QAT == 2)>;
     auto kern =
-        w4a16_tc_kernel<KB, MT, NSTAGE, NACC, NASTAGE, NSPLIT, NDQ, MOE, WGL, QAT, ZP, SPLITN>;
+        w4a16_tc_kernel<KB, MT, NSTAGE, NACC, NASTAGE, NSPLIT, NDQ, MOE, WGL, QAT, ZP, SPLITN, FP4>;
     // At least half of the SM's shared memory, so one CTA (and one TMEM
     // allocation of 512 columns) per SM.
     const int smem = std::max(L::kAlloc, 120 * 1024);
@@ -1098,10 +1247,18 @@ struct SplitPlan {
     size_t cnt_bytes, part_bytes;
 };
 
+// The arrival counters sit in a fixed region at the start of the workspace,
+// large enough for every row-tile count the split accepts, and the partial
+// sums after it: a call's partials (left in place) can then never lie where a
+// later call on the same workspace, with more row tiles, expects zeroed
+// counters.
+constexpr size_t kSplitCntBytes = 4096;
+constexpr int64_t kSplitMaxRowTiles = kSplitCntBytes / (4 * sizeof(unsigned int));
+
 bool plan_split(int64_t M, int64_t N, int64_t K, int sms, SplitPlan *sp) {
     if (M > 64 || (K % 256) != 0) return false;
     const int64_t n_rt = (N + 127) / 128, nkb = K / 256;
-    if (n_rt >= sms || nkb < 2 || n_rt > (1 << 20)) return false;
+    if (n_rt >= sms || nkb < 2 || n_rt > kSplitMaxRowTiles) return false;
     const int64_t units = n_rt * nkb;
     const int ctas = (int)std::min<int64_t>(sms, units);
     if (units * (ctas + 1) >= ((int64_t)1 << 32)) return false;   // device math is 32-bit
@@ -1114,7 +1271,7 @@ bool plan_split(int64_t M, int64_t N, int64_t K, int sms, SplitPlan *sp) {
     sp->ctas = ctas;
     sp->max_contrib = mc;
     sp->mt = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
-    sp->cnt_bytes = ((size_t)n_rt * 4 * sizeof(unsigned int) + 255) / 256 * 256;
+    sp->cnt_bytes = kSplitCntBytes;
     sp->part_bytes = (size_t)n_rt * mc * 128 * sp->mt * sizeof(float);
     return true;
 }
@@ -1320,6 +1477,56 @@ extern "C" w4_status w4_qat_gemm(const w4_bf16 *X, const w4_bf16 *W, w4_bf16 *Y,
     return launch_cfg<64, 256, 4, 1, 4, 1, 2, false, false, true>(tw, ts, tx, p, (int)items, st);
 }
 
+extern "C" w4_status w4_qat_gemm_dx(const w4_bf16 *dY, const w4_bf16 *W, w4_bf16 *dX, int64_t M,
+                                    int64_t N, int64_t K, int group, void *stream) {
+    if (group != 32) return W4_ERR_UNSUPPORTED;
+    if (M < 0 || N < 0 || K <= 0 || (K % 32) != 0) return W4_ERR_INVALID_ARG;
+    if (!w4host::aligned16(dY) || !w4host::aligned16(W) || !w4host::aligned16(dX))
+        return W4_ERR_INVALID_ARG;
+    if ((K % 64) != 0 || (N % 8) != 0) return W4_ERR_UNSUPPORTED;
+    if (M == 0) return W4_OK;
+    if (N > (1 << 24) || M > (1 << 30) || K > (1 << 30)) return W4_ERR_UNSUPPORTED;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (N == 0) return cudaMemsetAsync(dX, 0, (size_t)M * K * 2, st) == cudaSuccess
+                           ? W4_OK : w4host::launch_status();
+    // output rows of the kernel = K, contraction = N (64-wide k-blocks), tokens = M
+    GemmParams p = {};
+    p.Y = reinterpret_cast<uint16_t *>(dX);
+    p.M = M;
+    p.N = K;
+    p.K = N;
+    const int mt = M <= 64 ? 64 : 256;
+    p.rows_per_tile = 128;
+    p.n_row_tiles = ceil_div_i(K, 128);
+    p.n_tok_tiles = ceil_div_i(M, mt);
+    p.num_kb = ceil_div_i(N, 64);
+    CUtensorMap tw, ts, tx;
+    memset(&ts, 0, sizeof ts);
+    {
+        // dY [M, N]: 64-wide N boxes of mt tokens
+        cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+        cuuint64_t strides[1] = {(cuuint64_t)N * 2};
+        cuuint32_t box[2] = {64u, (cuuint32_t)mt};
+        if (!make_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dY, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+            return W4_ERR_CUDA;
+    }
+    {
+        // W [N, K]: 64 x 64 boxes (128-byte lines along K)
+        cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)N};
+        cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+        cuuint32_t box[2] = {64u, 64u};
+        if (!make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+            return W4_ERR_CUDA;
+    }
+    const int64_t items = (int64_t)p.n_row_tiles * p.n_tok_tiles;
+    if (items > (1 << 30)) return W4_ERR_UNSUPPORTED;
+    if (mt == 64)
+        return launch_cfg<64, 64, 4, 1, 4, 4, 2, false, false, 2>(tw, ts, tx, p, (int)items, st);
+    return launch_cfg<64, 256, 3, 1, 3, 1, 2, false, false, 2>(tw, ts, tx, p, (int)items, st);
+}
+
 extern "C" w4_status w4a16_gemm_zp(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S,
                                    const uint8_t *Z, w4_bf16 *Y, int64_t M, int64_t N, int64_t K,
                                    int group, void *stream) {
@@ -1378,6 +1585,75 @@ extern "C" w4_status w4a16_gemm_zp(const w4_bf16 *X, const int32_t *Wq, const w4
                                                                               (int)items, st);
 }
 
+namespace w4 {
+namespace {
+
+// W4A16 GEMM on FP4 codes (FP4 = 1: MXFP4, 2: NVFP4): the zero-point kernel's
+// tiles (128 weight rows x 64-wide k-blocks, scale bytes read directly by the
+// dequant warps) with the FP4 unpack in the weight prologue.
+template <int FP4>
+w4_status gemm_fp4(const w4_bf16 *X, const int32_t *Wq, const uint8_t *SB, float g, w4_bf16 *Y,
+                   int64_t M, int64_t N, int64_t K, void *stream) {
+    if (M < 0 || N < 0 || K <= 0 || (K % 32) != 0) return W4_ERR_INVALID_ARG;
+    if (!w4host::aligned16(X) || !w4host::aligned16(Wq) || !w4host::aligned16(Y) ||
+        SB == nullptr)
+        return W4_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return W4_OK;
+    if (N > (1 << 30) || M > (1 << 30) || K > (1 << 24)) return W4_ERR_UNSUPPORTED;
+    cudaStream_t st = (cudaStream_t)stream;
+    GemmParams p = {};
+    p.Z = SB;
+    p.fp4_g = g;
+    p.Y = reinterpret_cast<uint16_t *>(Y);
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    const int mt = M <= 64 ? 64 : 256;
+    p.rows_per_tile = 128;
+    p.n_row_tiles = ceil_div_i(N, 128);
+    p.n_tok_tiles = ceil_div_i(M, mt);
+    p.num_kb = ceil_div_i(K, 64);
+    CUtensorMap tw, ts, tx;
+    memset(&ts, 0, sizeof ts);
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+        cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+        cuuint32_t box[2] = {64u, (cuuint32_t)mt};
+        if (!make_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+            return W4_ERR_CUDA;
+    }
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)(K / 8), (cuuint64_t)N};
+        cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+        cuuint32_t box[2] = {8u, 128u};
+        if (!make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_INT32, 2, Wq, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_32B))
+            return W4_ERR_CUDA;
+    }
+    const int64_t items = (int64_t)p.n_row_tiles * p.n_tok_tiles;
+    if (items > (1 << 30)) return W4_ERR_UNSUPPORTED;
+    if (mt == 64)
+        return launch_cfg<64, 64, 8, 1, 8, 4, 2, false, false, false, false, false, FP4>(
+            tw, ts, tx, p, (int)items, st);
+    return launch_cfg<64, 256, 6, 1, 6, 2, 2, false, false, false, false, true, FP4>(
+        tw, ts, tx, p, (int)items, st);
+}
+
+}  // namespace
+}  // namespace w4
+
+extern "C" w4_status w4a16_gemm_mxfp4(const w4_bf16 *X, const int32_t *Wq, const uint8_t *E,
+                                      w4_bf16 *Y, int64_t M, int64_t N, int64_t K, void *stream) {
+    return gemm_fp4<1>(X, Wq, E, 1.0f, Y, M, N, K, stream);
+}
+
+extern "C" w4_status w4a16_gemm_nvfp4(const w4_bf16 *X, const int32_t *Wq, const uint8_t *S,
+                                      float g, w4_bf16 *Y, int64_t M, int64_t N, int64_t K,
+                                      void *stream) {
+    return gemm_fp4<2>(X, Wq, S, g, Y, M, N, K, stream);
+}
+
 extern "C" int64_t w4_moe_capacity(int64_t T, int topk, int E, int block) {
     if (T < 0 || topk <= 0 || E <= 0 || block <= 0) return 0;
     const int64_t cap = T * topk + (int64_t)E * (block - 1);
@@ -1393,7 +1669,9 @@ namespace {
 w4_status moe_launch(const w4_bf16 *A, int a_row_div, const int32_t *Wq, const w4_bf16 *S,
                      const int32_t *sorted_ids, const int32_t *expert_ids,
                      const int32_t *num_post_pad, int64_t cap, int block, int64_t num_slots,
-                     w4_bf16 *Y, int64_t N, int64_t K, int E, int64_t silu_inter, void *stream) {
+                     w4_bf16 *Y, int64_t N, int64_t K, int E, int64_t silu_inter, void *stream,
+                     int topk = 0, const float *comb_w = nullptr, w4_bf16 *comb_out = nullptr,
+                     unsigned int *comb_cnt = nullptr) {
     if (!w4host::aligned16(A) || !w4host::aligned16(Wq) || !w4host::aligned16(S) ||
         !w4host::aligned16(sorted_ids) || !w4host::aligned16(expert_ids) ||
         !w4host::aligned16(num_post_pad) || !w4host::aligned16(Y))
@@ -1423,6 +1701,10 @@ w4_status moe_launch(const w4_bf16 *A, int a_row_div, const int32_t *Wq, const w
     p.cap_blocks = (int)(cap / block);
     p.rows_per_tile = 128;
     p.silu_inter = (int)silu_inter;
+    p.topk = topk;
+    p.comb_w = comb_w;
+    p.comb_out = reinterpret_cast<uint16_t *>(comb_out);
+    p.comb_cnt = comb_cnt;
     // a SiLU*up tile covers 64 output columns (64 gate + 64 up rows)
     p.n_row_tiles = silu_inter > 0 ? ceil_div_i(silu_inter, 64) : ceil_div_i(N, 128);
     p.n_tok_tiles = 0;
@@ -1477,6 +1759,26 @@ extern "C" w4_status w4_moe_w4a16_gemm(const w4_bf16 *A, int a_row_div, const in
                                        int64_t N, int64_t K, int E, void *stream) {
     return w4::moe_launch(A, a_row_div, Wq, S, sorted_ids, expert_ids, num_post_pad, cap, block,
                           num_slots, C, N, K, E, 0, stream);
+}
+
+extern "C" size_t w4_moe_combine_counter_bytes(int64_t T, int64_t N) {
+    if (T <= 0 || N <= 0) return 0;
+    return (size_t)T * (size_t)((N + 127) / 128) * 4 * sizeof(unsigned int);
+}
+
+extern "C" w4_status w4_moe_w4a16_gemm_combine(const w4_bf16 *A, const int32_t *Wq,
+                                               const w4_bf16 *S, const int32_t *sorted_ids,
+                                               const int32_t *expert_ids,
+                                               const int32_t *num_post_pad, int64_t cap,
+                                               int block, int topk, const float *w, w4_bf16 *C,
+                                               unsigned int *counters, w4_bf16 *out, int64_t T,
+                                               int64_t N, int64_t K, int E, void *stream) {
+    if (topk < 1 || topk > 64 || T < 0 || w == nullptr || counters == nullptr ||
+        (reinterpret_cast<uintptr_t>(counters) & 15u) != 0 || !w4host::aligned16(out))
+        return W4_ERR_INVALID_ARG;
+    if (T > ((int64_t)1 << 30) / topk) return W4_ERR_UNSUPPORTED;
+    return w4::moe_launch(A, 1, Wq, S, sorted_ids, expert_ids, num_post_pad, cap, block,
+                          T * topk, C, N, K, E, 0, stream, topk, w, out, counters);
 }
 
 extern "C" w4_status w4_moe_w4a16_gemm_silu(const w4_bf16 *A, int a_row_div, const int32_t *Wq,

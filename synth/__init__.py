@@ -67,11 +67,15 @@ def router_logits(T: int, E: int, seed: int, index: int = 0, device="cpu"):
     return torch.randn((T, E), generator=g, dtype=torch.float32).to(device)
 
 
-def routing(T: int, E: int, topk: int, seed: int, index: int = 0):
+def routing(T: int, E: int, topk: int, seed: int, index: int = 0, skew: float = 0.0):
     """Router logits ~ N(0,1) [T, E] -> softmax -> top-k (ties to lower id).
-    Returns (topk_ids int32 [T, topk], topk_weights float32 [T, topk]) on CPU."""
+    skew > 0 adds -skew * log(1 + e) to expert e's logit (a Zipf-like load: the
+    low ids are hot).  Returns (topk_ids int32 [T, topk], topk_weights float32
+    [T, topk]) on CPU."""
     g = _gen(seed, index, "cpu")
     logits = torch.randn((T, E), generator=g, dtype=torch.float32)
+    if skew:
+        logits = logits - skew * torch.log1p(torch.arange(E, dtype=torch.float32))
     p = torch.softmax(logits, dim=-1)
     order = torch.argsort(-p, dim=-1, stable=True)[:, :topk]
     w = torch.gather(p, 1, order)
@@ -156,8 +160,8 @@ class MoEDecode:
     def tokens(self, T: int, device="cpu"):
         return normal_bf16((T, self.hidden), 1.0, self.seed, 100 + T, device)
 
-    def routing(self, T: int):
-        return routing(T, self.E, self.topk, self.seed, 200 + T)
+    def routing(self, T: int, skew: float = 0.0):
+        return routing(T, self.E, self.topk, self.seed, 200 + T, skew)
 
     def logits(self, T: int, device="cpu"):
         return router_logits(T, self.E, self.seed, 200 + T, device)

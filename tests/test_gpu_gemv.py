@@ -1,13 +1,14 @@
 """Parity of the decode-shaped W4A16 GEMM with the CPU oracle, through the C
 ABI.  1..8 activation rows with K a multiple of 256 take the warp-level MMA
-kernel (w4_gemv.cu); the other shapes here run the tensor-memory kernel at the
-same sizes.
+kernel (w4_gemv.cu); the other shapes here run the tensor-memory kernel at
+the same sizes (its stream-K split included, on one shared workspace).
 
 Shapes cover every launch configuration of the warp-level kernel: one and
 several passes of the warps over K (4096 each), with a partly idle last pass;
-row ranges of one to six 16-row tiles per CTA, including ones whose stages
-outnumber the ring's slots (refills) and more CTAs than SMs; ragged N (not a
-multiple of 16 or of 4, fewer rows than one tile, fewer rows than CTAs)."""
+row ranges of one to six 16-row tiles per CTA,
+including ones whose stages outnumber the ring's slots (refills); more CTAs
+than SMs; ragged N (not a multiple of 16 or of 4, fewer rows than one tile,
+fewer rows than CTAs) and ragged M."""
 import numpy as np
 import pytest
 import torch
@@ -30,6 +31,12 @@ pytestmark = pytest.mark.gpu
     (2, 9472, 8192),      # 4 tiles x 2 passes per CTA: slots refilled from the ring
     (3, 20000, 512),      # more CTAs than SMs (24 row quads each at most)
     (1, 14212, 256),      # just past one wave of 96-row CTAs
+    (16, 9472, 8192),     # two column tiles: 4 tiles x 2 passes, ring refills
+    (24, 9472, 8192),
+    (13, 20000, 512),     # more CTAs than SMs
+    (29, 20000, 2304),
+    (32, 14212, 256),
+    (9, 12288, 4096), (17, 12288, 4096), (32, 12288, 4096),   # the decode layer
 ])
 def test_gemv_shapes(M, N, K):
     X, Wq, S, Y = _gemm_case(M, N, K, seed=M * 31 + N + K)
@@ -44,7 +51,8 @@ def test_gemv_laplace_weights():
 
 
 @pytest.mark.parametrize("N,K,MB", [(256, 256, 8), (200, 1536, 8), (120, 4096, 8),
-                                    (40, 4352, 5), (100, 2048, 16)])
+                                    (40, 4352, 5), (100, 2048, 16), (130, 4352, 32),
+                                    (70, 2560, 27)])
 def test_gemv_one_hot_exact(N, K, MB):
     """X = rows of the identity: Y[m, n] = dq(W)[n, k0 + m] exactly (one
     nonzero product per output: checks the fragment K order against the
@@ -65,8 +73,9 @@ def test_gemv_one_hot_exact(N, K, MB):
     w4.w4_device_status()
 
 
-def test_gemv_deterministic_and_no_workspace():
-    M, N, K = 8, 4096 + 12, 4096
+@pytest.mark.parametrize("M", [5, 8])
+def test_gemv_deterministic_and_no_workspace(M):
+    N, K = 4096 + 12, 4096
     assert w4.w4a16_gemm_workspace_bytes(M, N, K) == 0
     X, Wq, S, Y1 = _gemm_case(M, N, K, seed=11)
     Xd, Wqd, Sd = _np_bf16(X).to(DEV), torch.from_numpy(Wq).to(DEV), _np_bf16(S).to(DEV)
@@ -75,10 +84,11 @@ def test_gemv_deterministic_and_no_workspace():
     w4.w4_device_status()
 
 
-def test_gemv_leaves_other_rows_of_y_alone():
+@pytest.mark.parametrize("M", [5, 11, 19])
+def test_gemv_leaves_other_rows_of_y_alone(M):
     """Y is written only at [0, M) x [0, N): the rest of a larger flat buffer
     keeps its sentinel."""
-    M, N, K = 5, 333, 1024
+    N, K = 333, 1024
     X, Wq, S, Y = _gemm_case(M, N, K, seed=21)
     flat = torch.full(((M + 3) * N,), -7.0, dtype=torch.bfloat16, device=DEV)
     w4.w4a16_gemm(_np_bf16(X).to(DEV), torch.from_numpy(Wq).to(DEV), _np_bf16(S).to(DEV),

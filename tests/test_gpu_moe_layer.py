@@ -101,6 +101,31 @@ def test_moe_layer_stage_by_stage(T):
     assert np.array_equal(bits(out), oracle.moe_combine(bits(C2), w.cpu().numpy(), topk))
 
 
+@pytest.mark.parametrize("T,E,N,K,block", [(16, 128, 4096, 1536, 16), (64, 128, 4096, 1536, 16),
+                                            (256, 128, 4096, 1536, 32), (7, 8, 200, 256, 64),
+                                            (33, 5, 136, 512, 16)])
+def test_moe_down_combine_fused(T, E, N, K, block):
+    """Down projection with the combine in its epilogue: C bit for bit the
+    plain grouped GEMM's, out bit for bit w4_moe_combine / the oracle's combine
+    of that C, twice on the same counters (left zero after each call)."""
+    topk = 8 if E >= 8 else 3
+    logits = _logits(T, E, seed=70 + T + N)
+    ids, w = w4.moe_gate_topk(torch.from_numpy(logits).to(DEV), topk)
+    H = synth.normal_bf16((T * topk, K), 1.0, seed=80 + T).to(DEV)
+    Wq, S, _ = _experts(E, N, K)
+    Wq_d, S_d = torch.from_numpy(Wq).to(DEV), _np_bf16(S).to(DEV)
+    s_d, e_d, n_d = w4.moe_align(ids, E, block)
+    cnt = torch.zeros(w4.w4_moe_combine_counter_bytes(T, N), dtype=torch.uint8, device=DEV)
+    C_ref = bits(w4.moe_gemm(H, 1, Wq_d, S_d, s_d, e_d, n_d, block, T * topk))
+    want = oracle.moe_combine(C_ref, w.cpu().numpy(), topk)
+    for call in range(2):
+        C, out = w4.moe_gemm_combine(H, Wq_d, S_d, s_d, e_d, n_d, block, w, cnt)
+        w4.w4_device_status()
+        assert np.array_equal(bits(C), C_ref), f"call {call}: C differs from the plain GEMM"
+        assert np.array_equal(bits(out), want), f"call {call}: combine not bit-exact"
+        assert int(cnt.count_nonzero()) == 0, f"call {call}: counters not reset"
+
+
 def _silu_ref(R, F):
     """h = silu(g) * u from the oracle's FP32 gate_up sums (float64 evaluation)."""
     g, u = R[:, :F].astype(np.float64), R[:, F:].astype(np.float64)

@@ -289,8 +289,8 @@ def _decode_weight():
                                      (32, True), (32, False), (64, True), (64, False)])
 def test_gemm_decode_config(M, split):
     """Decode GEMV sweep: 1..8 rows take the warp-level MMA kernel (no
-    workspace); 16..64 rows the tensor-memory kernel, with the stream-K split
-    (workspace) and without."""
+    workspace; `split` makes no difference there); 16..64 rows the
+    tensor-memory kernel, with the stream-K split (workspace) and without."""
     cfg = synth.Decode()
     Wq, S = _decode_weight()
     X = cfg.activations(M)
@@ -318,6 +318,23 @@ def test_gemm_split_workspace_left_zero_and_deterministic():
     # the unsplit schedule gives the same product within tolerance
     Y0 = bits(w4.gemm(Xd, Wqd, Sd, ws=None))
     assert_gemm_close(Y0, R, "unsplit ragged")
+
+
+def test_gemm_split_workspace_shared_across_shapes():
+    """One zeroed workspace serves a sequence of split GEMMs with different
+    row-tile counts: a call's parked partial sums never sit where a later call
+    with more row tiles keeps its arrival counters."""
+    M, K = 32, 2048
+    ws = torch.zeros(w4.w4a16_gemm_workspace_bytes(M, 12288, K) + (1 << 20), dtype=torch.uint8,
+                     device=DEV)
+    for N in (4096, 9472, 12288, 640, 12288):
+        X, Wq, S, _ = _gemm_case(M, N, K, seed=N)
+        assert w4.w4a16_gemm_workspace_bytes(M, N, K) > 0
+        Y = bits(w4.gemm(_np_bf16(X).to(DEV), torch.from_numpy(Wq).to(DEV), _np_bf16(S).to(DEV),
+                         ws=ws))
+        w4.w4_device_status()
+        _, R = oracle.w4a16_gemm(X, Wq, S)
+        assert_gemm_close(Y, R, f"shared workspace N={N}")
 
 
 @pytest.mark.parametrize("M", [512, 2048, 8192])

@@ -1,6 +1,7 @@
-"""Parity of the QAT forward GEMM (fake quantization fused into the weight
-prologue, w4_qat_gemm) with the CPU oracle: Y = X . fake_quant(W)^T, where the
-oracle materializes fake_quant(W) and multiplies; the GPU never writes it."""
+"""Parity of the QAT GEMMs with fake quantization fused into the weight
+prologue with the CPU oracle: the forward w4_qat_gemm, Y = X . fake_quant(W)^T,
+and the input gradient w4_qat_gemm_dx, dX = dY . fake_quant(W).  The oracle
+materializes fake_quant(W) and multiplies; the GPU never writes it."""
 import numpy as np
 import pytest
 import torch
@@ -103,3 +104,76 @@ def test_qat_gemm_matches_fake_quant_then_gemm():
     Wdq_gpu = bits(w4.fake_quant(Wd))
     _, R = oracle.gemm(bits(X), Wdq_gpu)
     assert_gemm_close(Y1, R, "fused vs materialized")
+
+
+# ---------------------------------------------------------------------------
+# Input gradient with the fused QDQ: dX = dY . fake_quant(W)
+# ---------------------------------------------------------------------------
+
+def _dx_case(M, N, K, seed, outliers=0.001):
+    W = synth.normal_bf16((N, K), 0.02, seed=seed, outlier_frac=outliers)
+    dY = synth.normal_bf16((M, N), 1.0, seed=seed + 1)
+    dX = bits(w4.qat_gemm_dx(dY.to(DEV), W.to(DEV)))
+    w4.w4_device_status()
+    Wdq, _ = oracle.fake_quant(bits(W))
+    _, R = oracle.gemm(bits(dY), np.ascontiguousarray(Wdq.T))
+    return dX, R
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 8, 64), (5, 104, 128), (64, 320, 640), (65, 264, 256),
+                                   (300, 1000, 1024), (512, 1024, 2048), (3, 136, 4096),
+                                   (17, 4096, 192)])
+def test_qat_gemm_dx_shapes(M, N, K):
+    """Ragged token tiles, a partial last 64-wide block of N and a partial
+    last 128-row tile of K."""
+    dX, R = _dx_case(M, N, K, seed=M + N + K)
+    assert_gemm_close(dX, R, f"qat dx M={M} N={N} K={K}")
+
+
+def test_qat_gemm_dx_one_hot_exact_with_edge_groups():
+    """dY = identity rows: dX[m, :] = fake_quant(W)[n0 + m, :] bit for bit, on
+    weights with zero, subnormal-scale, huge and tie groups."""
+    N, K = 192, 256
+    W = synth.normal_bf16((N, K), 0.02, seed=9, outlier_frac=0.01).clone()
+    W[3, 0:32] = 0.0
+    W[4, 32:64] = 1e-39
+    W[5, 64:96] = torch.linspace(-3e30, 3e30, 32).to(torch.bfloat16)
+    W[6, 96:128] = torch.tensor([0.5 * (i % 3 - 1) for i in range(32)]).to(torch.bfloat16)
+    Wd = W.to(DEV)
+    Wdq, _ = oracle.fake_quant(bits(W))
+    for n0 in range(0, N, 64):
+        dY = torch.zeros((64, N), dtype=torch.bfloat16)
+        dY[torch.arange(64), n0 + torch.arange(64)] = 1.0
+        dX = bits(w4.qat_gemm_dx(dY.to(DEV), Wd))
+        want = Wdq[n0:n0 + 64, :]
+        if not np.array_equal(dX, want):
+            bad = np.argwhere(dX != want)
+            raise AssertionError(f"one-hot mismatch at n0={n0}: {bad[:8].tolist()}")
+    w4.w4_device_status()
+
+
+def test_qat_gemm_dx_layer_shape_sampled():
+    """A QAT-stack layer (W[12288, 4096]) at 2048 tokens: dX [2048, 4096]; the
+    oracle checks 12 rows (every weight enters every checked element)."""
+    N, K, M = 12288, 4096, 2048
+    W = synth.normal_bf16((N, K), 0.02, seed=0, index=1, device=DEV, outlier_frac=0.001)
+    dY = synth.normal_bf16((M, N), 1.0, seed=0, index=3, device=DEV)
+    dX = w4.qat_gemm_dx(dY, W)
+    w4.w4_device_status()
+    rows = torch.linspace(0, M - 1, 12).long()
+    Wdq, _ = oracle.fake_quant(bits(W.cpu()))
+    _, R = oracle.gemm(bits(dY[rows.to(DEV)].cpu()), np.ascontiguousarray(Wdq.T))
+    assert_gemm_close(bits(dX[rows.to(DEV)]), R, "qat dx layer sampled")
+
+
+def test_qat_gemm_dx_matches_fake_quant_then_gemm_and_is_deterministic():
+    M, N, K = 128, 512, 1024
+    W = synth.normal_bf16((N, K), 0.02, seed=4)
+    dY = synth.normal_bf16((M, N), 1.0, seed=6)
+    dYd, Wd = dY.to(DEV), W.to(DEV)
+    a = bits(w4.qat_gemm_dx(dYd, Wd))
+    b = bits(w4.qat_gemm_dx(dYd, Wd))
+    assert np.array_equal(a, b)
+    Wdq_gpu = bits(w4.fake_quant(Wd))
+    _, R = oracle.gemm(bits(dY), np.ascontiguousarray(Wdq_gpu.T))
+    assert_gemm_close(a, R, "fused dx vs materialized")

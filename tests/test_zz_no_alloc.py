@@ -29,25 +29,28 @@ def _close_to_oracle(y_bits, R, what):
     assert not np.any(err > REL_TOL * np.abs(r) + 1e-3 * scale), what
 
 
-@pytest.mark.parametrize("M", [1, 16, 32])
-def test_noalloc_matches_workspace_entry_point_twice(M):
+@pytest.mark.parametrize("M,N", [(1, 12288), (16, 12288), (32, 12288), (48, 4096)])
+def test_noalloc_matches_workspace_entry_point_twice(M, N):
     """Two calls in a row give the very bits of w4a16_gemm with a caller
     workspace: both run the same schedule and add the split's partial sums in
     the same fixed order, so a wrongly zeroed counter in the shared array would
-    show as a difference.  M = 16 and 32 run the split (scratch in use); M = 1
-    the warp-level kernel, which needs none.  M = 16 is also checked against
-    the oracle's FP32-accumulated product."""
+    show as a difference.  M = 16, 32 and 48 run the split (scratch in use;
+    ~6 MB of the 8 MiB array for M = 48 on 4096 weight rows); M = 1 the
+    warp-level kernel, which needs none.  M > 1 is also checked against the
+    oracle's FP32-accumulated product."""
     L = w4.lib()
     cfg = synth.Decode()
     Wq_h, S_h = _decode_weight()
+    Wq_h, S_h = np.ascontiguousarray(Wq_h[:N]), np.ascontiguousarray(S_h[:N])
     dev = "cuda"
     Wq = torch.from_numpy(Wq_h).to(dev)
     S = torch.from_numpy(S_h.view(np.int16)).view(torch.bfloat16).to(dev)
     X = cfg.activations(M, dev)
-    N, K = cfg.N, cfg.K
+    K = cfg.K
     stream = torch.cuda.current_stream().cuda_stream
     need = L.w4a16_gemm_workspace_bytes(M, N, K)
     assert (need > 0) == (M > 8), "the split schedule (scratch) is what M > 8 exercises"
+    assert need <= (8 << 20)
     ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
     Y_ref = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     rc = L.w4a16_gemm(X.data_ptr(), Wq.data_ptr(), S.data_ptr(), Y_ref.data_ptr(), M, N, K, 32,
@@ -61,7 +64,7 @@ def test_noalloc_matches_workspace_entry_point_twice(M):
         torch.cuda.synchronize()
         assert np.array_equal(bits(Y), bits(Y_ref)), f"M={M} call {call}: not the same bits"
     assert L.w4_device_status(stream) == 0
-    if M == 16:
+    if M > 1:
         _, R = oracle.w4a16_gemm(bits(X), Wq_h, S_h)
         _close_to_oracle(bits(Y), R, f"M={M} against the oracle")
 
