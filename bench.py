@@ -51,11 +51,9 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # (profiles/ holds the summaries and commands); an entry is used only while the
 # kernel's source file is unchanged since the capture.
 NCU_TRAFFIC = {
-    ("gemm_m16", "decode"): {"bytes": 28514816 + 0, "file": "w4_gemm.cu", "src": "55760fa033783eae"},
-    ("gemm_m1", "decode"): {"bytes": 28345856 + 0, "file": "w4_gemv.cu", "src": "5ef23c66e376b90e"},
-    ("fake_quant", "decode"): {"bytes": 100690176 + 48219648, "file": "w4_quant.cu", "src": "b06ce5204a7ad78a"},
-    ("ste_backward", "decode"): {"bytes": 100671488 + 44970496, "file": "w4_quant.cu", "src": "b06ce5204a7ad78a"},
-    ("quantize_pack", "decode"): {"bytes": 100693248 + 6085376, "file": "w4_quant.cu", "src": "b06ce5204a7ad78a"},
+    ("gemm_m16", "decode"): {"bytes": 28514560 + 0, "file": "w4_gemm.cu", "src": "94e60b49eb034652"},
+    ("gemm_m1", "decode"): {"bytes": 28347904 + 0, "file": "w4_gemv.cu", "src": "4e2e44264b5b9b9b"},
+    ("ste_backward", "decode"): {"bytes": 100672512 + 46598656, "file": "w4_quant.cu", "src": "63bc5e9cb458e7cb"},
 }
 
 
