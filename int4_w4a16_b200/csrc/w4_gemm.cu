@@ -1410,8 +1410,8 @@ extern "C" w4_status w4a16_gemm(const w4_bf16 *X, const int32_t *Wq, const w4_bf
             items = p.n_row_tiles;
             if (!map_x(mt) || !map_w(256, R) || !map_s(R)) return W4_ERR_CUDA;
         }
-        if (mt == 16) return launch_cfg<256, 16, 6, 1, 3, 8, 2, false, true>(tw, ts, tx, p, items, st);
-        if (mt == 32) return launch_cfg<256, 32, 6, 1, 2, 8, 2, false, true>(tw, ts, tx, p, items, st);
+        if (mt == 16) return launch_cfg<256, 16, 6, 2, 3, 4, 2, false, true>(tw, ts, tx, p, items, st);
+        if (mt == 32) return launch_cfg<256, 32, 6, 2, 2, 4, 2, false, true>(tw, ts, tx, p, items, st);
         return launch_cfg<256, 64, 4, 1, 2, 4, 2, false>(tw, ts, tx, p, items, st);
     }
     // Prefill (and any K that is not a multiple of 256): 128-row tiles,

@@ -207,10 +207,11 @@ __device__ __forceinline__ void dec_word(uint32_t wg, uint32_t wh, uint32_t s2g,
     mma_bf16_m16n8k16(d, pg[2], ph[2], pg[3], ph[3], x.z, x.w);
 }
 
-// One chunk of a tile, rows g and (HI) g + 8: loads, then the four words.
+// One chunk of a tile, rows g and (HI) g + 8: loads, then the four words, the
+// even ones into acc and the odd ones into acc2 (two independent MMA chains).
 template <bool ZP, bool HI>
 __device__ __forceinline__ void dec_chunk(uint32_t slot, const LaneOff<ZP> &o, const uint4 (&x)[4],
-                                          float (&acc)[4]) {
+                                          float (&acc)[4], float (&acc2)[4]) {
     const uint4 wg = lds128(slot + o.w);
     const uint32_t sg = lds_u16(slot + o.s);
     const uint32_t zg = ZP ? lds_u8(slot + o.z) : 0u;
@@ -223,9 +224,9 @@ __device__ __forceinline__ void dec_chunk(uint32_t slot, const LaneOff<ZP> &o, c
     }
     const uint32_t s2g = sg | (sg << 16), s2h = sh | (sh << 16);
     dec_word<ZP, HI>(wg.x, wh.x, s2g, s2h, zg, zh, x[0], acc);
-    dec_word<ZP, HI>(wg.y, wh.y, s2g, s2h, zg, zh, x[1], acc);
+    dec_word<ZP, HI>(wg.y, wh.y, s2g, s2h, zg, zh, x[1], acc2);
     dec_word<ZP, HI>(wg.z, wh.z, s2g, s2h, zg, zh, x[2], acc);
-    dec_word<ZP, HI>(wg.w, wh.w, s2g, s2h, zg, zh, x[3], acc);
+    dec_word<ZP, HI>(wg.w, wh.w, s2g, s2h, zg, zh, x[3], acc2);
 }
 
 // Stage s = (pass s / ntiles, tile s % ntiles) into slot s % kNStage; out of
@@ -344,15 +345,15 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             const int nq = min(4, cta_quads - 4 * i);
             const bool full = nq == 4, hi_rows = nq > 2;       // rows 8..15 of the tile
             const uint32_t sb = base + (uint32_t)(slot * C::STAGE);
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int cl = 0; cl < kWarpChunks; ++cl) {
                 if (cl < na) {
                     const LaneOff<ZP> o(full, warp * kWarpChunks + cl, g, t);
                     if (hi_rows)
-                        dec_chunk<ZP, true>(sb, o, xf[cl], acc);
+                        dec_chunk<ZP, true>(sb, o, xf[cl], acc, acc2);
                     else
-                        dec_chunk<ZP, false>(sb, o, xf[cl], acc);
+                        dec_chunk<ZP, false>(sb, o, xf[cl], acc, acc2);
                 }
             }
             // This warp's shared-memory reads of the slot are complete; the last
@@ -366,7 +367,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             }
             // the tile's sums into this warp's partial sums
             const uint32_t ra = red + (uint32_t)(((warp * kMaxTiles + i) * 32 + lane) * 16);
-            float4 v = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            float4 v = make_float4(acc[0] + acc2[0], acc[1] + acc2[1], acc[2] + acc2[2],
+                                   acc[3] + acc2[3]);
             if (pass > 0) {
                 const float4 prev = lds128f(ra);
                 v = make_float4(prev.x + v.x, prev.y + v.y, prev.z + v.z, prev.w + v.w);
