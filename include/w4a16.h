@@ -298,8 +298,10 @@ w4_status w4_dequant_nvfp4(const int32_t *Wq, const uint8_t *S, float g, w4_bf16
  * W4A16 GEMM on FP4 weight groups: Y[M, N] = X[M, K] . Wdq^T with Wdq the
  * dequantized FP4 weights above, FP32 accumulation, one BF16 rounding.  The
  * codes are unpacked in registers (hardware E2M1 -> FP16 conversion, exact
- * FP32 scaling, BF16 rounding) and stored into tensor memory as the A
- * operand of tcgen05 BF16 MMAs, as in w4a16_gemm_zp's kernel.
+ * FP32 scaling, BF16 rounding): 1..8 rows with K % 512 == 0 and 16-byte-
+ * aligned scale bytes straight into warp-level MMA fragments (the decode
+ * kernel of w4a16_gemm), other shapes into tensor memory as the A operand of
+ * tcgen05 BF16 MMAs, as in w4a16_gemm_zp's kernel.
  *   X in [M, K] BF16;  Wq in [N, K/8];  E in [N, K/32] / S in [N, K/16];
  *   Y out [M, N] BF16.  Device pointers; asynchronous on `stream`.
  */

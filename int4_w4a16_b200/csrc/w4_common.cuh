@@ -585,6 +585,10 @@ w4_status gemv_launch(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S, w4_
 // 16-byte-aligned Z, W4_ERR_UNSUPPORTED otherwise.
 w4_status gemv_launch_zp(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S, const uint8_t *Z,
                          w4_bf16 *Y, int64_t M, int64_t N, int64_t K, void *stream);
+// The same for FP4 codes (fp4 = 1: MXFP4 with E8M0 bytes, 2: NVFP4 with E4M3
+// bytes under the tensor scale g); needs K % 512 == 0 and a 16-byte-aligned SB.
+w4_status gemv_launch_fp4(int fp4, const w4_bf16 *X, const int32_t *Wq, const uint8_t *SB,
+                          float g, w4_bf16 *Y, int64_t M, int64_t N, int64_t K, void *stream);
 
 inline bool aligned16(const void *p) {
     return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0;

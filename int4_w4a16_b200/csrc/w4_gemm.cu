@@ -1600,6 +1600,12 @@ w4_status gemm_fp4(const w4_bf16 *X, const int32_t *Wq, const uint8_t *SB, float
         return W4_ERR_INVALID_ARG;
     if (M == 0 || N == 0) return W4_OK;
     if (N > (1 << 30) || M > (1 << 30) || K > (1 << 24)) return W4_ERR_UNSUPPORTED;
+    // 1..8 activation rows: the warp-level MMA kernel (w4_gemv.cu) when K and
+    // the scale bytes suit its TMA boxes
+    if (w4host::gemv_supported(M, N, K)) {
+        const w4_status gs = w4host::gemv_launch_fp4(FP4, X, Wq, SB, g, Y, M, N, K, stream);
+        if (gs != W4_ERR_UNSUPPORTED) return gs;
+    }
     cudaStream_t st = (cudaStream_t)stream;
     GemmParams p = {};
     p.Z = SB;

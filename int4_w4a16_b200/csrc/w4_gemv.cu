@@ -4,9 +4,10 @@
 // What it computes (INT4 QAT blog, Fig. 4 and "zero-overhead unpacking";
 // reportify.cn "量化感知训练" [32][35]):  Y[m, n] = sum_k X[m, k] * dq(W)[n, k],
 // dq(W)[n, k] = bf16_rne(q[n, k] * S[n, k/32]) (or bf16_rne((q - z) * s) for
-// zero-point groups), FP32 accumulation, one BF16 rounding of the result -- the product of
-// w4_gemm.cu, for activation heights where streaming the packed weights from
-// HBM, not the math, sets the time.
+// zero-point groups, or the dequantized MXFP4 / NVFP4 value for E2M1 codes with
+// scale bytes, MR-GPTQ / QuTLASS FP4 summary), FP32 accumulation, one BF16
+// rounding of the result -- the product of w4_gemm.cu, for activation heights
+// where streaming the packed weights from HBM, not the math, sets the time.
 //
 // Design (B200-first):
 //  * one CTA per SM owns a contiguous range of output rows, cut at 4-row
@@ -55,13 +56,25 @@ constexpr int kMaxQuads = 4 * kMaxTiles;                 // 4-row units per CTA
 constexpr int kNStage = 4;
 constexpr int kMaxM = 8;
 
-template <bool ZP>
+// Weight formats of the kernel: INT4 codes with BF16 scales (symmetric, or
+// with a zero-point byte per group), or FP4 (E2M1) codes with one scale byte
+// per 32 (MXFP4, E8M0) or per 16 (NVFP4, E4M3) codes.
+enum : int { kFmtInt4 = 0, kFmtInt4Zp = 1, kFmtMxfp4 = 2, kFmtNvfp4 = 3 };
+__host__ __device__ constexpr bool fmt_has_s(int f) { return f <= kFmtInt4Zp; }   // BF16 scales
+__host__ __device__ constexpr bool fmt_has_z(int f) { return f >= kFmtInt4Zp; }   // byte box
+__host__ __device__ constexpr bool fmt_fp4(int f) { return f >= kFmtMxfp4; }
+// bytes of the byte box per row and 512-K block: zero points or E8M0 scales
+// (one per 32 codes), E4M3 scales (one per 16)
+__host__ __device__ constexpr int fmt_zbytes(int f) { return f == kFmtNvfp4 ? 32 : 16; }
+
+template <int F>
 struct DecCfg {
     // a stage as its TMA boxes land (a 16-row tile: one box per operand; a
     // partial tile: one 4-row box per 4-row unit, QW / QS / QZ apart)
+    static constexpr int ZB = fmt_zbytes(F);
     static constexpr int QW = kPassChunks * 4 * 64;               // words [chunk][4 rows][16]
-    static constexpr int QS = (kPassChunks / 2) * 4 * 16;         // scales [256 K][4 rows][8]
-    static constexpr int QZ = ZP ? (kPassChunks / 4) * 4 * 16 : 0;  // zero points [512 K][4][16]
+    static constexpr int QS = fmt_has_s(F) ? (kPassChunks / 2) * 4 * 16 : 0;  // [256 K][4][8]
+    static constexpr int QZ = fmt_has_z(F) ? (kPassChunks / 4) * 4 * ZB : 0;  // [512 K][4][ZB]
     static constexpr int SOFF = 4 * QW;                           // 32 KB of words first
     static constexpr int ZOFF = 4 * (QW + QS);
     static constexpr int STAGE = 4 * (QW + QS + QZ);
@@ -77,6 +90,7 @@ struct DecCfg {
 struct DecParams {
     const uint16_t *X;    // [M, K] BF16
     uint16_t *Y;          // [M, N] BF16
+    float g;              // NVFP4 tensor scale
     int M, N, K;
     int n_quads, ctas;    // 4-row units of N, CTAs they are cut over
     int kc, passes;       // K / 128 chunks, passes of 4096 K
@@ -143,26 +157,31 @@ __device__ __forceinline__ void dec_drain(uint32_t bar, uint32_t parity) {
 
 // Shared-memory offsets of one lane for the chunk ch of a stage.  A full tile
 // is one box per operand: words [chunk][16 rows][64 B], scales [256-K block]
-// [16 rows][16 B], zero points [512-K block][16 rows][16 B]; a partial tile
-// holds 4-row boxes ([chunk][4 rows][64 B], [block][4 rows][16 B]) QW / QS /
-// QZ apart.  Row g + 8 sits a fixed distance after row g.
-template <bool ZP>
+// [16 rows][16 B], bytes [512-K block][16 rows][ZB B]; a partial tile holds
+// 4-row boxes ([chunk][4 rows][64 B], [block][4 rows][16 B], [block][4 rows]
+// [ZB B]) QW / QS / QZ apart.  Row g + 8 sits a fixed distance after row g.
+// The lane's byte (or, for NVFP4, its two bytes) of its group of 32 codes
+// sits at group index (ch & 3) * 4 + t of the row's 512-K block.
+template <int F>
 struct LaneOff {
-    uint32_t w, s, z;       // row g: its 16 bytes of words, its scale, its zero point
+    uint32_t w, s, z;       // row g: its 16 bytes of words, its scale, its byte(s)
     uint32_t dw, ds, dz;    // row g + 8 minus row g
     __device__ __forceinline__ LaneOff(bool full, int ch, int g, int t) {
-        using C = DecCfg<ZP>;
-        const uint32_t su = (uint32_t)(((ch & 1) * 4 + t) * 2), zu = (uint32_t)((ch & 3) * 4 + t);
+        using C = DecCfg<F>;
+        constexpr int ZB = C::ZB;
+        const uint32_t su = (uint32_t)(((ch & 1) * 4 + t) * 2);
+        const uint32_t zu = (uint32_t)(((ch & 3) * 4 + t) * (ZB / 16));
         if (full) {
             w = (uint32_t)(ch * 1024 + g * 64 + t * 16);
             s = (uint32_t)(C::SOFF + (ch >> 1) * 256 + g * 16) + su;
-            z = (uint32_t)(C::ZOFF + (ch >> 2) * 256 + g * 16) + zu;
+            z = (uint32_t)(C::ZOFF + (ch >> 2) * 16 * ZB + g * ZB) + zu;
             dw = 512u;
-            ds = dz = 128u;
+            ds = 128u;
+            dz = 8u * ZB;
         } else {
             w = (uint32_t)((g >> 2) * C::QW + ch * 256 + (g & 3) * 64 + t * 16);
             s = (uint32_t)(C::SOFF + (g >> 2) * C::QS + (ch >> 1) * 64 + (g & 3) * 16) + su;
-            z = (uint32_t)(C::ZOFF + (g >> 2) * C::QZ + (ch >> 2) * 64 + (g & 3) * 16) + zu;
+            z = (uint32_t)(C::ZOFF + (g >> 2) * C::QZ + (ch >> 2) * 4 * ZB + (g & 3) * ZB) + zu;
             dw = 2u * C::QW;
             ds = 2u * C::QS;
             dz = 2u * C::QZ;
@@ -192,11 +211,11 @@ __device__ __forceinline__ uint32_t lds_u8(uint32_t addr) {
 }
 
 // One word pair (rows g and g + 8) of step j into the accumulators.
-template <bool ZP, bool HI>
+template <int F, bool HI>
 __device__ __forceinline__ void dec_word(uint32_t wg, uint32_t wh, uint32_t s2g, uint32_t s2h,
                                          uint32_t zg, uint32_t zh, const uint4 &x, float (&d)[4]) {
     uint32_t pg[4], ph[4] = {0u, 0u, 0u, 0u};
-    if (ZP) {
+    if (F == kFmtInt4Zp) {
         dequant_word_k8perm_zp(wg, s2g, zp_bias2(zg), pg);
         if (HI) dequant_word_k8perm_zp(wh, s2h, zp_bias2(zh), ph);
     } else {
@@ -207,37 +226,78 @@ __device__ __forceinline__ void dec_word(uint32_t wg, uint32_t wh, uint32_t s2g,
     mma_bf16_m16n8k16(d, pg[2], ph[2], pg[3], ph[3], x.z, x.w);
 }
 
+// FP4: one word pair with the group scales as FP32 (sg, sh) into the
+// accumulators; the codes come out in natural order (codes 2j, 2j + 1 in one
+// register), so these activations are not permuted.
+template <int F, bool HI>
+__device__ __forceinline__ void dec_word_fp4(uint32_t wg, uint32_t wh, float sg, float sh, float g,
+                                             const uint4 &x, float (&d)[4]) {
+    uint32_t pg[4], ph[4] = {0u, 0u, 0u, 0u};
+    if (F == kFmtMxfp4) {
+        dequant_word_mxfp4(wg, sg, pg);
+        if (HI) dequant_word_mxfp4(wh, sh, ph);
+    } else {
+        dequant_word_nvfp4(wg, sg, g, pg);
+        if (HI) dequant_word_nvfp4(wh, sh, g, ph);
+    }
+    mma_bf16_m16n8k16(d, pg[0], ph[0], pg[1], ph[1], x.x, x.y);
+    mma_bf16_m16n8k16(d, pg[2], ph[2], pg[3], ph[3], x.z, x.w);
+}
+
 // One chunk of a tile, rows g and (HI) g + 8: loads, then the four words, the
 // even ones into acc and the odd ones into acc2 (two independent MMA chains).
-template <bool ZP, bool HI>
-__device__ __forceinline__ void dec_chunk(uint32_t slot, const LaneOff<ZP> &o, const uint4 (&x)[4],
-                                          float (&acc)[4], float (&acc2)[4]) {
+template <int F, bool HI>
+__device__ __forceinline__ void dec_chunk(uint32_t slot, const LaneOff<F> &o, const uint4 (&x)[4],
+                                          float g, float (&acc)[4], float (&acc2)[4]) {
     const uint4 wg = lds128(slot + o.w);
-    const uint32_t sg = lds_u16(slot + o.s);
-    const uint32_t zg = ZP ? lds_u8(slot + o.z) : 0u;
     uint4 wh = make_uint4(0u, 0u, 0u, 0u);
-    uint32_t sh = 0u, zh = 0u;
-    if (HI) {
-        wh = lds128(slot + o.w + o.dw);
-        sh = lds_u16(slot + o.s + o.ds);
-        if (ZP) zh = lds_u8(slot + o.z + o.dz);
+    if (HI) wh = lds128(slot + o.w + o.dw);
+    if constexpr (fmt_fp4(F)) {
+        // MXFP4: one E8M0 byte for the chunk's 32 codes; NVFP4: two E4M3
+        // bytes, words 0-1 and words 2-3
+        float sg0, sg1, sh0 = 0.f, sh1 = 0.f;
+        if (F == kFmtMxfp4) {
+            sg0 = sg1 = e8m0_to_f32(lds_u8(slot + o.z));
+            if (HI) sh0 = sh1 = e8m0_to_f32(lds_u8(slot + o.z + o.dz));
+        } else {
+            const uint32_t zg = lds_u16(slot + o.z);
+            sg0 = e4m3_to_f32(zg & 0xFFu);
+            sg1 = e4m3_to_f32(zg >> 8);
+            if (HI) {
+                const uint32_t zh = lds_u16(slot + o.z + o.dz);
+                sh0 = e4m3_to_f32(zh & 0xFFu);
+                sh1 = e4m3_to_f32(zh >> 8);
+            }
+        }
+        dec_word_fp4<F, HI>(wg.x, wh.x, sg0, sh0, g, x[0], acc);
+        dec_word_fp4<F, HI>(wg.y, wh.y, sg0, sh0, g, x[1], acc2);
+        dec_word_fp4<F, HI>(wg.z, wh.z, sg1, sh1, g, x[2], acc);
+        dec_word_fp4<F, HI>(wg.w, wh.w, sg1, sh1, g, x[3], acc2);
+    } else {
+        const uint32_t sg = lds_u16(slot + o.s);
+        const uint32_t zg = (F == kFmtInt4Zp) ? lds_u8(slot + o.z) : 0u;
+        uint32_t sh = 0u, zh = 0u;
+        if (HI) {
+            sh = lds_u16(slot + o.s + o.ds);
+            if (F == kFmtInt4Zp) zh = lds_u8(slot + o.z + o.dz);
+        }
+        const uint32_t s2g = sg | (sg << 16), s2h = sh | (sh << 16);
+        dec_word<F, HI>(wg.x, wh.x, s2g, s2h, zg, zh, x[0], acc);
+        dec_word<F, HI>(wg.y, wh.y, s2g, s2h, zg, zh, x[1], acc2);
+        dec_word<F, HI>(wg.z, wh.z, s2g, s2h, zg, zh, x[2], acc);
+        dec_word<F, HI>(wg.w, wh.w, s2g, s2h, zg, zh, x[3], acc2);
     }
-    const uint32_t s2g = sg | (sg << 16), s2h = sh | (sh << 16);
-    dec_word<ZP, HI>(wg.x, wh.x, s2g, s2h, zg, zh, x[0], acc);
-    dec_word<ZP, HI>(wg.y, wh.y, s2g, s2h, zg, zh, x[1], acc2);
-    dec_word<ZP, HI>(wg.z, wh.z, s2g, s2h, zg, zh, x[2], acc);
-    dec_word<ZP, HI>(wg.w, wh.w, s2g, s2h, zg, zh, x[3], acc2);
 }
 
 // Stage s = (pass s / ntiles, tile s % ntiles) into slot s % kNStage; out of
 // line so that the compute loop keeps its registers.
-template <bool ZP>
+template <int F>
 __device__ __noinline__ void dec_issue(const CUtensorMap *tw, const CUtensorMap *ts,
                                        const CUtensorMap *tz, const CUtensorMap *tw4,
                                        const CUtensorMap *ts4, const CUtensorMap *tz4,
                                        uint32_t bars, uint32_t base, int row0, int cta_quads,
                                        int ntiles, int *issued, int s) {
-    using C = DecCfg<ZP>;
+    using C = DecCfg<F>;
     const int slot = s % kNStage, pass = s / ntiles, tile = s % ntiles;
     const int nq = min(4, cta_quads - 4 * tile);
     const uint32_t fb = bars + (uint32_t)(slot * 8);
@@ -247,27 +307,28 @@ __device__ __noinline__ void dec_issue(const CUtensorMap *tw, const CUtensorMap 
     mbar_arrive_expect_tx(fb, (uint32_t)(nq * (C::QW + C::QS + C::QZ)));
     if (nq == 4) {
         tma_load_3d(dst, tw, fb, 0, r, pass * kPassChunks);
-        tma_load_3d(dst + C::SOFF, ts, fb, 0, r, pass * (kPassChunks / 2));
-        if (ZP) tma_load_3d(dst + C::ZOFF, tz, fb, 0, r, pass * (kPassChunks / 4));
+        if (fmt_has_s(F)) tma_load_3d(dst + C::SOFF, ts, fb, 0, r, pass * (kPassChunks / 2));
+        if (fmt_has_z(F)) tma_load_3d(dst + C::ZOFF, tz, fb, 0, r, pass * (kPassChunks / 4));
     } else {
         for (int q = 0; q < nq; ++q) {
             tma_load_3d(dst + q * C::QW, tw4, fb, 0, r + 4 * q, pass * kPassChunks);
-            tma_load_3d(dst + C::SOFF + q * C::QS, ts4, fb, 0, r + 4 * q,
-                        pass * (kPassChunks / 2));
-            if (ZP)
+            if (fmt_has_s(F))
+                tma_load_3d(dst + C::SOFF + q * C::QS, ts4, fb, 0, r + 4 * q,
+                            pass * (kPassChunks / 2));
+            if (fmt_has_z(F))
                 tma_load_3d(dst + C::ZOFF + q * C::QZ, tz4, fb, 0, r + 4 * q,
                             pass * (kPassChunks / 4));
         }
     }
 }
 
-template <bool ZP>
+template <int F>
 __global__ void __launch_bounds__(kDecThreads, 1)
     w4a16_dec_kernel(const __grid_constant__ CUtensorMap tw, const __grid_constant__ CUtensorMap ts,
                      const __grid_constant__ CUtensorMap tz, const __grid_constant__ CUtensorMap tw4,
                      const __grid_constant__ CUtensorMap ts4, const __grid_constant__ CUtensorMap tz4,
                      const DecParams p) {
-    using C = DecCfg<ZP>;
+    using C = DecCfg<F>;
     extern __shared__ __align__(1024) uint8_t dec_smem[];
     __shared__ __align__(8) uint64_t full_bar[kNStage];     // stage landed (TMA bytes)
     __shared__ uint32_t slot_done[kNStage];                 // warps done with a slot (grows)
@@ -310,12 +371,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     load_x(0);
 
 #define DEC_ISSUE(s_)                                                                        \
-    dec_issue<ZP>(&tw, &ts, &tz, &tw4, &ts4, &tz4, smem_u32(&full_bar[0]), base, row0, cta_quads, \
+    dec_issue<F>(&tw, &ts, &tz, &tw4, &ts4, &tz4, smem_u32(&full_bar[0]), base, row0, cta_quads, \
                   ntiles, &issued, (s_))
     if (threadIdx.x == 0) {
         tma_prefetch_desc(&tw);
-        tma_prefetch_desc(&ts);
-        if (ZP) tma_prefetch_desc(&tz);
+        if (fmt_has_s(F)) tma_prefetch_desc(&ts);
+        if (fmt_has_z(F)) tma_prefetch_desc(&tz);
         for (int i = 0; i < kNStage; ++i) {
             mbar_init(smem_u32(&full_bar[i]), 1u);
             slot_done[i] = 0u;
@@ -334,7 +395,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
         for (int cl = 0; cl < kWarpChunks; ++cl)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) xf[cl][j] = permute_chunk8(xr[cl][j]);
+            for (int j = 0; j < 4; ++j)
+                xf[cl][j] = fmt_fp4(F) ? xr[cl][j] : permute_chunk8(xr[cl][j]);
         for (int i = 0; i < ntiles; ++i) {
             const int s = pass * ntiles + i;
             const int slot = s % kNStage;
@@ -349,11 +411,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
             for (int cl = 0; cl < kWarpChunks; ++cl) {
                 if (cl < na) {
-                    const LaneOff<ZP> o(full, warp * kWarpChunks + cl, g, t);
+                    const LaneOff<F> o(full, warp * kWarpChunks + cl, g, t);
                     if (hi_rows)
-                        dec_chunk<ZP, true>(sb, o, xf[cl], acc, acc2);
+                        dec_chunk<F, true>(sb, o, xf[cl], p.g, acc, acc2);
                     else
-                        dec_chunk<ZP, false>(sb, o, xf[cl], acc, acc2);
+                        dec_chunk<F, false>(sb, o, xf[cl], p.g, acc, acc2);
                 }
             }
             // This warp's shared-memory reads of the slot are complete; the last
@@ -406,14 +468,15 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 // Host side
 // ---------------------------------------------------------------------------
 
-template <bool ZP>
+template <int F>
 w4_status dec_launch(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S, const uint8_t *Z,
-                     w4_bf16 *Y, int M, int N, int K, cudaStream_t stream) {
-    using C = DecCfg<ZP>;
+                     float g, w4_bf16 *Y, int M, int N, int K, cudaStream_t stream) {
+    using C = DecCfg<F>;
     const int sms = w4host::num_sms();
     DecParams p = {};
     p.X = reinterpret_cast<const uint16_t *>(X);
     p.Y = reinterpret_cast<uint16_t *>(Y);
+    p.g = g;
     p.M = M;
     p.N = N;
     p.K = K;
@@ -428,9 +491,9 @@ w4_status dec_launch(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S, cons
     const size_t smem = (size_t)C::SMEM;
 
     // packed words as [K / 128 chunks][N rows][16 words],
-    // scales as [K / 256 blocks][N rows][8 groups], zero points as [K / 512
-    // blocks][N rows][16 groups]: 16-row boxes for whole tiles, 4-row boxes for
-    // a CTA's partial last tile
+    // BF16 scales as [K / 256 blocks][N rows][8 groups], zero points or FP4
+    // scale bytes as [K / 512 blocks][N rows][16 or 32 bytes]: 16-row boxes for
+    // whole tiles, 4-row boxes for a CTA's partial last tile
     CUtensorMap tw, ts, tz, tw4, ts4, tz4;
     for (int rows : {16, 4}) {
         CUtensorMap *mw = rows == 16 ? &tw : &tw4, *ms = rows == 16 ? &ts : &ts4;
@@ -444,7 +507,7 @@ w4_status dec_launch(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S, cons
                                      CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
                 return W4_ERR_CUDA;
         }
-        {
+        if (fmt_has_s(F)) {
             cuuint64_t dims[3] = {8u, (cuuint64_t)N, (cuuint64_t)(K / 256)};
             cuuint64_t strides[2] = {(cuuint64_t)K / 16, 16u};
             cuuint32_t box[3] = {8u, (cuuint32_t)rows, (cuuint32_t)(kPassChunks / 2)};
@@ -453,18 +516,19 @@ w4_status dec_launch(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S, cons
                                      CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
                 return W4_ERR_CUDA;
         }
-        if (ZP) {
-            cuuint64_t dims[3] = {16u, (cuuint64_t)N, (cuuint64_t)(K / 512)};
-            cuuint64_t strides[2] = {(cuuint64_t)K / 32, 16u};
-            cuuint32_t box[3] = {16u, (cuuint32_t)rows, (cuuint32_t)(kPassChunks / 4)};
+        if (fmt_has_z(F)) {
+            constexpr int ZB = C::ZB;
+            cuuint64_t dims[3] = {(cuuint64_t)ZB, (cuuint64_t)N, (cuuint64_t)(K / 512)};
+            cuuint64_t strides[2] = {(cuuint64_t)K / 512 * ZB, (cuuint64_t)ZB};
+            cuuint32_t box[3] = {(cuuint32_t)ZB, (cuuint32_t)rows, (cuuint32_t)(kPassChunks / 4)};
             if (w4host::encode_tiled(mz, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(Z),
                                      dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
                 return W4_ERR_CUDA;
-        } else {
-            *mz = *ms;                               // not read
         }
+        if (!fmt_has_s(F)) *ms = *mz;                // not read
+        if (!fmt_has_z(F)) *mz = *ms;                // not read
     }
-    auto kern = w4a16_dec_kernel<ZP>;
+    auto kern = w4a16_dec_kernel<F>;
     static bool configured = false;
     if (!configured) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
@@ -490,15 +554,27 @@ bool w4host::gemv_supported(int64_t M, int64_t N, int64_t K) {
 w4_status w4host::gemv_launch(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S, w4_bf16 *Y,
                               int64_t M, int64_t N, int64_t K, void *stream) {
     if (!gemv_supported(M, N, K)) return W4_ERR_UNSUPPORTED;
-    return w4::dec_launch<false>(X, Wq, S, nullptr, Y, (int)M, (int)N, (int)K,
-                                 (cudaStream_t)stream);
+    return w4::dec_launch<w4::kFmtInt4>(X, Wq, S, nullptr, 1.0f, Y, (int)M, (int)N, (int)K,
+                                        (cudaStream_t)stream);
 }
 
 w4_status w4host::gemv_launch_zp(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S,
                                  const uint8_t *Z, w4_bf16 *Y, int64_t M, int64_t N, int64_t K,
                                  void *stream) {
     if (!gemv_supported(M, N, K) || (K % 512) != 0 || !aligned16(Z)) return W4_ERR_UNSUPPORTED;
-    return w4::dec_launch<true>(X, Wq, S, Z, Y, (int)M, (int)N, (int)K, (cudaStream_t)stream);
+    return w4::dec_launch<w4::kFmtInt4Zp>(X, Wq, S, Z, 1.0f, Y, (int)M, (int)N, (int)K,
+                                          (cudaStream_t)stream);
+}
+
+w4_status w4host::gemv_launch_fp4(int fp4, const w4_bf16 *X, const int32_t *Wq, const uint8_t *SB,
+                                  float g, w4_bf16 *Y, int64_t M, int64_t N, int64_t K,
+                                  void *stream) {
+    if (!gemv_supported(M, N, K) || (K % 512) != 0 || !aligned16(SB)) return W4_ERR_UNSUPPORTED;
+    if (fp4 == 1)
+        return w4::dec_launch<w4::kFmtMxfp4>(X, Wq, nullptr, SB, 1.0f, Y, (int)M, (int)N, (int)K,
+                                             (cudaStream_t)stream);
+    return w4::dec_launch<w4::kFmtNvfp4>(X, Wq, nullptr, SB, g, Y, (int)M, (int)N, (int)K,
+                                         (cudaStream_t)stream);
 }
 
 cudaError_t w4host::gemv_device_status(unsigned int *flag) {

@@ -193,8 +193,12 @@ def _nv_weights(N, K, seed):
     return oq, oS, og, _dev_u8(pack_codes(oq)), _dev_u8(oS)
 
 
+# 1..8 rows with K % 512 == 0 take the warp-level decode kernel (one and
+# several passes over K, ring refills, more CTAs than SMs, ragged N); the
+# others the tensor-memory tile
 SHAPES = [(1, 1, 32), (1, 300, 4096), (5, 100, 128), (64, 300, 640), (65, 257, 256),
-          (300, 1000, 1024), (512, 1024, 2048), (3, 129, 96)]
+          (300, 1000, 1024), (512, 1024, 2048), (3, 129, 96), (8, 4099, 2048), (7, 1000, 1536),
+          (2, 9472, 8192), (3, 20000, 512), (1, 14212, 512), (4, 37, 4608)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)
@@ -217,12 +221,12 @@ def test_gemm_nvfp4_shapes(M, N, K):
     assert_gemm_close(Y, R, f"nvfp4 M={M} N={N} K={K}")
 
 
-def _one_hot_check(run, Wdq, K):
-    for m0 in range(0, K, 64):
-        X = torch.zeros((64, K), dtype=torch.bfloat16)
-        X[torch.arange(64), m0 + torch.arange(64)] = 1.0
+def _one_hot_check(run, Wdq, K, MB=64):
+    for m0 in range(0, K, MB):
+        X = torch.zeros((MB, K), dtype=torch.bfloat16)
+        X[torch.arange(MB), m0 + torch.arange(MB)] = 1.0
         Y = bits(run(X.to(DEV)))
-        want = Wdq[:, m0:m0 + 64].T
+        want = Wdq[:, m0:m0 + MB].T
         if not np.array_equal(Y, want):
             bad = np.argwhere(Y != want)
             raise AssertionError(f"one-hot mismatch at m0={m0}: {bad[:8].tolist()}")
@@ -239,14 +243,27 @@ def test_gemm_fp4_one_hot_exact():
     w4.w4_device_status()
 
 
-@pytest.mark.parametrize("M", [16, 2048])
+def test_gemm_fp4_one_hot_exact_decode_kernel():
+    """The same with 8-row one-hot blocks, which the warp-level decode kernel
+    takes (K % 512 == 0): every code position of the natural-order unpack
+    meets its activation."""
+    N, K = 120, 1024
+    oq, oE, Wq, E = _mx_weights(N, K, seed=13)
+    _one_hot_check(lambda X: w4.gemm_mxfp4(X, Wq, E), oracle.dequant_mxfp4(oq, oE), K, MB=8)
+    oq, oS, og, Wq, S = _nv_weights(N, K, seed=14)
+    _one_hot_check(lambda X: w4.gemm_nvfp4(X, Wq, S, og), oracle.dequant_nvfp4(oq, oS, og), K,
+                   MB=8)
+    w4.w4_device_status()
+
+
+@pytest.mark.parametrize("M", [1, 8, 16, 2048])
 def test_gemm_fp4_layer_shape_sampled(M):
-    """The decode layer's weight (12288 x 4096) at 16 and 2048 tokens; the
-    oracle checks 12 rows of Y spread over M."""
+    """The decode layer's weight (12288 x 4096) at 1, 8, 16 and 2048 tokens;
+    the oracle checks up to 12 rows of Y spread over M."""
     N, K = 12288, 4096
     W = bits(synth.normal_bf16((N, K), 0.02, seed=6, outlier_frac=0.001))
     X = synth.normal_bf16((M, K), 1.0, seed=7)
-    rows = torch.linspace(0, M - 1, 12).long()
+    rows = torch.unique(torch.linspace(0, M - 1, 12).long())
     oq, oE = oracle.quantize_mxfp4(W)
     Y = w4.gemm_mxfp4(X.to(DEV), _dev_u8(pack_codes(oq)), _dev_u8(oE))
     _, R = oracle.gemm(bits(X[rows]), oracle.dequant_mxfp4(oq, oE))
