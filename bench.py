@@ -804,9 +804,9 @@ def bench_qat_gemm(w4, dev, peaks, Ms, reps, flush):
 
 def bench_fp4(w4, dev, peaks, reps, flush):
     """Micro-scaled FP4 weights (MXFP4 and NVFP4) on the decode layer's shape
-    W[12288, 4096]: the W4A16 GEMM at M = 1 (GB/s of packed codes + scales +
-    activations + output) and M = 2048 (TFLOP/s), and the quantizers (GB/s of
-    BF16 in + codes and scales out)."""
+    W[12288, 4096]: the W4A16 GEMM at M = 1 and 16 (GB/s of packed codes +
+    scales + activations + output) and M = 2048 (TFLOP/s), and the quantizers
+    (GB/s of BF16 in + codes and scales out)."""
     cfg = synth.Decode()
     W = cfg.weight(dev)
     N, K = cfg.N, cfg.K
@@ -818,7 +818,7 @@ def bench_fp4(w4, dev, peaks, reps, flush):
             ("mxfp4", mx[0], mx[1], lambda X, Y: w4.w4a16_gemm_mxfp4(X, mx[0], mx[1], Y)),
             ("nvfp4", nv[0], nv[1], lambda X, Y: w4.w4a16_gemm_nvfp4(X, nv[0], nv[1], g, Y))):
         r = {}
-        for M in (1, 2048):
+        for M in (1, 16, 2048):
             X = cfg.activations(M, dev) if M <= 64 else synth.normal_bf16((M, K), 1.0, 0, 600, dev)
             Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
             f = lambda: run(X, Y)

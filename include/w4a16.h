@@ -250,7 +250,9 @@ w4_status w4_dequant_zp(const int32_t *Wq, const w4_bf16 *S, const uint8_t *Z, w
  * fp32 accumulation, BF16 output (the zero point is subtracted in the same
  * register unpack as w4a16_gemm's constant bias, no extra instruction).  1..8
  * rows with K % 512 == 0 and a 16-byte-aligned Z take the warp-level decode
- * kernel; every other shape the tensor-memory kernel with 64-wide k-blocks.
+ * kernel, 9..64 rows with K % 256 == 0 and a 16-byte-aligned Z the 256-wide
+ * tensor-memory decode tiles (no workspace), every other shape the
+ * tensor-memory kernel with 64-wide k-blocks.
  * K a multiple of 32; group 32; X, Wq, S, Y 16-byte aligned; Z not NULL.
  * Device pointers; the call is asynchronous on `stream`.
  */
@@ -301,7 +303,8 @@ w4_status w4_dequant_nvfp4(const int32_t *Wq, const uint8_t *S, float g, w4_bf16
  * FP32 scaling, BF16 rounding): 1..8 rows with K % 512 == 0 and 16-byte-
  * aligned scale bytes straight into warp-level MMA fragments (the decode
  * kernel of w4a16_gemm), other shapes into tensor memory as the A operand of
- * tcgen05 BF16 MMAs, as in w4a16_gemm_zp's kernel.
+ * tcgen05 BF16 MMAs (9..64 rows with K % 256 == 0 on the 256-wide decode
+ * tiles, the rest on the 64-wide tile), as in w4a16_gemm_zp.
  *   X in [M, K] BF16;  Wq in [N, K/8];  E in [N, K/32] / S in [N, K/16];
  *   Y out [M, N] BF16.  Device pointers; asynchronous on `stream`.
  */

@@ -227,7 +227,7 @@ __device__ __forceinline__ int unit_owner(uint32_t x, const GemmParams &p) {
 
 // Shared-memory layout, all offsets from a 1024-aligned base.
 template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT, bool BF16W = false,
-          bool SMEM_A = false>
+          bool SMEM_A = false, bool A_IN_TMEM = true>
 struct Layout {
     // weight tile of up to 128 rows: packed INT4 words, or BF16 weights (QAT)
     static constexpr int kWBytes = BF16W ? 128 * KB * 2 : 128 * KB / 2;
@@ -246,7 +246,8 @@ struct Layout {
     static constexpr int kAlloc = kBytes + 1024;            // slack for 1024-alignment
     static_assert(kWBytes % 1024 == 0 && kXSub % 1024 == 0, "1024-byte aligned tiles");
     static_assert(kStage % 1024 == 0, "stage size");
-    static_assert(NACC * NSPLIT * MT + NASTAGE * (KB / 2) <= kTmemCols, "TMEM budget");
+    static_assert(NACC * NSPLIT * MT + (A_IN_TMEM ? NASTAGE * (KB / 2) : 0) <= kTmemCols,
+                  "TMEM budget");
 };
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
@@ -326,18 +327,31 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
     constexpr int kAccSets = SPLITN ? 1 : NSPLIT;   // accumulators per work item
     // QAT = 1: forward (fake quantization of W in the weight prologue, A in
     // TMEM); QAT = 2: input gradient dX = dY . fake_quant(W), A = fake_quant(W)^T
-    // tile in shared memory
+    // tile in shared memory; QAT = 3: forward with the QDQ written back in place
+    // over the weight tile, which the MMA then reads as A from shared memory
+    // (tensor memory holds only accumulators)
     constexpr bool kQdx = (QAT == 2);
-    using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE, kAccSets, (QAT != 0), kQdx>;
-    static_assert(!QAT || (KB == 64 && !MOE && QAT <= 2),
+    constexpr bool kQin = (QAT == 3);
+    using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE, kAccSets, (QAT != 0), kQdx, (QAT <= 1)>;
+    static_assert(!QAT || (KB == 64 && !MOE && QAT <= 3),
                   "QAT: 64-wide k-blocks of dense BF16 weights");
-    static_assert(!kQdx || NSTAGE == NASTAGE, "QAT input gradient: one release per k-block");
+    static_assert(!(kQdx || kQin) || NSTAGE == NASTAGE,
+                  "A in shared memory: one release per k-block");
+    static_assert(MT <= 256 || (SPLITN && MT / NSPLIT <= 256 && QAT >= 2),
+                  "more than 256 tokens per item: token-split issuers, A in shared memory");
     static_assert(!SPLITN || (KB == 64 && !MOE && !WGL && MT % (16 * NSPLIT) == 0),
                   "token-split issuers: dense 64-wide k-blocks, N per issuer a multiple of 16");
-    static_assert(!ZP || (KB == 64 && !MOE && !QAT), "zero points: dense 64-wide k-blocks");
+    static_assert(!ZP || ((KB == 64 || KB == 256) && !MOE && !QAT),
+                  "zero points: dense k-blocks");
     // FP4 = 1: MXFP4 (a scale byte per 32 codes), 2: NVFP4 (a scale byte per 16)
-    static_assert(FP4 == 0 || (KB == 64 && !MOE && !QAT && !ZP && FP4 <= 2),
-                  "FP4 codes: dense 64-wide k-blocks");
+    static_assert(FP4 == 0 || ((KB == 64 || KB == 256) && !MOE && !QAT && !ZP && FP4 <= 2),
+                  "FP4 codes: dense k-blocks");
+    // 256-wide k-blocks with zero points or FP4 scales: the row's bytes of the
+    // k-block (8 zero points / E8M0 scales, 16 E4M3 scales) are read directly
+    // by the dequant warps; FP4 codes unpack in natural order, so the
+    // activation chunks keep theirs (the reorder warps only join the barrier)
+    constexpr bool kByteScales = (KB == 256) && (ZP || FP4 != 0);
+    static_assert(!kByteScales || !WGL, "byte scales: flat warp layout");
     constexpr int kWords = KB / 8;             // packed words per row per k-block
     constexpr int kAStageCols = KB / 2;        // TMEM columns per A stage
     constexpr int kAccCols = kAccSets * MT;    // TMEM columns per work item accumulator
@@ -418,7 +432,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tm_w);
-        if (KB == 256) tma_prefetch_desc(&tm_s);
+        if (KB == 256 && FP4 == 0) tma_prefetch_desc(&tm_s);
         if (!MOE) tma_prefetch_desc(&tm_x);
     }
     if (warp == kAllocWarp) {
@@ -478,7 +492,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                 }
                 if (lane == 0) {
                     const uint32_t wbytes = QAT ? (uint32_t)R * KB * 2u : (uint32_t)R * (KB / 2);
-                    const uint32_t sbytes = (KB == 256) ? (uint32_t)R * 16u : 0u;
+                    const uint32_t sbytes = (KB == 256 && FP4 == 0) ? (uint32_t)R * 16u : 0u;
                     const uint32_t xbytes = MOE ? 0u : (uint32_t)L::kXBytes;
                     mbar_arrive_expect_tx(full_bar(s), wbytes + sbytes + xbytes);
                     if (MOE && p.silu_inter > 0) {
@@ -503,15 +517,21 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                         tma_load_2d(w_stage(s), &tm_w, full_bar(s), row0, kb * KB);
                         tma_load_2d(w_stage(s) + L::kWBytes / 2, &tm_w, full_bar(s), row0 + 64,
                                     kb * KB);
-                        tma_load_2d(x_stage(s), &tm_x, full_bar(s), kb * KB, tt * MT);
+#pragma unroll
+                        for (int h = 0; h < (MT + 255) / 256; ++h)
+                            tma_load_2d(x_stage(s) + h * 256 * 128, &tm_x, full_bar(s), kb * KB,
+                                        tt * MT + h * 256);
                     } else {
                         tma_load_2d(w_stage(s), &tm_w, full_bar(s), QAT ? kb * KB : kb * kWords,
                                     row0);
-                        if (KB == 256) tma_load_2d(s_stage(s), &tm_s, full_bar(s), kb * 8, row0);
+                        if (KB == 256 && FP4 == 0)
+                            tma_load_2d(s_stage(s), &tm_s, full_bar(s), kb * 8, row0);
 #pragma unroll
                         for (int u = 0; u < KB / 64; ++u)
-                            tma_load_2d(x_stage(s) + u * L::kXSub, &tm_x, full_bar(s),
-                                        kb * KB + u * 64, tt * MT);
+#pragma unroll
+                            for (int h = 0; h < (MT + 255) / 256; ++h)
+                                tma_load_2d(x_stage(s) + u * L::kXSub + h * 256 * 128, &tm_x,
+                                            full_bar(s), kb * KB + u * 64, tt * MT + h * 256);
                     }
                 }
                 if (MOE) {
@@ -566,6 +586,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                 srow = p.S + base;
             }
             const uint8_t *zrow = (ZP && srow != nullptr) ? p.Z + (srow - p.S) : nullptr;
+            if (ZP && KB == 256 && valid) zrow = p.Z + row * gpr;
             // FP4: the row's scale bytes, one per 32 (MX) or 16 (NV) codes
             constexpr int kFpg = FP4 == 2 ? 4 : 2;       // scale bytes per k-block
             const int64_t fgpr = (FP4 == 2) ? p.K / 16 : gpr;
@@ -617,6 +638,38 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                     mbar_arrive(afull_bar(a));
                     continue;
                 }
+                if constexpr (kQin) {
+                    // QAT forward, in place: the row's 64 BF16 weights (two groups
+                    // of 32, one 128-byte swizzled line of the stage) go through
+                    // the exact group QDQ and are written back where they were;
+                    // the line is this thread's alone, and the stage is reused
+                    // only after the MMAs that read it complete
+                    if (!warp_wait(full_bar(s), (it / NSTAGE) & 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    uint32_t v[2][16], o[2][16];
+                    uint32_t addr[8];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        addr[c] = w_stage(s) + swz((uint32_t)(lrow * 128 + c * 16), 128);
+                        const uint4 x = lds128(addr[c]);
+                        v[c >> 2][4 * (c & 3)] = x.x;
+                        v[c >> 2][4 * (c & 3) + 1] = x.y;
+                        v[c >> 2][4 * (c & 3) + 2] = x.z;
+                        v[c >> 2][4 * (c & 3) + 3] = x.w;
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) qdq::fake_quant_group(v[h], o[h]);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        sts128(addr[c], make_uint4(o[c >> 2][4 * (c & 3)], o[c >> 2][4 * (c & 3) + 1],
+                                                   o[c >> 2][4 * (c & 3) + 2],
+                                                   o[c >> 2][4 * (c & 3) + 3]));
+                    fence_proxy_async_smem();       // generic writes -> tensor-core reads
+                    mbar_arrive(afull_bar(a));
+                    continue;
+                }
                 if constexpr (QAT == 1) {
                     // QAT forward: the row's 64 BF16 weights (two groups of 32,
                     // 128-byte swizzled line) go through the exact group QDQ of the
@@ -655,7 +708,19 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                 static_assert(KB == 256 || G == 2, "direct-load scales: one chunk pair per k-block");
                 uint32_t sc[G] = {}, zb[G] = {};
                 float fs[kFpg];
-                if constexpr (FP4 != 0) {
+                uint4 kbytes = make_uint4(0u, 0u, 0u, 0u);     // kByteScales: the k-block's bytes
+                if constexpr (kByteScales) {
+                    const uint8_t *src = ZP ? zrow : frow;
+                    if (src != nullptr) {
+                        if (FP4 == 2) {
+                            kbytes = __ldg(reinterpret_cast<const uint4 *>(src) + kb);
+                        } else {
+                            const uint2 b8 = __ldg(reinterpret_cast<const uint2 *>(src) + kb);
+                            kbytes.x = b8.x;
+                            kbytes.y = b8.y;
+                        }
+                    }
+                } else if constexpr (FP4 != 0) {
                     // the k-block's FP4 group scales as FP32 (exact conversions)
 #pragma unroll
                     for (int j = 0; j < kFpg; ++j) {
@@ -690,10 +755,18 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                                        swz((uint32_t)(lrow * (KB / 2) + (j + jj) * 16), KB / 2));
                 };
                 auto load_scales = [&](int j) -> uint32_t {
-                    return KB == 256 ? lds32(s_stage(s) + lrow * 16 + j * 2) : 0u;
+                    return (KB == 256 && FP4 == 0) ? lds32(s_stage(s) + lrow * 16 + j * 2) : 0u;
+                };
+                // byte b of the k-block's direct-loaded bytes
+                auto kbyte = [&](int b) -> uint32_t {
+                    const uint32_t wv = (b >> 2) == 0 ? kbytes.x
+                                      : (b >> 2) == 1 ? kbytes.y
+                                      : (b >> 2) == 2 ? kbytes.z : kbytes.w;
+                    return (wv >> (8 * (b & 3))) & 0xFFu;
                 };
                 // Two chunks (8 packed words) become 32 TMEM columns, 2 BF16 per column.
-                auto unpack_pair = [&](const uint4 (&w)[2], uint32_t s_pair, uint32_t (&o)[32]) {
+                auto unpack_pair = [&](const uint4 (&w)[2], uint32_t s_pair, uint32_t (&o)[32],
+                                       int jpair) {
                     uint32_t scp[2];
                     if (KB == 256) {
                         scp[0] = bf16x2_splat((uint16_t)(s_pair & 0xFFFFu));
@@ -708,7 +781,15 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             uint32_t t4[4];
-                            if (kXPerm) dequant_word_k8perm(ws[q], scp[jj], t4);
+                            const int c = jpair + jj;           // chunk of the k-block
+                            if (kByteScales && FP4 == 1)
+                                dequant_word_mxfp4(ws[q], e8m0_to_f32(kbyte(c)), t4);
+                            else if (kByteScales && FP4 == 2)
+                                dequant_word_nvfp4(ws[q], e4m3_to_f32(kbyte(2 * c + (q >> 1))),
+                                                   p.fp4_g, t4);
+                            else if (kByteScales && ZP)
+                                dequant_word_k8perm_zp(ws[q], scp[jj], zp_bias2(kbyte(c)), t4);
+                            else if (kXPerm) dequant_word_k8perm(ws[q], scp[jj], t4);
                             else if (FP4 == 1) dequant_word_mxfp4(ws[q], fs[jj], t4);
                             else if (FP4 == 2)
                                 dequant_word_nvfp4(ws[q], fs[(2 * jj + (q >> 1)) % kFpg], p.fp4_g,
@@ -728,7 +809,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                 uint4 cur[2];
                 load_pair(0, cur);
                 uint32_t o[2][32];
-                unpack_pair(cur, load_scales(0), o[0]);
+                unpack_pair(cur, load_scales(0), o[0], 0);
                 if (!warp_wait(aslot_free_bar(it), aslot_free_parity(it), abort_flag)) {
                     ok = false;
                     break;
@@ -745,7 +826,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                         s_nxt = load_scales(j + 2);
                     }
                     tmem_st_x32(a_col + (uint32_t)(j * 16), o[jp & 1]);
-                    if (jp + 1 < kPairs) unpack_pair(cur, s_nxt, o[(jp + 1) & 1]);
+                    if (jp + 1 < kPairs) unpack_pair(cur, s_nxt, o[(jp + 1) & 1], j + 2);
                 }
                 tmem_wait_st();
                 tc_fence_before_sync();
@@ -779,7 +860,7 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                 constexpr int kStride = 32 * (kPermWarps > 0 ? kPermWarps : 1);
                 static_assert(kChunks % (kStride * kBatch) == 0, "whole batches");
 #pragma unroll 1
-                for (int c0 = pw * 32 + lane; c0 < kChunks; c0 += kStride * kBatch) {
+                for (int c0 = pw * 32 + lane; FP4 == 0 && c0 < kChunks; c0 += kStride * kBatch) {
                     uint32_t addr[kBatch];
                     uint4 v[kBatch];
 #pragma unroll
@@ -860,6 +941,9 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
                             const uint32_t acc_flag = (kb > kb0 || u >= kU0Step) ? 1u : 0u;
                             if (kQdx)
                                 tc_mma_ss(d_tmem, smem_desc_k_sw128(a_smem(a) + (u & 3) * 32),
+                                          smem_desc_k_sw128(baddr), kIdesc, acc_flag);
+                            else if (kQin)
+                                tc_mma_ss(d_tmem, smem_desc_k_sw128(w_stage(s) + (u & 3) * 32),
                                           smem_desc_k_sw128(baddr), kIdesc, acc_flag);
                             else
                                 tc_mma_ts(d_tmem, a_tmem + u * 8, smem_desc_k_sw128(baddr), kIdesc,
@@ -1190,7 +1274,8 @@ template <int KB, int MT, int NSTAGE, int NACC, int NASTAGE, int NSPLIT, int NDQ
           bool WGL = false, int QAT = 0, bool ZP = false, bool SPLITN = false, int FP4 = 0>
 w4_status launch_cfg(const CUtensorMap &tw, const CUtensorMap &ts, const CUtensorMap &tx,
                      const GemmParams &p, int num_items_max, cudaStream_t stream) {
-    using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE, (SPLITN ? 1 : NSPLIT), (QAT != 0), (QAT == 2)>;
+    using L = Layout<KB, MT, NSTAGE, NACC, NASTAGE, (SPLITN ? 1 : NSPLIT), (QAT != 0), (QAT == 2),
+                     (QAT <= 1)>;
     auto kern =
         w4a16_tc_kernel<KB, MT, NSTAGE, NACC, NASTAGE, NSPLIT, NDQ, MOE, WGL, QAT, ZP, SPLITN, FP4>;
     // At least half of the SM's shared memory, so one CTA (and one TMEM
@@ -1445,7 +1530,12 @@ extern "C" w4_status w4_qat_gemm(const w4_bf16 *X, const w4_bf16 *W, w4_bf16 *Y,
     p.M = M;
     p.N = N;
     p.K = K;
-    const int mt = M <= 64 ? 64 : 256;
+    // more than 64 tokens: 256-token work items with the QDQ written back over
+    // the weight tile (A from shared memory), which leaves tensor memory to two
+    // accumulator sets, so one item's epilogue overlaps the next item's MMAs --
+    // unless 256-token items would leave SMs idle (64-token items then)
+    int mt = M <= 64 ? 64 : 256;
+    if (mt == 256 && (int64_t)ceil_div_i(N, 128) * ceil_div_i(M, 256) < w4host::num_sms()) mt = 64;
     p.rows_per_tile = 128;
     p.n_row_tiles = ceil_div_i(N, 128);
     p.n_tok_tiles = ceil_div_i(M, mt);
@@ -1455,7 +1545,7 @@ extern "C" w4_status w4_qat_gemm(const w4_bf16 *X, const w4_bf16 *W, w4_bf16 *Y,
     {
         cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
         cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-        cuuint32_t box[2] = {64u, (cuuint32_t)mt};
+        cuuint32_t box[2] = {64u, (cuuint32_t)std::min(mt, 256)};
         if (!make_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, dims, strides, box,
                       CU_TENSOR_MAP_SWIZZLE_128B))
             return W4_ERR_CUDA;
@@ -1472,9 +1562,9 @@ extern "C" w4_status w4_qat_gemm(const w4_bf16 *X, const w4_bf16 *W, w4_bf16 *Y,
     const int64_t items = (int64_t)p.n_row_tiles * p.n_tok_tiles;
     if (items > (1 << 30)) return W4_ERR_UNSUPPORTED;
     if (mt == 64)
-        return launch_cfg<64, 64, 8, 1, 8, 4, 2, false, false, true>(tw, ts, tx, p, (int)items, st);
-    // one issuer: with the QDQ prologue, more issuers measured no faster
-    return launch_cfg<64, 256, 4, 1, 4, 1, 2, false, false, true>(tw, ts, tx, p, (int)items, st);
+        return launch_cfg<64, 64, 8, 1, 8, 4, 2, false, false, 1>(tw, ts, tx, p, (int)items, st);
+    return launch_cfg<64, 256, 4, 2, 4, 2, 2, false, false, 3, false, true>(tw, ts, tx, p,
+                                                                           (int)items, st);
 }
 
 extern "C" w4_status w4_qat_gemm_dx(const w4_bf16 *dY, const w4_bf16 *W, w4_bf16 *dX, int64_t M,
@@ -1495,7 +1585,8 @@ extern "C" w4_status w4_qat_gemm_dx(const w4_bf16 *dY, const w4_bf16 *W, w4_bf16
     p.M = M;
     p.N = K;
     p.K = N;
-    const int mt = M <= 64 ? 64 : 256;
+    int mt = M <= 64 ? 64 : 256;
+    if (mt == 256 && (int64_t)ceil_div_i(K, 128) * ceil_div_i(M, 256) < w4host::num_sms()) mt = 64;
     p.rows_per_tile = 128;
     p.n_row_tiles = ceil_div_i(K, 128);
     p.n_tok_tiles = ceil_div_i(M, mt);
@@ -1503,10 +1594,10 @@ extern "C" w4_status w4_qat_gemm_dx(const w4_bf16 *dY, const w4_bf16 *W, w4_bf16
     CUtensorMap tw, ts, tx;
     memset(&ts, 0, sizeof ts);
     {
-        // dY [M, N]: 64-wide N boxes of mt tokens
+        // dY [M, N]: 64-wide N boxes of up to 256 tokens
         cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
         cuuint64_t strides[1] = {(cuuint64_t)N * 2};
-        cuuint32_t box[2] = {64u, (cuuint32_t)mt};
+        cuuint32_t box[2] = {64u, (cuuint32_t)std::min(mt, 256)};
         if (!make_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dY, dims, strides, box,
                       CU_TENSOR_MAP_SWIZZLE_128B))
             return W4_ERR_CUDA;
@@ -1524,8 +1615,20 @@ extern "C" w4_status w4_qat_gemm_dx(const w4_bf16 *dY, const w4_bf16 *W, w4_bf16
     if (items > (1 << 30)) return W4_ERR_UNSUPPORTED;
     if (mt == 64)
         return launch_cfg<64, 64, 4, 1, 4, 4, 2, false, false, 2>(tw, ts, tx, p, (int)items, st);
-    return launch_cfg<64, 256, 3, 1, 3, 1, 2, false, false, 2>(tw, ts, tx, p, (int)items, st);
+    // two accumulator sets (A is in shared memory), two issuers over the
+    // 256 tokens
+    return launch_cfg<64, 256, 3, 2, 3, 2, 2, false, false, 2, false, true>(tw, ts, tx, p,
+                                                                           (int)items, st);
 }
+
+namespace w4 {
+namespace {
+template <bool ZP, int FP4>
+w4_status decode_tiles_bytes(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S,
+                             const uint8_t *SB, float g, w4_bf16 *Y, int64_t M, int64_t N,
+                             int64_t K, cudaStream_t st);
+}  // namespace
+}  // namespace w4
 
 extern "C" w4_status w4a16_gemm_zp(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S,
                                    const uint8_t *Z, w4_bf16 *Y, int64_t M, int64_t N, int64_t K,
@@ -1544,6 +1647,9 @@ extern "C" w4_status w4a16_gemm_zp(const w4_bf16 *X, const int32_t *Wq, const w4
         if (gs != W4_ERR_UNSUPPORTED) return gs;
     }
     cudaStream_t st = (cudaStream_t)stream;
+    // up to 64 rows: the 256-wide decode tiles, zero points read directly
+    if (M <= 64 && (K % 256) == 0 && w4host::aligned16(Z))
+        return decode_tiles_bytes<true, 0>(X, Wq, S, Z, 1.0f, Y, M, N, K, st);
     GemmParams p = {};
     p.S = reinterpret_cast<const uint16_t *>(S);
     p.Z = Z;
@@ -1588,6 +1694,74 @@ extern "C" w4_status w4a16_gemm_zp(const w4_bf16 *X, const int32_t *Wq, const w4
 namespace w4 {
 namespace {
 
+// Decode-shaped GEMM (9..64 rows, K % 256 == 0) on zero-point groups or FP4
+// codes: the 256-wide tensor-memory tiles of w4a16_gemm without a workspace
+// (rows split evenly over the SMs, each tile all of K), the byte scales read
+// directly by the dequant warps.  S: BF16 scales (zero points only); SB: the
+// zero points or FP4 scale bytes.
+template <bool ZP, int FP4>
+w4_status decode_tiles_bytes(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S,
+                             const uint8_t *SB, float g, w4_bf16 *Y, int64_t M, int64_t N,
+                             int64_t K, cudaStream_t st) {
+    const int sms = w4host::num_sms();
+    GemmParams p = {};
+    p.S = reinterpret_cast<const uint16_t *>(S);
+    p.Z = SB;
+    p.fp4_g = g;
+    p.Y = reinterpret_cast<uint16_t *>(Y);
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    const int mt = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+    int R = std::min<int64_t>(128, std::max<int64_t>(1, ceil_div_i(N, sms)));
+    while (R < 128 && ceil_div_i(N, R) > sms) ++R;
+    p.rows_per_tile = R;
+    p.n_row_tiles = ceil_div_i(N, R);
+    p.n_tok_tiles = 1;
+    p.num_kb = (int)(K / 256);
+    CUtensorMap tw, ts, tx;
+    memset(&ts, 0, sizeof ts);
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+        cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+        cuuint32_t box[2] = {64u, (cuuint32_t)mt};
+        if (!make_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+            return W4_ERR_CUDA;
+    }
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)(K / 8), (cuuint64_t)N};
+        cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+        cuuint32_t box[2] = {32u, (cuuint32_t)R};
+        if (!make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_INT32, 2, Wq, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+            return W4_ERR_CUDA;
+    }
+    if (FP4 == 0) {
+        cuuint64_t dims[2] = {(cuuint64_t)(K / 32), (cuuint64_t)N};
+        cuuint64_t strides[1] = {(cuuint64_t)(K / 16)};
+        cuuint32_t box[2] = {8u, (cuuint32_t)R};
+        if (!make_map(&ts, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, S, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+            return W4_ERR_CUDA;
+    }
+    const int items = p.n_row_tiles;
+    if (mt == 16)
+        return launch_cfg<256, 16, 6, 2, 3, 4, 2, false, false, 0, ZP, false, FP4>(tw, ts, tx, p,
+                                                                                  items, st);
+    if (mt == 32)
+        return launch_cfg<256, 32, 6, 2, 2, 4, 2, false, false, 0, ZP, false, FP4>(tw, ts, tx, p,
+                                                                                  items, st);
+    return launch_cfg<256, 64, 4, 1, 2, 4, 2, false, false, 0, ZP, false, FP4>(tw, ts, tx, p, items,
+                                                                              st);
+}
+
+}  // namespace
+}  // namespace w4
+
+namespace w4 {
+namespace {
+
 // W4A16 GEMM on FP4 codes (FP4 = 1: MXFP4, 2: NVFP4): the zero-point kernel's
 // tiles (128 weight rows x 64-wide k-blocks, scale bytes read directly by the
 // dequant warps) with the FP4 unpack in the weight prologue.
@@ -1607,6 +1781,9 @@ w4_status gemm_fp4(const w4_bf16 *X, const int32_t *Wq, const uint8_t *SB, float
         if (gs != W4_ERR_UNSUPPORTED) return gs;
     }
     cudaStream_t st = (cudaStream_t)stream;
+    // up to 64 rows: the 256-wide decode tiles
+    if (M <= 64 && (K % 256) == 0 && w4host::aligned16(SB))
+        return decode_tiles_bytes<false, FP4>(X, Wq, nullptr, SB, g, Y, M, N, K, st);
     GemmParams p = {};
     p.Z = SB;
     p.fp4_g = g;

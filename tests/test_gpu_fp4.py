@@ -194,11 +194,14 @@ def _nv_weights(N, K, seed):
 
 
 # 1..8 rows with K % 512 == 0 take the warp-level decode kernel (one and
-# several passes over K, ring refills, more CTAs than SMs, ragged N); the
-# others the tensor-memory tile
+# several passes over K, ring refills, more CTAs than SMs, ragged N); 9..64
+# rows with K % 256 == 0 the 256-wide decode tiles; the others the 64-wide
+# tensor-memory tile
 SHAPES = [(1, 1, 32), (1, 300, 4096), (5, 100, 128), (64, 300, 640), (65, 257, 256),
           (300, 1000, 1024), (512, 1024, 2048), (3, 129, 96), (8, 4099, 2048), (7, 1000, 1536),
-          (2, 9472, 8192), (3, 20000, 512), (1, 14212, 512), (4, 37, 4608)]
+          (2, 9472, 8192), (3, 20000, 512), (1, 14212, 512), (4, 37, 4608), (16, 300, 4096),
+          (9, 1000, 1024), (32, 4099, 2048), (64, 129, 768), (24, 12288, 4096),
+          (17, 20000, 512)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)

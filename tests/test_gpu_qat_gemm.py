@@ -177,3 +177,25 @@ def test_qat_gemm_dx_matches_fake_quant_then_gemm_and_is_deterministic():
     Wdq_gpu = bits(w4.fake_quant(Wd))
     _, R = oracle.gemm(bits(dY), np.ascontiguousarray(Wdq_gpu.T))
     assert_gemm_close(a, R, "fused dx vs materialized")
+
+
+def test_qat_gemms_one_hot_several_token_tiles():
+    """More than 256 tokens run several 256-token work items per weight tile
+    (the forward with the QDQ written back over the weight tile, both with two
+    accumulator sets): one-hot rows give fake_quant(W) bit for bit across the
+    items and the ragged end."""
+    N, K, M = 384, 512, 320
+    W = synth.normal_bf16((N, K), 0.02, seed=17, outlier_frac=0.01).clone()
+    W[7, 32:64] = 1e-39                                   # subnormal scale
+    W[9, 64:96] = 0.0
+    Wdq, _ = oracle.fake_quant(bits(W))
+    Wd = W.to(DEV)
+    X = torch.zeros((M, K), dtype=torch.bfloat16)
+    X[torch.arange(M), torch.arange(M)] = 1.0
+    Y = bits(w4.qat_gemm(X.to(DEV), Wd))                  # Y[m, n] = Wdq[n, m]
+    assert np.array_equal(Y, Wdq[:, :M].T)
+    dY = torch.zeros((M, N), dtype=torch.bfloat16)
+    dY[torch.arange(M), torch.arange(M)] = 1.0
+    dX = bits(w4.qat_gemm_dx(dY.to(DEV), Wd))             # dX[m, :] = Wdq[m, :]
+    assert np.array_equal(dX, Wdq[:M, :])
+    w4.w4_device_status()

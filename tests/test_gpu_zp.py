@@ -53,9 +53,14 @@ def test_quantize_pack_zp_layer_shape():
     assert np.array_equal(Z.cpu().numpy(), oZ)
 
 
+# 9..64 rows with K % 256 == 0 take the 256-wide decode tiles (zero points read
+# directly by the dequant warps): 16-, 32- and 64-token tiles, ragged N and M,
+# more row tiles than SMs
 @pytest.mark.parametrize("M,N,K", [(1, 1, 64), (1, 300, 4096), (5, 100, 128), (64, 300, 640),
                                    (65, 257, 256), (300, 1000, 1024), (512, 1024, 2048),
-                                   (3, 129, 96)])
+                                   (3, 129, 96), (16, 300, 4096), (9, 1000, 1024),
+                                   (32, 4099, 2048), (64, 129, 768), (24, 12288, 4096),
+                                   (17, 20000, 512)])
 def test_gemm_zp_shapes(M, N, K):
     W = _edge_weights(N, K, seed=M + N + K)
     X = synth.normal_bf16((M, K), 1.0, seed=M + 7)
