@@ -204,7 +204,8 @@ w4_status w4a16_gemm_noalloc(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 
  * group must be 32; 16-byte aligned, contiguous rows.
  */
 w4_status w4_qat_gemm(const w4_bf16 *X, const w4_bf16 *W, w4_bf16 *Y, int64_t M, int64_t N,
-                      int64_t K, int group, void *stream);
+                      int64_t K, int group, void *workspace, size_t workspace_bytes,
+                      void *stream);
 
 /*
  * QAT input gradient with the same fusion -- [QAT] fake quantization with a
@@ -220,7 +221,19 @@ w4_status w4_qat_gemm(const w4_bf16 *X, const w4_bf16 *W, w4_bf16 *Y, int64_t M,
  * aligned, contiguous rows.  N == 0 writes dX = 0.
  */
 w4_status w4_qat_gemm_dx(const w4_bf16 *dY, const w4_bf16 *W, w4_bf16 *dX, int64_t M, int64_t N,
-                         int64_t K, int group, void *stream);
+                         int64_t K, int group, void *workspace, size_t workspace_bytes,
+                         void *stream);
+
+/* Bytes of workspace the split schedule of the QAT GEMMs uses: up to 256 tokens
+ * in one token tile and fewer 128-row output tiles than half the SMs (rows = N for
+ * w4_qat_gemm, K for w4_qat_gemm_dx; contraction = K, resp. N) cut the
+ * (row tile, 64-wide k-block) units evenly over the SMs and add the parked
+ * FP32 partial sums in ascending k order (deterministic), as w4a16_gemm's
+ * split does; 0 when the shape runs unsplit.  The workspace follows
+ * w4a16_gemm's rules (256-byte aligned, all zero before its first use, left
+ * with its counters zero; NULL or too small: unsplit, same results within
+ * the GEMM tolerance).  Host-only. */
+size_t w4_qat_gemm_workspace_bytes(int64_t M, int64_t rows, int64_t contraction);
 
 /*
  * Asymmetric (zero-point) groups -- [BAS] §2.1 (affine map q = clamp(round(x/s)

@@ -29,6 +29,7 @@ __all__ = [
     "w4_quantize_pack", "w4_dequant", "w4a16_gemm", "w4_moe_capacity", "w4_moe_align",
     "w4_moe_w4a16_gemm", "w4_moe_w4a16_gemm_silu", "w4_moe_gate_topk", "w4_moe_block_size",
     "w4_silu_mul", "moe_gemm_silu", "w4_qat_gemm", "qat_gemm", "w4_qat_gemm_dx", "qat_gemm_dx",
+    "w4_qat_gemm_workspace_bytes",
     "w4_quantize_pack_zp", "w4_dequant_zp", "w4a16_gemm_zp", "quantize_pack_zp", "dequant_zp",
     "gemm_zp",
     "w4_quantize_pack_mxfp4", "w4_dequant_mxfp4", "w4_nvfp4_tensor_scale",
@@ -86,8 +87,8 @@ def lib() -> ctypes.CDLL:
             "w4_moe_w4a16_gemm_silu": [_P, _INT, _P, _P, _P, _P, _P, _I64, _INT, _I64, _P,
                                        _I64, _I64, _INT, _P],
             "w4_moe_gate_topk": [_P, _I64, _INT, _INT, _P, _P, _P],
-            "w4_qat_gemm": [_P, _P, _P, _I64, _I64, _I64, _INT, _P],
-            "w4_qat_gemm_dx": [_P, _P, _P, _I64, _I64, _I64, _INT, _P],
+            "w4_qat_gemm": [_P, _P, _P, _I64, _I64, _I64, _INT, _P, ctypes.c_size_t, _P],
+            "w4_qat_gemm_dx": [_P, _P, _P, _I64, _I64, _I64, _INT, _P, ctypes.c_size_t, _P],
             "w4_quantize_pack_zp": [_P, _P, _P, _P, _I64, _I64, _INT, _P],
             "w4_dequant_zp": [_P, _P, _P, _P, _I64, _I64, _INT, _P],
             "w4a16_gemm_zp": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _INT, _P],
@@ -110,6 +111,8 @@ def lib() -> ctypes.CDLL:
             f.restype = ctypes.c_int
         L.w4a16_gemm_workspace_bytes.argtypes = [_I64, _I64, _I64]
         L.w4a16_gemm_workspace_bytes.restype = ctypes.c_size_t
+        L.w4_qat_gemm_workspace_bytes.argtypes = [_I64, _I64, _I64]
+        L.w4_qat_gemm_workspace_bytes.restype = ctypes.c_size_t
         L.w4_moe_capacity.argtypes = [_I64, _INT, _INT, _INT]
         L.w4_moe_capacity.restype = ctypes.c_int64
         L.w4_moe_block_size.argtypes = [_I64, _INT, _INT]
@@ -359,7 +362,19 @@ def w4_moe_w4a16_gemm_silu(A, a_row_div: int, Wq, S, sorted_ids, expert_ids, num
         _stream(stream)))
 
 
-def w4_qat_gemm(X, W, Y, group: int = GROUP, stream=None) -> None:
+def _ws_args(ws, need: int, device):
+    """ws: "auto" (the module's zeroed per-device buffer), None, or a zeroed
+    uint8 CUDA tensor -> (pointer, bytes)."""
+    if isinstance(ws, str):
+        ws = workspace(device, need) if need > 0 else None
+    return (_ptr(ws), ws.numel() * ws.element_size()) if ws is not None else (None, 0)
+
+
+def w4_qat_gemm_workspace_bytes(M: int, rows: int, contraction: int) -> int:
+    return int(lib().w4_qat_gemm_workspace_bytes(M, rows, contraction))
+
+
+def w4_qat_gemm(X, W, Y, group: int = GROUP, ws="auto", stream=None) -> None:
     """Y = X . fake_quant(W)^T, the QDQ fused into the GEMM's weight prologue."""
     _dtype(X, torch.bfloat16, "X")
     M, K = X.shape
@@ -367,11 +382,12 @@ def w4_qat_gemm(X, W, Y, group: int = GROUP, stream=None) -> None:
     N = W.shape[0]
     _arg(W, torch.bfloat16, (N, K), "W")
     _arg(Y, torch.bfloat16, (M, N), "Y")
-    _check("w4_qat_gemm", lib().w4_qat_gemm(_ptr(X), _ptr(W), _ptr(Y), M, N, K, group,
-                                            _stream(stream)))
+    wptr, wbytes = _ws_args(ws, w4_qat_gemm_workspace_bytes(M, N, K), X.device)
+    _check("w4_qat_gemm", lib().w4_qat_gemm(_ptr(X), _ptr(W), _ptr(Y), M, N, K, group, wptr,
+                                            wbytes, _stream(stream)))
 
 
-def w4_qat_gemm_dx(dY, W, dX, group: int = GROUP, stream=None) -> None:
+def w4_qat_gemm_dx(dY, W, dX, group: int = GROUP, ws="auto", stream=None) -> None:
     """dX = dY . fake_quant(W), the QDQ fused into the GEMM's weight prologue."""
     _dtype(dY, torch.bfloat16, "dY")
     M, N = dY.shape
@@ -379,8 +395,9 @@ def w4_qat_gemm_dx(dY, W, dX, group: int = GROUP, stream=None) -> None:
     K = W.shape[1]
     _arg(W, torch.bfloat16, (N, K), "W")
     _arg(dX, torch.bfloat16, (M, K), "dX")
+    wptr, wbytes = _ws_args(ws, w4_qat_gemm_workspace_bytes(M, K, N), dY.device)
     _check("w4_qat_gemm_dx", lib().w4_qat_gemm_dx(_ptr(dY), _ptr(W), _ptr(dX), M, N, K, group,
-                                                  _stream(stream)))
+                                                  wptr, wbytes, _stream(stream)))
 
 
 def w4_quantize_pack_zp(W, Wq, S, Z, group: int = GROUP, stream=None) -> None:
@@ -667,15 +684,15 @@ def moe_gemm_silu(A, a_row_div, Wq, S, sorted_ids, expert_ids, num_post_pad, blo
     return H
 
 
-def qat_gemm(X: torch.Tensor, W: torch.Tensor) -> torch.Tensor:
+def qat_gemm(X: torch.Tensor, W: torch.Tensor, ws="auto") -> torch.Tensor:
     Y = torch.empty((X.shape[0], W.shape[0]), dtype=torch.bfloat16, device=X.device)
-    w4_qat_gemm(X, W, Y)
+    w4_qat_gemm(X, W, Y, ws=ws)
     return Y
 
 
-def qat_gemm_dx(dY: torch.Tensor, W: torch.Tensor) -> torch.Tensor:
+def qat_gemm_dx(dY: torch.Tensor, W: torch.Tensor, ws="auto") -> torch.Tensor:
     dX = torch.empty((dY.shape[0], W.shape[1]), dtype=torch.bfloat16, device=dY.device)
-    w4_qat_gemm_dx(dY, W, dX)
+    w4_qat_gemm_dx(dY, W, dX, ws=ws)
     return dX
 
 

@@ -27,12 +27,15 @@
 //    E2M1 conversion (cvt.rn.satfinite.e2m1x2.f32) rounds it to nearest even
 //    with saturation; -0 codes are cleared to +0.
 //  * NVFP4: the group scale is the IEEE FP64 quotient amax / (6 g) rounded to
-//    E4M3 from its bits; each element compares |w| with the rounding
-//    thresholds t * s * g (t in 0.25, 0.75, ..., 5), which are exact in FP64
-//    (3 + 4 + 24 significant bits).  That is the same decision as rounding the
-//    quotient w / (s g): an 8-bit w over a 28-bit step is either exactly a
-//    threshold or at least 2^-31 relative away from it, far more than one
-//    FP64 rounding.
+//    E4M3 from its bits; an element's code is the hardware E2M1 rounding of
+//    w * fl32(1 / (s g)) when the rounding of that FP32 quotient scaled by
+//    1 - 2^-19 and by 1 + 2^-19 agree (the quotient is then at least that far
+//    from every rounding midpoint, and its error is below 2^-22); otherwise
+//    |w| is compared with the rounding thresholds t * s * g (t in 0.25, 0.75,
+//    ..., 5), which are exact in FP64 (3 + 4 + 24 significant bits).  That is
+//    the same decision as rounding the quotient w / (s g): an 8-bit w over a
+//    28-bit step is either exactly a threshold or at least 2^-31 relative away
+//    from it, far more than one FP64 rounding.
 #include <algorithm>
 
 #include "w4_common.cuh"
@@ -227,6 +230,15 @@ __global__ void __launch_bounds__(kThreads) quant_nvfp4_kernel(const uint4 *__re
             const double tq[7] = {0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0};
 #pragma unroll
             for (int i = 0; i < 7; ++i) th[i] = tq[i] * step;   // exact
+            // Fast path: r = w * fl32(1 / step) in FP32 is within 2^-22 of w /
+            // step (relative); rounding r * (1 -+ 2^-19) with the hardware E2M1
+            // conversion gives the same code at both ends unless the exact
+            // quotient is within that band of a rounding midpoint (a tie
+            // included), and then it is the code of the exact quotient.  Pairs
+            // whose two ends differ take the exact FP64 thresholds.
+            const bool fast = step > 0x1p-100;
+            const float rs = fast ? (float)(1.0 / step) : 0.0f;
+            constexpr float kLo = 1.0f - 0x1p-19f, kHi = 1.0f + 0x1p-19f;
 #pragma unroll
             for (int wd = 0; wd < 2; ++wd) {
                 uint32_t w = 0;
@@ -234,11 +246,22 @@ __global__ void __launch_bounds__(kThreads) quant_nvfp4_kernel(const uint4 *__re
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         const uint32_t x = v[8 * h + 4 * wd + k];
-                        w |= e2m1_code_thresholds(bf16_lo(x), th) << (8 * k);
-                        w |= e2m1_code_thresholds(bf16_hi(x), th) << (8 * k + 4);
+                        const float a = bf16_lo(x), b = bf16_hi(x);
+                        uint32_t byte;
+                        bool exact = !fast;
+                        if (fast) {
+                            const float ra = __fmul_rn(a, rs), rb = __fmul_rn(b, rs);
+                            const uint32_t lo = e2m1x2_from_f32(__fmul_rn(ra, kLo), __fmul_rn(rb, kLo));
+                            const uint32_t hi = e2m1x2_from_f32(__fmul_rn(ra, kHi), __fmul_rn(rb, kHi));
+                            byte = lo;
+                            exact = lo != hi;
+                        }
+                        if (exact)
+                            byte = e2m1_code_thresholds(a, th) | (e2m1_code_thresholds(b, th) << 4);
+                        w |= byte << (8 * k);
                     }
                 }
-                words[2 * h + wd] = w;
+                words[2 * h + wd] = clear_negative_zeros(w);
             }
         }
         __stcs(Wq + gp, make_uint4(words[0], words[1], words[2], words[3]));

@@ -1515,13 +1515,74 @@ extern "C" w4_status w4a16_gemm(const w4_bf16 *X, const int32_t *Wq, const w4_bf
                                                                                (int)items, st);
 }
 
+namespace w4 {
+namespace {
+
+// Stream-K plan for a QAT GEMM with a single token tile (M <= 256): the
+// (128-row tile, 64-wide k-block) units cut evenly over the SMs, as in the
+// decode split, when the row tiles alone would leave most SMs idle (fewer than
+// half the SMs: measured, the split costs more than it gains above that, e.g.
+// the forward at 96 row tiles and 256 tokens).
+bool plan_split_qat(int64_t M, int64_t rows, int64_t contraction, int sms, SplitPlan *sp) {
+    if (M > 256) return false;
+    const int64_t n_rt = (rows + 127) / 128, nkb = (contraction + 63) / 64;
+    if (2 * n_rt > sms || nkb < 2 || n_rt > kSplitMaxRowTiles) return false;
+    const int64_t units = n_rt * nkb;
+    const int ctas = (int)std::min<int64_t>(sms, units);
+    if (units * (ctas + 1) >= ((int64_t)1 << 32)) return false;
+    auto owner = [&](int64_t x) { return (int)(((x + 1) * ctas - 1) / units); };
+    int mc = 1;
+    for (int64_t rt = 0; rt < n_rt; ++rt)
+        mc = std::max(mc, owner(rt * nkb + nkb - 1) - owner(rt * nkb) + 1);
+    sp->n_rt = (int)n_rt;
+    sp->nkb = (int)nkb;
+    sp->ctas = ctas;
+    sp->max_contrib = mc;
+    sp->mt = M <= 64 ? 64 : 256;
+    sp->cnt_bytes = kSplitCntBytes;
+    sp->part_bytes = (size_t)n_rt * mc * 128 * sp->mt * sizeof(float);
+    return true;
+}
+
+// Applies a QAT split plan to the kernel parameters (false: run unsplit).
+bool use_split_qat(GemmParams &p, int64_t M, int64_t rows, int64_t contraction, void *workspace,
+                   size_t workspace_bytes, int *items) {
+    SplitPlan sp;
+    if (workspace == nullptr ||
+        !plan_split_qat(M, rows, contraction, w4host::num_sms(), &sp) ||
+        workspace_bytes < sp.cnt_bytes + sp.part_bytes)
+        return false;
+    p.n_row_tiles = sp.n_rt;
+    p.split = 1;
+    p.units = (int64_t)sp.n_rt * sp.nkb;
+    p.ctas = sp.ctas;
+    p.max_contrib = sp.max_contrib;
+    p.ws_cnt = reinterpret_cast<unsigned int *>(workspace);
+    p.ws_part = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + sp.cnt_bytes);
+    *items = sp.ctas;
+    return true;
+}
+
+}  // namespace
+}  // namespace w4
+
+extern "C" size_t w4_qat_gemm_workspace_bytes(int64_t M, int64_t rows, int64_t contraction) {
+    SplitPlan sp;
+    if (M <= 0 || rows <= 0 || contraction <= 0) return 0;
+    if (!plan_split_qat(M, rows, contraction, w4host::num_sms(), &sp)) return 0;
+    return sp.cnt_bytes + sp.part_bytes;
+}
+
 extern "C" w4_status w4_qat_gemm(const w4_bf16 *X, const w4_bf16 *W, w4_bf16 *Y, int64_t M,
-                                 int64_t N, int64_t K, int group, void *stream) {
+                                 int64_t N, int64_t K, int group, void *workspace,
+                                 size_t workspace_bytes, void *stream) {
     if (group != 32) return W4_ERR_UNSUPPORTED;
     if (M < 0 || N < 0 || K <= 0 || (K % 32) != 0) return W4_ERR_INVALID_ARG;
     if (!w4host::aligned16(X) || !w4host::aligned16(W) || !w4host::aligned16(Y))
         return W4_ERR_INVALID_ARG;
     if ((K % 64) != 0) return W4_ERR_UNSUPPORTED;
+    if (workspace != nullptr && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return W4_ERR_INVALID_ARG;
     if (M == 0 || N == 0) return W4_OK;
     if (N > (1 << 30) || M > (1 << 30) || K > (1 << 24)) return W4_ERR_UNSUPPORTED;
     cudaStream_t st = (cudaStream_t)stream;
@@ -1532,10 +1593,10 @@ extern "C" w4_status w4_qat_gemm(const w4_bf16 *X, const w4_bf16 *W, w4_bf16 *Y,
     p.K = K;
     // more than 64 tokens: 256-token work items with the QDQ written back over
     // the weight tile (A from shared memory), which leaves tensor memory to two
-    // accumulator sets, so one item's epilogue overlaps the next item's MMAs --
-    // unless 256-token items would leave SMs idle (64-token items then)
-    int mt = M <= 64 ? 64 : 256;
-    if (mt == 256 && (int64_t)ceil_div_i(N, 128) * ceil_div_i(M, 256) < w4host::num_sms()) mt = 64;
+    // accumulator sets, so one item's epilogue overlaps the next item's MMAs
+    // (64-token items to fill idle SMs measured slower: each token tile pays
+    // the QDQ of every weight tile again)
+    const int mt = M <= 64 ? 64 : 256;
     p.rows_per_tile = 128;
     p.n_row_tiles = ceil_div_i(N, 128);
     p.n_tok_tiles = ceil_div_i(M, mt);
@@ -1559,21 +1620,26 @@ extern "C" w4_status w4_qat_gemm(const w4_bf16 *X, const w4_bf16 *W, w4_bf16 *Y,
                       CU_TENSOR_MAP_SWIZZLE_128B))
             return W4_ERR_CUDA;
     }
-    const int64_t items = (int64_t)p.n_row_tiles * p.n_tok_tiles;
-    if (items > (1 << 30)) return W4_ERR_UNSUPPORTED;
+    if ((int64_t)p.n_row_tiles * p.n_tok_tiles > (1 << 30)) return W4_ERR_UNSUPPORTED;
+    int items = p.n_row_tiles * p.n_tok_tiles;
+    // one token tile and fewer row tiles than SMs: stream-K over the k-blocks
+    use_split_qat(p, M, N, K, workspace, workspace_bytes, &items);
     if (mt == 64)
-        return launch_cfg<64, 64, 8, 1, 8, 4, 2, false, false, 1>(tw, ts, tx, p, (int)items, st);
-    return launch_cfg<64, 256, 4, 2, 4, 2, 2, false, false, 3, false, true>(tw, ts, tx, p,
-                                                                           (int)items, st);
+        return launch_cfg<64, 64, 8, 1, 8, 4, 2, false, false, 1>(tw, ts, tx, p, items, st);
+    return launch_cfg<64, 256, 4, 2, 4, 2, 2, false, false, 3, false, true>(tw, ts, tx, p, items,
+                                                                           st);
 }
 
 extern "C" w4_status w4_qat_gemm_dx(const w4_bf16 *dY, const w4_bf16 *W, w4_bf16 *dX, int64_t M,
-                                    int64_t N, int64_t K, int group, void *stream) {
+                                    int64_t N, int64_t K, int group, void *workspace,
+                                    size_t workspace_bytes, void *stream) {
     if (group != 32) return W4_ERR_UNSUPPORTED;
     if (M < 0 || N < 0 || K <= 0 || (K % 32) != 0) return W4_ERR_INVALID_ARG;
     if (!w4host::aligned16(dY) || !w4host::aligned16(W) || !w4host::aligned16(dX))
         return W4_ERR_INVALID_ARG;
     if ((K % 64) != 0 || (N % 8) != 0) return W4_ERR_UNSUPPORTED;
+    if (workspace != nullptr && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return W4_ERR_INVALID_ARG;
     if (M == 0) return W4_OK;
     if (N > (1 << 24) || M > (1 << 30) || K > (1 << 30)) return W4_ERR_UNSUPPORTED;
     cudaStream_t st = (cudaStream_t)stream;
@@ -1585,8 +1651,7 @@ extern "C" w4_status w4_qat_gemm_dx(const w4_bf16 *dY, const w4_bf16 *W, w4_bf16
     p.M = M;
     p.N = K;
     p.K = N;
-    int mt = M <= 64 ? 64 : 256;
-    if (mt == 256 && (int64_t)ceil_div_i(K, 128) * ceil_div_i(M, 256) < w4host::num_sms()) mt = 64;
+    const int mt = M <= 64 ? 64 : 256;
     p.rows_per_tile = 128;
     p.n_row_tiles = ceil_div_i(K, 128);
     p.n_tok_tiles = ceil_div_i(M, mt);
@@ -1611,14 +1676,17 @@ extern "C" w4_status w4_qat_gemm_dx(const w4_bf16 *dY, const w4_bf16 *W, w4_bf16
                       CU_TENSOR_MAP_SWIZZLE_128B))
             return W4_ERR_CUDA;
     }
-    const int64_t items = (int64_t)p.n_row_tiles * p.n_tok_tiles;
-    if (items > (1 << 30)) return W4_ERR_UNSUPPORTED;
+    if ((int64_t)p.n_row_tiles * p.n_tok_tiles > (1 << 30)) return W4_ERR_UNSUPPORTED;
+    int items = p.n_row_tiles * p.n_tok_tiles;
+    // one token tile and fewer row tiles than SMs (K = 4096 has only 32):
+    // stream-K over the contraction
+    use_split_qat(p, M, K, N, workspace, workspace_bytes, &items);
     if (mt == 64)
-        return launch_cfg<64, 64, 4, 1, 4, 4, 2, false, false, 2>(tw, ts, tx, p, (int)items, st);
+        return launch_cfg<64, 64, 4, 1, 4, 4, 2, false, false, 2>(tw, ts, tx, p, items, st);
     // two accumulator sets (A is in shared memory), two issuers over the
     // 256 tokens
-    return launch_cfg<64, 256, 3, 2, 3, 2, 2, false, false, 2, false, true>(tw, ts, tx, p,
-                                                                           (int)items, st);
+    return launch_cfg<64, 256, 3, 2, 3, 2, 2, false, false, 2, false, true>(tw, ts, tx, p, items,
+                                                                           st);
 }
 
 namespace w4 {

@@ -138,11 +138,15 @@ def test_moe_glue_validation_host_only():
 
 def test_qat_gemm_validation_host_only():
     L = w4.lib()
-    assert L.w4_qat_gemm(A16, A16, A16, 4, 8, 64, 64, None) == 2      # group != 32
-    assert L.w4_qat_gemm(A16, A16, A16, 4, 8, 48, 32, None) == 1      # K % 32 != 0
-    assert L.w4_qat_gemm(A16, A16, A16, 4, 8, 96, 32, None) == 2      # K % 64 != 0
-    assert L.w4_qat_gemm(MIS, A16, A16, 4, 8, 64, 32, None) == 1      # misaligned X
-    assert L.w4_qat_gemm(A16, A16, A16, 0, 8, 64, 32, None) == 0      # empty: no launch
+    assert L.w4_qat_gemm(A16, A16, A16, 4, 8, 64, 64, None, 0, None) == 2      # group != 32
+    assert L.w4_qat_gemm(A16, A16, A16, 4, 8, 48, 32, None, 0, None) == 1      # K % 32 != 0
+    assert L.w4_qat_gemm(A16, A16, A16, 4, 8, 96, 32, None, 0, None) == 2      # K % 64 != 0
+    assert L.w4_qat_gemm(MIS, A16, A16, 4, 8, 64, 32, None, 0, None) == 1      # misaligned X
+    assert L.w4_qat_gemm(A16, A16, A16, 0, 8, 64, 32, None, 0, None) == 0      # empty: no launch
+    assert L.w4_qat_gemm(A16, A16, A16, 4, 8, 64, 32, A16 + 16, 4096, None) == 1  # ws not 256-aligned
+    assert L.w4_qat_gemm_dx(A16, A16, A16, 4, 8, 64, 64, None, 0, None) == 2   # group != 32
+    assert L.w4_qat_gemm_dx(A16, A16, A16, 4, 12, 64, 32, None, 0, None) == 2  # N % 8 != 0
+    assert L.w4_qat_gemm_dx(A16, A16, A16, 0, 8, 64, 32, None, 0, None) == 0   # empty: no launch
 
 
 def test_zero_point_validation_host_only():

@@ -199,3 +199,30 @@ def test_qat_gemms_one_hot_several_token_tiles():
     dX = bits(w4.qat_gemm_dx(dY.to(DEV), Wd))             # dX[m, :] = Wdq[m, :]
     assert np.array_equal(dX, Wdq[:M, :])
     w4.w4_device_status()
+
+
+@pytest.mark.parametrize("M", [1, 64, 200, 256])
+def test_qat_gemms_split_matches_unsplit(M):
+    """Up to 256 tokens the QAT GEMMs cut the (row tile, k-block) units over
+    the SMs (workspace): same product as the unsplit schedule within the GEMM
+    tolerance, deterministic, counters left zero, and against the oracle."""
+    N, K = 4096, 4096
+    assert w4.w4_qat_gemm_workspace_bytes(M, N, K) > 0          # 32 row tiles < SMs / 2
+    W = synth.normal_bf16((N, K), 0.02, seed=M, outlier_frac=0.001)
+    X = synth.normal_bf16((M, K), 1.0, seed=M + 1)
+    dY = synth.normal_bf16((M, N), 1.0, seed=M + 2)
+    Wd, Xd, dYd = W.to(DEV), X.to(DEV), dY.to(DEV)
+    ws = torch.zeros(max(w4.w4_qat_gemm_workspace_bytes(M, N, K), 256), dtype=torch.uint8,
+                     device=DEV)
+    Wdq, _ = oracle.fake_quant(bits(W))
+    Y1, Y2 = bits(w4.qat_gemm(Xd, Wd, ws=ws)), bits(w4.qat_gemm(Xd, Wd, ws=ws))
+    D1, D2 = bits(w4.qat_gemm_dx(dYd, Wd, ws=ws)), bits(w4.qat_gemm_dx(dYd, Wd, ws=ws))
+    w4.w4_device_status()
+    assert np.array_equal(Y1, Y2) and np.array_equal(D1, D2)
+    assert int(ws[:4096].count_nonzero()) == 0, "split counters not reset"
+    _, R = oracle.gemm(bits(X), Wdq)
+    assert_gemm_close(Y1, R, f"qat split M={M}")
+    assert_gemm_close(bits(w4.qat_gemm(Xd, Wd, ws=None)), R, f"qat unsplit M={M}")
+    _, Rd = oracle.gemm(bits(dY), np.ascontiguousarray(Wdq.T))
+    assert_gemm_close(D1, Rd, f"qat dx split M={M}")
+    assert_gemm_close(bits(w4.qat_gemm_dx(dYd, Wd, ws=None)), Rd, f"qat dx unsplit M={M}")
