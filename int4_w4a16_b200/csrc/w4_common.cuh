@@ -156,6 +156,23 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  A GEMM launched with programmatic stream
+// serialization may become resident while the kernel before it on the stream
+// still runs; it sets up its barriers and prefetches its tensor maps (kernel
+// parameters), then waits here, before its first global-memory access, until
+// that kernel has completed and its writes are visible.  Every such kernel
+// reaches the wait on every path, so completion stays transitive along the
+// stream.  The trigger lets the next kernel on the stream be scheduled as soon
+// as every CTA of this one has started.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void griddep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor), no multicast
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *m) {
@@ -604,6 +621,24 @@ inline w4_status launch_status() {
 }
 
 int num_sms();
+
+// Launch with programmatic stream serialization (the kernel must execute
+// griddep_wait() before touching global memory; see w4::griddep_wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<Args &&>(args)...);
+}
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
 CUresult encode_tiled(CUtensorMap *map, CUtensorMapDataType dtype, cuuint32_t rank,

@@ -435,6 +435,11 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
         if (KB == 256 && FP4 == 0) tma_prefetch_desc(&tm_s);
         if (!MOE) tma_prefetch_desc(&tm_x);
     }
+    // the kernel before this one on the stream may still be running: no global
+    // memory (and no tensor memory, which a co-resident CTA of it may hold)
+    // is touched before it completes
+    griddep_wait();
+    griddep_launch_dependents();
     if (warp == kAllocWarp) {
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
         tmem_relinquish();
@@ -1304,7 +1309,12 @@ w4_status launch_cfg(const CUtensorMap &tw, const CUtensorMap &ts, const CUtenso
             return W4_ERR_UNSUPPORTED;
     }
     const int grid = std::max(1, std::min(num_items_max, w4host::num_sms()));
-    kern<<<grid, gemm_threads(NDQ, KB, NSPLIT, WGL), smem, stream>>>(tw, ts, tx, p);
+    const cudaError_t e = w4host::launch_pdl(kern, dim3(grid), dim3(gemm_threads(NDQ, KB, NSPLIT, WGL)),
+                                             (size_t)smem, stream, tw, ts, tx, p);
+    if (e != cudaSuccess) {
+        w4host::set_cuda_error(e);
+        return W4_ERR_CUDA;
+    }
     return w4host::launch_status();
 }
 
@@ -1496,7 +1506,7 @@ extern "C" w4_status w4a16_gemm(const w4_bf16 *X, const int32_t *Wq, const w4_bf
             if (!map_x(mt) || !map_w(256, R) || !map_s(R)) return W4_ERR_CUDA;
         }
         if (mt == 16) return launch_cfg<256, 16, 6, 2, 3, 4, 2, false, true>(tw, ts, tx, p, items, st);
-        if (mt == 32) return launch_cfg<256, 32, 6, 2, 2, 4, 2, false, true>(tw, ts, tx, p, items, st);
+        if (mt == 32) return launch_cfg<256, 32, 6, 2, 2, 4, 2, false, false>(tw, ts, tx, p, items, st);
         return launch_cfg<256, 64, 4, 1, 2, 4, 2, false>(tw, ts, tx, p, items, st);
     }
     // Prefill (and any K that is not a multiple of 256): 128-row tiles,

@@ -352,7 +352,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
     // this warp's two chunks of the activations in B-fragment order (tokens >=
     // M and K beyond the end are zero): lane (g, t) holds token g's
-    // K = 128c + 32t + 8j + (0..7).  Pass 0's requests go out first of all.
+    // K = 128c + 32t + 8j + (0..7).  Pass 0's requests go out ahead of the
+    // first weight stages.
     uint4 xr[kWarpChunks][4];
     int na = 0;
     auto load_x = [&](int pass) {
@@ -368,8 +369,6 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                                           (size_t)(c_first + cl) * kChunkK + 32 * t + 8 * j);
             }
     };
-    load_x(0);
-
 #define DEC_ISSUE(s_)                                                                        \
     dec_issue<F>(&tw, &ts, &tz, &tw4, &ts4, &tz4, smem_u32(&full_bar[0]), base, row0, cta_quads, \
                   ntiles, &issued, (s_))
@@ -384,8 +383,14 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         abort_flag = 0;
         issued = 0;
         fence_mbar_init();
-        for (int s = 0; s < min(nstages, kNStage); ++s) DEC_ISSUE(s);
     }
+    // the kernel before this one on the stream may still be running: its
+    // outputs (X among them) are read only after it completes
+    griddep_wait();
+    griddep_launch_dependents();
+    load_x(0);
+    if (threadIdx.x == 0)
+        for (int s = 0; s < min(nstages, kNStage); ++s) DEC_ISSUE(s);
     __syncthreads();
 
     bool ok = true;
@@ -536,7 +541,12 @@ w4_status dec_launch(const w4_bf16 *X, const int32_t *Wq, const w4_bf16 *S, cons
             return w4host::launch_status();
         configured = true;
     }
-    kern<<<p.ctas, kDecThreads, smem, stream>>>(tw, ts, tz, tw4, ts4, tz4, p);
+    const cudaError_t e = w4host::launch_pdl(kern, dim3(p.ctas), dim3(kDecThreads), (size_t)smem,
+                                             stream, tw, ts, tz, tw4, ts4, tz4, p);
+    if (e != cudaSuccess) {
+        w4host::set_cuda_error(e);
+        return W4_ERR_CUDA;
+    }
     return w4host::launch_status();
 }
 

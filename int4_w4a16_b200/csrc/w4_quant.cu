@@ -169,6 +169,7 @@ __global__ void __launch_bounds__(kThreads, kQuantBlocksPerSm) quant_kernel(cons
                                                          uint32_t *__restrict__ Wq,
                                                          uint16_t *__restrict__ S,
                                                          int64_t ngroups) {
+    griddep_launch_dependents();       // a GEMM after this waits for its completion
     const int64_t T = (int64_t)gridDim.x * blockDim.x;
     for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < ngroups;
          base += kGroupsInFlight * T) {
@@ -297,9 +298,21 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint4 *__restri
 //   s = bf16_rne(fl32(fl32(x_max - x_min) / 15)),
 //   z = clamp(rint_even(0 - fl32(x_min / s)), 0, 15),
 //   q = clamp(rint_even(fl32(x / s)) + z, 0, 15),   q = z = 0 when s == 0.
-// The quotients are IEEE divisions: x / s is not bounded by the group's
-// range here (a narrow group far from zero has |x / s| up to ~3840), so the
-// reciprocal-and-snap rounding of the symmetric path does not carry over.
+// The scale's quotient is an IEEE division (its numerator is any fp32
+// difference, not a BF16 value).  The per-element quotients need none: the
+// symmetric path's argument carries over with a wider range.  For a normal
+// BF16 scale, |x / s| <= 256 * 15 * (1 + 2^-8) < 3856 (two distinct BF16
+// values differ by at least 1/256 of the larger magnitude), and x / s is
+// either exactly a half-integer or more than 1/510 away from every one
+// (both operands have 8-bit significands).  So t = x * rcp.approx(s), off by
+// at most 3856 * 2^-23 < 4.6e-4, snapped to the 2^-9 grid by one fused
+// multiply-add against 1.5 * 2^14 (ulp 2^-9 on [2^14, 2^15)), lands on the
+// half-integer exactly for a tie and stays strictly on its own side
+// otherwise; adding 1.5 * 2^23 - 1.5 * 2^14 then rounds it to an integer,
+// ties to even, as rint_even(fl32(x / s)) does (fl32 moves a quotient below
+// 4096 by at most 2^-13, never onto or across a half-integer).  The zero point
+// is the same code of x_min, negated: rint_even(-v) = -rint_even(v).  Zero,
+// subnormal and huge scales (and non-finite groups) keep the IEEE divisions.
 
 __device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
     uint32_t d;
@@ -312,44 +325,83 @@ __device__ __forceinline__ uint32_t bf16x2_min(uint32_t a, uint32_t b) {
     return d;
 }
 
-// One thread per group of 32 weights: Wq (4 words), S, Z.
+constexpr float kSnapZ = 24576.0f;         // 1.5 * 2^14: ulp 2^-9 around it
+constexpr float kToIntZ = 12558336.0f;     // 1.5 * 2^23 - 1.5 * 2^14 (exact in fp32)
+
+// bits(1.5 * 2^23 + rint_even(x / s)) on the fast path (|x / s| < 4096).
+__device__ __forceinline__ uint32_t zp_code_bits(float x, float r) {
+    return __float_as_uint(__fadd_rn(__fmaf_rn(x, r, kSnapZ), kToIntZ));
+}
+
+// One group of 32 weights (16 words, natural order) -> Wq[g] (4 words), S[g], Z[g].
+__device__ __forceinline__ void quant_zp_group(const uint32_t (&v)[16], uint4 *Wq, uint16_t *S,
+                                               uint8_t *Z, int64_t g) {
+    uint32_t mx = v[0], mn = v[0];
+#pragma unroll
+    for (int j = 1; j < 16; ++j) {
+        mx = bf16x2_max(mx, v[j]);
+        mn = bf16x2_min(mn, v[j]);
+    }
+    const float xmax = fmaxf(lo_f(mx), hi_f(mx));
+    const float xmin = fminf(lo_f(mn), hi_f(mn));
+    const float s32 = __fdiv_rn(__fsub_rn(xmax, xmin), 15.0f);
+    const __nv_bfloat16 sb = __float2bfloat16_rn(s32);
+    const float s = __bfloat162float(sb);
+    uint32_t words[4] = {0u, 0u, 0u, 0u};
+    uint32_t z = 0u;
+    if (s >= 1.17549435e-38f && s <= 1.2676506e30f) {
+        const float r = rcp_approx(s);
+        // z = clamp(-rint_even(x_min / s), 0, 15); codes relative to 1.5 * 2^23
+        z = (uint32_t)__vimin_s32_relu((int)(0x4B400000u - zp_code_bits(xmin, r)), 15);
+        const uint32_t zoff = z - 0x4B400000u;
+        const uint64_t r2 = f2_splat(r), snap2 = f2_splat(kSnapZ), toint2 = f2_splat(kToIntZ);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const uint64_t c = f2_add(f2_fma(f2_from_bf16x2(v[j]), r2, snap2), toint2);
+            const uint32_t q0 = (uint32_t)__vimin_s32_relu((int)((uint32_t)c + zoff), 15);
+            const uint32_t q1 = (uint32_t)__vimin_s32_relu((int)((uint32_t)(c >> 32) + zoff), 15);
+            words[j >> 2] |= (q0 | (q1 << 4)) << (8 * (j & 3));
+        }
+    } else if (s != 0.0f) {
+        const float zf = fminf(fmaxf(rintf(__fsub_rn(0.0f, __fdiv_rn(xmin, s))), 0.0f), 15.0f);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const float x2[2] = {lo_f(v[j]), hi_f(v[j])};
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float c = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(x2[h], s)), zf), 0.0f), 15.0f);
+                const int i = 2 * j + h;               // element of the group
+                words[i >> 3] |= (uint32_t)c << (4 * (i & 7));
+            }
+        }
+        z = (uint32_t)zf;
+    }
+    __stcs(Wq + g, make_uint4(words[0], words[1], words[2], words[3]));
+    S[g] = *reinterpret_cast<const uint16_t *>(&sb);
+    Z[g] = (uint8_t)z;
+}
+
+// One thread per group of 32 weights, two groups in flight per thread.
 template <bool V8>
 __global__ void __launch_bounds__(kThreads, kQuantBlocksPerSm)
     quant_zp_kernel(const uint32_t *__restrict__ W, uint4 *__restrict__ Wq,
                     uint16_t *__restrict__ S, uint8_t *__restrict__ Z, int64_t ngroups) {
+    griddep_launch_dependents();       // a GEMM after this waits for its completion
     const int64_t T = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < ngroups; g += T) {
-        uint32_t v[16];
-        load_group<V8>(W + 16 * g, v);
-        uint32_t mx = v[0], mn = v[0];
+    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < ngroups;
+         base += kGroupsInFlight * T) {
+        uint32_t v[kGroupsInFlight][16];
 #pragma unroll
-        for (int j = 1; j < 16; ++j) {
-            mx = bf16x2_max(mx, v[j]);
-            mn = bf16x2_min(mn, v[j]);
+        for (int u = 0; u < kGroupsInFlight; ++u) {
+            const int64_t g = base + u * T;
+            if (g < ngroups) load_group<V8>(W + 16 * g, v[u]);
         }
-        const float xmax = fmaxf(lo_f(mx), hi_f(mx));
-        const float xmin = fminf(lo_f(mn), hi_f(mn));
-        const float s32 = __fdiv_rn(__fsub_rn(xmax, xmin), 15.0f);
-        const __nv_bfloat16 sb = __float2bfloat16_rn(s32);
-        const float s = __bfloat162float(sb);
-        uint32_t words[4] = {0u, 0u, 0u, 0u};
-        float zf = 0.0f;
-        if (s != 0.0f) {
-            zf = fminf(fmaxf(rintf(__fsub_rn(0.0f, __fdiv_rn(xmin, s))), 0.0f), 15.0f);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const float x2[2] = {lo_f(v[j]), hi_f(v[j])};
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const float c = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(x2[h], s)), zf), 0.0f), 15.0f);
-                    const int i = 2 * j + h;               // element of the group
-                    words[i >> 3] |= (uint32_t)c << (4 * (i & 7));
-                }
-            }
+        for (int u = 0; u < kGroupsInFlight; ++u) {
+            const int64_t g = base + u * T;
+            if (g >= ngroups) break;
+            quant_zp_group(v[u], Wq, S, Z, g);
         }
-        __stcs(Wq + g, make_uint4(words[0], words[1], words[2], words[3]));
-        S[g] = *reinterpret_cast<const uint16_t *>(&sb);
-        Z[g] = (uint8_t)zf;
     }
 }
 
@@ -481,7 +533,7 @@ extern "C" w4_status w4_quantize_pack_zp(const w4_bf16 *W, int32_t *Wq, w4_bf16 
     if (!w4host::aligned16(S) || Z == nullptr) return W4_ERR_INVALID_ARG;
     const int64_t ngroups = rows * K / 32;
     if (ngroups == 0) return W4_OK;
-    const int grid = grid_for(ngroups, 1);
+    const int grid = grid_for(ngroups, kGroupsInFlight);
     const uint32_t *w = reinterpret_cast<const uint32_t *>(W);
     uint4 *q = reinterpret_cast<uint4 *>(Wq);
     uint16_t *s = reinterpret_cast<uint16_t *>(S);

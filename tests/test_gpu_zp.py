@@ -27,6 +27,26 @@ def _edge_weights(N, K, seed):
         W[5, 160:192] = torch.linspace(100.0, 100.5, 32).to(torch.bfloat16)  # narrow, far from 0
         W[6, 192:224] = 1e-39 * torch.linspace(-1, 1, 32).to(torch.bfloat16)  # subnormal range
         W[7, 224:256] = torch.tensor([0.25 * (i % 7 - 3) for i in range(32)]).to(torch.bfloat16)
+    if N > 13:
+        t = 2.0 ** -126
+        groups = {
+            # s = 1, z = 7: exact ties x / s = k + 1/2 of both parities
+            8: [-7.0, 8.0] + [k + 0.5 for k in range(-7, 8)] + [float(k) for k in range(-6, 8)] + [0.0],
+            # s = 0.5, z = 7: ties at odd multiples of 0.25
+            9: [-3.5, 4.0] + [0.25 * (2 * k + 1) for k in range(-7, 8)] + [0.5 * k for k in range(-6, 8)] + [0.0],
+            # s = 1.5 (significand 192): ties at odd multiples of 0.75
+            10: [-10.5, 12.0] + [0.75 * (2 * k + 1) for k in range(-7, 8)] + [1.5 * k for k in range(-6, 8)] + [0.0],
+            # all negative: z = 15, ties below zero
+            11: [-15.0, 0.0] + [-(k + 0.5) for k in range(15)] + [-float(k) for k in range(1, 15)] + [-7.0],
+            # s = 2^-126, the smallest scale of the reciprocal path: ties of subnormal weights
+            12: [0.0, 15 * t] + [(k + 0.5) * t for k in range(15)] + [k * t for k in range(1, 15)] + [7 * t],
+            # s = 2^101, above the reciprocal path's range: IEEE divisions
+            13: [-7 * 2.0 ** 101, 8 * 2.0 ** 101] + [(k + 0.5) * 2.0 ** 101 for k in range(-7, 8)]
+                + [k * 2.0 ** 101 for k in range(-6, 8)] + [0.0],
+        }
+        for row, vals in groups.items():
+            assert len(vals) == 32
+            W[row, 0:32] = torch.tensor(vals, dtype=torch.float64).to(torch.bfloat16)
     return W
 
 

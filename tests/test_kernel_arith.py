@@ -13,6 +13,11 @@ cast to float32 is the single rounding of the fused operation.
    other BF16/BF16 quotient (at least 1/510 from any half-integer) on its side;
    the add then rounds to an integer, ties to even.  Checked on every BF16
    magnitude below 128 group maxima, with the reciprocal perturbed both ways.
+3. The zero-point quantizer's codes rint_half_even(fl32(x / s)), |x / s| < 3856,
+   are formed the same way on the 2^-9 grid (snap constant 1.5*2^14).  Checked
+   for every finite BF16 x in that range against every BF16 significand of s at
+   three exponents (the subnormal edge, 1, 2^90), with every fp32 reciprocal
+   within one ulp of 1/s and with a two-ulp perturbation both ways.
 """
 import numpy as np
 import pytest
@@ -59,6 +64,31 @@ def test_snap_rounding_matches_ieee_quotient(rel):
         # the code is the low byte of the float's bits
         low = (c.view(np.uint32) & 0xFF).astype(np.uint8).view(np.int8)
         assert np.array_equal(low.astype(np.float64), ref)
+
+
+SNAP_Z = 24576.0                  # 1.5 * 2^14: ulp 2^-9 on [2^14, 2^15)
+TOINT_Z = 12582912.0 - 24576.0    # 1.5 * 2^23 - 1.5 * 2^14
+
+
+@pytest.mark.parametrize("s_exp", [-126, 0, 90])
+def test_zero_point_snap_rounding_matches_ieee_quotient(s_exp):
+    finite = np.arange(0, 0x7F80, dtype=np.uint32)
+    mags = (finite << 16).view(np.float32).astype(np.float64)
+    allx = np.concatenate([mags, -mags[1:]])
+    for S in range(128, 256):
+        s = S * 2.0 ** (s_exp - 7)                     # a normal BF16 scale
+        x = allx[np.abs(allx) <= 3856.0 * s]
+        ref = np.rint((x.astype(np.float32) / F32(s)).astype(np.float64))
+        r0 = F32(1.0 / s)
+        rs = [np.nextafter(r0, F32(0)), r0, np.nextafter(r0, F32(np.inf)),
+              F32(float(r0) * (1.0 + 2.0 ** -22)), F32(float(r0) * (1.0 - 2.0 ** -22))]
+        for r in rs:
+            # fma(x, r, 1.5*2^14) lies in [2^14, 2^15): its one rounding puts
+            # x*r (exact in float64) on the 2^-9 grid, ties to even
+            k = np.rint(x * float(r) * 512.0)
+            c = _f32(SNAP_Z + k / 512.0 + TOINT_Z)       # fadd: round to an integer
+            q = c.astype(np.float64) - MAGIC
+            assert np.array_equal(q, ref), (S, float(r))
 
 
 def _bf16_rne(x64: np.ndarray) -> np.ndarray:
