@@ -26,16 +26,20 @@
 //    below the first rounding threshold 0.25 can underflow), and the hardware
 //    E2M1 conversion (cvt.rn.satfinite.e2m1x2.f32) rounds it to nearest even
 //    with saturation; -0 codes are cleared to +0.
-//  * NVFP4: the group scale is the IEEE FP64 quotient amax / (6 g) rounded to
-//    E4M3 from its bits; an element's code is the hardware E2M1 rounding of
-//    w * fl32(1 / (s g)) when the rounding of that FP32 quotient scaled by
-//    1 - 2^-19 and by 1 + 2^-19 agree (the quotient is then at least that far
-//    from every rounding midpoint, and its error is below 2^-22); otherwise
-//    |w| is compared with the rounding thresholds t * s * g (t in 0.25, 0.75,
-//    ..., 5), which are exact in FP64 (3 + 4 + 24 significant bits).  That is
-//    the same decision as rounding the quotient w / (s g): an 8-bit w over a
-//    28-bit step is either exactly a threshold or at least 2^-31 relative away
-//    from it, far more than one FP64 rounding.
+//  * NVFP4: both decisions take an FP32 quotient with a relative error below
+//    2^-22 and round it, with the hardware conversion, scaled by 1 - 2^-b and
+//    by 1 + 2^-b; when the two agree the exact quotient lies between them, so
+//    that is its rounding (a tie, or any quotient within the band of a
+//    rounding midpoint, gives two different codes).  Otherwise the decision is
+//    taken exactly in FP64.  The group scale: amax * fl32(1 / fl32(6 g)) with
+//    b = 20 through the E4M3 conversion (nearest even, saturating at 448),
+//    else the IEEE FP64 quotient amax / (6 g) rounded to E4M3 from its bits.
+//    An element: w * fl32(1 / fl32(s g)) with b = 19 through the E2M1
+//    conversion, else |w| compared with the rounding thresholds t * s * g
+//    (t in 0.25, 0.75, ..., 5), which are exact in FP64 (3 + 4 + 24
+//    significant bits).  That is the same decision as rounding the quotient
+//    w / (s g): an 8-bit w over a 28-bit step is either exactly a threshold or
+//    at least 2^-31 relative away from it, far more than one FP64 rounding.
 #include <algorithm>
 
 #include "w4_common.cuh"
@@ -134,16 +138,42 @@ __global__ void __launch_bounds__(kThreads) dequant_mxfp4_kernel(const uint4 *__
 // ---- NVFP4 ------------------------------------------------------------------
 // Tensor amax: the largest |w| as BF16 bits (sign cleared), max-reduced into
 // *amax_bits (zeroed by the host first).
-__global__ void __launch_bounds__(kThreads) amax_bf16_kernel(const uint32_t *__restrict__ W,
+// W is 4-byte aligned: the pairs before its first 16-byte boundary and after
+// the last whole 16 bytes are read one word at a time, the rest 16 bytes at a
+// time, four loads in flight per thread.  Non-negative BF16 values order like
+// their bits, so the max is a per-half unsigned max.
+__global__ void __launch_bounds__(kThreads, 4) amax_bf16_kernel(const uint32_t *__restrict__ W,
                                                              int64_t n_pairs,
                                                              const uint16_t *__restrict__ tail,
                                                              unsigned int *amax_bits) {
     const int64_t T = (int64_t)gridDim.x * blockDim.x;
-    uint32_t m = 0;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_pairs; i += T) {
-        const uint32_t a = __ldcs(W + i) & 0x7FFF7FFFu;
-        m = max(m, max(a & 0xFFFFu, a >> 16));
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t head =
+        min(n_pairs, (int64_t)(((16u - (uint32_t)(reinterpret_cast<uintptr_t>(W) & 15u)) & 15u) / 4u));
+    const int64_t n16 = (n_pairs - head) / 4;
+    const uint4 *W4 = reinterpret_cast<const uint4 *>(W + head);
+    uint32_t m2 = 0;                                   // two running maxima, one per half
+    for (int64_t base = tid; base < n16; base += 4 * T) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (base + u * T < n16) v[u] = __ldcs(W4 + base + u * T);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (base + u * T < n16) {
+                m2 = __vmaxu2(m2, v[u].x & 0x7FFF7FFFu);
+                m2 = __vmaxu2(m2, v[u].y & 0x7FFF7FFFu);
+                m2 = __vmaxu2(m2, v[u].z & 0x7FFF7FFFu);
+                m2 = __vmaxu2(m2, v[u].w & 0x7FFF7FFFu);
+            }
     }
+    // the unaligned head and the ragged end
+    const int64_t rest = head + (n_pairs - head - 4 * n16);
+    for (int64_t i = tid; i < rest; i += T) {
+        const int64_t j = i < head ? i : head + 4 * n16 + (i - head);
+        m2 = __vmaxu2(m2, __ldcs(W + j) & 0x7FFF7FFFu);
+    }
+    uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
     if (tail != nullptr && blockIdx.x == 0 && threadIdx.x == 0) m = max(m, (uint32_t)(*tail & 0x7FFFu));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
@@ -192,7 +222,110 @@ __device__ __forceinline__ uint32_t e2m1_code_thresholds(float w, const double (
     return (c != 0u && w < 0.0f) ? (c | 8u) : c;
 }
 
-// One thread = two groups of 16 BF16 weights (64 bytes) -> 4 words + 2 scale bytes.
+// The two codes of a BF16 pair (low half in bits 0..3) by the exact FP64
+// thresholds of the step E4M3(sc) * g; out of line, taken rarely.
+__device__ __noinline__ uint32_t e2m1_pair_exact(uint32_t x, uint32_t sc, double gd) {
+    const double step = e4m3_value_f64(sc) * gd;                  // exact
+    const double tq[7] = {0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0};
+    double th[7];
+#pragma unroll
+    for (int i = 0; i < 7; ++i) th[i] = tq[i] * step;             // exact
+    return e2m1_code_thresholds(bf16_lo(x), th) | (e2m1_code_thresholds(bf16_hi(x), th) << 4);
+}
+
+// Two FP32 values -> two E4M3 codes (a in bits 0..7, b in bits 8..15), nearest
+// even, saturating at 448.
+__device__ __forceinline__ uint32_t e4m3x2_from_f32(float a, float b) {
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(d) : "f"(a), "f"(b));
+    return d;
+}
+
+// Packed pairs of FP32 (sm_100 f32x2 multiply, each lane rounded to nearest
+// even as the scalar form): the two BF16 halves of a word widened exactly, a
+// splat, the lane-wise product, and the lanes back.
+__device__ __forceinline__ uint64_t f2_from_bf16x2_fp4(uint32_t w) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(w << 16), "r"(w & 0xFFFF0000u));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_splat_fp4(float x) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t e2m1x2_from_f2(uint64_t d) {
+    uint32_t r;
+    asm("{\n\t.reg .f32 lo, hi;\n\t.reg .b8 t;\n\tmov.b64 {lo, hi}, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, hi, lo;\n\tcvt.u32.u8 %0, t;\n\t}"
+        : "=r"(r)
+        : "l"(d));
+    return r;
+}
+
+constexpr int kNvPairsInFlight = 2;
+
+// One group of 16 BF16 weights (v[0..7]) -> two words of codes; returns the
+// group's E4M3 scale code.  r6g = fl32(1 / fl32(6 g)) and fast (g in
+// [2^-100, 2^100]) are per tensor.
+__device__ __forceinline__ uint32_t nvfp4_group(const uint32_t *v, float g, double gd, float r6g,
+                                                bool fast, uint32_t *words) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m = __vmaxu2(m, v[j] & 0x7FFF7FFFu);
+    const float amax = __uint_as_float(max(m & 0xFFFFu, m >> 16) << 16);
+    uint32_t sc = 0xFFu;
+    if (fast) {
+        // the quotient amax / (6 g) to within 1.5 * 2^-23; both ends of the
+        // 2^-20 band round alike unless it is near an E4M3 midpoint
+        const float q = __fmul_rn(amax, r6g);
+        const uint32_t two = e4m3x2_from_f32(__fmul_rn(q, 1.0f - 0x1p-20f), __fmul_rn(q, 1.0f + 0x1p-20f));
+        if (q <= 0x1p20f && (two & 0xFFu) == (two >> 8)) sc = two & 0xFFu;
+    }
+    if (sc == 0xFFu) sc = e4m3_code_f64(__ddiv_rn((double)amax, 6.0 * gd));
+    if (sc == 0u) {                                 // the scale rounds to 0: zeros
+        words[0] = words[1] = 0u;
+        return 0u;
+    }
+    if (fast) {
+        // rs = fl32(1 / fl32(E4M3(sc) * g)) is within 2^-23 of 1 / step, so
+        // w * rs is within 2^-22 of w / step; the band ends fold into rs
+        const float e = e4m3_to_f32(sc);
+        const float rs = __frcp_rn(__fmul_rn(e, g));
+        const uint64_t lo2 = f2_splat_fp4(__fmul_rn(rs, 1.0f - 0x1p-19f));
+        const uint64_t hi2 = f2_splat_fp4(__fmul_rn(rs, 1.0f + 0x1p-19f));
+#pragma unroll
+        for (int wd = 0; wd < 2; ++wd) {
+            uint32_t w = 0;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t x = v[4 * wd + k];
+                const uint64_t x2 = f2_from_bf16x2_fp4(x);
+                const uint32_t lo = e2m1x2_from_f2(f2_mul(x2, lo2));
+                const uint32_t hi = e2m1x2_from_f2(f2_mul(x2, hi2));
+                w |= (lo == hi ? lo : e2m1_pair_exact(x, sc, gd)) << (8 * k);
+            }
+            words[wd] = clear_negative_zeros(w);
+        }
+    } else {
+#pragma unroll
+        for (int wd = 0; wd < 2; ++wd) {
+            uint32_t w = 0;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) w |= e2m1_pair_exact(v[4 * wd + k], sc, gd) << (8 * k);
+            words[wd] = clear_negative_zeros(w);
+        }
+    }
+    return sc;
+}
+
+// One thread = two groups of 16 BF16 weights (64 bytes) -> 4 words + 2 scale
+// bytes, two such pairs in flight.
 __global__ void __launch_bounds__(kThreads) quant_nvfp4_kernel(const uint4 *__restrict__ W,
                                                                const float *__restrict__ g_dev,
                                                                uint4 *__restrict__ Wq,
@@ -201,72 +334,36 @@ __global__ void __launch_bounds__(kThreads) quant_nvfp4_kernel(const uint4 *__re
     const int64_t T = (int64_t)gridDim.x * blockDim.x;
     const float g = *g_dev;
     const double gd = (double)g;
-    const double six_g = 6.0 * gd;
-    for (int64_t gp = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; gp < npairs; gp += T) {
-        uint32_t v[16];
+    const bool fast = g >= 0x1p-100f && g <= 0x1p100f;
+    const float r6g = fast ? __frcp_rn(__fmul_rn(6.0f, g)) : 0.0f;
+    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < npairs;
+         base += kNvPairsInFlight * T) {
+        uint32_t v[kNvPairsInFlight][16];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const uint4 x = __ldcs(W + 4 * gp + c);
-            v[4 * c] = x.x;
-            v[4 * c + 1] = x.y;
-            v[4 * c + 2] = x.z;
-            v[4 * c + 3] = x.w;
-        }
-        uint32_t words[4];
-        uint32_t sc2 = 0;
+        for (int u = 0; u < kNvPairsInFlight; ++u) {
+            const int64_t gp = base + u * T;
+            if (gp < npairs) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {                    // group h: v[8h .. 8h + 7]
-            uint32_t m = 0;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const uint32_t a = v[8 * h + j] & 0x7FFF7FFFu;
-                m = max(m, max(a & 0xFFFFu, a >> 16));
-            }
-            const double amax = (double)__uint_as_float(m << 16);
-            const uint32_t sc = e4m3_code_f64(__ddiv_rn(amax, six_g));
-            sc2 |= sc << (8 * h);
-            const double step = e4m3_value_f64(sc) * gd;          // exact
-            double th[7];
-            const double tq[7] = {0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0};
-#pragma unroll
-            for (int i = 0; i < 7; ++i) th[i] = tq[i] * step;   // exact
-            // Fast path: r = w * fl32(1 / step) in FP32 is within 2^-22 of w /
-            // step (relative); rounding r * (1 -+ 2^-19) with the hardware E2M1
-            // conversion gives the same code at both ends unless the exact
-            // quotient is within that band of a rounding midpoint (a tie
-            // included), and then it is the code of the exact quotient.  Pairs
-            // whose two ends differ take the exact FP64 thresholds.
-            const bool fast = step > 0x1p-100;
-            const float rs = fast ? (float)(1.0 / step) : 0.0f;
-            constexpr float kLo = 1.0f - 0x1p-19f, kHi = 1.0f + 0x1p-19f;
-#pragma unroll
-            for (int wd = 0; wd < 2; ++wd) {
-                uint32_t w = 0;
-                if (step > 0.0) {
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint32_t x = v[8 * h + 4 * wd + k];
-                        const float a = bf16_lo(x), b = bf16_hi(x);
-                        uint32_t byte;
-                        bool exact = !fast;
-                        if (fast) {
-                            const float ra = __fmul_rn(a, rs), rb = __fmul_rn(b, rs);
-                            const uint32_t lo = e2m1x2_from_f32(__fmul_rn(ra, kLo), __fmul_rn(rb, kLo));
-                            const uint32_t hi = e2m1x2_from_f32(__fmul_rn(ra, kHi), __fmul_rn(rb, kHi));
-                            byte = lo;
-                            exact = lo != hi;
-                        }
-                        if (exact)
-                            byte = e2m1_code_thresholds(a, th) | (e2m1_code_thresholds(b, th) << 4);
-                        w |= byte << (8 * k);
-                    }
+                for (int c = 0; c < 4; ++c) {
+                    const uint4 x = __ldcs(W + 4 * gp + c);
+                    v[u][4 * c] = x.x;
+                    v[u][4 * c + 1] = x.y;
+                    v[u][4 * c + 2] = x.z;
+                    v[u][4 * c + 3] = x.w;
                 }
-                words[2 * h + wd] = clear_negative_zeros(w);
             }
         }
-        __stcs(Wq + gp, make_uint4(words[0], words[1], words[2], words[3]));
-        S[2 * gp] = (uint8_t)(sc2 & 0xFFu);
-        S[2 * gp + 1] = (uint8_t)(sc2 >> 8);
+#pragma unroll
+        for (int u = 0; u < kNvPairsInFlight; ++u) {
+            const int64_t gp = base + u * T;
+            if (gp >= npairs) break;
+            uint32_t words[4];
+            const uint32_t s0 = nvfp4_group(&v[u][0], g, gd, r6g, fast, &words[0]);
+            const uint32_t s1 = nvfp4_group(&v[u][8], g, gd, r6g, fast, &words[2]);
+            __stcs(Wq + gp, make_uint4(words[0], words[1], words[2], words[3]));
+            S[2 * gp] = (uint8_t)s0;                   // S is only byte-aligned
+            S[2 * gp + 1] = (uint8_t)s1;
+        }
     }
 }
 
@@ -339,9 +436,9 @@ extern "C" w4_status w4_nvfp4_tensor_scale(const w4_bf16 *W, int64_t n, float *g
     if (cudaMemsetAsync(g, 0, sizeof(float), st) != cudaSuccess) return w4host::launch_status();
     const int64_t pairs = n / 2;
     const uint16_t *tail = (n & 1) ? reinterpret_cast<const uint16_t *>(W) + (n - 1) : nullptr;
-    const int grid = (int)std::min<int64_t>(std::max<int64_t>(1, (pairs + kThreads * 8 - 1) /
-                                                                     (kThreads * 8)),
-                                            (int64_t)w4host::num_sms() * 8);
+    const int grid = (int)std::min<int64_t>(std::max<int64_t>(1, (pairs + kThreads * 16 - 1) /
+                                                                     (kThreads * 16)),
+                                            (int64_t)w4host::num_sms() * 4);
     amax_bf16_kernel<<<grid, kThreads, 0, st>>>(reinterpret_cast<const uint32_t *>(W), pairs, tail,
                                                 reinterpret_cast<unsigned int *>(g));
     tensor_scale_kernel<<<1, 1, 0, st>>>(reinterpret_cast<unsigned int *>(g));
@@ -355,7 +452,8 @@ extern "C" w4_status w4_quantize_pack_nvfp4(const w4_bf16 *W, const float *g, in
     if (g == nullptr || (reinterpret_cast<uintptr_t>(g) & 3u) != 0) return W4_ERR_INVALID_ARG;
     const int64_t npairs = rows * K / 32;
     if (npairs == 0) return W4_OK;
-    quant_nvfp4_kernel<<<grid_for(npairs), kThreads, 0, (cudaStream_t)stream>>>(
+    quant_nvfp4_kernel<<<grid_for((npairs + kNvPairsInFlight - 1) / kNvPairsInFlight), kThreads, 0,
+                         (cudaStream_t)stream>>>(
         reinterpret_cast<const uint4 *>(W), g, reinterpret_cast<uint4 *>(Wq), S, npairs);
     return w4host::launch_status();
 }

@@ -435,6 +435,19 @@ __global__ void __launch_bounds__(gemm_threads(NDQ, KB, NSPLIT, WGL), 1)
         if (KB == 256 && FP4 == 0) tma_prefetch_desc(&tm_s);
         if (!MOE) tma_prefetch_desc(&tm_x);
     }
+    // Decode tiles: warm L2 with this CTA's first weight and scale tiles (its
+    // work items follow from the parameters alone) while the kernel before it
+    // drains; measured faster chained behind another GEMM, where the warp-level
+    // decode kernel measured slower with the same prefetch.
+    if (KB == 256 && !MOE && !QAT && threadIdx.x == 0) {
+        ItemIter I = make_iter(p, p.n_row_tiles * p.n_tok_tiles);
+        int rt, tt, kb0, kb1, left = 32;
+        while (left > 0 && next_item(I, p, rt, tt, kb0, kb1))
+            for (int kb = kb0; kb < kb1 && left > 0; ++kb, --left) {
+                tma_prefetch_l2_2d(&tm_w, kb * kWords, rt * p.rows_per_tile);
+                if (FP4 == 0) tma_prefetch_l2_2d(&tm_s, kb * 8, rt * p.rows_per_tile);
+            }
+    }
     // the kernel before this one on the stream may still be running: no global
     // memory (and no tensor memory, which a co-resident CTA of it may hold)
     // is touched before it completes

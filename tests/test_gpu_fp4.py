@@ -140,6 +140,37 @@ def test_quantize_nvfp4_every_bf16_value():
     _check_nv(small.reshape(-1, 256))
 
 
+def _nv_tie_groups(amax_t: float) -> np.ndarray:
+    """Groups of 16 whose amax runs through every positive BF16 value up to
+    amax_t (the tensor's amax, so g = fl32(amax_t / 2688)), each holding the
+    E2M1 rounding midpoints of its expected step (E4M3(amax / 6), +-0.25 ..
+    +-5 of it) and a zero; rows of 16 groups, zero-padded."""
+    vals = (np.arange(1, 0x7F80, dtype=np.uint32) << 16).view(np.float32)
+    vals = vals[vals <= amax_t]
+    # torch's E4M3 conversion does not saturate: clamp at 448 first
+    step = torch.from_numpy(np.minimum(vals / np.float32(6.0), np.float32(448.0)))
+    step = step.to(torch.float8_e4m3fn).float().numpy()
+    tq = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32)
+    el = step[:, None] * tq[None, :]
+    grp = np.concatenate([vals[:, None], el, -el, np.zeros((len(vals), 1), np.float32)], axis=1)
+    assert not np.any(grp.view(np.uint32) & 0xFFFF)          # all exact in BF16
+    g_bits = (grp.view(np.uint32) >> 16).astype(np.uint16)
+    pad = (-len(g_bits)) % 16
+    g_bits = np.concatenate([g_bits, np.zeros((pad, 16), np.uint16)])
+    return g_bits.reshape(-1, 256)
+
+
+@pytest.mark.parametrize("amax_t", [2688.0, 2944.0])
+def test_quantize_nvfp4_scale_and_code_ties(amax_t):
+    """At g = 1 (tensor amax 2688) many group scales amax / 6 are exact E4M3
+    midpoints and the elements exact E2M1 midpoints of their step: both
+    decisions reach their exact FP64 path and must round ties to the even code.
+    At g = fl32(2944 / 2688) the quotients fall near the midpoints instead."""
+    W = _nv_tie_groups(amax_t)
+    assert (W[:, :].view(np.uint16) & 0x7FFF).max() == np.float32(amax_t).view(np.uint32) >> 16
+    _check_nv(W)
+
+
 def test_quantize_nvfp4_row_scales_span_e4m3():
     """Rows scaled by 2^0 .. 2^-40 under one tensor scale: group scales run
     through every E4M3 binade, the subnormals and zero."""
@@ -170,6 +201,22 @@ def test_nvfp4_tensor_scale_odd_length():
     g = torch.empty(1, dtype=torch.float32, device=DEV)
     w4.w4_nvfp4_tensor_scale(W.to(DEV), g)
     assert g.item() == float(np.float32(7.0) / np.float32(2688.0))
+
+
+@pytest.mark.parametrize("where", [0, 3, 500, 1998])
+def test_nvfp4_tensor_scale_unaligned_views(where):
+    """Views starting 4, 8 and 12 bytes past a 16-byte boundary: the amax pass
+    reads the pairs before the first boundary and after the last whole 16
+    bytes one word at a time; the largest value sits in the head, the middle
+    or the ragged end."""
+    base = synth.normal_bf16((1, 4096), 0.02, seed=6).reshape(-1).to(DEV)
+    for off in (2, 4, 6):
+        W = base[off:off + 2002]
+        W[where] = -5.0
+        g = torch.empty(1, dtype=torch.float32, device=DEV)
+        w4.w4_nvfp4_tensor_scale(W, g)
+        assert g.item() == float(np.float32(5.0) / np.float32(2688.0)), (off, where)
+        W[where] = 0.0
 
 
 def test_fp4_quantize_layer_shape():
