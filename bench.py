@@ -51,11 +51,11 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # (profiles/ holds the summaries and commands); an entry is used only while the
 # kernel's source file is unchanged since the capture.
 NCU_TRAFFIC = {
-    ("gemm_m16", "decode"): {"bytes": 28519168 + 0, "file": "w4_gemm.cu", "src": "a9f5ca1fc2175494"},
-    ("gemm_m1", "decode"): {"bytes": 28344064 + 0, "file": "w4_gemv.cu", "src": "4ebd40701504f1ee"},
-    ("fake_quant", "decode"): {"bytes": 100691456 + 50415872, "file": "w4_quant.cu", "src": "63bc5e9cb458e7cb"},
-    ("ste_backward", "decode"): {"bytes": 100672512 + 45052160, "file": "w4_quant.cu", "src": "63bc5e9cb458e7cb"},
-    ("quantize_pack", "decode"): {"bytes": 100688128 + 5947392, "file": "w4_quant.cu", "src": "63bc5e9cb458e7cb"},
+    ("gemm_m16", "decode"): {"bytes": 28523008 + 0, "file": "w4_gemm.cu", "src": "389a57b5497f8f27"},
+    ("gemm_m1", "decode"): {"bytes": 28345088 + 0, "file": "w4_gemv.cu", "src": "bee317c18421180b"},
+    ("fake_quant", "decode"): {"bytes": 100688640 + 47492864, "file": "w4_quant.cu", "src": "daef7cabc96462d0"},
+    ("ste_backward", "decode"): {"bytes": 100670976 + 45220864, "file": "w4_quant.cu", "src": "daef7cabc96462d0"},
+    ("quantize_pack", "decode"): {"bytes": 100686848 + 5896448, "file": "w4_quant.cu", "src": "daef7cabc96462d0"},
 }
 
 
