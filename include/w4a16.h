@@ -42,6 +42,12 @@
  *     enqueues kernels on `stream` and returns; it never synchronizes, never
  *     allocates device memory and keeps no pointer after it returns.  Scratch
  *     memory, where a schedule uses some, is passed in by the caller.
+ *   - The GEMM kernels are launched with programmatic stream serialization:
+ *     they may become resident while the previous kernel on `stream` still
+ *     runs, but read and write no buffer (weights, scales, activations,
+ *     outputs, workspace) before it has completed, so stream order is as for
+ *     a plain launch.  Before that point they only set up shared memory and
+ *     may issue L2 prefetches (cache hints) of their own weight tiles.
  *   - group must be 32 (else W4_ERR_UNSUPPORTED); K must be a positive
  *     multiple of 32.
  *   - A kernel launch failure returns W4_ERR_CUDA (w4_last_cuda_error() gives

@@ -301,6 +301,31 @@ def test_gemm_decode_config(M, split):
     assert_gemm_close(Y, R, f"decode M={M} split={split}")
 
 
+@pytest.mark.parametrize("M", [1, 8, 16, 32])
+def test_gemm_reads_weights_the_previous_kernel_wrote(M):
+    """The GEMMs may become resident (and warm L2 with their weight tiles)
+    while the kernel before them on the stream still runs.  Here that kernel
+    overwrites the packed weights and scales the GEMM reads, right after a GEMM
+    on the old contents: the product must be that of the new weights."""
+    N, K = 4096, 2048
+    Wa = synth.normal_bf16((N, K), 0.02, seed=11).to(DEV)
+    Wb = synth.normal_bf16((N, K), 0.5, seed=12).to(DEV)
+    X = synth.normal_bf16((M, K), 1.0, seed=13).to(DEV)
+    Wq = torch.empty((N, K // 8), dtype=torch.int32, device=DEV)
+    S = torch.empty((N, K // 32), dtype=torch.bfloat16, device=DEV)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=DEV)
+    for _ in range(3):
+        w4.w4_quantize_pack(Wa, Wq, S)
+        w4.w4a16_gemm(X, Wq, S, Y)
+        w4.w4_quantize_pack(Wb, Wq, S)
+        w4.w4a16_gemm(X, Wq, S, Y)
+    w4.w4_device_status()
+    oWq, oS = oracle.quantize_pack(bits(Wb.cpu()))
+    assert np.array_equal(Wq.cpu().numpy(), oWq)
+    _, R = oracle.w4a16_gemm(bits(X.cpu()), oWq, oS)
+    assert_gemm_close(bits(Y), R, f"weights rewritten before the GEMM, M={M}")
+
+
 def test_gemm_split_workspace_left_zero_and_deterministic():
     M, N, K = 16, 4096 + 200, 2048          # ragged last row tile, 8 k-blocks
     X, Wq, S, Y1 = _gemm_case(M, N, K, seed=5)
