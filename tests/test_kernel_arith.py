@@ -18,6 +18,12 @@ cast to float32 is the single rounding of the fused operation.
    for every finite BF16 x in that range against every BF16 significand of s at
    three exponents (the subnormal edge, 1, 2^90), with every fp32 reciprocal
    within one ulp of 1/s and with a two-ulp perturbation both ways.
+4. The NVFP4 quantizer's two band decisions: an FP32 quotient (group scale:
+   amax * fl32(1 / fl32(6 g)); element: w * fl32(1 / fl32(E4M3(sc) * g)), the
+   band folded into the reciprocal) is rounded at both ends of a relative band
+   (2^-20, 2^-19); wherever the two ends agree, that code is the oracle's
+   rounding of the FP64 quotient.  Checked for every BF16 value in range under
+   several tensor scales; the FP32 arithmetic is numpy's IEEE float32.
 """
 import numpy as np
 import pytest
@@ -89,6 +95,50 @@ def test_zero_point_snap_rounding_matches_ieee_quotient(s_exp):
             c = _f32(SNAP_Z + k / 512.0 + TOINT_Z)       # fadd: round to an integer
             q = c.astype(np.float64) - MAGIC
             assert np.array_equal(q, ref), (S, float(r))
+
+
+_TENSOR_SCALES = [1.0, float(np.float32(2944.0) / np.float32(2688.0)),
+                  float(np.float32(0.07) / np.float32(2688.0)), float(np.float32(3.1e-25))]
+
+
+def _finite_positive_bf16():
+    return (np.arange(1, 0x7F80, dtype=np.uint32) << 16).view(np.float32)
+
+
+@pytest.mark.parametrize("g", _TENSOR_SCALES)
+def test_nvfp4_scale_band_decision(g):
+    g32 = F32(g)
+    enc = np.vectorize(oracle.e4m3_encode, otypes=[np.int64])
+    amax = _finite_positive_bf16()
+    amax = amax[amax.astype(np.float64) <= 2688.0 * float(g32) * (1 + 2.0 ** -20)]
+    r6g = F32(1.0) / (F32(6.0) * g32)                    # fl32(1 / fl32(6 g))
+    q = amax * r6g
+    lo = enc((q * F32(1.0 - 2.0 ** -20)).astype(np.float64))
+    hi = enc((q * F32(1.0 + 2.0 ** -20)).astype(np.float64))
+    ref = enc(amax.astype(np.float64) / (6.0 * float(g32)))
+    agree = lo == hi
+    assert np.array_equal(lo[agree], ref[agree])
+    assert (~agree).sum() <= max(200, len(amax) // 50)  # the FP64 path stays rare
+
+
+@pytest.mark.parametrize("g", _TENSOR_SCALES)
+def test_nvfp4_element_band_decision(g):
+    g32 = F32(g)
+    enc = np.vectorize(oracle.e2m1_encode, otypes=[np.int64])
+    w_all = _finite_positive_bf16()
+    w_all = np.concatenate([w_all, -w_all])
+    for sc in (0x01, 0x07, 0x08, 0x2B, 0x38, 0x51, 0x7E):
+        e = F32(oracle.e4m3_value(sc))
+        step = float(e) * float(g32)                         # exact in FP64
+        w = w_all[np.abs(w_all.astype(np.float64)) <= 7.0 * step]
+        rs = F32(1.0) / (e * g32)                            # fl32(1 / fl32(E4M3(sc) g))
+        lo = enc((w * (rs * F32(1.0 - 2.0 ** -19))).astype(np.float64)) & 7
+        hi = enc((w * (rs * F32(1.0 + 2.0 ** -19))).astype(np.float64)) & 7
+        ref = enc(w.astype(np.float64) / step) & 7            # magnitudes: the sign is w's
+        agree = lo == hi
+        assert agree.sum() > 0
+        assert np.array_equal(lo[agree], ref[agree]), (sc, g)
+        assert (~agree).sum() <= max(50, len(w) // 100)
 
 
 def _bf16_rne(x64: np.ndarray) -> np.ndarray:
